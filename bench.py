@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Benchmark of the fused pair-bias attention (features -> folded MLP ->
+masked attention with the bias kept on chip) on the N=128 jets, P=128 slots,
+H=8, D=16 workload.
+
+One step = one call of pair_attention_forward over one batch of synthetic
+jets (one kernel launch). Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank processes its own batch (jets are
+independent; no collective on the data path), so per-GPU work is fixed and
+the scaling is weak. Timing: CUDA events on the launching stream, bracketed
+by a barrier and a synchronize, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from part_pair_bias_b200 import configs, synth  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+MLP_FLOP_PER_PAIR = 2 * (4 * 64 + 64 * 64 + 64 * 64 + 64 * 8)          # 17,920 (algorithmic)
+MMA_FLOP_PER_ROW = 2 * (16 * 64 + 64 * 64 + 64 * 64 + 64 * 16)         # 20,480 (issued per tile row)
+PROFILE = os.path.join(ROOT, "profiles", "k_fused_n128_p128.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "part_pair_bias_b200", "csrc", f)
+                  for f in ("pb_kernels.cuh", "pb_device.cuh", "pairbias.cu")]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="n128_p128")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def pair_counts(b):
+    m = b.mult.astype(np.int64)
+    unordered = m * (m + 1) // 2
+    tiles = (unordered + 127) // 128
+    return int(unordered.sum()), int(tiles.sum()), int((m * m).sum())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d.get("bf16_tflops"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def kernel_sha():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    if not os.path.exists(PROFILE):
+        return None
+    kv = {}
+    for line in open(PROFILE):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha") != kernel_sha():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, reasons) taken while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.rows, self.proc, self.window = [], None, None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        inside = [r for t, r in self.rows if t0 <= t <= t1]
+        note = None
+        if not inside:  # region shorter than the sampling period: nearest samples after its start
+            inside = [r for t, r in self.rows if t >= t0][:3] or [self.rows[-1][1]]
+            note = "timed region shorter than the 50 ms sampling period; nearest samples"
+        sm = [float(r[1]) for r in inside if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in inside if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+               "reasons": reasons, "samples": len(inside)}
+        if note:
+            out["note"] = note
+        return out
+
+
+def cpu_baseline(b, seconds):
+    """The fp64 oracle, as it stands, on the host cores: full batches until
+    `seconds` have passed (at least one)."""
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        oracle.forward(b)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    return {"value": passes * b.N / dt, "unit": "jets/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{passes} pass(es) over the full {b.N}-jet batch, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------- our path
+
+def run_ours(args, world, rank, local):
+    from part_pair_bias_b200 import ops
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl = args.workload
+    b = synth.make_jets(**configs.workload(wl, seed=args.seed + rank))
+    unordered, tiles, ordered = pair_counts(b)
+    mlp = ops.folded_mlp(b.params, dev)
+
+    set_bytes = 4 * b.E.nbytes + (b.mask.nbytes if b.mask is not None else b.ptr.nbytes) + 4 * b.q.nbytes
+    R = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes) + 1))
+    sets = []
+    for _ in range(R):
+        jets = ops.jets_to_device(b, dev)
+        q, k, v = (ops.bf16_to_device(x, dev) for x in (b.q, b.k, b.v))
+        sets.append((jets, q, k, v, torch.empty_like(q)))
+
+    def step(i):
+        jets, q, k, v, out = sets[i % R]
+        ops.pair_attention_forward(jets, mlp, None, q, k, v, out)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if ops.get_device_status():
+        raise RuntimeError("device status set during warm-up")
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_index = vis.split(",")[local] if vis else str(local)
+    sampler = ClockSampler(gpu_index) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record()
+    for i in range(K):
+        ev_s[i].record()
+        step(args.warmup + i)
+        ev_e[i].record()
+    end.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.summary(t0, t1) if sampler else None
+    if sampler:
+        sampler.stop()
+    ms = start.elapsed_time(end)
+    launch_ms = statistics.mean(ev_s[i].elapsed_time(ev_e[i]) for i in range(K))
+    status = ops.get_device_status()
+
+    # end to end through the public API from pinned host buffers
+    host = dict(E=torch.from_numpy(b.E).pin_memory(), px=torch.from_numpy(b.px).pin_memory(),
+                py=torch.from_numpy(b.py).pin_memory(), pz=torch.from_numpy(b.pz).pin_memory(),
+                mask=torch.from_numpy(b.mask).pin_memory(),
+                q=torch.from_numpy(b.q.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                k=torch.from_numpy(b.k.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                v=torch.from_numpy(b.v.view(np.int16)).view(torch.bfloat16).pin_memory())
+    jets, q, k, v, out = sets[0]
+    dst = dict(E=jets.E, px=jets.px, py=jets.py, pz=jets.pz, mask=jets.mask, q=q, k=k, v=v)
+    out_host = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    Ke = max(1, min(K, 500))
+
+    def e2e_step():
+        for name, t in host.items():
+            dst[name].copy_(t, non_blocking=True)
+        ops.pair_attention_forward(jets, mlp, None, q, k, v, out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record()
+    for _ in range(Ke):
+        e2e_step()
+    ee.record()
+    torch.cuda.synchronize()
+    e2e_ms = es.elapsed_time(ee)
+    status |= ops.get_device_status()
+
+    t = torch.tensor([ms, e2e_ms, launch_ms, float(status)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        dist.destroy_process_group()
+    ms, e2e_ms, launch_ms, status = t.tolist()
+    if rank != 0:
+        return
+    if status:
+        raise RuntimeError(f"device status bits {int(status):#x} during the timed region")
+
+    jets_total = b.N * K * world
+    value = jets_total / (ms / 1e3)
+    peak_tf, hbm_gbs, peak_src = measured_peaks()
+    alg_flop = unordered * MLP_FLOP_PER_PAIR
+    achieved_tf = alg_flop / (launch_ms / 1e3) / 1e12
+    exec_tf = tiles * 128 * MMA_FLOP_PER_ROW / (launch_ms / 1e3) / 1e12
+    dense_tf = b.N * b.P * b.P * MLP_FLOP_PER_PAIR / (launch_ms / 1e3) / 1e12
+    traffic = profiled_traffic()
+    line = {
+        "metric": "jets/s for fused pair-bias attention (P=128,H=8,D=16); % bf16 tensor peak",
+        "value": value,
+        "unit": "jets/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16 MLP operands, bf16 Q/K/V/out, fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": wl, "jets_per_gpu": b.N, "P": b.P, "H": 8, "D": 16, "layout": b.layout,
+                   "mean_multiplicity": float(b.mult.mean()), "path": "fused (bias on chip)",
+                   "l2": f"{R} rotating input sets of {set_bytes / 2**20:.1f} MiB (> 2x L2)",
+                   "parallelism": f"data-parallel over jets x{world}, no collective"},
+        "pairs_per_s": ordered * K * world / (ms / 1e3),
+        "gpu_launches": K,
+        "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved_tf / peak_tf, "traffic": traffic,
+                     "kernel": "k_fused", "launch_ms": launch_ms,
+                     "flop_per_launch": alg_flop,
+                     "flop_convention": "algorithmic: 17,920 per valid unordered pair (incl. diagonal)",
+                     "exec_tflops": exec_tf, "dense_equiv_tflops": dense_tf,
+                     "peak_source": f"{peak_src} bf16 dense burst (f16 runs at the same tensor rate)"},
+        "clocks": clocks,
+        "e2e": {"value": b.N * Ke * world / (e2e_ms / 1e3), "unit": "jets/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores, on the same workload and metric;
+    each step is a bounded sample of 16 jets of the batch."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    b = synth.make_jets(**configs.workload(args.workload, seed=args.seed))
+    per = 16
+    samples = [synth.slice_jets(b, lo, min(b.N, lo + per)) for lo in range(0, b.N, per)]
+    for i in range(args.warmup):
+        oracle.forward(samples[i % len(samples)])
+    t0 = time.perf_counter()
+    jets = 0
+    for i in range(args.steps):
+        s = samples[i % len(samples)]
+        oracle.forward(s)
+        jets += s.N
+    dt = time.perf_counter() - t0
+    value = jets / dt
+    cores = oracle.threads()
+    line = {
+        "metric": "jets/s for fused pair-bias attention (P=128,H=8,D=16); % bf16 tensor peak",
+        "value": value, "unit": "jets/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / max(1, args.steps), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "jets_per_step": per, "P": b.P, "H": 8, "D": 16},
+        "cpu_baseline": {"value": value, "unit": "jets/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per} jets of the {b.N}-jet batch per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": "jets/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

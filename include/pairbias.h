@@ -1,0 +1,157 @@
+/*
+ * pairbias.h -- C ABI of the B200 (sm_100a) Particle-Transformer pair-bias library.
+ *
+ * The operations are those of "Event Classification with Masked Transformer
+ * Autoencoders" (ml4sci_cms_e2e26 README):
+ *   - section "Fusion 2 -- Pairwise Features + Conv1d MLP -> FusedPairMLP":
+ *     four Lorentz-invariant features per particle pair (ln kT, ln z, ln dR,
+ *     ln m^2) and the pair-embedding MLP 4 -> 64 -> 64 -> 64 -> 8 with its
+ *     batch-norm affines folded into the weights and GELU after each hidden
+ *     layer, producing one attention bias per head, U[h, i, j];
+ *   - section "Fusion 3 -- Self-Attention + Additive Bias -> Fused Triton
+ *     Attention": softmax(Q K^T / sqrt(D) + U) V with masked keys excluded.
+ * Feature definitions: dy = y_a - y_b (rapidity), dphi wrapped to (-pi, pi],
+ * dR = sqrt(dy^2 + dphi^2), kT = min(pT) dR, z = min(pT) / (pT_a + pT_b),
+ * m^2 = (E_a + E_b)^2 - |p_a + p_b|^2, each feature ln(max(x, 1e-8)).
+ * Diagonal pairs (i == j) are included. Masked query rows of the attention
+ * output are 0.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers owned by the caller, except in
+ *     pb_fold_affine (host). Nothing is allocated inside the library.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream), launches exactly one kernel and
+ *     does not synchronise. Host-side argument errors return before any
+ *     launch; device-side problems (an invalid ptr array, a bounded wait that
+ *     ran out) set bits of a per-device status word, read with
+ *     pb_get_device_status.
+ *   - H must be 8 and D must be 16 (the MLP output width fixes H);
+ *     1 <= P <= 256. Other values return PB_EUNSUPPORTED.
+ *   - Q, K, V, out and U pointers must be 16-byte aligned; momentum, mask and
+ *     ptr arrays 4-byte aligned (mask: 1-byte). Violations return PB_EINVAL.
+ *   - bf16 values travel as raw uint16_t bit patterns.
+ *   - Every element of every output is written: entries of masked pairs of
+ *     feat and U are 0, masked query rows of out are 0.
+ *   - On error, pb_last_error() returns a message (thread-local).
+ */
+#ifndef PAIRBIAS_H
+#define PAIRBIAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PB_OK = 0,
+  PB_EINVAL = 1,        /* null / misaligned pointer, negative size, bad dtype  */
+  PB_EUNSUPPORTED = 2,  /* H != 8, D != 16, P outside [1, 256]                   */
+  PB_ECUDA = 3,         /* a CUDA runtime call failed (launch, attribute, copy)  */
+  PB_EDEVICE = 4        /* the device status word reported an error              */
+} pb_status;
+
+typedef enum { PB_BF16 = 0, PB_F32 = 1 } pb_dtype;
+
+/* Device status bits (pb_get_device_status). */
+#define PB_DEV_TIMEOUT 1u   /* a bounded wait inside a kernel ran out; outputs invalid */
+#define PB_DEV_BADPTR 2u    /* a packed jet had ptr[n] > ptr[n+1], more than P tokens,
+                               or reached past `tokens`; that jet was skipped          */
+
+/* One batch of jets. Exactly one layout is used.
+ * Padded (ptr == NULL): E, px, py, pz and mask are [N*P] (jet n, slot s at
+ *   n*P + s); mask != 0 marks a valid particle, any pattern is allowed.
+ *   Q/K/V/out are [N, H, P, D].
+ * Packed (ptr != NULL, mask ignored): jet n owns tokens ptr[n] .. ptr[n+1]-1
+ *   of the [tokens] momentum arrays ("ptr" jet boundaries as in
+ *   lloca.backbone.transformer_v2.Transformer.forward); every token is valid;
+ *   P is the largest multiplicity allowed; Q/K/V/out are [tokens, H, D].
+ * Momenta are energy-first (E, px, py, pz), fp32, GeV. */
+typedef struct pb_jets {
+  const float *E, *px, *py, *pz;
+  const uint8_t *mask;
+  const int32_t *ptr;
+  int32_t N;
+  int32_t P;
+  int64_t tokens;        /* packed only: length of the momentum arrays */
+} pb_jets;
+
+/* Folded pair-embedding MLP, fp32, device pointers, row-major [out][in]. */
+typedef struct pb_mlp {
+  const float *W1, *b1;  /* [64][4], [64]  (input affine and layer-1 affine folded in) */
+  const float *W2, *b2;  /* [64][64], [64] (layer-2 affine folded in)                  */
+  const float *W3, *b3;  /* [64][64], [64] (layer-3 affine folded in)                  */
+  const float *W4, *b4;  /* [8][64], [8]   (plain output Linear)                       */
+} pb_mlp;
+
+/* Unfolded MLP as a model holds it, host pointers, fp32:
+ *   x = a0*f + c0;  h_k = GELU(a_k*(W_k h_{k-1} + b_k) + c_k), k = 1..3;
+ *   U = W4 h_3 + b4.  (a_k, c_k are the eval-mode batch-norm scale and shift.) */
+typedef struct pb_mlp_unfolded {
+  const float *a0, *c0;              /* [4]                      */
+  const float *W1, *b1, *a1, *c1;    /* [64][4], [64], [64], [64] */
+  const float *W2, *b2, *a2, *c2;    /* [64][64], [64] x 3        */
+  const float *W3, *b3, *a3, *c3;    /* [64][64], [64] x 3        */
+  const float *W4, *b4;              /* [8][64], [8]              */
+} pb_mlp_unfolded;
+
+/* Offsets (in floats) of the folded parameters inside the flat buffer that
+ * pb_fold_affine writes; PB_FOLDED_FLOATS is its length. */
+enum {
+  PB_OFF_W1 = 0, PB_OFF_B1 = 256, PB_OFF_W2 = 320, PB_OFF_B2 = 4416,
+  PB_OFF_W3 = 4480, PB_OFF_B3 = 8576, PB_OFF_W4 = 8640, PB_OFF_B4 = 9152,
+  PB_FOLDED_FLOATS = 9160
+};
+
+/* pairfeat_compute -- the four pair features of every slot pair.
+ * feat: fp32 [N, P, P, 4], channel order (ln kT, ln z, ln dR, ln m^2);
+ * feat[n, i, j] == feat[n, j, i] bit for bit; pairs with a masked (or, packed,
+ * absent) end are 0. Source: "Fusion 2" (features half). */
+pb_status pairfeat_compute(const pb_jets *jets, float *feat, void *stream);
+
+/* pairbias_mlp_forward -- features and folded MLP, materialising the bias.
+ * U: [N, 8, P, P] in `dtype` (PB_BF16 raw bits or PB_F32); U[n,h,i,j] ==
+ * U[n,h,j,i]; entries with a masked end are 0. The MLP runs on tcgen05 tensor
+ * cores with f16 operands and fp32 accumulation; hidden activations never
+ * leave the chip. Source: "Fusion 2". */
+pb_status pairbias_mlp_forward(const pb_jets *jets, const pb_mlp *mlp, void *U, pb_dtype dtype,
+                               void *stream);
+
+/* pair_attention_forward -- masked multi-head attention with the pair bias.
+ * Exactly one of `mlp` and `U` is non-NULL:
+ *   mlp != NULL: the fused path -- features, MLP and attention in one kernel;
+ *                the bias is produced and consumed on chip, never in HBM;
+ *   U   != NULL: the bias is read from a bf16 [N, 8, P, P] array (as written
+ *                by pairbias_mlp_forward with PB_BF16).
+ * q, k, v, out: bf16 in the layout of `jets` (padded [N,H,P,D], packed
+ * [tokens,H,D]). out = softmax(q k^T / sqrt(D) + U) v over valid keys, with
+ * fp32 scores, softmax and accumulation; masked query rows are 0.
+ * Source: "Fusion 3" (with the bias of "Fusion 2"). */
+pb_status pair_attention_forward(const pb_jets *jets, const pb_mlp *mlp, const uint16_t *U,
+                                 int H, int D, const uint16_t *q, const uint16_t *k,
+                                 const uint16_t *v, uint16_t *out, void *stream);
+
+/* pb_get_device_status -- synchronise `stream`, then read and clear the
+ * status word of the current device. *bits (may be NULL) receives the
+ * PB_DEV_* bits. Returns PB_OK when no bit was set, PB_EDEVICE otherwise,
+ * PB_ECUDA if the synchronisation itself failed. */
+pb_status pb_get_device_status(void *stream, uint32_t *bits);
+
+/* pb_fold_affine -- host helper, not on the GPU path: fold the batch-norm
+ * affines of an unfolded MLP into Linear weights and biases (the eval-time
+ * folding of "Fusion 2"), computing in double and rounding once to fp32.
+ * out: host buffer of PB_FOLDED_FLOATS floats, laid out by the PB_OFF_*
+ * offsets. Returns PB_EINVAL for a NULL pointer. */
+pb_status pb_fold_affine(const pb_mlp_unfolded *in, float *out);
+
+/* pb_last_error -- message for the last non-OK status of this thread. */
+const char *pb_last_error(void);
+
+/* pb_version -- library version string. */
+const char *pb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAIRBIAS_H */

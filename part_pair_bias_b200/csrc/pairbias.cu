@@ -1,0 +1,257 @@
+// pairbias.cu -- C-ABI entry points of the pair-bias library (include/pairbias.h).
+//
+// Host side only validates arguments, picks the template instance for P
+// (<= 128 or <= 256), sizes a persistent grid from the SM count and the
+// occupancy of that instance, and launches exactly one kernel on the caller's
+// stream. Nothing is allocated and nothing is synchronised here.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "pairbias.h"
+#include "pb_kernels.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+pb_status fail(pb_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Per-device launch facts, filled once per device and kernel instance.
+constexpr int kMaxDev = 64;
+struct DevInfo {
+  int sms = 0;
+};
+DevInfo g_dev[kMaxDev];
+std::mutex g_mu;
+
+pb_status device_sms(int* dev_out, int* sms_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDev) return fail(PB_ECUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev[dev].sms == 0) {
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(PB_ECUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    g_dev[dev].sms = sms;
+  }
+  *dev_out = dev;
+  *sms_out = g_dev[dev].sms;
+  return PB_OK;
+}
+
+// Raise the dynamic shared-memory limit of `kernel` (once per device) and
+// return the persistent grid size: SMs x resident CTAs, at most `work`.
+template <class K>
+pb_status prepare(K kernel, size_t smem, int threads, int work, int* grid) {
+  int dev = 0, sms = 0;
+  pb_status st = device_sms(&dev, &sms);
+  if (st != PB_OK) return st;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(%zu B smem): %s", smem, cudaGetErrorString(e));
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "occupancy query: %s", cudaGetErrorString(e));
+  if (per_sm < 1) return fail(PB_ECUDA, "kernel does not fit on an SM (%zu B smem)", smem);
+  long long g = (long long)sms * per_sm;
+  if (g > work) g = work;
+  *grid = (int)(g < 1 ? 1 : g);
+  return PB_OK;
+}
+
+pb_status launched(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(PB_ECUDA, "%s launch: %s", what, cudaGetErrorString(e));
+  return PB_OK;
+}
+
+pb_status check_jets(const pb_jets* j, pb::JetArgs* out) {
+  if (!j) return fail(PB_EINVAL, "jets is NULL");
+  if (j->N < 0) return fail(PB_EINVAL, "N = %d < 0", j->N);
+  if (j->P < 1 || j->P > 256) return fail(PB_EUNSUPPORTED, "P = %d outside [1, 256]", j->P);
+  *out = pb::JetArgs{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, j->P, 0};
+  if (j->N == 0) return PB_OK;  // nothing to read or write: pointers may be NULL
+  if (!j->E || !j->px || !j->py || !j->pz) return fail(PB_EINVAL, "a momentum pointer is NULL");
+  if (!aligned(j->E, 4) || !aligned(j->px, 4) || !aligned(j->py, 4) || !aligned(j->pz, 4))
+    return fail(PB_EINVAL, "momentum arrays must be 4-byte aligned");
+  if (j->ptr) {
+    if (!aligned(j->ptr, 4)) return fail(PB_EINVAL, "ptr must be 4-byte aligned");
+    if (j->tokens < 0) return fail(PB_EINVAL, "tokens = %lld < 0", (long long)j->tokens);
+  } else if (!j->mask) {
+    return fail(PB_EINVAL, "padded layout needs a mask (or pass ptr for the packed layout)");
+  }
+  *out = pb::JetArgs{j->E, j->px, j->py, j->pz, j->ptr ? nullptr : j->mask, j->ptr, j->N, j->P,
+                     (long long)j->tokens};
+  return PB_OK;
+}
+
+pb_status check_mlp(const pb_mlp* w, pb::MlpArgs* out) {
+  if (!w) return fail(PB_EINVAL, "mlp is NULL");
+  if (!w->W1 || !w->b1 || !w->W2 || !w->b2 || !w->W3 || !w->b3 || !w->W4 || !w->b4)
+    return fail(PB_EINVAL, "an MLP parameter pointer is NULL");
+  *out = pb::MlpArgs{w->W1, w->b1, w->W2, w->b2, w->W3, w->b3, w->W4, w->b4};
+  return PB_OK;
+}
+
+constexpr int kGroups = 2;  // tensor-core tile groups per CTA (128 threads each)
+
+template <int PM>
+pb_status run_pairfeat(const pb::JetArgs& J, float* feat, cudaStream_t s) {
+  auto k = pb::k_pairfeat<PM>;
+  const size_t smem = sizeof(pb::Particles<PM>);
+  int grid = 0;
+  pb_status st = prepare(k, smem, 256, J.N, &grid);
+  if (st != PB_OK) return st;
+  k<<<grid, 256, smem, s>>>(J, feat);
+  return launched("k_pairfeat");
+}
+
+template <int PM, bool F32>
+pb_status run_mlp_bias(const pb::JetArgs& J, const pb::MlpArgs& W, void* U, cudaStream_t s) {
+  auto k = pb::k_mlp_bias<PM, kGroups, F32>;
+  const size_t smem = sizeof(pb::MlpBiasSmem<PM, kGroups>);
+  int grid = 0;
+  pb_status st = prepare(k, smem, kGroups * 128, J.N, &grid);
+  if (st != PB_OK) return st;
+  k<<<grid, kGroups * 128, smem, s>>>(J, W, U);
+  return launched("k_mlp_bias");
+}
+
+template <int PM>
+pb_status run_attn_bias(const pb::JetArgs& J, const pb::QkvArgs& X, const uint16_t* U, cudaStream_t s) {
+  auto k = pb::k_attn_bias<PM>;
+  const size_t smem = sizeof(pb::AttnSmem<PM>);
+  int grid = 0;
+  pb_status st = prepare(k, smem, 256, J.N, &grid);
+  if (st != PB_OK) return st;
+  k<<<grid, 256, smem, s>>>(J, X, U);
+  return launched("k_attn_bias");
+}
+
+template <int PM>
+pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s) {
+  auto k = pb::k_fused<PM, kGroups>;
+  const size_t smem = sizeof(pb::FusedSmem<PM, kGroups>);
+  int grid = 0;
+  pb_status st = prepare(k, smem, kGroups * 128, J.N, &grid);
+  if (st != PB_OK) return st;
+  k<<<grid, kGroups * 128, smem, s>>>(J, W, X);
+  return launched("k_fused");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pb_last_error(void) { return g_err; }
+
+const char* pb_version(void) { return "pairbias-b200 0.1 (sm_100a)"; }
+
+pb_status pairfeat_compute(const pb_jets* jets, float* feat, void* stream) {
+  pb::JetArgs J;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK || J.N == 0) return st;
+  if (!feat || !aligned(feat, 16)) return fail(PB_EINVAL, "feat must be a non-NULL 16-byte aligned pointer");
+  if (J.N == 0) return PB_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return J.P <= 128 ? run_pairfeat<128>(J, feat, s) : run_pairfeat<256>(J, feat, s);
+}
+
+pb_status pairbias_mlp_forward(const pb_jets* jets, const pb_mlp* mlp, void* U, pb_dtype dtype, void* stream) {
+  pb::JetArgs J;
+  pb::MlpArgs W;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK || J.N == 0) return st;
+  if ((st = check_mlp(mlp, &W)) != PB_OK) return st;
+  if (!U || !aligned(U, 16)) return fail(PB_EINVAL, "U must be a non-NULL 16-byte aligned pointer");
+  if (dtype != PB_BF16 && dtype != PB_F32) return fail(PB_EINVAL, "dtype %d is not PB_BF16 or PB_F32", (int)dtype);
+  if (J.N == 0) return PB_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == PB_F32)
+    return J.P <= 128 ? run_mlp_bias<128, true>(J, W, U, s) : run_mlp_bias<256, true>(J, W, U, s);
+  return J.P <= 128 ? run_mlp_bias<128, false>(J, W, U, s) : run_mlp_bias<256, false>(J, W, U, s);
+}
+
+pb_status pair_attention_forward(const pb_jets* jets, const pb_mlp* mlp, const uint16_t* U, int H, int D,
+                                 const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                                 void* stream) {
+  pb::JetArgs J;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK) return st;
+  if (H != pb::kH || D != pb::kD) return fail(PB_EUNSUPPORTED, "H = %d, D = %d; only H = 8, D = 16", H, D);
+  if ((mlp == nullptr) == (U == nullptr)) return fail(PB_EINVAL, "pass exactly one of mlp and U");
+  if (J.N == 0) return PB_OK;
+  if (!q || !k || !v || !out) return fail(PB_EINVAL, "q, k, v and out must be non-NULL");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || (U && !aligned(U, 16)))
+    return fail(PB_EINVAL, "q, k, v, out and U must be 16-byte aligned");
+  pb::QkvArgs X{q, k, v, out};
+  if (J.N == 0) return PB_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (mlp) {
+    pb::MlpArgs W;
+    if ((st = check_mlp(mlp, &W)) != PB_OK) return st;
+    return J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
+  }
+  return J.P <= 128 ? run_attn_bias<128>(J, X, U, s) : run_attn_bias<256>(J, X, U, s);
+}
+
+pb_status pb_get_device_status(void* stream, uint32_t* bits) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  unsigned int word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, pb::g_status, sizeof word);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(pb::g_status, &zero, sizeof zero);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "status word copy: %s", cudaGetErrorString(e));
+  if (bits) *bits = word;
+  if (word) return fail(PB_EDEVICE, "device status bits 0x%x", word);
+  return PB_OK;
+}
+
+pb_status pb_fold_affine(const pb_mlp_unfolded* in, float* out) {
+  if (!in || !out) return fail(PB_EINVAL, "NULL argument");
+  const float* need[] = {in->a0, in->c0, in->W1, in->b1, in->a1, in->c1, in->W2, in->b2,
+                         in->a2, in->c2, in->W3, in->b3, in->a3, in->c3, in->W4, in->b4};
+  for (const float* p : need)
+    if (!p) return fail(PB_EINVAL, "an unfolded parameter pointer is NULL");
+  // layer 1: a1*(W1 (a0 f + c0) + b1) + c1 = (a1 W1 a0) f + a1 (W1 c0 + b1) + c1
+  for (int o = 0; o < 64; ++o) {
+    double bias = in->b1[o];
+    for (int i = 0; i < 4; ++i) {
+      const double w = in->W1[o * 4 + i];
+      out[PB_OFF_W1 + o * 4 + i] = (float)((double)in->a1[o] * w * (double)in->a0[i]);
+      bias += w * (double)in->c0[i];
+    }
+    out[PB_OFF_B1 + o] = (float)((double)in->a1[o] * bias + (double)in->c1[o]);
+  }
+  // layers 2, 3: a*(W h + b) + c = (a W) h + (a b + c)
+  const float* Ws[2] = {in->W2, in->W3};
+  const float* bs[2] = {in->b2, in->b3};
+  const float* as[2] = {in->a2, in->a3};
+  const float* cs[2] = {in->c2, in->c3};
+  const int offW[2] = {PB_OFF_W2, PB_OFF_W3}, offB[2] = {PB_OFF_B2, PB_OFF_B3};
+  for (int L = 0; L < 2; ++L)
+    for (int o = 0; o < 64; ++o) {
+      for (int i = 0; i < 64; ++i)
+        out[offW[L] + o * 64 + i] = (float)((double)as[L][o] * (double)Ws[L][o * 64 + i]);
+      out[offB[L] + o] = (float)((double)as[L][o] * (double)bs[L][o] + (double)cs[L][o]);
+    }
+  memcpy(out + PB_OFF_W4, in->W4, sizeof(float) * 8 * 64);
+  memcpy(out + PB_OFF_B4, in->b4, sizeof(float) * 8);
+  return PB_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+"""Thin Python binding of the C-ABI library ``libpairbias.so``.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. PyTorch provides device memory and streams. The library is loaded
+on first use and its absence is an error -- there is no fallback.
+
+Entry points mirror ``include/pairbias.h``: ``pairfeat_compute``,
+``pairbias_mlp_forward``, ``pair_attention_forward``,
+``get_device_status`` and the host helper ``fold_affine``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpairbias.so")
+
+PB_OK, PB_EINVAL, PB_EUNSUPPORTED, PB_ECUDA, PB_EDEVICE = range(5)
+PB_BF16, PB_F32 = 0, 1
+PB_DEV_TIMEOUT, PB_DEV_BADPTR = 1, 2
+H, D = 8, 16
+
+# offsets of the folded parameters in the flat buffer (PB_OFF_* in the header)
+FOLDED_OFFSETS = dict(W1=(0, (64, 4)), b1=(256, (64,)), W2=(320, (64, 64)), b2=(4416, (64,)),
+                      W3=(4480, (64, 64)), b3=(8576, (64,)), W4=(8640, (8, 64)), b4=(9152, (8,)))
+FOLDED_FLOATS = 9160
+
+
+class PairBiasError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"pairbias status {status}: {msg}")
+        self.status = status
+
+
+class _Jets(C.Structure):
+    _fields_ = [("E", C.c_void_p), ("px", C.c_void_p), ("py", C.c_void_p), ("pz", C.c_void_p),
+                ("mask", C.c_void_p), ("ptr", C.c_void_p), ("N", C.c_int32), ("P", C.c_int32),
+                ("tokens", C.c_int64)]
+
+
+class _Mlp(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("W1", "b1", "W2", "b2", "W3", "b3", "W4", "b4")]
+
+
+class _MlpUnfolded(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("a0", "c0", "W1", "b1", "a1", "c1", "W2", "b2", "a2", "c2",
+                                          "W3", "b3", "a3", "c3", "W4", "b4")]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """Load libpairbias.so (built by ``__graft_entry__.build()``); fail loudly if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build()")
+            L = C.CDLL(LIB_PATH)
+            vp = C.c_void_p
+            L.pairfeat_compute.argtypes = [C.POINTER(_Jets), vp, vp]
+            L.pairbias_mlp_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, vp]
+            L.pair_attention_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, C.c_int,
+                                                 vp, vp, vp, vp, vp]
+            L.pb_get_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
+            L.pb_fold_affine.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float)]
+            L.pb_last_error.restype = C.c_char_p
+            L.pb_version.restype = C.c_char_p
+            for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward,
+                      L.pb_get_device_status, L.pb_fold_affine):
+                f.restype = C.c_int
+            _lib = L
+        return _lib
+
+
+def _check(st: int) -> None:
+    if st != PB_OK:
+        raise PairBiasError(st, lib().pb_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dp(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+@dataclass
+class Jets:
+    """Device tensors of one jet batch (see pb_jets in the header)."""
+
+    E: torch.Tensor
+    px: torch.Tensor
+    py: torch.Tensor
+    pz: torch.Tensor
+    mask: Optional[torch.Tensor]
+    ptr: Optional[torch.Tensor]
+    N: int
+    P: int
+
+    @property
+    def tokens(self) -> int:
+        return int(self.E.numel())
+
+    def struct(self) -> _Jets:
+        return _Jets(_dp(self.E), _dp(self.px), _dp(self.py), _dp(self.pz), _dp(self.mask), _dp(self.ptr),
+                     int(self.N), int(self.P), self.tokens if self.ptr is not None else 0)
+
+
+@dataclass
+class FoldedMLP:
+    """Folded MLP parameters in one flat fp32 device buffer (PB_OFF_* layout)."""
+
+    flat: torch.Tensor
+
+    def struct(self) -> _Mlp:
+        base = self.flat.data_ptr()
+        return _Mlp(**{k: base + 4 * off for k, (off, _s) in FOLDED_OFFSETS.items()})
+
+
+def fold_affine(params: Dict[str, np.ndarray]) -> np.ndarray:
+    """Fold the batch-norm affines of an unfolded MLP (host, C library)."""
+    arrs = {k: np.ascontiguousarray(v, np.float32) for k, v in params.items()}
+    st = _MlpUnfolded(**{n: arrs[n].ctypes.data for n, _t in _MlpUnfolded._fields_})
+    out = np.zeros(FOLDED_FLOATS, np.float32)
+    _check(lib().pb_fold_affine(C.byref(st), out.ctypes.data_as(C.POINTER(C.c_float))))
+    return out
+
+
+def folded_mlp(params: Dict[str, np.ndarray], device="cuda") -> FoldedMLP:
+    return FoldedMLP(torch.from_numpy(fold_affine(params)).to(device))
+
+
+def jets_to_device(b, device="cuda") -> Jets:
+    """Momenta, mask / ptr of a ``synth.JetBatch`` as device tensors."""
+    t = lambda a, dt: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device=device, dtype=dt)
+    return Jets(t(b.E, torch.float32), t(b.px, torch.float32), t(b.py, torch.float32), t(b.pz, torch.float32),
+                t(b.mask, torch.uint8), t(b.ptr, torch.int32), int(b.N), int(b.P))
+
+
+def bf16_to_device(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """Raw bf16 bit patterns (uint16) -> a torch.bfloat16 device tensor."""
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def pairfeat_compute(jets: Jets, feat: torch.Tensor, stream=None) -> None:
+    """feat: float32 [N, P, P, 4] on the device."""
+    assert feat.dtype == torch.float32 and feat.is_contiguous()
+    js = jets.struct()
+    _check(lib().pairfeat_compute(C.byref(js), feat.data_ptr(), _stream(stream)))
+
+
+def pairbias_mlp_forward(jets: Jets, mlp: FoldedMLP, U: torch.Tensor, stream=None) -> None:
+    """U: bfloat16 or float32 [N, 8, P, P] on the device."""
+    assert U.is_contiguous() and U.dtype in (torch.bfloat16, torch.float32)
+    js, ms = jets.struct(), mlp.struct()
+    dtype = PB_F32 if U.dtype == torch.float32 else PB_BF16
+    _check(lib().pairbias_mlp_forward(C.byref(js), C.byref(ms), U.data_ptr(), dtype, _stream(stream)))
+
+
+def pair_attention_forward(jets: Jets, mlp: Optional[FoldedMLP], U: Optional[torch.Tensor], q: torch.Tensor,
+                           k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """Fused (mlp given) or bias-reading (U given, bf16) attention; bf16 q/k/v/out."""
+    for t in (q, k, v, out):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    if U is not None:
+        assert U.dtype == torch.bfloat16 and U.is_contiguous()
+    js = jets.struct()
+    ms = mlp.struct() if mlp is not None else None
+    _check(lib().pair_attention_forward(C.byref(js), C.byref(ms) if ms is not None else None,
+                                        _dp(U), H, D, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        out.data_ptr(), _stream(stream)))
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the device status bits."""
+    bits = C.c_uint32(0)
+    st = lib().pb_get_device_status(_stream(stream), C.byref(bits))
+    if st not in (PB_OK, PB_EDEVICE):
+        _check(st)
+    return int(bits.value)
+
+
+def version() -> str:
+    return lib().pb_version().decode()

@@ -86,7 +86,9 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def _multiplicities(rng, n, dist, lo, hi, lam):
+def _multiplicities(rng, n, dist, lo, hi, lam, mults=None):
+    if mults is not None:
+        return np.asarray(mults, dtype=np.int32).reshape(n)
     if dist == "uniform":
         return rng.integers(lo, hi + 1, size=n).astype(np.int32)
     if dist == "poisson":
@@ -98,6 +100,9 @@ def _multiplicities(rng, n, dist, lo, hi, lam):
 
 def _constituents(rng, m, pt_lo, pt_hi, prongs):
     """Massless constituents of one jet, as float64 (E, px, py, pz) columns."""
+    if m == 0:
+        z = np.zeros(0)
+        return z, z, z, z
     jet_pt = rng.uniform(pt_lo, pt_hi)
     frac = rng.dirichlet(np.ones(m))
     pt = jet_pt * frac
@@ -135,11 +140,12 @@ def make_params(rng) -> Dict[str, np.ndarray]:
 def make_jets(*, N: int, P: int, layout: str = "padded", dist: str = "poisson",
               mult_lo: int = 2, mult_hi: Optional[int] = None, lam: float = 40.0,
               pt_lo: float = 500.0, pt_hi: float = 550.0, prongs: int = 1,
-              mask_mode: str = "prefix", seed: int = 0) -> JetBatch:
+              mask_mode: str = "prefix", seed: int = 0, mults=None) -> JetBatch:
     """Draw one batch of jets, MLP parameters and Q/K/V from PCG64(seed).
 
     ``mask_mode="prefix"`` puts the m valid particles in slots 0..m-1;
     ``"scrambled"`` places them in m random slots of the P (padded only).
+    ``mults`` fixes the multiplicity of every jet instead of drawing it.
     Draw order: parameters, multiplicities, per-jet kinematics, slot
     permutations, Q, K, V.
     """
@@ -147,7 +153,7 @@ def make_jets(*, N: int, P: int, layout: str = "padded", dist: str = "poisson",
         mult_hi = P
     rng = np.random.Generator(np.random.PCG64(seed))
     params = make_params(rng)
-    mult = _multiplicities(rng, N, dist, mult_lo, mult_hi, lam)
+    mult = _multiplicities(rng, N, dist, mult_lo, mult_hi, lam, mults)
     kin = [_constituents(rng, int(m), pt_lo, pt_hi, prongs) for m in mult]
 
     if layout == "padded":

@@ -1,0 +1,119 @@
+"""Comparison helpers shared by the GPU parity tests.
+
+Tolerances (the benchmark's stated bars, with the readings of where they
+apply):
+  features  |g - o| <= 1e-5 * max(1, |o|): a relative error on the physical
+            quantity, with an absolute floor where the logarithm crosses 0;
+  bias U    max |g - o| <= 3e-2 and relative L2 <= 1e-2 over valid pairs
+            (for a bf16 U add half a bf16 ulp of o, its storage rounding);
+  attention relative L2 <= 1e-2 over valid query rows; masked rows exactly 0.
+"""
+import numpy as np
+import torch
+
+from part_pair_bias_b200 import ops, synth
+
+FEAT_REL = 1e-5
+U_MAXABS = 3e-2
+U_RELL2 = 1e-2
+ATT_RELL2 = 1e-2
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def valid_pairs(b):
+    """bool [N, P, P]: both ends valid (padded per-jet view for both layouts)."""
+    if b.layout == "padded":
+        m = b.mask.reshape(b.N, b.P).astype(bool)
+    else:
+        m = np.arange(b.P)[None, :] < b.mult[:, None]
+    return m[:, :, None] & m[:, None, :]
+
+
+def valid_rows(b, shape):
+    """bool broadcast of valid query rows over an attention output."""
+    if b.layout == "padded":
+        return np.broadcast_to(b.mask.reshape(b.N, 1, b.P, 1).astype(bool), shape)
+    return np.ones(shape, bool)
+
+
+def check_features(got, ref, b):
+    vp = valid_pairs(b)
+    g, o = got[vp], ref[vp]
+    err = np.abs(g - o) / np.maximum(1.0, np.abs(o))
+    assert err.max() <= FEAT_REL, f"feature error {err.max():.3e} > {FEAT_REL}"
+    assert np.all(got[~vp] == 0.0), "masked pairs must be 0"
+    assert np.array_equal(got, got.transpose(0, 2, 1, 3)), "feat[i,j] != feat[j,i]"
+    return float(err.max())
+
+
+def bf16_half_ulp(x):
+    """Half the bf16 spacing at |x| (the storage rounding bound)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 0.5 * 2.0 ** (e - 7)
+
+
+def check_bias(got, ref, b, bf16=False):
+    vp = np.broadcast_to(valid_pairs(b)[:, None], got.shape)
+    g, o = got[vp], ref[vp]
+    tol = U_MAXABS + (bf16_half_ulp(o) if bf16 else 0.0)
+    err = np.abs(g - o)
+    assert np.all(err <= tol), f"U max-abs error {err.max():.3e} (bf16={bf16})"
+    rel = np.linalg.norm(g - o) / np.linalg.norm(o)
+    assert rel <= U_RELL2, f"U rel L2 {rel:.3e}"
+    assert np.all(got[~vp] == 0.0), "masked pairs of U must be 0"
+    assert np.array_equal(got, got.transpose(0, 1, 3, 2)), "U[i,j] != U[j,i]"
+    return float(err.max()), float(rel)
+
+
+def check_attention(got, ref, b):
+    vr = valid_rows(b, got.shape)
+    g, o = got[vr], ref[vr]
+    rel = np.linalg.norm(g - o) / np.linalg.norm(o)
+    assert rel <= ATT_RELL2, f"attention rel L2 {rel:.3e}"
+    assert np.all(got[~vr] == 0.0), "masked query rows must be 0"
+    return float(rel)
+
+
+def jet_rows(b, out_full, jets):
+    """Rows of a full-batch output belonging to the listed jets, in the
+    layout that ``synth.slice_jets`` produces for each jet."""
+    if b.layout == "padded":
+        return [out_full[n:n + 1] for n in jets]
+    return [out_full[b.ptr[n]:b.ptr[n + 1]] for n in jets]
+
+
+class Device:
+    """One batch on the device: jets, folded MLP and bf16 q/k/v."""
+
+    def __init__(self, b, dev="cuda"):
+        self.b = b
+        self.jets = ops.jets_to_device(b, dev)
+        self.mlp = ops.folded_mlp(b.params, dev)
+        self.q, self.k, self.v = (ops.bf16_to_device(x, dev) for x in (b.q, b.k, b.v))
+
+    def features(self):
+        f = torch.full((self.b.N, self.b.P, self.b.P, 4), float("nan"), device=self.q.device)
+        ops.pairfeat_compute(self.jets, f)
+        return f
+
+    def bias(self, dtype=torch.float32):
+        U = torch.full((self.b.N, 8, self.b.P, self.b.P), float("nan"), device=self.q.device, dtype=dtype)
+        ops.pairbias_mlp_forward(self.jets, self.mlp, U)
+        return U
+
+    def fused(self):
+        out = torch.full_like(self.q, float("nan"))
+        ops.pair_attention_forward(self.jets, self.mlp, None, self.q, self.k, self.v, out)
+        return out
+
+    def with_bias(self, U_bf16):
+        out = torch.full_like(self.q, float("nan"))
+        ops.pair_attention_forward(self.jets, None, U_bf16, self.q, self.k, self.v, out)
+        return out
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    return synth.bf16_bits_to_f64(synth.f32_to_bf16_bits(x.astype(np.float32)))

@@ -1,0 +1,101 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every declared
+symbol, rejects bad arguments on the host, and its batch-norm folding agrees
+with the oracle's unfolded MLP."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+from scipy.special import erf
+
+from part_pair_bias_b200 import ops, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pairbias.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from part_pair_bias_b200 import build
+    build.build()
+    return ops.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(\w+)\s*\(", text, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert {"pairfeat_compute", "pairbias_mlp_forward", "pair_attention_forward",
+            "pb_get_device_status", "pb_fold_affine", "pb_last_error", "pb_version"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in pairbias.h but not exported"
+    assert ops.version().startswith("pairbias-b200")
+
+
+def _jets(N=2, P=8, ptr=False, aligned=True):
+    buf = np.zeros(64, np.float32)
+    base = buf.ctypes.data + (0 if aligned else 1)
+    m = np.ones(N * P, np.uint8)
+    p = np.zeros(N + 1, np.int32)
+    js = ops._Jets(base, base, base, base, m.ctypes.data, p.ctypes.data if ptr else None, N, P, 0)
+    return js, (buf, m, p)
+
+
+def test_host_validation(L):
+    js, keep = _jets()
+    dummy = np.zeros(64, np.float32)
+    d = dummy.ctypes.data
+    assert L.pairfeat_compute(None, d, None) == ops.PB_EINVAL
+    assert "NULL" in ops.lib().pb_last_error().decode()
+    js.P = 0
+    assert L.pairfeat_compute(C.byref(js), d, None) == ops.PB_EUNSUPPORTED
+    js.P = 257
+    assert L.pairfeat_compute(C.byref(js), d, None) == ops.PB_EUNSUPPORTED
+    js.P = 8
+    js.N = -1
+    assert L.pairfeat_compute(C.byref(js), d, None) == ops.PB_EINVAL
+    js.N = 2
+    assert L.pairfeat_compute(C.byref(js), d + 4, None) == ops.PB_EINVAL   # feat not 16-byte aligned
+    js.mask = None
+    assert L.pairfeat_compute(C.byref(js), d, None) == ops.PB_EINVAL       # padded without mask
+    js2, keep2 = _jets(aligned=False)
+    assert L.pairfeat_compute(C.byref(js2), d, None) == ops.PB_EINVAL      # misaligned momenta
+    js3, keep3 = _jets()
+    mlp = ops._Mlp(*([d] * 8))
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 4, 16, d, d, d, d, None) == ops.PB_EUNSUPPORTED
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 32, d, d, d, d, None) == ops.PB_EUNSUPPORTED
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), d, 8, 16, d, d, d, d, None) == ops.PB_EINVAL
+    assert L.pair_attention_forward(C.byref(js3), None, None, 8, 16, d, d, d, d, None) == ops.PB_EINVAL
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 16, d + 2, d, d, d, None) == ops.PB_EINVAL
+    assert L.pairbias_mlp_forward(C.byref(js3), C.byref(mlp), d, 7, None) == ops.PB_EINVAL
+    bad = ops._Mlp(*([d] * 7 + [0]))
+    assert L.pairbias_mlp_forward(C.byref(js3), C.byref(bad), d, 0, None) == ops.PB_EINVAL
+    # N = 0 is a no-op that needs no device
+    js3.N = 0
+    assert L.pairfeat_compute(C.byref(js3), d, None) == ops.PB_OK
+
+
+def test_fold_affine_matches_unfolded_oracle(L, oracle_lib):
+    """The folded network (product host helper) equals the oracle's unfolded
+    MLP up to the fp32 rounding of the folded parameters."""
+    rng = np.random.default_rng(21)
+    for seed in range(3):
+        p = synth.make_params(np.random.default_rng(seed))
+        flat = ops.fold_affine(p).astype(np.float64)
+        get = lambda name: flat[ops.FOLDED_OFFSETS[name][0]:][:int(np.prod(ops.FOLDED_OFFSETS[name][1]))].reshape(
+            ops.FOLDED_OFFSETS[name][1])
+        gelu = lambda x: 0.5 * x * (1 + erf(x / np.sqrt(2)))
+        for _ in range(50):
+            f = rng.uniform(-18.4, 12, 4)
+            h = gelu(get("W1") @ f + get("b1"))
+            h = gelu(get("W2") @ h + get("b2"))
+            h = gelu(get("W3") @ h + get("b3"))
+            u = get("W4") @ h + get("b4")
+            ref = oracle_lib.mlp_row(f, p)
+            assert np.max(np.abs(u - ref)) < 2e-5 * max(1.0, np.max(np.abs(ref)))
+    assert L.pb_fold_affine(None, None) == ops.PB_EINVAL

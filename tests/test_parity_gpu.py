@@ -1,0 +1,168 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small workloads are compared element by element in full; the large ones run
+at full size on the GPU (the launch the benchmark times) and are compared on
+sampled jets that the oracle computes one range at a time. Edge cases: odd P,
+scrambled masks, empty / one-particle / full jets, P = 256 jets whose bias
+does not fit on chip (query-block path), packed jets, an invalid ptr array.
+"""
+import numpy as np
+import pytest
+import torch
+
+from part_pair_bias_b200 import configs, ops, synth
+from tests import parity as pt
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    torch.cuda.set_device(0)
+    ops.lib()
+    yield
+    assert ops.get_device_status() == 0
+
+
+_BATCHES = {}
+
+
+def batch(name, **over):
+    key = (name, tuple(sorted(over.items())))
+    if key not in _BATCHES:
+        _BATCHES[key] = synth.make_jets(**configs.workload(name, seed=0, **over))
+    return _BATCHES[key]
+
+
+def sample_ranges(b):
+    """Jet ranges the oracle recomputes for a large batch."""
+    N = b.N
+    if N <= 128:
+        return [(0, N)]
+    w = 16 if N <= 512 else 32
+    rs = [(0, w), (N // 2, N // 2 + w), (N - w, N)]
+    big = int(np.argmax(b.mult))  # the widest jet (query-block path when m > 128)
+    if not any(lo <= big < hi for lo, hi in rs):
+        rs.append((big, big + 1))
+    return rs
+
+
+def per_jet(b, full, lo, hi):
+    if b.layout == "padded" or full.shape[0] == b.N:
+        return full[lo:hi]
+    return full[b.ptr[lo]:b.ptr[hi]]
+
+
+ALL = ["pr1_n8_p32", "n128_p128", "n512_p128", "packed_8192", "n256_p256_3prong"]
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_features(oracle_lib, name):
+    b = batch(name)
+    d = pt.Device(b)
+    got = pt.to_np(d.features())
+    assert ops.get_device_status() == 0
+    for lo, hi in sample_ranges(b):
+        s = synth.slice_jets(b, lo, hi)
+        pt.check_features(got[lo:hi], oracle_lib.features(s), s)
+
+
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_bias(oracle_lib, name, dtype):
+    b = batch(name)
+    d = pt.Device(b)
+    got = pt.to_np(d.bias(dtype))
+    assert ops.get_device_status() == 0
+    for lo, hi in sample_ranges(b):
+        s = synth.slice_jets(b, lo, hi)
+        pt.check_bias(got[lo:hi], oracle_lib.pair_bias(s), s, bf16=dtype == torch.bfloat16)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_fused_attention(oracle_lib, name):
+    b = batch(name)
+    d = pt.Device(b)
+    got = pt.to_np(d.fused())
+    assert ops.get_device_status() == 0
+    for lo, hi in sample_ranges(b):
+        s = synth.slice_jets(b, lo, hi)
+        pt.check_attention(per_jet(b, got, lo, hi), oracle_lib.forward(s), s)
+
+
+@pytest.mark.parametrize("name", ["pr1_n8_p32", "n128_p128", "n512_p128", "n256_p256_3prong"])
+def test_materialised_bias_then_attention(oracle_lib, name):
+    """The standalone path: bf16 U written to HBM, then attention reading it."""
+    b = batch(name)
+    d = pt.Device(b)
+    U = d.bias(torch.bfloat16)
+    got = pt.to_np(d.with_bias(U))
+    assert ops.get_device_status() == 0
+    for lo, hi in sample_ranges(b):
+        s = synth.slice_jets(b, lo, hi)
+        pt.check_attention(per_jet(b, got, lo, hi), oracle_lib.forward(s), s)
+
+
+@pytest.mark.parametrize("name", ["pr1_n8_p32", "n128_p128"])
+def test_attention_kernel_alone(oracle_lib, name):
+    """Attention with the oracle's own bias (rounded to bf16) isolates the
+    attention kernel: the oracle sees exactly the bias the kernel reads."""
+    b = batch(name)
+    d = pt.Device(b)
+    U = pt.bf16_round(oracle_lib.pair_bias(b))
+    Ud = torch.from_numpy(U.astype(np.float32)).to(torch.bfloat16).cuda()
+    got = pt.to_np(d.with_bias(Ud))
+    rel = pt.check_attention(got, oracle_lib.attention(b, U), b)
+    assert rel < 5e-3
+
+
+def test_odd_p_scrambled_masks_and_degenerate_jets(oracle_lib):
+    b = synth.make_jets(N=8, P=37, mults=[0, 1, 2, 37, 17, 36, 5, 33], mask_mode="scrambled", seed=3)
+    d = pt.Device(b)
+    pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
+    pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
+    got = pt.to_np(d.fused())
+    pt.check_attention(got, oracle_lib.forward(b), b)
+    assert np.all(got[0] == 0.0)                     # empty jet: every row masked
+    assert ops.get_device_status() == 0
+
+
+def test_wide_jets_query_block_path(oracle_lib):
+    """P = 256 with jets above 128 particles: the bias of a whole jet no longer
+    fits on chip and the fused kernel tiles queries."""
+    b = synth.make_jets(N=5, P=256, mults=[256, 200, 129, 128, 3], pt_lo=800, pt_hi=1000, prongs=3, seed=5)
+    d = pt.Device(b)
+    pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
+    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    assert ops.get_device_status() == 0
+
+
+def test_packed_with_empty_jets(oracle_lib):
+    b = synth.make_jets(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6)
+    d = pt.Device(b)
+    pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
+    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    assert ops.get_device_status() == 0
+
+
+def test_invalid_ptr_sets_status_and_skips_jet():
+    b = synth.make_jets(N=3, P=32, layout="packed", mults=[10, 10, 10], seed=7)
+    d = pt.Device(b)
+    d.jets.ptr = torch.tensor([0, 20, 10, 30], dtype=torch.int32, device="cuda")  # jet 1 runs backwards
+    f = d.features()
+    bits = ops.get_device_status()
+    assert bits & ops.PB_DEV_BADPTR
+    assert torch.all(f[1] == 0)
+    assert ops.get_device_status() == 0              # reading clears the word
+
+
+def test_deterministic_and_empty_batch():
+    b = batch("n128_p128")
+    d = pt.Device(b)
+    o1, o2 = d.fused(), d.fused()
+    assert torch.equal(o1, o2)
+    e = synth.make_jets(N=0, P=16, mults=np.zeros(0, int), seed=1)
+    de = pt.Device(e)
+    ops.pair_attention_forward(de.jets, de.mlp, None, de.q, de.k, de.v, torch.empty_like(de.q))
+    assert ops.get_device_status() == 0
