@@ -107,7 +107,7 @@ pb_status check_mlp(const pb_mlp* w, pb::MlpArgs* out) {
   return PB_OK;
 }
 
-constexpr int kGroups = 2;  // tensor-core tile groups per CTA (128 threads each)
+constexpr int kGroups = 4;  // tensor-core tile groups per CTA (128 threads each)
 
 template <int PM>
 pb_status run_pairfeat(const pb::JetArgs& J, float* feat, cudaStream_t s) {

@@ -117,7 +117,14 @@ __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
 // construction when called with (min, max). m^2 uses the light-cone form
 // (E_s - pz_s)(E_s + pz_s) - px_s^2 - py_s^2 of the pair sum s, in fp64, which
 // equals the definition (E_a+E_b)^2 - |p_a+p_b|^2 without its cancellation.
-template <int PM>
+// kFastLog selects the hardware log2 approximation (absolute error ~1e-7 in
+// ln); the feature output path uses the accurate logf.
+template <bool kFastLog>
+__device__ __forceinline__ float flog(float x) {
+  return kFastLog ? __logf(x) : logf(x);
+}
+
+template <int PM, bool kFastLog = false>
 __device__ __forceinline__ void pair_feat(const Particles<PM>& S, int a, int b, float f[4]) {
   const double dy = S.y[a] - S.y[b];
   double dphi = S.phi[a] - S.phi[b];
@@ -125,14 +132,14 @@ __device__ __forceinline__ void pair_feat(const Particles<PM>& S, int a, int b, 
   else if (dphi <= -kPi) dphi += 2.0 * kPi;
   const float fy = (float)dy, fp = (float)dphi;
   const float dr2 = fmaf(fy, fy, fp * fp);
-  const float lndr = 0.5f * logf(dr2);  // -inf for dR = 0, clamped below
+  const float lndr = 0.5f * flog<kFastLog>(dr2);  // -inf for dR = 0, clamped below
   const float lnptmin = fminf(S.lnpt[a], S.lnpt[b]);
   f[0] = fmaxf(lnptmin + lndr, kLnEps);
-  f[1] = fmaxf(lnptmin - logf(S.pt[a] + S.pt[b]), kLnEps);
+  f[1] = fmaxf(lnptmin - flog<kFastLog>(S.pt[a] + S.pt[b]), kLnEps);
   f[2] = fmaxf(lndr, kLnEps);
   const double sx = S.px[a] + S.px[b], sy = S.py[a] + S.py[b];
   const double m2 = fma(S.wm[a] + S.wm[b], S.wp[a] + S.wp[b], -(sx * sx + sy * sy));
-  f[3] = m2 > 1e-8 ? logf((float)m2) : kLnEps;
+  f[3] = m2 > 1e-8 ? flog<kFastLog>((float)m2) : kLnEps;
 }
 
 // ----------------------------------------------------- k_pairfeat (features)
@@ -156,6 +163,18 @@ __global__ void __launch_bounds__(256) k_pairfeat(JetArgs J, float* __restrict__
 }
 
 // ================================================================ MLP engine
+//
+// Numerics of the tensor-core MLP (all exact rescalings are powers of two):
+//   layer 1: y1 = W1 f + b1 with f and W1 split into f16 hi + lo parts, the
+//            bias through a column of ones, so y1 carries ~22 bits;
+//   hidden:  the stored activation is h = y (1 + tanh(a y + b y^3)) = 2 GELU(y)
+//            in packed f16x2 (a, b fitted minimax to the erf GELU: max
+//            deviation 2.7e-4); the next layer's weights carry the factor 1/2;
+//   layers 2..4: f16 operands, fp32 accumulation in TMEM, each bias entering
+//            through two constant A columns (1, 1) against (hi(b), lo(b)).
+
+constexpr int kAK = 80;    // A-tile / weight K width: 64 activations + 16 bias columns
+constexpr int kSBO = kAK / 8 * 128;  // byte stride between 8-row groups (1280)
 
 // Element index of (row r, column k) of an f16 tile with K columns in the
 // tensor-core canonical K-major layout without swizzle: 8x8 core matrices of
@@ -167,15 +186,13 @@ __device__ __forceinline__ int cofs(int r, int k, int K) {
 
 template <int NG>
 struct MlpSmem {
-  __half A[NG][kTileM * kHid];  // per-group activation tile (layer-1 uses the first 16 columns)
-  __half W1[64 * 16];           // [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0]
-  __half W2[64 * 64];
-  __half W3[64 * 64];
-  __half W4[16 * 64];           // rows 8..15 are zero (N = 16 MMA)
-  float b2[64], b3[64], b4[8];
+  __half A[NG][kTileM * kAK];  // per-group activation tile; columns 64, 65 hold 1.0 during a pass
+  __half W1[64 * 16];          // [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0], K = 16 layout
+  __half W2[64 * kAK];         // [W2/2 | hi(b2) lo(b2) 0 ...]
+  __half W3[64 * kAK];
+  __half W4[16 * kAK];         // rows 8..15 zero (N = 16 MMA)
   uint64_t mbar[NG];
   uint32_t tmem_base;
-  int abort_flag;
 };
 
 // f16 hi/lo split: x = hi + lo to about 22 bits.
@@ -198,19 +215,34 @@ __device__ void load_weights(MlpSmem<NG>& S, const MlpArgs& W) {
     }
     S.W1[cofs(n, k, 16)] = v;
   }
-  for (int i = threadIdx.x; i < 64 * 64; i += blockDim.x) {
-    const int n = i >> 6, k = i & 63;
-    S.W2[cofs(n, k, 64)] = __float2half_rn(W.W2[i]);
-    S.W3[cofs(n, k, 64)] = __float2half_rn(W.W3[i]);
+  // hidden layers: the stored activation is 2 GELU, so the weights carry 1/2
+  for (int i = threadIdx.x; i < 64 * kAK; i += blockDim.x) {
+    const int n = i / kAK, k = i % kAK;
+    __half v2 = __float2half_rn(0.f), v3 = v2, hi, lo;
+    if (k < 64) {
+      v2 = __float2half_rn(0.5f * W.W2[n * 64 + k]);
+      v3 = __float2half_rn(0.5f * W.W3[n * 64 + k]);
+    } else if (k < 66) {
+      split_half(W.b2[n], hi, lo);
+      v2 = (k == 64) ? hi : lo;
+      split_half(W.b3[n], hi, lo);
+      v3 = (k == 64) ? hi : lo;
+    }
+    S.W2[cofs(n, k, kAK)] = v2;
+    S.W3[cofs(n, k, kAK)] = v3;
   }
-  for (int i = threadIdx.x; i < 16 * 64; i += blockDim.x) {
-    const int n = i >> 6, k = i & 63;
-    S.W4[cofs(n, k, 64)] = __float2half_rn(n < 8 ? W.W4[n * 64 + k] : 0.f);
-  }
-  for (int i = threadIdx.x; i < 64; i += blockDim.x) {
-    S.b2[i] = W.b2[i];
-    S.b3[i] = W.b3[i];
-    if (i < 8) S.b4[i] = W.b4[i];
+  for (int i = threadIdx.x; i < 16 * kAK; i += blockDim.x) {
+    const int n = i / kAK, k = i % kAK;
+    __half v = __float2half_rn(0.f), hi, lo;
+    if (n < 8) {
+      if (k < 64) {
+        v = __float2half_rn(0.5f * W.W4[n * 64 + k]);
+      } else if (k < 66) {
+        split_half(W.b4[n], hi, lo);
+        v = (k == 64) ? hi : lo;
+      }
+    }
+    S.W4[cofs(n, k, kAK)] = v;
   }
 }
 
@@ -220,7 +252,6 @@ __device__ void mlp_setup(MlpSmem<NG>& S, const MlpArgs& W) {
   load_weights<NG>(S, W);
   if (threadIdx.x == 0) {
     for (int g = 0; g < NG; ++g) mbar_init(&S.mbar[g], 1);
-    S.abort_flag = 0;
     fence_mbar_init();
   }
   if ((threadIdx.x >> 5) == 0) tmem_alloc(&S.tmem_base, NG * 64);
@@ -245,8 +276,14 @@ __device__ void mlp_teardown(MlpSmem<NG>& S, bool aborted, const uint32_t* phase
   if ((threadIdx.x >> 5) == 0) tmem_dealloc(S.tmem_base, NG * 64);
 }
 
-// GELU(x) = x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)).
-__device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// 2 GELU(y) for two packed f16 values: y (1 + tanh(y (a + b y^2))).
+__device__ __forceinline__ uint32_t gelu2_f16x2(uint32_t y) {
+  const uint32_t kA = 0x3A67u * 0x10001u;  // f16 0.80029297 in both halves
+  const uint32_t kB = 0x2871u * 0x10001u;  // f16 0.03469849 in both halves
+  const uint32_t y2 = hmul2(y, y);
+  const uint32_t u = hmul2(y, hfma2(y2, kB, kA));
+  return hfma2(y, htanh2(u), y);
+}
 
 // Pair enumerations of one MLP pass: row p -> compact particles (a, b).
 struct TriPairs {  // unordered pairs a <= b, p = b(b+1)/2 + a
@@ -270,7 +307,7 @@ struct RectPairs {  // ordered pairs (i0 + p / m, p % m): a query block against 
 // 128g .. 128g+127) takes tiles g, g+NG, ...; thread row r of a group owns
 // TMEM lane r (its warp's lane quadrant). For each valid row the sink gets
 // (p, a, b, u[8]). Returns false if the group aborted on a timed-out wait.
-template <int PM, int NG, class Pairs, class Sink>
+template <int PM, int NG, bool kFastLog, class Pairs, class Sink>
 __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, const Pairs& pairs,
                          Sink& sink, uint32_t& phase) {
   const int g = threadIdx.x >> 7;
@@ -285,6 +322,11 @@ __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, con
   constexpr uint32_t kId64 = idesc_f16_m128(64), kId16 = idesc_f16_m128(16);
   const int ntiles = (npairs + kTileM - 1) / kTileM;
   bool ok = true;
+  // The bias columns of this thread's activation row: (1, 1, 0, ..., 0). They
+  // are rewritten on every pass because the tiles double as scratch between
+  // passes (the fused kernel stages K and V there).
+  *reinterpret_cast<uint4*>(A + cofs(row, 64, kAK)) = make_uint4(0x3C003C00u, 0u, 0u, 0u);
+  *reinterpret_cast<uint4*>(A + cofs(row, 72, kAK)) = make_uint4(0u, 0u, 0u, 0u);
 
   // Publish this thread's operand writes and TMEM reads, meet the group, issue
   // one layer's MMAs from the leader, wait for them to complete.
@@ -295,11 +337,11 @@ __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, con
     if (leader) {
       tc_fence_after();
       if (L == 0) {
-        mma_f16(t_d, smem_desc(a_addr, 128, 256), smem_desc(w_addr[0], 128, 256), kId64, 0);
+        mma_f16(t_d, smem_desc(a_addr, 128, kSBO), smem_desc(w_addr[0], 128, 256), kId64, 0);
       } else {
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-          mma_f16(t_d, smem_desc(a_addr + 256u * s, 128, 1024), smem_desc(w_addr[L] + 256u * s, 128, 1024),
+        for (int s = 0; s < kAK / 16; ++s)
+          mma_f16(t_d, smem_desc(a_addr + 256u * s, 128, kSBO), smem_desc(w_addr[L] + 256u * s, 128, kSBO),
                   L == 3 ? kId16 : kId64, s > 0 ? 1u : 0u);
       }
       mma_commit(&S.mbar[g]);
@@ -310,21 +352,19 @@ __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, con
     return true;
   };
 
-  // TMEM accumulator row -> (+bias) -> GELU -> f16 -> next layer's A tile.
-  auto hidden = [&](const float* bias) {
-    float v[64];
-    tmem_ld64_wait(t_ld, v);
+  // TMEM accumulator row (bias included) -> 2 GELU in f16x2 -> next A tile.
+  auto hidden = [&]() {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t w[4];
+    for (int half = 0; half < 2; ++half) {
+      float v[32];
+      tmem_ld32_wait(t_ld + 32u * half, v);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int col = 8 * c + 2 * j;
-        const float x0 = v[col] + (bias ? bias[col] : 0.f);
-        const float x1 = v[col + 1] + (bias ? bias[col + 1] : 0.f);
-        w[j] = pack_half2(gelu(x0), gelu(x1));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = gelu2_f16x2(cvt_f16x2(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]));
+        *reinterpret_cast<uint4*>(A + cofs(row, 32 * half + 8 * c, kAK)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      *reinterpret_cast<uint4*>(A + cofs(row, 8 * c, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   };
 
@@ -335,7 +375,7 @@ __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, con
     float f[4] = {0.f, 0.f, 0.f, 0.f};
     if (valid) {
       pairs.map(p, a, b);
-      pair_feat<PM>(P, min(a, b), max(a, b), f);
+      pair_feat<PM, kFastLog>(P, min(a, b), max(a, b), f);
     }
     // layer-1 operand row: [hi(f) | hi(f) | lo(f) | 1 1 0 0] against
     // [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0] gives W1 f + b1 to ~22 bits
@@ -346,20 +386,18 @@ __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, con
       const __half one = __float2half_rn(valid ? 1.f : 0.f), zero = __float2half_rn(0.f);
       __half r0[8] = {hi[0], hi[1], hi[2], hi[3], hi[0], hi[1], hi[2], hi[3]};
       __half r1[8] = {lo[0], lo[1], lo[2], lo[3], one, one, zero, zero};
-      *reinterpret_cast<uint4*>(A + cofs(row, 0, 16)) = *reinterpret_cast<uint4*>(r0);
-      *reinterpret_cast<uint4*>(A + cofs(row, 8, 16)) = *reinterpret_cast<uint4*>(r1);
+      *reinterpret_cast<uint4*>(A + cofs(row, 0, kAK)) = *reinterpret_cast<uint4*>(r0);
+      *reinterpret_cast<uint4*>(A + cofs(row, 8, kAK)) = *reinterpret_cast<uint4*>(r1);
     }
     if (!layer(0)) return false;
-    hidden(nullptr);
+    hidden();
     if (!layer(1)) return false;
-    hidden(S.b2);
+    hidden();
     if (!layer(2)) return false;
-    hidden(S.b3);
+    hidden();
     if (!layer(3)) return false;
     float u[8];
     tmem_ld8_wait(t_ld, u);
-#pragma unroll
-    for (int h = 0; h < 8; ++h) u[h] += S.b4[h];
     if (valid) sink(p, a, b, u);
   }
   // the TMEM reads of the last tile must finish before anyone reuses it
@@ -426,7 +464,7 @@ __global__ void __launch_bounds__(NG * 128) k_mlp_bias(JetArgs J, MlpArgs W, voi
     zero_masked_pairs<PM, F32OUT>(S.part, U, n, J.P);
     const int m = S.part.m;
     GlobalUSink<PM, F32OUT> sink{&S.part, U, n, J.P};
-    const bool ok = mlp_pass<PM, NG>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, phase);
+    const bool ok = mlp_pass<PM, NG, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, phase);
     aborted = __syncthreads_or(!ok) != 0;
     if (aborted) break;
   }
@@ -601,9 +639,16 @@ __global__ void __launch_bounds__(256) k_attn_bias(JetArgs J, QkvArgs X, const u
 // ======================================================= k_fused (one pass)
 
 // The bias of the jet's pairs lives in shared memory as 8 f16 (one per head)
-// per pair: the whole upper triangle when it fits (kUCapPairs pairs, i.e.
-// m <= 128), otherwise one query block against all keys at a time.
-constexpr int kUCapPairs = 128 * 129 / 2;
+// per pair: the whole upper triangle when it fits (UCap pairs), otherwise one
+// query block against all keys at a time. UCap is what is left of the
+// per-CTA shared memory after the MLP tiles and the particles.
+constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
+
+template <int PM, int NG>
+struct FusedLayout {
+  static constexpr int kFixed = (int)(sizeof(MlpSmem<NG>) + sizeof(Particles<PM>)) + 1024;
+  static constexpr int kUCap = (kSmemLimit - kFixed) / 16;
+};
 
 struct SmemUSink {
   uint4* U8;
@@ -633,7 +678,7 @@ template <int PM, int NG>
 struct FusedSmem {
   MlpSmem<NG> mlp;
   Particles<PM> part;
-  uint4 U8[kUCapPairs];
+  uint4 U8[FusedLayout<PM, NG>::kUCap];
 };
 
 template <int PM, int NG>
@@ -643,24 +688,25 @@ __global__ void __launch_bounds__(NG * 128) k_fused(JetArgs J, MlpArgs W, QkvArg
   mlp_setup<NG>(S.mlp, W);
   // during attention the activation tiles hold K and V
   float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
-  constexpr int kStageFloats = NG * kTileM * kHid / 2;
+  constexpr int kStageFloats = NG * kTileM * kAK / 2;
+  constexpr int kUCap = FusedLayout<PM, NG>::kUCap;
   uint32_t phase = 0;
   bool aborted = false;
   for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
     stage_jet<PM>(S.part, J, n);
     const int m = S.part.m;
     SmemUSink sink{S.U8};
-    if (m * (m + 1) / 2 <= kUCapPairs) {
-      const bool ok = mlp_pass<PM, NG>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, phase);
+    if (m * (m + 1) / 2 <= kUCap) {
+      const bool ok = mlp_pass<PM, NG, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, phase);
       aborted = __syncthreads_or(!ok) != 0;
       if (aborted) break;
       TriUBias ub{reinterpret_cast<const __half*>(S.U8)};
       attention_block<PM>(S.part, J, X, n, 0, m, stage, kStageFloats, ub);
     } else {
-      const int qb = kUCapPairs / m;
+      const int qb = kUCap / m;
       for (int i0 = 0; i0 < m; i0 += qb) {
         const int i1 = min(m, i0 + qb);
-        const bool ok = mlp_pass<PM, NG>(S.mlp, S.part, (i1 - i0) * m, RectPairs{i0, m}, sink, phase);
+        const bool ok = mlp_pass<PM, NG, true>(S.mlp, S.part, (i1 - i0) * m, RectPairs{i0, m}, sink, phase);
         aborted = __syncthreads_or(!ok) != 0;
         if (aborted) break;
         RectUBias ub{reinterpret_cast<const __half*>(S.U8), i0, m};

@@ -166,3 +166,14 @@ def test_deterministic_and_empty_batch():
     de = pt.Device(e)
     ops.pair_attention_forward(de.jets, de.mlp, None, de.q, de.k, de.v, torch.empty_like(de.q))
     assert ops.get_device_status() == 0
+
+
+def test_many_jets_per_cta(oracle_lib):
+    """More jets than resident CTAs: every CTA runs several jets in a row, so
+    any state left over from one jet (shared-memory scratch, barrier phases,
+    TMEM) would corrupt the next."""
+    b = synth.make_jets(N=700, P=24, dist="uniform", mult_lo=1, mult_hi=24, mask_mode="scrambled", seed=8)
+    d = pt.Device(b)
+    pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
+    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    assert ops.get_device_status() == 0
