@@ -191,6 +191,11 @@ __host__ __device__ constexpr uint32_t idesc_f16_m128(int n) {
          | ((uint32_t)(128 >> 4) << 24); // M / 16
 }
 
+// Same for bf16 A and B.
+__host__ __device__ constexpr uint32_t idesc_bf16_m128(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor, no swizzle (interleaved core matrices of
 // 8 rows x 16 bytes). lbo = byte distance between the two K-adjacent core
 // matrices of one MMA, sbo = byte distance between 8-row groups.
@@ -256,6 +261,27 @@ __device__ __forceinline__ uint32_t htanh2(uint32_t a) {
   uint32_t r;
   asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(a));
   return r;
+}
+
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ float ex2(float x) {

@@ -167,14 +167,23 @@ __global__ void __launch_bounds__(256) k_pairfeat(JetArgs J, float* __restrict__
 // Numerics of the tensor-core MLP (all exact rescalings are powers of two):
 //   layer 1: y1 = W1 f + b1 with f and W1 split into f16 hi + lo parts, the
 //            bias through a column of ones, so y1 carries ~22 bits;
-//   hidden:  the stored activation is h = y (1 + tanh(a y + b y^3)) = 2 GELU(y)
-//            in packed f16x2 (a, b fitted minimax to the erf GELU: max
-//            deviation 2.7e-4); the next layer's weights carry the factor 1/2;
-//   layers 2..4: f16 operands, fp32 accumulation in TMEM, each bias entering
-//            through two constant A columns (1, 1) against (hi(b), lo(b)).
+//   hidden:  the accumulator row (bias included) is converted to packed f16
+//            and activated on two pipes: 5 of every 8 columns with the tanh
+//            form h = y (1 + tanh(a y + b y^3)) = 2 GELU(y) (one MUFU op per
+//            two values; a, b fitted minimax to the erf GELU, max deviation
+//            2.7e-4), the other 3 with h = relu(y) + s q(s), s = min(|y|, 3.5),
+//            q a degree-6 polynomial fitted to GELU - relu (f16 evaluation,
+//            max deviation 4.8e-3), on the FMA pipe only. The next layer's
+//            weights carry 1/2 on the tanh columns;
+//   layers 2..4: f16 operands, fp32 accumulation in TMEM; each bias enters
+//            through an extra K step: a constant tile of ones times the
+//            weights' (hi(b), lo(b)) columns.
 
-constexpr int kAK = 80;    // A-tile / weight K width: 64 activations + 16 bias columns
-constexpr int kSBO = kAK / 8 * 128;  // byte stride between 8-row groups (1280)
+constexpr int kAK = 64;              // activation tile width
+constexpr int kWK = 80;              // weight K width: 64 activations + 16 bias columns
+constexpr int kASBO = kAK / 8 * 128;   // 8-row group stride of an activation tile (1024 B)
+constexpr int kWSBO = kWK / 8 * 128;   // 8-row group stride of a weight tile (1280 B)
+constexpr int kTanhChunks = 5;       // of the 8 eight-column chunks of a hidden layer
 
 // Element index of (row r, column k) of an f16 tile with K columns in the
 // tensor-core canonical K-major layout without swizzle: 8x8 core matrices of
@@ -184,16 +193,21 @@ __device__ __forceinline__ int cofs(int r, int k, int K) {
   return (((r >> 3) * (K >> 3) + (k >> 3)) << 6) + ((r & 7) << 3) + (k & 7);
 }
 
-template <int NG>
+// NG tile groups of 128 threads; each group keeps SL tiles in flight (slots
+// SL*g .. SL*g+SL-1), so one tile's epilogue overlaps another's MMAs.
+template <int NG, int SL>
 struct MlpSmem {
-  __half A[NG][kTileM * kAK];  // per-group activation tile; columns 64, 65 hold 1.0 during a pass
-  __half W1[64 * 16];          // [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0], K = 16 layout
-  __half W2[64 * kAK];         // [W2/2 | hi(b2) lo(b2) 0 ...]
-  __half W3[64 * kAK];
-  __half W4[16 * kAK];         // rows 8..15 zero (N = 16 MMA)
-  uint64_t mbar[NG];
+  __half A[NG * SL][kTileM * kAK];  // per-slot activation tile (layer 1 uses its first 16 columns)
+  __half Ones[kTileM * 16];         // [1 1 0 ... 0] per row: the bias K step
+  __half W1[64 * 16];               // [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0], K = 16 layout
+  __half W2[64 * kWK];              // [W2 scaled per column | hi(b2) lo(b2) 0 ...]
+  __half W3[64 * kWK];
+  __half W4[16 * kWK];              // rows 8..15 zero (N = 16 MMA)
+  uint64_t mbar[NG * SL];
   uint32_t tmem_base;
 };
+
+__host__ __device__ constexpr int kTmemCols(int ng, int sl) { return ng * sl * 64; }
 
 // f16 hi/lo split: x = hi + lo to about 22 bits.
 __device__ __forceinline__ void split_half(float x, __half& hi, __half& lo) {
@@ -201,79 +215,111 @@ __device__ __forceinline__ void split_half(float x, __half& hi, __half& lo) {
   lo = __float2half_rn(x - __half2float(hi));
 }
 
-template <int NG>
-__device__ void load_weights(MlpSmem<NG>& S, const MlpArgs& W) {
-  for (int i = threadIdx.x; i < 64 * 16; i += blockDim.x) {
-    const int n = i >> 4, k = i & 15;
-    __half v = __float2half_rn(0.f), hi, lo;
-    if (k < 12) {
-      split_half(W.W1[n * 4 + (k & 3)], hi, lo);
-      v = (k >= 4 && k < 8) ? lo : hi;
-    } else if (k < 14) {
-      split_half(W.b1[n], hi, lo);
-      v = (k == 12) ? hi : lo;
-    }
-    S.W1[cofs(n, k, 16)] = v;
+__device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+// Scale of input column k of layers 2..4: the tanh columns hold 2 GELU.
+__device__ __forceinline__ float act_scale(int k) { return (k >> 3) < kTanhChunks ? 0.5f : 1.0f; }
+
+// Weight tiles in the canonical layout. All global loads of a thread are
+// issued before any conversion so that their latencies overlap.
+template <int NG, int SL>
+__device__ void load_weights(MlpSmem<NG, SL>& S, const MlpArgs& W) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  constexpr int kPer = (2 * 1024 + 255) / 256;  // float4 loads of W2 and W3 per thread (>= 256 threads)
+  float4 w[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int q = tid + j * nthr;
+    w[j] = q < 2048 ? reinterpret_cast<const float4*>(q < 1024 ? W.W2 : W.W3)[q & 1023] : make_float4(0, 0, 0, 0);
   }
-  // hidden layers: the stored activation is 2 GELU, so the weights carry 1/2
-  for (int i = threadIdx.x; i < 64 * kAK; i += blockDim.x) {
-    const int n = i / kAK, k = i % kAK;
-    __half v2 = __float2half_rn(0.f), v3 = v2, hi, lo;
-    if (k < 64) {
-      v2 = __float2half_rn(0.5f * W.W2[n * 64 + k]);
-      v3 = __float2half_rn(0.5f * W.W3[n * 64 + k]);
-    } else if (k < 66) {
-      split_half(W.b2[n], hi, lo);
-      v2 = (k == 64) ? hi : lo;
-      split_half(W.b3[n], hi, lo);
-      v3 = (k == 64) ? hi : lo;
+  const float4 w4 = tid < 128 ? reinterpret_cast<const float4*>(W.W4)[tid] : make_float4(0, 0, 0, 0);
+  const float4 w1 = tid < 64 ? reinterpret_cast<const float4*>(W.W1)[tid] : make_float4(0, 0, 0, 0);
+  const float bias1 = tid < 64 ? W.b1[tid] : 0.f;
+  const float bias2 = tid < 64 ? W.b2[tid] : 0.f;
+  const float bias3 = tid < 64 ? W.b3[tid] : 0.f;
+  const float bias4 = tid < 8 ? W.b4[tid] : 0.f;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int q = tid + j * nthr;
+    if (q < 2048) {
+      const int e = (q & 1023) * 4, n = e >> 6, k = e & 63;  // 4 consecutive k of one chunk
+      const float sc = act_scale(k);
+      __half* dst = (q < 1024 ? S.W2 : S.W3) + cofs(n, k, kWK);
+      reinterpret_cast<uint2*>(dst)[0] =
+          make_uint2(h2bits(__float2half_rn(sc * w[j].x), __float2half_rn(sc * w[j].y)),
+                     h2bits(__float2half_rn(sc * w[j].z), __float2half_rn(sc * w[j].w)));
     }
-    S.W2[cofs(n, k, kAK)] = v2;
-    S.W3[cofs(n, k, kAK)] = v3;
   }
-  for (int i = threadIdx.x; i < 16 * kAK; i += blockDim.x) {
-    const int n = i / kAK, k = i % kAK;
-    __half v = __float2half_rn(0.f), hi, lo;
-    if (n < 8) {
-      if (k < 64) {
-        v = __float2half_rn(0.5f * W.W4[n * 64 + k]);
-      } else if (k < 66) {
-        split_half(W.b4[n], hi, lo);
-        v = (k == 64) ? hi : lo;
-      }
+  if (tid < 128) {  // W4 rows 0..7, zero rows 8..15
+    const int e = tid * 4, n = e >> 6, k = e & 63;
+    const float sc = act_scale(k);
+    reinterpret_cast<uint2*>(S.W4 + cofs(n, k, kWK))[0] =
+        make_uint2(h2bits(__float2half_rn(sc * w4.x), __float2half_rn(sc * w4.y)),
+                   h2bits(__float2half_rn(sc * w4.z), __float2half_rn(sc * w4.w)));
+    reinterpret_cast<uint2*>(S.W4 + cofs(8 + n, k, kWK))[0] = make_uint2(0u, 0u);
+  }
+  if (tid < 64) {  // layer-1 row n = tid, and the bias columns of W2, W3, W4
+    const int n = tid;
+    __half h[4], l[4], bh, bl;
+    split_half(w1.x, h[0], l[0]);
+    split_half(w1.y, h[1], l[1]);
+    split_half(w1.z, h[2], l[2]);
+    split_half(w1.w, h[3], l[3]);
+    split_half(bias1, bh, bl);
+    const __half z = __float2half_rn(0.f);
+    *reinterpret_cast<uint4*>(S.W1 + cofs(n, 0, 16)) =
+        make_uint4(h2bits(h[0], h[1]), h2bits(h[2], h[3]), h2bits(l[0], l[1]), h2bits(l[2], l[3]));
+    *reinterpret_cast<uint4*>(S.W1 + cofs(n, 8, 16)) =
+        make_uint4(h2bits(h[0], h[1]), h2bits(h[2], h[3]), h2bits(bh, bl), h2bits(z, z));
+    split_half(bias2, bh, bl);
+    *reinterpret_cast<uint4*>(S.W2 + cofs(n, 64, kWK)) = make_uint4(h2bits(bh, bl), 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(S.W2 + cofs(n, 72, kWK)) = make_uint4(0u, 0u, 0u, 0u);
+    split_half(bias3, bh, bl);
+    *reinterpret_cast<uint4*>(S.W3 + cofs(n, 64, kWK)) = make_uint4(h2bits(bh, bl), 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(S.W3 + cofs(n, 72, kWK)) = make_uint4(0u, 0u, 0u, 0u);
+    if (n < 16) {  // thread n < 8 holds b4[n]; rows 8..15 get zeros
+      split_half(n < 8 ? bias4 : 0.f, bh, bl);
+      *reinterpret_cast<uint4*>(S.W4 + cofs(n, 64, kWK)) = make_uint4(h2bits(bh, bl), 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(S.W4 + cofs(n, 72, kWK)) = make_uint4(0u, 0u, 0u, 0u);
     }
-    S.W4[cofs(n, k, kAK)] = v;
+  }
+  for (int r = tid; r < kTileM; r += nthr) {
+    *reinterpret_cast<uint4*>(S.Ones + cofs(r, 0, 16)) = make_uint4(0x3C003C00u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(S.Ones + cofs(r, 8, 16)) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
-// Once per CTA: weights, mbarriers, TMEM (warp 0 allocates NG*64 columns).
-template <int NG>
-__device__ void mlp_setup(MlpSmem<NG>& S, const MlpArgs& W) {
-  load_weights<NG>(S, W);
+// Once per CTA: weights, mbarriers, TMEM (warp 0 allocates NG*SL*64 columns).
+template <int NG, int SL>
+__device__ void mlp_setup(MlpSmem<NG, SL>& S, const MlpArgs& W) {
+  load_weights<NG, SL>(S, W);
   if (threadIdx.x == 0) {
-    for (int g = 0; g < NG; ++g) mbar_init(&S.mbar[g], 1);
+    for (int i = 0; i < NG * SL; ++i) mbar_init(&S.mbar[i], 1);
     fence_mbar_init();
   }
-  if ((threadIdx.x >> 5) == 0) tmem_alloc(&S.tmem_base, NG * 64);
+  if ((threadIdx.x >> 5) == 0) tmem_alloc(&S.tmem_base, kTmemCols(NG, SL));
   fence_proxy_async_smem();  // weight tiles are read by the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 }
 
-template <int NG>
-__device__ void mlp_teardown(MlpSmem<NG>& S, bool aborted, const uint32_t* phase) {
+template <int NG, int SL>
+__device__ void mlp_teardown(MlpSmem<NG, SL>& S, bool aborted, const uint32_t* phase) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (aborted && (threadIdx.x & 127) == 0) {
-    // A wait that ran out may leave the group's last commit in flight: give it
-    // one more bounded wait before the TMEM it writes is released.
+    // A wait that ran out may leave a slot's last commit in flight: give each
+    // slot one more bounded wait before the TMEM they write is released.
     const int g = threadIdx.x >> 7;
-    if (g < NG) mbar_wait(&S.mbar[g], phase[0] ^ 1u);
+    if (g < NG)
+      for (int s = 0; s < SL; ++s) mbar_wait(&S.mbar[SL * g + s], ((*phase >> s) & 1u) ^ 1u);
   }
   __syncthreads();
-  if ((threadIdx.x >> 5) == 0) tmem_dealloc(S.tmem_base, NG * 64);
+  if ((threadIdx.x >> 5) == 0) tmem_dealloc(S.tmem_base, kTmemCols(NG, SL));
 }
 
 // 2 GELU(y) for two packed f16 values: y (1 + tanh(y (a + b y^2))).
@@ -283,6 +329,21 @@ __device__ __forceinline__ uint32_t gelu2_f16x2(uint32_t y) {
   const uint32_t y2 = hmul2(y, y);
   const uint32_t u = hmul2(y, hfma2(y2, kB, kA));
   return hfma2(y, htanh2(u), y);
+}
+
+// GELU(y) for two packed f16 values on the FMA pipe only:
+// relu(y) + s q(s), s = min(|y|, 3.5), q(s) = c1 + c2 s + ... + c6 s^5.
+__device__ __forceinline__ uint32_t gelu_poly_f16x2(uint32_t y) {
+  uint32_t s, r;
+  asm("and.b32 %0, %1, 0x7FFF7FFF;" : "=r"(s) : "r"(y));
+  asm("min.f16x2 %0, %1, %2;" : "=r"(s) : "r"(s), "r"(0x43004300u));
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(y), "r"(0u));
+  uint32_t q = hfma2(0x98779877u, s, 0x25652565u);  // c6 s + c5
+  q = hfma2(q, s, 0xAB11AB11u);                     // + c4
+  q = hfma2(q, s, 0xAB4AAB4Au);                     // + c3
+  q = hfma2(q, s, 0x371E371Eu);                     // + c2
+  q = hfma2(q, s, 0xB814B814u);                     // + c1
+  return hfma2(q, s, r);
 }
 
 // Pair enumerations of one MLP pass: row p -> compact particles (a, b).
@@ -304,71 +365,93 @@ struct RectPairs {  // ordered pairs (i0 + p / m, p % m): a query block against 
 };
 
 // Runs the 4-layer MLP over `npairs` rows in 128-row tiles. Group g (threads
-// 128g .. 128g+127) takes tiles g, g+NG, ...; thread row r of a group owns
-// TMEM lane r (its warp's lane quadrant). For each valid row the sink gets
-// (p, a, b, u[8]). Returns false if the group aborted on a timed-out wait.
-template <int PM, int NG, bool kFastLog, class Pairs, class Sink>
-__device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, const Pairs& pairs,
-                         Sink& sink, uint32_t& phase) {
+// 128g .. 128g+127) takes tiles g, g+NG, ... and keeps up to SL of them in
+// flight (each slot: activation tile, 64 TMEM columns, an mbarrier): while
+// the tensor cores run one slot's layer, the group computes another slot's
+// epilogue. Thread row r of a group owns TMEM lane r. For each valid row the
+// sink gets (p, a, b, u[8]). Bit s of *phase tracks slot s's mbarrier parity.
+// Returns false if the group aborted on a timed-out wait.
+template <int PM, int NG, int SL, bool kFastLog, class Pairs, class Sink>
+__device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Particles<PM>& P, int npairs, const Pairs& pairs,
+                         Sink& sink, uint32_t* phase) {
+  static_assert(SL == 1 || SL == 2, "one or two tiles in flight per group");
   const int g = threadIdx.x >> 7;
   const int row = threadIdx.x & 127;
   const uint32_t bar_id = 1 + g;
   const bool leader = row == 0;
-  const uint32_t t_d = S.tmem_base + (uint32_t)(g * 64);
-  const uint32_t t_ld = S.tmem_base + ((uint32_t)(row & 96) << 16) + (uint32_t)(g * 64);
-  __half* A = S.A[g];
-  const uint32_t a_addr = smem_u32(A);
   const uint32_t w_addr[4] = {smem_u32(S.W1), smem_u32(S.W2), smem_u32(S.W3), smem_u32(S.W4)};
+  const uint32_t ones_addr = smem_u32(S.Ones);
   constexpr uint32_t kId64 = idesc_f16_m128(64), kId16 = idesc_f16_m128(16);
   const int ntiles = (npairs + kTileM - 1) / kTileM;
   bool ok = true;
-  // The bias columns of this thread's activation row: (1, 1, 0, ..., 0). They
-  // are rewritten on every pass because the tiles double as scratch between
-  // passes (the fused kernel stages K and V there).
-  *reinterpret_cast<uint4*>(A + cofs(row, 64, kAK)) = make_uint4(0x3C003C00u, 0u, 0u, 0u);
-  *reinterpret_cast<uint4*>(A + cofs(row, 72, kAK)) = make_uint4(0u, 0u, 0u, 0u);
 
-  // Publish this thread's operand writes and TMEM reads, meet the group, issue
-  // one layer's MMAs from the leader, wait for them to complete.
-  auto layer = [&](int L) -> bool {
+  // slot s: activation tile A0 + s*kTileElems, TMEM columns t_d0 + 64 s,
+  // mbarrier S.mbar[SL g + s]; selected arithmetically (no local-memory arrays)
+  constexpr int kTileElems = kTileM * kAK;
+  __half* const A0 = S.A[SL * g];
+  const uint32_t a_addr0 = smem_u32(A0);
+  const uint32_t t_d0 = S.tmem_base + (uint32_t)(SL * g * 64);
+  const uint32_t lane_off = (uint32_t)(row & 96) << 16;
+
+  // Publish this thread's operand writes and TMEM reads, meet the group and
+  // have the leader issue layer L of slot s; completion arrives on its mbarrier.
+  auto issue = [&](int s, int L) -> bool {
     fence_proxy_async_smem();
     tc_fence_before();
     if (named_bar_or(bar_id, 128, !ok)) return false;
     if (leader) {
       tc_fence_after();
+      const uint32_t a_addr = a_addr0 + (uint32_t)(s * kTileElems * 2);
+      const uint32_t d = t_d0 + 64u * s;
       if (L == 0) {
-        mma_f16(t_d, smem_desc(a_addr, 128, kSBO), smem_desc(w_addr[0], 128, 256), kId64, 0);
+        mma_f16(d, smem_desc(a_addr, 128, kASBO), smem_desc(w_addr[0], 128, 256), kId64, 0);
       } else {
+        const uint32_t w = L == 1 ? w_addr[1] : (L == 2 ? w_addr[2] : w_addr[3]);
+        const uint32_t id = L == 3 ? kId16 : kId64;
+        // bias step first (initialises the accumulator), then the 64 activations
+        mma_f16(d, smem_desc(ones_addr, 128, 256), smem_desc(w + 1024u, 128, kWSBO), id, 0u);
 #pragma unroll
-        for (int s = 0; s < kAK / 16; ++s)
-          mma_f16(t_d, smem_desc(a_addr + 256u * s, 128, kSBO), smem_desc(w_addr[L] + 256u * s, 128, kSBO),
-                  L == 3 ? kId16 : kId64, s > 0 ? 1u : 0u);
+        for (int k = 0; k < kAK / 16; ++k)
+          mma_f16(d, smem_desc(a_addr + 256u * k, 128, kASBO), smem_desc(w + 256u * k, 128, kWSBO), id, 1u);
       }
-      mma_commit(&S.mbar[g]);
+      mma_commit(&S.mbar[SL * g + s]);
     }
-    ok = mbar_wait(&S.mbar[g], phase);
-    phase ^= 1u;
-    tc_fence_after();
     return true;
   };
+  auto wait = [&](int s) {
+    const bool done = mbar_wait(&S.mbar[SL * g + s], (*phase >> s) & 1u);
+    ok = ok && done;
+    *phase ^= 1u << s;
+    tc_fence_after();
+  };
 
-  // TMEM accumulator row (bias included) -> 2 GELU in f16x2 -> next A tile.
-  auto hidden = [&]() {
+  // TMEM accumulator row (bias included) -> activation in f16x2 -> the slot's A tile.
+  auto hidden = [&](int s) {
+    __half* As = A0 + s * kTileElems;
+    const uint32_t t = t_d0 + 64u * s + lane_off;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       float v[32];
-      tmem_ld32_wait(t_ld + 32u * half, v);
+      tmem_ld32_wait(t + 32u * half, v);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        const int chunk = 4 * half + c;
         uint32_t w[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w[j] = gelu2_f16x2(cvt_f16x2(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]));
-        *reinterpret_cast<uint4*>(A + cofs(row, 32 * half + 8 * c, kAK)) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t y = cvt_f16x2(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]);
+          w[j] = chunk < kTanhChunks ? gelu2_f16x2(y) : gelu_poly_f16x2(y);
+        }
+        *reinterpret_cast<uint4*>(As + cofs(row, 8 * chunk, kAK)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   };
 
-  for (int t = g; t < ntiles; t += NG) {
+  // Features of tile t into slot s's layer-1 operand row: [hi(f) | hi(f) |
+  // lo(f) | 1 1 0 0] against [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0]
+  // gives W1 f + b1 to ~22 bits. Returns the row's pair index (-1 if beyond
+  // npairs) and its particles.
+  auto start = [&](int s, int t, int& p_out, int& a_out, int& b_out) -> bool {
     const int p = t * kTileM + row;
     const bool valid = p < npairs;
     int a = 0, b = 0;
@@ -377,30 +460,64 @@ __device__ bool mlp_pass(MlpSmem<NG>& S, const Particles<PM>& P, int npairs, con
       pairs.map(p, a, b);
       pair_feat<PM, kFastLog>(P, min(a, b), max(a, b), f);
     }
-    // layer-1 operand row: [hi(f) | hi(f) | lo(f) | 1 1 0 0] against
-    // [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0] gives W1 f + b1 to ~22 bits
-    {
-      __half hi[4], lo[4];
+    p_out = valid ? p : -1;
+    a_out = a;
+    b_out = b;
+    __half hi[4], lo[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) split_half(f[i], hi[i], lo[i]);
-      const __half one = __float2half_rn(valid ? 1.f : 0.f), zero = __float2half_rn(0.f);
-      __half r0[8] = {hi[0], hi[1], hi[2], hi[3], hi[0], hi[1], hi[2], hi[3]};
-      __half r1[8] = {lo[0], lo[1], lo[2], lo[3], one, one, zero, zero};
-      *reinterpret_cast<uint4*>(A + cofs(row, 0, kAK)) = *reinterpret_cast<uint4*>(r0);
-      *reinterpret_cast<uint4*>(A + cofs(row, 8, kAK)) = *reinterpret_cast<uint4*>(r1);
-    }
-    if (!layer(0)) return false;
-    hidden();
-    if (!layer(1)) return false;
-    hidden();
-    if (!layer(2)) return false;
-    hidden();
-    if (!layer(3)) return false;
-    float u[8];
-    tmem_ld8_wait(t_ld, u);
-    if (valid) sink(p, a, b, u);
+    for (int i = 0; i < 4; ++i) split_half(f[i], hi[i], lo[i]);
+    const __half one = __float2half_rn(valid ? 1.f : 0.f), zero = __float2half_rn(0.f);
+    __half* As = A0 + s * kTileElems;
+    *reinterpret_cast<uint4*>(As + cofs(row, 0, kAK)) =
+        make_uint4(h2bits(hi[0], hi[1]), h2bits(hi[2], hi[3]), h2bits(hi[0], hi[1]), h2bits(hi[2], hi[3]));
+    *reinterpret_cast<uint4*>(As + cofs(row, 8, kAK)) =
+        make_uint4(h2bits(lo[0], lo[1]), h2bits(lo[2], lo[3]), h2bits(one, one), h2bits(zero, zero));
+    return issue(s, 0);
+  };
+
+  // per-slot state: tile index (-1 = idle), next layer, row's pair and particles
+  int tile0 = -1, tile1 = -1, lay0 = 0, lay1 = 0;
+  int p0 = -1, a0 = 0, b0 = 0, p1 = -1, a1 = 0, b1 = 0;
+  int next = g;
+  if (next < ntiles) {
+    tile0 = next;
+    next += NG;
+    lay0 = 1;
+    if (!start(0, tile0, p0, a0, b0)) return false;
   }
-  // the TMEM reads of the last tile must finish before anyone reuses it
+  if (SL == 2 && next < ntiles) {
+    tile1 = next;
+    next += NG;
+    lay1 = 1;
+    if (!start(1, tile1, p1, a1, b1)) return false;
+  }
+#pragma unroll 1
+  for (int s = 0; tile0 >= 0 || tile1 >= 0; s = (SL == 2) ? (s ^ 1) : 0) {
+    int& tile = s ? tile1 : tile0;
+    int& lay = s ? lay1 : lay0;
+    if (tile < 0) continue;
+    wait(s);
+    if (lay <= 3) {
+      hidden(s);
+      if (!issue(s, lay)) return false;
+      ++lay;
+    } else {
+      float u[8];
+      tmem_ld8_wait(t_d0 + 64u * s + lane_off, u);
+      const int p = s ? p1 : p0;
+      if (p >= 0) sink(p, s ? a1 : a0, s ? b1 : b0, u);
+      if (next < ntiles) {
+        tile = next;
+        next += NG;
+        lay = 1;
+        const bool started = s ? start(1, tile, p1, a1, b1) : start(0, tile, p0, a0, b0);
+        if (!started) return false;
+      } else {
+        tile = -1;
+      }
+    }
+  }
+  // the TMEM reads of the last tiles must finish before anyone reuses them
   tc_fence_before();
   return ok;
 }
@@ -448,27 +565,27 @@ __device__ void zero_masked_pairs(const Particles<PM>& S, void* U, int n, int P)
 
 template <int PM, int NG>
 struct MlpBiasSmem {
-  MlpSmem<NG> mlp;
+  MlpSmem<NG, 2> mlp;
   Particles<PM> part;
 };
 
 template <int PM, int NG, bool F32OUT>
-__global__ void __launch_bounds__(NG * 128) k_mlp_bias(JetArgs J, MlpArgs W, void* __restrict__ U) {
+__global__ void __launch_bounds__(NG * 128, 1) k_mlp_bias(JetArgs J, MlpArgs W, void* __restrict__ U) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   MlpBiasSmem<PM, NG>& S = *reinterpret_cast<MlpBiasSmem<PM, NG>*>(smem_raw);
-  mlp_setup<NG>(S.mlp, W);
-  uint32_t phase = 0;
+  mlp_setup<NG, 2>(S.mlp, W);
+  uint32_t phase = 0u;
   bool aborted = false;
   for (int n = blockIdx.x; n < J.N; n += gridDim.x) {
     stage_jet<PM>(S.part, J, n);
     zero_masked_pairs<PM, F32OUT>(S.part, U, n, J.P);
     const int m = S.part.m;
     GlobalUSink<PM, F32OUT> sink{&S.part, U, n, J.P};
-    const bool ok = mlp_pass<PM, NG, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, phase);
+    const bool ok = mlp_pass<PM, NG, 2, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, &phase);
     aborted = __syncthreads_or(!ok) != 0;
     if (aborted) break;
   }
-  mlp_teardown<NG>(S.mlp, aborted, &phase);
+  mlp_teardown<NG, 2>(S.mlp, aborted, &phase);
 }
 
 // ========================================================== attention engine
@@ -644,9 +761,17 @@ __global__ void __launch_bounds__(256) k_attn_bias(JetArgs J, QkvArgs X, const u
 // per-CTA shared memory after the MLP tiles and the particles.
 constexpr int kSmemLimit = 232448;  // 227 KB per CTA on sm_100
 
+// Tiles in flight per group in the fused kernel: two for P <= 128 (the bias
+// triangle of such jets is small), one for P = 256 (room for wider jets).
+template <int PM>
+struct FusedSlots {
+  static constexpr int value = PM <= 128 ? 2 : 1;
+};
+
 template <int PM, int NG>
 struct FusedLayout {
-  static constexpr int kFixed = (int)(sizeof(MlpSmem<NG>) + sizeof(Particles<PM>)) + 1024;
+  static constexpr int kSL = FusedSlots<PM>::value;
+  static constexpr int kFixed = (int)(sizeof(MlpSmem<NG, kSL>) + sizeof(Particles<PM>)) + 1024;
   static constexpr int kUCap = (kSmemLimit - kFixed) / 16;
 };
 
@@ -676,28 +801,29 @@ struct RectUBias {  // U of (query i, key j) at index (i - i0) * m + j
 
 template <int PM, int NG>
 struct FusedSmem {
-  MlpSmem<NG> mlp;
+  MlpSmem<NG, FusedLayout<PM, NG>::kSL> mlp;
   Particles<PM> part;
   uint4 U8[FusedLayout<PM, NG>::kUCap];
 };
 
 template <int PM, int NG>
-__global__ void __launch_bounds__(NG * 128) k_fused(JetArgs J, MlpArgs W, QkvArgs X) {
+__global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, QkvArgs X) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FusedSmem<PM, NG>& S = *reinterpret_cast<FusedSmem<PM, NG>*>(smem_raw);
-  mlp_setup<NG>(S.mlp, W);
+  constexpr int SL = FusedLayout<PM, NG>::kSL;
+  mlp_setup<NG, SL>(S.mlp, W);
   // during attention the activation tiles hold K and V
   float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
-  constexpr int kStageFloats = NG * kTileM * kAK / 2;
+  constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
   constexpr int kUCap = FusedLayout<PM, NG>::kUCap;
-  uint32_t phase = 0;
+  uint32_t phase = 0u;
   bool aborted = false;
   for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
     stage_jet<PM>(S.part, J, n);
     const int m = S.part.m;
     SmemUSink sink{S.U8};
     if (m * (m + 1) / 2 <= kUCap) {
-      const bool ok = mlp_pass<PM, NG, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, phase);
+      const bool ok = mlp_pass<PM, NG, SL, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, &phase);
       aborted = __syncthreads_or(!ok) != 0;
       if (aborted) break;
       TriUBias ub{reinterpret_cast<const __half*>(S.U8)};
@@ -706,7 +832,7 @@ __global__ void __launch_bounds__(NG * 128) k_fused(JetArgs J, MlpArgs W, QkvArg
       const int qb = kUCap / m;
       for (int i0 = 0; i0 < m; i0 += qb) {
         const int i1 = min(m, i0 + qb);
-        const bool ok = mlp_pass<PM, NG, true>(S.mlp, S.part, (i1 - i0) * m, RectPairs{i0, m}, sink, phase);
+        const bool ok = mlp_pass<PM, NG, SL, true>(S.mlp, S.part, (i1 - i0) * m, RectPairs{i0, m}, sink, &phase);
         aborted = __syncthreads_or(!ok) != 0;
         if (aborted) break;
         RectUBias ub{reinterpret_cast<const __half*>(S.U8), i0, m};
@@ -717,7 +843,7 @@ __global__ void __launch_bounds__(NG * 128) k_fused(JetArgs J, MlpArgs W, QkvArg
     zero_masked_rows<PM>(S.part, J, X.out, n);
     __syncthreads();
   }
-  mlp_teardown<NG>(S.mlp, aborted, &phase);
+  mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
 }
 
 }  // namespace pb
