@@ -167,6 +167,23 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 64 columns of a 16-bit accumulator row (one f16 per TMEM column) as 32
+// packed f16x2 words: word i holds columns 2i (low half) and 2i+1 (high).
+__device__ __forceinline__ void tmem_ld64_f16_wait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.pack::16b.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, float* v) {
   uint32_t r[8];
   asm volatile(
@@ -181,10 +198,10 @@ __device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, float* v) {
 
 // ------------------------------------------------------------------- tcgen05
 
-// Instruction descriptor for kind::f16 with f16 A and B, fp32 accumulate,
-// both operands K-major, M = 128.
-__host__ __device__ constexpr uint32_t idesc_f16_m128(int n) {
-  return (1u << 4)                       // D format: f32
+// Instruction descriptor for kind::f16 with f16 A and B, both operands
+// K-major, M = 128; D is fp32 (default) or f16.
+__host__ __device__ constexpr uint32_t idesc_f16_m128(int n, bool f32_acc = true) {
+  return ((f32_acc ? 1u : 0u) << 4)      // D format: f32 or f16
          | (0u << 7) | (0u << 10)        // A, B format: f16
          | (0u << 15) | (0u << 16)       // A, B K-major
          | ((uint32_t)(n >> 3) << 17)    // N / 8

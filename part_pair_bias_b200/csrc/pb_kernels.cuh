@@ -167,15 +167,16 @@ __global__ void __launch_bounds__(256) k_pairfeat(JetArgs J, float* __restrict__
 // Numerics of the tensor-core MLP (all exact rescalings are powers of two):
 //   layer 1: y1 = W1 f + b1 with f and W1 split into f16 hi + lo parts, the
 //            bias through a column of ones, so y1 carries ~22 bits;
-//   hidden:  the accumulator row (bias included) is converted to packed f16
-//            and activated on two pipes: 5 of every 8 columns with the tanh
+//   hidden:  layers 1..3 accumulate in f16 in TMEM (the row is read back as
+//            packed f16x2, so no conversion is needed) and are activated on
+//            two pipes: 5 of every 8 columns with the tanh
 //            form h = y (1 + tanh(a y + b y^3)) = 2 GELU(y) (one MUFU op per
 //            two values; a, b fitted minimax to the erf GELU, max deviation
 //            2.7e-4), the other 3 with h = relu(y) + s q(s), s = min(|y|, 3.5),
 //            q a degree-6 polynomial fitted to GELU - relu (f16 evaluation,
 //            max deviation 4.8e-3), on the FMA pipe only. The next layer's
 //            weights carry 1/2 on the tanh columns;
-//   layers 2..4: f16 operands, fp32 accumulation in TMEM; each bias enters
+//   layers 2..4: f16 operands; layer 4 accumulates in fp32; each bias enters
 //            through an extra K step: a constant tile of ones times the
 //            weights' (hi(b), lo(b)) columns.
 
@@ -381,7 +382,8 @@ __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Particles<PM>& P, int npairs,
   const bool leader = row == 0;
   const uint32_t w_addr[4] = {smem_u32(S.W1), smem_u32(S.W2), smem_u32(S.W3), smem_u32(S.W4)};
   const uint32_t ones_addr = smem_u32(S.Ones);
-  constexpr uint32_t kId64 = idesc_f16_m128(64), kId16 = idesc_f16_m128(16);
+  // layers 1..3 accumulate in f16 (read back packed, no conversion), layer 4 in fp32
+  constexpr uint32_t kId64 = idesc_f16_m128(64, false), kId16 = idesc_f16_m128(16, true);
   const int ntiles = (npairs + kTileM - 1) / kTileM;
   bool ok = true;
 
@@ -425,25 +427,18 @@ __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Particles<PM>& P, int npairs,
     tc_fence_after();
   };
 
-  // TMEM accumulator row (bias included) -> activation in f16x2 -> the slot's A tile.
+  // TMEM accumulator row (bias included, f16) -> activation in f16x2 -> the slot's A tile.
   auto hidden = [&](int s) {
     __half* As = A0 + s * kTileElems;
-    const uint32_t t = t_d0 + 64u * s + lane_off;
+    uint32_t y[32];
+    tmem_ld64_f16_wait(t_d0 + 64u * s + lane_off, y);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float v[32];
-      tmem_ld32_wait(t + 32u * half, v);
+    for (int chunk = 0; chunk < 8; ++chunk) {
+      uint32_t w[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int chunk = 4 * half + c;
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t y = cvt_f16x2(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]);
-          w[j] = chunk < kTanhChunks ? gelu2_f16x2(y) : gelu_poly_f16x2(y);
-        }
-        *reinterpret_cast<uint4*>(As + cofs(row, 8 * chunk, kAK)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      for (int j = 0; j < 4; ++j)
+        w[j] = chunk < kTanhChunks ? gelu2_f16x2(y[4 * chunk + j]) : gelu_poly_f16x2(y[4 * chunk + j]);
+      *reinterpret_cast<uint4*>(As + cofs(row, 8 * chunk, kAK)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   };
 
