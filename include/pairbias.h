@@ -20,9 +20,9 @@
  *   - All array arguments are DEVICE pointers owned by the caller, except in
  *     pb_fold_affine (host). Nothing is allocated inside the library.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
- *     NULL = the legacy default stream), launches exactly one kernel and
- *     does not synchronise. Host-side argument errors return before any
- *     launch; device-side problems (an invalid ptr array, a bounded wait that
+ *     NULL = the legacy default stream), launches exactly one kernel (the
+ *     balanced fused path as a cooperative launch) and does not synchronise.
+ *     Host-side argument errors return before any launch; device-side problems (an invalid ptr array, a bounded wait that
  *     ran out) set bits of a per-device status word, read with
  *     pb_get_device_status.
  *   - H must be 8 and D must be 16 (the MLP output width fixes H);
@@ -113,24 +113,43 @@ pb_status pairfeat_compute(const pb_jets *jets, float *feat, void *stream);
 /* pairbias_mlp_forward -- features and folded MLP, materialising the bias.
  * U: [N, 8, P, P] in `dtype` (PB_BF16 raw bits or PB_F32); U[n,h,i,j] ==
  * U[n,h,j,i]; entries with a masked end are 0. The MLP runs on tcgen05 tensor
- * cores with f16 operands and fp32 accumulation; hidden activations never
- * leave the chip. Source: "Fusion 2". */
+ * cores with f16 operands (hidden layers accumulate in f16, the output layer
+ * in fp32); hidden activations never leave the chip. Source: "Fusion 2". */
 pb_status pairbias_mlp_forward(const pb_jets *jets, const pb_mlp *mlp, void *U, pb_dtype dtype,
                                void *stream);
 
 /* pair_attention_forward -- masked multi-head attention with the pair bias.
  * Exactly one of `mlp` and `U` is non-NULL:
  *   mlp != NULL: the fused path -- features, MLP and attention in one kernel;
- *                the bias is produced and consumed on chip, never in HBM;
+ *                the bias is produced and consumed on chip (shared memory,
+ *                or with a workspace the L2-resident records), never read
+ *                back from HBM;
  *   U   != NULL: the bias is read from a bf16 [N, 8, P, P] array (as written
  *                by pairbias_mlp_forward with PB_BF16).
  * q, k, v, out: bf16 in the layout of `jets` (padded [N,H,P,D], packed
  * [tokens,H,D]). out = softmax(q k^T / sqrt(D) + U) v over valid keys, with
  * fp32 scores, softmax and accumulation; masked query rows are 0.
+ * workspace / workspace_bytes: optional, fused path only (see
+ * pb_workspace_bytes); NULL / 0 otherwise.
  * Source: "Fusion 3" (with the bias of "Fusion 2"). */
 pb_status pair_attention_forward(const pb_jets *jets, const pb_mlp *mlp, const uint16_t *U,
                                  int H, int D, const uint16_t *q, const uint16_t *k,
-                                 const uint16_t *v, uint16_t *out, void *stream);
+                                 const uint16_t *v, uint16_t *out, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/* pb_workspace_bytes -- size of the optional workspace of the fused path.
+ * With a workspace of at least this size (device memory, 256-byte aligned,
+ * zero-filled before its first use; every call leaves its first 256 bytes
+ * zero again), pair_attention_forward(mlp != NULL) spreads the MLP tiles of
+ * all jets evenly over all SMs and keeps each pair's 8 biases in the
+ * workspace (16 bytes per pair, read back from L2) between the MLP and the
+ * attention; this needs N <= 8192 and, padded, N*P <= 2^21. Without one (NULL
+ * or too small) each CTA runs whole jets and keeps their bias in shared
+ * memory. Returns 0 when the balanced path does not apply to `jets`. A call
+ * that reports PB_DEV_TIMEOUT may leave the workspace header non-zero: zero it
+ * again before reuse. Calls sharing one workspace must not overlap on the
+ * device. */
+size_t pb_workspace_bytes(const pb_jets *jets);
 
 /* pb_get_device_status -- synchronise `stream`, then read and clear the
  * status word of the current device. *bits (may be NULL) receives the

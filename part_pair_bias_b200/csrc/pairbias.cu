@@ -153,6 +153,36 @@ pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArg
   return launched("k_fused");
 }
 
+constexpr long long kGridMaxMaskBytes = 1ll << 21;  // padded N*P scanned by every CTA in phase 0
+
+bool grid_applies(const pb::JetArgs& J) {
+  if (J.N < 1 || J.N > pb::kGridMaxJets) return false;
+  if (!J.ptr && (long long)J.N * J.P > kGridMaxMaskBytes) return false;
+  return true;
+}
+
+template <int PM>
+pb_status run_fused_grid(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, void* ws,
+                         cudaStream_t s) {
+  auto k = pb::k_fused_grid<PM>;
+  const size_t smem = sizeof(pb::FusedGridSmem<PM>);
+  int dev = 0, sms = 0;
+  pb_status st = device_sms(&dev, &sms);
+  if (st != PB_OK) return st;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(%zu B smem): %s", smem, cudaGetErrorString(e));
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 512, smem);
+  if (e != cudaSuccess || per_sm < 1) return fail(PB_ECUDA, "k_fused_grid does not fit on an SM");
+  long long g = sms;  // one CTA per SM, all resident
+  if (g > 8ll * J.N) g = 8ll * J.N;
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  void* args[] = {(void*)&J, (void*)&W, (void*)&X, (void*)&wsb};
+  e = cudaLaunchCooperativeKernel((const void*)k, dim3((unsigned)g), dim3(512), args, smem, s);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "k_fused_grid cooperative launch: %s", cudaGetErrorString(e));
+  return PB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -186,9 +216,15 @@ pb_status pairbias_mlp_forward(const pb_jets* jets, const pb_mlp* mlp, void* U, 
   return J.P <= 128 ? run_mlp_bias<128, false>(J, W, U, s) : run_mlp_bias<256, false>(J, W, U, s);
 }
 
+size_t pb_workspace_bytes(const pb_jets* jets) {
+  pb::JetArgs J;
+  if (check_jets(jets, &J) != PB_OK || !grid_applies(J)) return 0;
+  return pb::grid_workspace_bytes(J.N, J.P, J.tokens, J.ptr != nullptr);
+}
+
 pb_status pair_attention_forward(const pb_jets* jets, const pb_mlp* mlp, const uint16_t* U, int H, int D,
                                  const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
-                                 void* stream) {
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   pb::JetArgs J;
   pb_status st = check_jets(jets, &J);
   if (st != PB_OK) return st;
@@ -204,6 +240,12 @@ pb_status pair_attention_forward(const pb_jets* jets, const pb_mlp* mlp, const u
   if (mlp) {
     pb::MlpArgs W;
     if ((st = check_mlp(mlp, &W)) != PB_OK) return st;
+    if (workspace) {
+      if (!aligned(workspace, 256)) return fail(PB_EINVAL, "workspace must be 256-byte aligned");
+      if (grid_applies(J) &&
+          workspace_bytes >= pb::grid_workspace_bytes(J.N, J.P, J.tokens, J.ptr != nullptr))
+        return J.P <= 128 ? run_fused_grid<128>(J, W, X, workspace, s) : run_fused_grid<256>(J, W, X, workspace, s);
+    }
     return J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
   }
   return J.P <= 128 ? run_attn_bias<128>(J, X, U, s) : run_attn_bias<256>(J, X, U, s);

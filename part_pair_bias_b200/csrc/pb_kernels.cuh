@@ -372,9 +372,26 @@ struct RectPairs {  // ordered pairs (i0 + p / m, p % m): a query block against 
 // epilogue. Thread row r of a group owns TMEM lane r. For each valid row the
 // sink gets (p, a, b, u[8]). Bit s of *phase tracks slot s's mbarrier parity.
 // Returns false if the group aborted on a timed-out wait.
-template <int PM, int NG, int SL, bool kFastLog, class Pairs, class Sink>
-__device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Particles<PM>& P, int npairs, const Pairs& pairs,
-                         Sink& sink, uint32_t* phase) {
+// A source of MLP rows for one pass: ntiles() tiles; row(t, r, ...) gives
+// the features of row r of tile t and the (p, a, b) its sink receives, or
+// false for a padding row.
+template <int PM, class Pairs, bool kFastLog>
+struct JetTiles {  // the pairs of one staged jet
+  const Particles<PM>* P;
+  int npairs;
+  Pairs pairs;
+  __device__ __forceinline__ int ntiles() const { return (npairs + kTileM - 1) / kTileM; }
+  __device__ __forceinline__ bool row(int t, int r, int& p, int& a, int& b, float f[4]) const {
+    p = t * kTileM + r;
+    if (p >= npairs) return false;
+    pairs.map(p, a, b);
+    pair_feat<PM, kFastLog>(*P, min(a, b), max(a, b), f);
+    return true;
+  }
+};
+
+template <int NG, int SL, class Source, class Sink>
+__device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Source& src, Sink& sink, uint32_t* phase) {
   static_assert(SL == 1 || SL == 2, "one or two tiles in flight per group");
   const int g = threadIdx.x >> 7;
   const int row = threadIdx.x & 127;
@@ -384,7 +401,7 @@ __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Particles<PM>& P, int npairs,
   const uint32_t ones_addr = smem_u32(S.Ones);
   // layers 1..3 accumulate in f16 (read back packed, no conversion), layer 4 in fp32
   constexpr uint32_t kId64 = idesc_f16_m128(64, false), kId16 = idesc_f16_m128(16, true);
-  const int ntiles = (npairs + kTileM - 1) / kTileM;
+  const int ntiles = src.ntiles();
   bool ok = true;
 
   // slot s: activation tile A0 + s*kTileElems, TMEM columns t_d0 + 64 s,
@@ -444,16 +461,15 @@ __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Particles<PM>& P, int npairs,
 
   // Features of tile t into slot s's layer-1 operand row: [hi(f) | hi(f) |
   // lo(f) | 1 1 0 0] against [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0]
-  // gives W1 f + b1 to ~22 bits. Returns the row's pair index (-1 if beyond
-  // npairs) and its particles.
+  // gives W1 f + b1 to ~22 bits. Returns the row's sink key (-1 for a padding
+  // row) and its particles.
   auto start = [&](int s, int t, int& p_out, int& a_out, int& b_out) -> bool {
-    const int p = t * kTileM + row;
-    const bool valid = p < npairs;
-    int a = 0, b = 0;
+    int p = -1, a = 0, b = 0;
     float f[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) {
-      pairs.map(p, a, b);
-      pair_feat<PM, kFastLog>(P, min(a, b), max(a, b), f);
+    const bool valid = src.row(t, row, p, a, b, f);
+    if (!valid) {
+      f[0] = f[1] = f[2] = f[3] = 0.f;
+      a = b = 0;
     }
     p_out = valid ? p : -1;
     a_out = a;
@@ -576,7 +592,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_mlp_bias(JetArgs J, MlpArgs W, 
     zero_masked_pairs<PM, F32OUT>(S.part, U, n, J.P);
     const int m = S.part.m;
     GlobalUSink<PM, F32OUT> sink{&S.part, U, n, J.P};
-    const bool ok = mlp_pass<PM, NG, 2, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, &phase);
+    const bool ok = mlp_pass<NG, 2>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, m * (m + 1) / 2, TriPairs{}}, sink, &phase);
     aborted = __syncthreads_or(!ok) != 0;
     if (aborted) break;
   }
@@ -611,19 +627,28 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float* f) {
 // Masked multi-head attention for queries [i_lo, i_hi) of the staged jet,
 // all valid keys, on CUDA cores: one thread per (query, head), keys streamed
 // from shared memory in chunks of 8 with an online (running-max) softmax in
-// the log2 domain. ubias(i, j, h) returns U[h, i, j]. `stage` holds K and V
-// of up to `stage_floats / (32 m)` heads at a time as fp32.
+// the log2 domain, for heads [h_lo, h_hi). ubias(i, j, h) returns U[h, i, j].
+// `stage` holds K and V of up to `stage_floats / (32 m)` heads at a time as fp32.
 template <int PM, class UBias>
 __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int i_lo,
-                                int i_hi, float* stage, int stage_floats, const UBias& ubias) {
+                                int i_hi, float* stage, int stage_floats, const UBias& ubias, int h_lo = 0,
+                                int h_hi = kH) {
   const int m = S.m;
   const int nq = i_hi - i_lo;
   const int tid = threadIdx.x, nthr = blockDim.x;
   if (m <= 0 || nq <= 0) return;
   const int HR = min(kH, stage_floats / (32 * m));
   const float qscale = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
-  for (int h0 = 0; h0 < kH; h0 += HR) {
-    const int hr = min(HR, kH - h0);
+  for (int h0 = h_lo; h0 < h_hi; h0 += HR) {
+    const int hr = min(HR, h_hi - h0);
+    // this thread's first query row is fetched before the staging barrier so
+    // that its memory latency overlaps the K/V staging
+    uint4 qraw0 = make_uint4(0, 0, 0, 0), qraw1 = qraw0;
+    if (tid < hr * nq) {
+      const uint16_t* qp = X.q + qkv_off<PM>(S, J, n, h0 + tid / nq, i_lo + tid % nq);
+      qraw0 = *reinterpret_cast<const uint4*>(qp);
+      qraw1 = *reinterpret_cast<const uint4*>(qp + 8);
+    }
     for (int idx = tid; idx < hr * m * 4; idx += nthr) {
       const int part = idx & 3, j = (idx >> 2) % m, hh = (idx >> 2) / m;
       const uint16_t* src = (part < 2 ? X.k : X.v) + qkv_off<PM>(S, J, n, h0 + hh, j) + (part & 1) * 8;
@@ -637,9 +662,13 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
     for (int item = tid; item < hr * nq; item += nthr) {
       const int hh = item / nq, i = i_lo + item % nq, h = h0 + hh;
       float q[16];
-      const uint16_t* qp = X.q + qkv_off<PM>(S, J, n, h, i);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(qp), q);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(qp + 8), q + 8);
+      if (item != tid) {
+        const uint16_t* qp = X.q + qkv_off<PM>(S, J, n, h, i);
+        qraw0 = *reinterpret_cast<const uint4*>(qp);
+        qraw1 = *reinterpret_cast<const uint4*>(qp + 8);
+      }
+      bf16x8_to_f32(qraw0, q);
+      bf16x8_to_f32(qraw1, q + 8);
 #pragma unroll
       for (int d = 0; d < 16; ++d) q[d] *= qscale;
       float o[16];
@@ -656,16 +685,16 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
           s[jj] = -INFINITY;
           if (j < m) {
             const float4* kr = reinterpret_cast<const float4*>(kv + j * 32);
-            float acc = 0.f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains instead of one of 16
 #pragma unroll
             for (int d4 = 0; d4 < 4; ++d4) {
               const float4 k4 = kr[d4];
-              acc = fmaf(q[4 * d4], k4.x, acc);
-              acc = fmaf(q[4 * d4 + 1], k4.y, acc);
-              acc = fmaf(q[4 * d4 + 2], k4.z, acc);
-              acc = fmaf(q[4 * d4 + 3], k4.w, acc);
+              acc[d4] = fmaf(q[4 * d4], k4.x, acc[d4]);
+              acc[d4] = fmaf(q[4 * d4 + 1], k4.y, acc[d4]);
+              acc[d4] = fmaf(q[4 * d4 + 2], k4.z, acc[d4]);
+              acc[d4] = fmaf(q[4 * d4 + 3], k4.w, acc[d4]);
             }
-            s[jj] = fmaf(ubias(i, j, h), kLog2e, acc);
+            s[jj] = fmaf(ubias(i, j, h), kLog2e, (acc[0] + acc[1]) + (acc[2] + acc[3]));
             cmax = fmaxf(cmax, s[jj]);
           }
         }
@@ -818,7 +847,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
     const int m = S.part.m;
     SmemUSink sink{S.U8};
     if (m * (m + 1) / 2 <= kUCap) {
-      const bool ok = mlp_pass<PM, NG, SL, true>(S.mlp, S.part, m * (m + 1) / 2, TriPairs{}, sink, &phase);
+      const bool ok = mlp_pass<NG, SL>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, m * (m + 1) / 2, TriPairs{}}, sink, &phase);
       aborted = __syncthreads_or(!ok) != 0;
       if (aborted) break;
       TriUBias ub{reinterpret_cast<const __half*>(S.U8)};
@@ -827,7 +856,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
       const int qb = kUCap / m;
       for (int i0 = 0; i0 < m; i0 += qb) {
         const int i1 = min(m, i0 + qb);
-        const bool ok = mlp_pass<PM, NG, SL, true>(S.mlp, S.part, (i1 - i0) * m, RectPairs{i0, m}, sink, &phase);
+        const bool ok = mlp_pass<NG, SL>(S.mlp, JetTiles<PM, RectPairs, true>{&S.part, (i1 - i0) * m, RectPairs{i0, m}}, sink, &phase);
         aborted = __syncthreads_or(!ok) != 0;
         if (aborted) break;
         RectUBias ub{reinterpret_cast<const __half*>(S.U8), i0, m};
@@ -839,6 +868,296 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
     __syncthreads();
   }
   mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
+}
+
+// ================================================= k_fused_grid (balanced)
+//
+// The fused path spread over the whole GPU. One CTA per SM, all resident
+// (cooperative launch); a caller-provided workspace holds two barrier
+// counters and the bias records of every pair (8 f16 per pair, 16 bytes,
+// 2 MB for 128 jets of ~40 particles: it stays in the 126 MB L2).
+//   phase 0  every CTA derives the same jet table: the number of 128-row MLP
+//            tiles of each jet and their exclusive prefix T (shared memory);
+//   phase A  the T[N] tiles are split evenly over the CTAs; a CTA stages up
+//            to kBatch jets of its range at a time and streams their tiles
+//            through the MLP pipeline without draining between jets; each
+//            row's 8 biases go to record T[n] * 128 + p of the workspace;
+//   barrier  (bounded; counters reset by the last CTA to leave)
+//   phase B  the 8 N (jet, head) attention items, weighted by the jet's tiles,
+//            are split evenly over the CTAs and run with the bias read back
+//            from the records.
+// Jets of any multiplicity up to P use the unordered triangle.
+
+constexpr int kGridMaxJets = 8192;    // jet-table capacity (shared memory)
+constexpr size_t kWsHeader = 256;     // barrier counters, then the records
+
+template <int PM>
+struct GridCfg {
+  static constexpr int kBatch = PM <= 128 ? 4 : 2;  // jets staged at once in phase A
+};
+
+template <int PM>
+struct BatchInfo {  // the jets of one phase-A batch
+  int K;                                  // jets in the batch
+  int tbeg[GridCfg<PM>::kBatch + 1];      // prefix of their tiles within the batch
+  int t_lo[GridCfg<PM>::kBatch];          // first tile of each jet taken by this CTA
+  int npairs[GridCfg<PM>::kBatch];
+  long long rowbase[GridCfg<PM>::kBatch]; // record index of the jet's pair 0
+};
+
+template <int PM>
+struct FusedGridSmem {
+  MlpSmem<4, 2> mlp;                       // activation tiles double as scratch in phases 0 and B
+  Particles<PM> ring[GridCfg<PM>::kBatch];
+  int T[kGridMaxJets + 1];                 // exclusive prefix of tiles per jet
+  BatchInfo<PM> batch;
+  int warp_sums[32];
+  int flag;
+};
+
+// Tiles of a staged batch, in order; row keys are record indices.
+template <int PM>
+struct BatchTiles {
+  const Particles<PM>* ring;
+  const BatchInfo<PM>* B;
+  __device__ __forceinline__ int ntiles() const { return B->tbeg[B->K]; }
+  __device__ __forceinline__ bool row(int bt, int r, int& p, int& a, int& b, float f[4]) const {
+    int k = 0;
+#pragma unroll
+    for (int q = 1; q < GridCfg<PM>::kBatch; ++q) k += (q < B->K && B->tbeg[q] <= bt) ? 1 : 0;
+    const int pl = (B->t_lo[k] + bt - B->tbeg[k]) * kTileM + r;
+    if (pl >= B->npairs[k]) return false;
+    TriPairs{}.map(pl, a, b);
+    pair_feat<PM, true>(ring[k], min(a, b), max(a, b), f);
+    p = (int)(B->rowbase[k] + pl);  // record index (fits: < 2^31 for N <= 8192, P <= 256)
+    return true;
+  }
+};
+
+struct RecordSink {  // the 8 biases of a pair as 8 f16 in one 16-byte record
+  uint4* rec;
+  __device__ __forceinline__ void operator()(int p, int, int, const float* u) const {
+    rec[p] = make_uint4(pack_half2(u[0], u[1]), pack_half2(u[2], u[3]), pack_half2(u[4], u[5]),
+                        pack_half2(u[6], u[7]));
+  }
+};
+
+struct RecordUBias {  // U[h, i, j] from the jet's records (unordered-pair index)
+  const __half* rec;   // record 0 of the jet, as halves
+  __device__ __forceinline__ float operator()(int i, int j, int h) const {
+    const int hi = max(i, j), lo = min(i, j);
+    return __half2float(rec[(size_t)(hi * (hi + 1) / 2 + lo) * 8 + h]);
+  }
+};
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier over `nblk` resident CTAs on a counter that only grows
+// within a launch. Bounded: returns false (status raised) if it runs out.
+__device__ bool grid_barrier(unsigned long long* ctr, unsigned nblk, int* smem_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned long long old = atomicAdd(ctr, 1ull);
+    const unsigned long long target = (old / nblk + 1) * nblk;
+    bool ok = true;
+    unsigned long long t0 = 0;
+    for (uint32_t it = 0; ld_acquire_u64(ctr) < target; ++it) {
+      if ((it & 63u) == 63u) {
+        const unsigned long long now = global_ns();
+        if (t0 == 0) {
+          t0 = now;
+        } else if (now - t0 > kWaitNs) {
+          raise_status(kStTimeout);
+          ok = false;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *smem_flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *smem_flag != 0;
+}
+
+// Valid particles of jet n without staging them (phase 0).
+__device__ __forceinline__ int jet_count(const JetArgs& J, int n, int lane) {
+  if (J.ptr) {
+    const long long lo = J.ptr[n], hi = J.ptr[n + 1];
+    return (lo < 0 || hi < lo || hi > J.tokens || hi - lo > J.P) ? 0 : (int)(hi - lo);
+  }
+  int c = 0;
+  for (int s0 = 0; s0 < J.P; s0 += 32) {
+    const int sl = s0 + lane;
+    c += __popc(__ballot_sync(0xffffffffu, sl < J.P && J.mask[(long long)n * J.P + sl] != 0));
+  }
+  return c;
+}
+
+template <int PM>
+__global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, QkvArgs X, unsigned char* ws) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  FusedGridSmem<PM>& S = *reinterpret_cast<FusedGridSmem<PM>*>(smem_raw);
+  constexpr int NG = 4, SL = 2, JB = GridCfg<PM>::kBatch;
+  unsigned long long* bar_ctr = reinterpret_cast<unsigned long long*>(ws);
+  unsigned long long* exit_ctr = bar_ctr + 1;
+  uint4* rec = reinterpret_cast<uint4*>(ws + kWsHeader);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const int G = gridDim.x, b = blockIdx.x;
+  const int N = J.N;
+
+  // ---------------------------------------------------------------- phase 0
+  // tiles per jet into T[n + 1] (one warp per jet), then an exclusive scan
+  for (int n = warp; n < N; n += nwarp) {
+    const int m = jet_count(J, n, lane);
+    if (lane == 0) S.T[n + 1] = (m * (m + 1) / 2 + kTileM - 1) / kTileM;
+  }
+  if (tid == 0) S.T[0] = 0;
+  __syncthreads();
+  {
+    // each thread scans a contiguous chunk, warps then the block combine
+    const int per = (N + blockDim.x - 1) / blockDim.x;
+    const int c0 = 1 + tid * per, c1 = min(N + 1, c0 + per);
+    int sum = 0;
+    for (int i = c0; i < c1; ++i) sum += S.T[i];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) S.warp_sums[warp] = incl;
+    __syncthreads();
+    int woff = 0;
+    for (int w = 0; w < warp; ++w) woff += S.warp_sums[w];
+    int run = woff + incl - sum;
+    __syncthreads();
+    for (int i = c0; i < c1; ++i) {
+      run += S.T[i];
+      S.T[i] = run;
+    }
+  }
+  __syncthreads();
+  const long long Ttot = S.T[N];
+
+  mlp_setup<NG, SL>(S.mlp, W);
+  uint32_t phase = 0u;
+  bool aborted = false;
+
+  // ---------------------------------------------------------------- phase A
+  {
+    const long long lo = Ttot * b / G, hi = Ttot * (b + 1) / G;
+    // first jet whose tiles reach past lo
+    int n = 0;
+    {
+      int l = 0, r = N;  // smallest n with T[n + 1] > lo
+      while (l < r) {
+        const int mid = (l + r) >> 1;
+        if (S.T[mid + 1] > lo) r = mid; else l = mid + 1;
+      }
+      n = l;
+    }
+    while (!aborted && n < N && S.T[n] < hi) {
+      // gather up to JB jets with tiles in [lo, hi)
+      if (tid == 0) {
+        int K = 0, acc = 0;
+        int nn = n;
+        while (K < JB && nn < N && S.T[nn] < hi) {
+          const long long a0 = max((long long)S.T[nn], lo), a1 = min((long long)S.T[nn + 1], hi);
+          if (a1 > a0) {
+            S.batch.tbeg[K] = acc;
+            S.batch.t_lo[K] = (int)(a0 - S.T[nn]);
+            S.batch.rowbase[K] = (long long)S.T[nn] * kTileM;
+            S.batch.npairs[K] = nn;  // jet index for now; replaced after staging
+            acc += (int)(a1 - a0);
+            ++K;
+          }
+          ++nn;
+        }
+        S.batch.tbeg[K] = acc;
+        S.batch.K = K;
+        S.flag = nn;  // next jet to look at
+      }
+      __syncthreads();
+      const int K = S.batch.K;
+      const int n_next = S.flag;
+      for (int k = 0; k < K; ++k) stage_jet<PM>(S.ring[k], J, S.batch.npairs[k]);
+      if (tid == 0)
+        for (int k = 0; k < K; ++k) S.batch.npairs[k] = S.ring[k].m * (S.ring[k].m + 1) / 2;
+      __syncthreads();
+      RecordSink sink{rec};
+      const bool ok = mlp_pass<NG, SL>(S.mlp, BatchTiles<PM>{S.ring, &S.batch}, sink, &phase);
+      aborted = __syncthreads_or(!ok) != 0;
+      n = n_next;
+    }
+  }
+
+  // --------------------------------------------------------------- barrier
+  const bool passed = grid_barrier(bar_ctr, (unsigned)G, &S.flag);
+  aborted = aborted || !passed;
+
+  // ---------------------------------------------------------------- phase B
+  if (!aborted) {
+    // item (n, h) costs tiles_n + 1; its start is 8 (T[n] + n) + h (tiles_n + 1)
+    const long long C = 8ll * (Ttot + N);
+    const long long lo = C * b / G, hi = C * (b + 1) / G;
+    int n = 0;
+    {
+      int l = 0, r = N;  // smallest n whose items end past lo
+      while (l < r) {
+        const int mid = (l + r) >> 1;
+        if (8ll * ((long long)S.T[mid + 1] + mid + 1) > lo) r = mid; else l = mid + 1;
+      }
+      n = l;
+    }
+    float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
+    constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
+    for (; n < N && 8ll * ((long long)S.T[n] + n) < hi; ++n) {
+      const long long base = 8ll * ((long long)S.T[n] + n);
+      const long long c = (long long)(S.T[n + 1] - S.T[n]) + 1;
+      int h_lo = 0, h_hi = 0;
+      for (int h = 0; h < kH; ++h) {
+        const long long st = base + h * c;
+        if (st < lo) h_lo = h + 1;
+        if (st < hi) h_hi = h + 1;
+      }
+      if (h_lo >= h_hi) continue;
+      stage_jet<PM>(S.ring[0], J, n);
+      RecordUBias ub{reinterpret_cast<const __half*>(rec + (size_t)S.T[n] * kTileM)};
+      attention_block<PM>(S.ring[0], J, X, n, 0, S.ring[0].m, stage, kStageFloats, ub, h_lo, h_hi);
+      if (h_lo == 0) zero_masked_rows<PM>(S.ring[0], J, X.out, n);
+      __syncthreads();
+    }
+  }
+
+  mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
+  // the last CTA to leave resets both counters for the next launch
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(exit_ctr, 1ull) == (unsigned long long)(G - 1)) {
+      atomicExch(bar_ctr, 0ull);
+      atomicExch(exit_ctr, 0ull);
+      __threadfence();
+    }
+  }
+}
+
+// Workspace bytes of the balanced path: header + one 16-byte record per row
+// of every jet's tiles (bounded from N, P and, packed, the token count).
+__host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long tokens, bool packed) {
+  const long long per_jet_tiles = ((long long)P * (P + 1) / 2 + kTileM - 1) / kTileM;
+  long long rows = (long long)N * per_jet_tiles * kTileM;
+  if (packed) {
+    // sum over jets of ceil(m(m+1)/2 / 128) * 128 <= tokens (P + 1) / 2 + 127 N
+    const long long alt = tokens * (P + 1) / 2 + (long long)(kTileM - 1) * N + kTileM;
+    rows = alt < rows ? alt : rows;
+  }
+  return kWsHeader + (size_t)rows * 16;
 }
 
 }  // namespace pb

@@ -70,7 +70,9 @@ def lib():
             L.pairfeat_compute.argtypes = [C.POINTER(_Jets), vp, vp]
             L.pairbias_mlp_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, vp]
             L.pair_attention_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, C.c_int,
-                                                 vp, vp, vp, vp, vp]
+                                                 vp, vp, vp, vp, vp, C.c_size_t, vp]
+            L.pb_workspace_bytes.argtypes = [C.POINTER(_Jets)]
+            L.pb_workspace_bytes.restype = C.c_size_t
             L.pb_get_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
             L.pb_fold_affine.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float)]
             L.pb_last_error.restype = C.c_char_p
@@ -170,18 +172,35 @@ def pairbias_mlp_forward(jets: Jets, mlp: FoldedMLP, U: torch.Tensor, stream=Non
     _check(lib().pairbias_mlp_forward(C.byref(js), C.byref(ms), U.data_ptr(), dtype, _stream(stream)))
 
 
+def workspace_bytes(jets: Jets) -> int:
+    """Bytes of the optional workspace of the fused path (0 if it does not apply)."""
+    js = jets.struct()
+    return int(lib().pb_workspace_bytes(C.byref(js)))
+
+
+def workspace_for(jets: Jets, device="cuda") -> Optional[torch.Tensor]:
+    """A zero-filled workspace tensor for the fused path, or None."""
+    n = workspace_bytes(jets)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
 def pair_attention_forward(jets: Jets, mlp: Optional[FoldedMLP], U: Optional[torch.Tensor], q: torch.Tensor,
-                           k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, stream=None) -> None:
-    """Fused (mlp given) or bias-reading (U given, bf16) attention; bf16 q/k/v/out."""
+                           k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Fused (mlp given) or bias-reading (U given, bf16) attention; bf16 q/k/v/out.
+    An optional uint8 workspace (``workspace_for``) selects the fused path
+    that balances the MLP tiles of all jets over all SMs."""
     for t in (q, k, v, out):
         assert t.dtype == torch.bfloat16 and t.is_contiguous()
     if U is not None:
         assert U.dtype == torch.bfloat16 and U.is_contiguous()
     js = jets.struct()
     ms = mlp.struct() if mlp is not None else None
+    ws_ptr = _dp(workspace)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().pair_attention_forward(C.byref(js), C.byref(ms) if ms is not None else None,
                                         _dp(U), H, D, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                        out.data_ptr(), _stream(stream)))
+                                        out.data_ptr(), ws_ptr, ws_len, _stream(stream)))
 
 
 def get_device_status(stream=None) -> int:

@@ -104,9 +104,17 @@ class Device:
         ops.pairbias_mlp_forward(self.jets, self.mlp, U)
         return U
 
-    def fused(self):
+    def fused(self, balanced=False):
+        """The fused path; balanced=True passes a workspace (all-SM MLP split)."""
         out = torch.full_like(self.q, float("nan"))
-        ops.pair_attention_forward(self.jets, self.mlp, None, self.q, self.k, self.v, out)
+        ws = None
+        if balanced:
+            ws = ops.workspace_for(self.jets, self.q.device)
+            assert ws is not None
+        ops.pair_attention_forward(self.jets, self.mlp, None, self.q, self.k, self.v, out, workspace=ws)
+        if balanced:
+            torch.cuda.synchronize()
+            assert torch.all(ws[:256] == 0), "the workspace header must be left zero"
         return out
 
     def with_bias(self, U_bf16):

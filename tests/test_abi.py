@@ -31,7 +31,8 @@ def declared_functions():
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
     assert {"pairfeat_compute", "pairbias_mlp_forward", "pair_attention_forward",
-            "pb_get_device_status", "pb_fold_affine", "pb_last_error", "pb_version"} <= set(names)
+            "pb_get_device_status", "pb_fold_affine", "pb_last_error", "pb_version",
+            "pb_workspace_bytes"} <= set(names)
     for n in names:
         assert hasattr(L, n), f"{n} declared in pairbias.h but not exported"
     assert ops.version().startswith("pairbias-b200")
@@ -67,14 +68,17 @@ def test_host_validation(L):
     assert L.pairfeat_compute(C.byref(js2), d, None) == ops.PB_EINVAL      # misaligned momenta
     js3, keep3 = _jets()
     mlp = ops._Mlp(*([d] * 8))
-    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 4, 16, d, d, d, d, None) == ops.PB_EUNSUPPORTED
-    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 32, d, d, d, d, None) == ops.PB_EUNSUPPORTED
-    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), d, 8, 16, d, d, d, d, None) == ops.PB_EINVAL
-    assert L.pair_attention_forward(C.byref(js3), None, None, 8, 16, d, d, d, d, None) == ops.PB_EINVAL
-    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 16, d + 2, d, d, d, None) == ops.PB_EINVAL
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 4, 16, d, d, d, d, None, 0, None) == ops.PB_EUNSUPPORTED
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 32, d, d, d, d, None, 0, None) == ops.PB_EUNSUPPORTED
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), d, 8, 16, d, d, d, d, None, 0, None) == ops.PB_EINVAL
+    assert L.pair_attention_forward(C.byref(js3), None, None, 8, 16, d, d, d, d, None, 0, None) == ops.PB_EINVAL
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 16, d + 2, d, d, d, None, 0, None) == ops.PB_EINVAL
     assert L.pairbias_mlp_forward(C.byref(js3), C.byref(mlp), d, 7, None) == ops.PB_EINVAL
     bad = ops._Mlp(*([d] * 7 + [0]))
     assert L.pairbias_mlp_forward(C.byref(js3), C.byref(bad), d, 0, None) == ops.PB_EINVAL
+    # misaligned workspace on the fused path
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 16, d, d, d, d, d + 16, 1 << 20,
+                                    None) == ops.PB_EINVAL
     # N = 0 is a no-op that needs no device
     js3.N = 0
     assert L.pairfeat_compute(C.byref(js3), d, None) == ops.PB_OK
@@ -99,3 +103,18 @@ def test_fold_affine_matches_unfolded_oracle(L, oracle_lib):
             ref = oracle_lib.mlp_row(f, p)
             assert np.max(np.abs(u - ref)) < 2e-5 * max(1.0, np.max(np.abs(ref)))
     assert L.pb_fold_affine(None, None) == ops.PB_EINVAL
+
+
+def test_workspace_size_rules(L):
+    """The balanced fused path's workspace: header + 16 bytes per row of every
+    jet's 128-row tiles; 0 where the path does not apply."""
+    js, keep = _jets(N=128, P=128)
+    tiles = (128 * 129 // 2 + 127) // 128
+    assert L.pb_workspace_bytes(C.byref(js)) == 256 + 128 * tiles * 128 * 16
+    js.N = 9000                       # more jets than the jet table holds
+    assert L.pb_workspace_bytes(C.byref(js)) == 0
+    js.N = 0
+    assert L.pb_workspace_bytes(C.byref(js)) == 0
+    js4, keep4 = _jets(N=8192, P=128, ptr=True)
+    js4.tokens = 327680               # packed: bounded by the token count
+    assert L.pb_workspace_bytes(C.byref(js4)) == 256 + (327680 * 129 // 2 + 127 * 8192 + 128) * 16

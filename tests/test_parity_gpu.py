@@ -81,10 +81,11 @@ def test_bias(oracle_lib, name, dtype):
 
 
 @pytest.mark.parametrize("name", ALL)
-def test_fused_attention(oracle_lib, name):
+@pytest.mark.parametrize("balanced", [False, True])
+def test_fused_attention(oracle_lib, name, balanced):
     b = batch(name)
     d = pt.Device(b)
-    got = pt.to_np(d.fused())
+    got = pt.to_np(d.fused(balanced))
     assert ops.get_device_status() == 0
     for lo, hi in sample_ranges(b):
         s = synth.slice_jets(b, lo, hi)
@@ -122,9 +123,11 @@ def test_odd_p_scrambled_masks_and_degenerate_jets(oracle_lib):
     d = pt.Device(b)
     pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
     pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
-    got = pt.to_np(d.fused())
-    pt.check_attention(got, oracle_lib.forward(b), b)
-    assert np.all(got[0] == 0.0)                     # empty jet: every row masked
+    ref = oracle_lib.forward(b)
+    for balanced in (False, True):
+        got = pt.to_np(d.fused(balanced))
+        pt.check_attention(got, ref, b)
+        assert np.all(got[0] == 0.0)                 # empty jet: every row masked
     assert ops.get_device_status() == 0
 
 
@@ -134,7 +137,9 @@ def test_wide_jets_query_block_path(oracle_lib):
     b = synth.make_jets(N=5, P=256, mults=[256, 200, 129, 128, 3], pt_lo=800, pt_hi=1000, prongs=3, seed=5)
     d = pt.Device(b)
     pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
-    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)   # whole triangles in the records
     assert ops.get_device_status() == 0
 
 
@@ -142,7 +147,9 @@ def test_packed_with_empty_jets(oracle_lib):
     b = synth.make_jets(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6)
     d = pt.Device(b)
     pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
-    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
     assert ops.get_device_status() == 0
 
 
@@ -162,6 +169,8 @@ def test_deterministic_and_empty_batch():
     d = pt.Device(b)
     o1, o2 = d.fused(), d.fused()
     assert torch.equal(o1, o2)
+    w1, w2 = d.fused(True), d.fused(True)          # balanced path: same bits on a reused workspace
+    assert torch.equal(w1, w2)
     e = synth.make_jets(N=0, P=16, mults=np.zeros(0, int), seed=1)
     de = pt.Device(e)
     ops.pair_attention_forward(de.jets, de.mlp, None, de.q, de.k, de.v, torch.empty_like(de.q))
@@ -175,5 +184,7 @@ def test_many_jets_per_cta(oracle_lib):
     b = synth.make_jets(N=700, P=24, dist="uniform", mult_lo=1, mult_hi=24, mask_mode="scrambled", seed=8)
     d = pt.Device(b)
     pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
-    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
     assert ops.get_device_status() == 0
