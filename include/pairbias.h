@@ -151,6 +151,33 @@ pb_status pair_attention_forward(const pb_jets *jets, const pb_mlp *mlp, const u
  * device. */
 size_t pb_workspace_bytes(const pb_jets *jets);
 
+/* PB_STATIC_SCRATCH_BYTES -- size of the library's static per-device scratch
+ * array used by pair_attention_forward_noalloc (32 MiB). */
+#define PB_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* pair_attention_forward_noalloc -- the fused path of pair_attention_forward
+ * (mlp given) with the balanced kernel, for callers that cannot allocate
+ * device memory: instead of a caller workspace it uses a static device array
+ * inside the library, PB_STATIC_SCRATCH_BYTES per device. The paper has no
+ * counterpart; it is an interface variant, the arithmetic is that of
+ * pair_attention_forward.
+ *   Arguments as in pair_attention_forward (bf16 q/k/v/out, H = 8, D = 16).
+ *   Rejects (PB_EUNSUPPORTED, message with both sizes) a batch whose
+ *   pb_workspace_bytes bound is 0 or exceeds PB_STATIC_SCRATCH_BYTES; this is
+ *   decided on the host from N, P and tokens before any device call.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture. Every call then clears the array's 256-byte
+ *   header (barrier counters) on `stream` with cudaMemsetAsync and launches
+ *   one cooperative kernel. It calls no cudaMalloc, cudaFree or other
+ *   allocating routine.
+ *   All calls on a device share the one array: calls that overlap on the
+ *   device (unordered streams, concurrent host threads) race and produce
+ *   wrong results; order them on one stream. */
+pb_status pair_attention_forward_noalloc(const pb_jets *jets, const pb_mlp *mlp, int H, int D,
+                                         const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                         uint16_t *out, void *stream);
+
 /* pb_get_device_status -- synchronise `stream`, then read and clear the
  * status word of the current device. *bits (may be NULL) receives the
  * PB_DEV_* bits. Returns PB_OK when no bit was set, PB_EDEVICE otherwise,

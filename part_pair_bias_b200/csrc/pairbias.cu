@@ -183,6 +183,32 @@ pb_status run_fused_grid(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::Q
   return PB_OK;
 }
 
+// Scratch of pair_attention_forward_noalloc: the balanced kernel's workspace
+// (barrier counters, then the bias records) as a file-scope device array, so
+// that this entry point allocates nothing. Each device holds its own copy,
+// zero at module load; all calls on a device share it.
+static __device__ __align__(256) unsigned char g_static_scratch[PB_STATIC_SCRATCH_BYTES];
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in for the symbol).
+void* g_static_scratch_ptr[kMaxDev] = {};
+
+pb_status static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDev) return fail(PB_ECUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return fail(PB_ECUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return PB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -249,6 +275,35 @@ pb_status pair_attention_forward(const pb_jets* jets, const pb_mlp* mlp, const u
     return J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
   }
   return J.P <= 128 ? run_attn_bias<128>(J, X, U, s) : run_attn_bias<256>(J, X, U, s);
+}
+
+pb_status pair_attention_forward_noalloc(const pb_jets* jets, const pb_mlp* mlp, int H, int D, const uint16_t* q,
+                                         const uint16_t* k, const uint16_t* v, uint16_t* out, void* stream) {
+  pb::JetArgs J;
+  pb::MlpArgs W;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK) return st;
+  if (H != pb::kH || D != pb::kD) return fail(PB_EUNSUPPORTED, "H = %d, D = %d; only H = 8, D = 16", H, D);
+  if ((st = check_mlp(mlp, &W)) != PB_OK) return st;
+  if (J.N == 0) return PB_OK;
+  if (!q || !k || !v || !out) return fail(PB_EINVAL, "q, k, v and out must be non-NULL");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return fail(PB_EINVAL, "q, k, v and out must be 16-byte aligned");
+  if (!grid_applies(J))
+    return fail(PB_EUNSUPPORTED, "static-scratch path needs 1 <= N <= %d and, padded, N*P <= %lld (N = %d, P = %d)",
+                pb::kGridMaxJets, kGridMaxMaskBytes, J.N, J.P);
+  const size_t need = pb::grid_workspace_bytes(J.N, J.P, J.tokens, J.ptr != nullptr);
+  if (need > (size_t)PB_STATIC_SCRATCH_BYTES)
+    return fail(PB_EUNSUPPORTED, "batch needs %zu bytes of scratch, the static scratch holds %zu (N = %d, P = %d)",
+                need, (size_t)PB_STATIC_SCRATCH_BYTES, J.N, J.P);
+  void* ws = nullptr;
+  if ((st = static_scratch(&ws)) != PB_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the barrier counters must start at zero (a timed-out call may leave them set)
+  cudaError_t e = cudaMemsetAsync(ws, 0, pb::kWsHeader, s);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "clearing the static scratch header: %s", cudaGetErrorString(e));
+  const pb::QkvArgs X{q, k, v, out};
+  return J.P <= 128 ? run_fused_grid<128>(J, W, X, ws, s) : run_fused_grid<256>(J, W, X, ws, s);
 }
 
 pb_status pb_get_device_status(void* stream, uint32_t* bits) {

@@ -6,7 +6,8 @@ on first use and its absence is an error -- there is no fallback.
 
 Entry points mirror ``include/pairbias.h``: ``pairfeat_compute``,
 ``pairbias_mlp_forward``, ``pair_attention_forward``,
-``get_device_status`` and the host helper ``fold_affine``.
+``pair_attention_forward_noalloc``, ``get_device_status`` and the host
+helper ``fold_affine``.
 """
 from __future__ import annotations
 
@@ -25,6 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libpairbias.so")
 PB_OK, PB_EINVAL, PB_EUNSUPPORTED, PB_ECUDA, PB_EDEVICE = range(5)
 PB_BF16, PB_F32 = 0, 1
 PB_DEV_TIMEOUT, PB_DEV_BADPTR = 1, 2
+PB_STATIC_SCRATCH_BYTES = 32 << 20
 H, D = 8, 16
 
 # offsets of the folded parameters in the flat buffer (PB_OFF_* in the header)
@@ -71,6 +73,8 @@ def lib():
             L.pairbias_mlp_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, vp]
             L.pair_attention_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, C.c_int,
                                                  vp, vp, vp, vp, vp, C.c_size_t, vp]
+            L.pair_attention_forward_noalloc.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.c_int, C.c_int,
+                                                         vp, vp, vp, vp, vp]
             L.pb_workspace_bytes.argtypes = [C.POINTER(_Jets)]
             L.pb_workspace_bytes.restype = C.c_size_t
             L.pb_get_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
@@ -78,7 +82,7 @@ def lib():
             L.pb_last_error.restype = C.c_char_p
             L.pb_version.restype = C.c_char_p
             for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward,
-                      L.pb_get_device_status, L.pb_fold_affine):
+                      L.pair_attention_forward_noalloc, L.pb_get_device_status, L.pb_fold_affine):
                 f.restype = C.c_int
             _lib = L
         return _lib
@@ -201,6 +205,17 @@ def pair_attention_forward(jets: Jets, mlp: Optional[FoldedMLP], U: Optional[tor
     _check(lib().pair_attention_forward(C.byref(js), C.byref(ms) if ms is not None else None,
                                         _dp(U), H, D, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                         out.data_ptr(), ws_ptr, ws_len, _stream(stream)))
+
+
+def pair_attention_forward_noalloc(jets: Jets, mlp: FoldedMLP, q: torch.Tensor, k: torch.Tensor,
+                                   v: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """The fused path on the library's static per-device scratch (no
+    allocation anywhere); calls on one device must not overlap."""
+    for t in (q, k, v, out):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    js, ms = jets.struct(), mlp.struct()
+    _check(lib().pair_attention_forward_noalloc(C.byref(js), C.byref(ms), H, D, q.data_ptr(), k.data_ptr(),
+                                                v.data_ptr(), out.data_ptr(), _stream(stream)))
 
 
 def get_device_status(stream=None) -> int:

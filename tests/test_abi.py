@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
     assert {"pairfeat_compute", "pairbias_mlp_forward", "pair_attention_forward",
             "pb_get_device_status", "pb_fold_affine", "pb_last_error", "pb_version",
-            "pb_workspace_bytes"} <= set(names)
+            "pb_workspace_bytes", "pair_attention_forward_noalloc"} <= set(names)
     for n in names:
         assert hasattr(L, n), f"{n} declared in pairbias.h but not exported"
     assert ops.version().startswith("pairbias-b200")
@@ -76,8 +76,10 @@ def test_host_validation(L):
     assert L.pairbias_mlp_forward(C.byref(js3), C.byref(mlp), d, 7, None) == ops.PB_EINVAL
     bad = ops._Mlp(*([d] * 7 + [0]))
     assert L.pairbias_mlp_forward(C.byref(js3), C.byref(bad), d, 0, None) == ops.PB_EINVAL
-    # misaligned workspace on the fused path
-    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 16, d, d, d, d, d + 16, 1 << 20,
+    # misaligned workspace on the fused path (16 bytes past a 256-byte boundary)
+    wbuf = np.zeros(1024, np.uint8)
+    ws = (wbuf.ctypes.data + 255) // 256 * 256 + 16
+    assert L.pair_attention_forward(C.byref(js3), C.byref(mlp), None, 8, 16, d, d, d, d, ws, 1 << 20,
                                     None) == ops.PB_EINVAL
     # N = 0 is a no-op that needs no device
     js3.N = 0
@@ -118,3 +120,22 @@ def test_workspace_size_rules(L):
     js4, keep4 = _jets(N=8192, P=128, ptr=True)
     js4.tokens = 327680               # packed: bounded by the token count
     assert L.pb_workspace_bytes(C.byref(js4)) == 256 + (327680 * 129 // 2 + 127 * 8192 + 128) * 16
+
+
+def test_noalloc_host_rejections(L):
+    """The static-scratch entry point decides on the host, before any device
+    call, that a batch does not fit its scratch or its kernel."""
+    js, keep = _jets(N=256, P=256)
+    d = np.zeros(64, np.float32).ctypes.data
+    mlp = ops._Mlp(*([d] * 8))
+    need = 256 + 256 * ((256 * 257 // 2 + 127) // 128) * 128 * 16
+    assert need > ops.PB_STATIC_SCRATCH_BYTES
+    assert L.pair_attention_forward_noalloc(C.byref(js), C.byref(mlp), 8, 16, d, d, d, d, None) == ops.PB_EUNSUPPORTED
+    assert "static scratch" in L.pb_last_error().decode()
+    js.N = 9000                       # beyond the balanced kernel's jet table
+    assert L.pair_attention_forward_noalloc(C.byref(js), C.byref(mlp), 8, 16, d, d, d, d, None) == ops.PB_EUNSUPPORTED
+    js.N = 2
+    assert L.pair_attention_forward_noalloc(C.byref(js), None, 8, 16, d, d, d, d, None) == ops.PB_EINVAL
+    assert L.pair_attention_forward_noalloc(C.byref(js), C.byref(mlp), 8, 16, d + 2, d, d, d, None) == ops.PB_EINVAL
+    js.N = 0                          # nothing to do: no device needed
+    assert L.pair_attention_forward_noalloc(C.byref(js), C.byref(mlp), 8, 16, d, d, d, d, None) == ops.PB_OK

@@ -1,0 +1,47 @@
+"""The allocation-free fused entry point (static per-device scratch) against
+the allocating one, through the C ABI, on two calls in a row.
+
+Collected last on purpose: it must hold both in a fresh process, where the
+first call performs the per-device set-up, and after every other test has
+run on the same device.
+"""
+import numpy as np
+import pytest
+import torch
+
+from part_pair_bias_b200 import configs, ops, synth
+from tests import parity as pt
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    torch.cuda.set_device(0)
+    ops.lib()
+    yield
+    assert ops.get_device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["pr1_n8_p32", "n128_p128"])
+def test_noalloc_matches_fused_entry_point(name):
+    b = synth.make_jets(**configs.workload(name, seed=0))
+    d = pt.Device(b)
+    ref = pt.to_np(d.fused())                     # the existing entry point, no workspace
+    assert ops.get_device_status() == 0
+    for _call in range(2):
+        out = torch.full_like(d.q, float("nan"))
+        ops.pair_attention_forward_noalloc(d.jets, d.mlp, d.q, d.k, d.v, out)
+        assert ops.get_device_status() == 0
+        pt.check_attention(pt.to_np(out), ref, b)  # rel L2 <= 1e-2, masked rows exactly 0
+
+
+def test_noalloc_rejects_batches_beyond_the_static_scratch():
+    b = synth.make_jets(N=256, P=256, mults=np.full(256, 4), seed=2)
+    d = pt.Device(b)
+    out = torch.empty_like(d.q)
+    with pytest.raises(ops.PairBiasError) as ei:
+        ops.pair_attention_forward_noalloc(d.jets, d.mlp, d.q, d.k, d.v, out)
+    assert ei.value.status == ops.PB_EUNSUPPORTED
+    assert "static scratch" in str(ei.value)
