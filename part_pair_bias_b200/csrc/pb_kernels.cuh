@@ -627,8 +627,57 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float* f) {
 // Masked multi-head attention for queries [i_lo, i_hi) of the staged jet,
 // all valid keys, on CUDA cores: one thread per (query, head), keys streamed
 // from shared memory in chunks of 8 with an online (running-max) softmax in
-// the log2 domain, for heads [h_lo, h_hi). ubias(i, j, h) returns U[h, i, j].
+// the log2 domain, for heads [h_lo, h_hi). `ubias.row(i, h)` returns a cursor
+// whose next() yields U[h, i, 0], U[h, i, 1], ... in key order.
 // `stage` holds K and V of up to `stage_floats / (32 m)` heads at a time as fp32.
+// Full chunks run without predicates; only the last, partial chunk checks j < m.
+template <bool kTail, class Cursor>
+__device__ __forceinline__ void attention_chunk(const float* kv, int j0, int m, const float* q, Cursor& cur,
+                                                float* o, float& l, float& mx) {
+  float s[8];
+  float cmax = mx;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    s[jj] = -INFINITY;
+    if (!kTail || j0 + jj < m) {
+      const float4* kr = reinterpret_cast<const float4*>(kv + (j0 + jj) * 32);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains instead of one of 16
+#pragma unroll
+      for (int d4 = 0; d4 < 4; ++d4) {
+        const float4 k4 = kr[d4];
+        acc[d4] = fmaf(q[4 * d4], k4.x, acc[d4]);
+        acc[d4] = fmaf(q[4 * d4 + 1], k4.y, acc[d4]);
+        acc[d4] = fmaf(q[4 * d4 + 2], k4.z, acc[d4]);
+        acc[d4] = fmaf(q[4 * d4 + 3], k4.w, acc[d4]);
+      }
+      s[jj] = fmaf(cur.next(), kLog2e, (acc[0] + acc[1]) + (acc[2] + acc[3]));
+      cmax = fmaxf(cmax, s[jj]);
+    }
+  }
+  // every chunk holds at least one valid key, so cmax is finite
+  const float corr = ex2(mx - cmax);
+  l *= corr;
+#pragma unroll
+  for (int d = 0; d < 16; ++d) o[d] *= corr;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    if (!kTail || j0 + jj < m) {
+      const float pj = ex2(s[jj] - cmax);
+      l += pj;
+      const float4* vr = reinterpret_cast<const float4*>(kv + (j0 + jj) * 32 + 16);
+#pragma unroll
+      for (int d4 = 0; d4 < 4; ++d4) {
+        const float4 v4 = vr[d4];
+        o[4 * d4] = fmaf(pj, v4.x, o[4 * d4]);
+        o[4 * d4 + 1] = fmaf(pj, v4.y, o[4 * d4 + 1]);
+        o[4 * d4 + 2] = fmaf(pj, v4.z, o[4 * d4 + 2]);
+        o[4 * d4 + 3] = fmaf(pj, v4.w, o[4 * d4 + 3]);
+      }
+    }
+  }
+  mx = cmax;
+}
+
 template <int PM, class UBias>
 __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int i_lo,
                                 int i_hi, float* stage, int stage_floats, const UBias& ubias, int h_lo = 0,
@@ -676,51 +725,10 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
       for (int d = 0; d < 16; ++d) o[d] = 0.f;
       float l = 0.f, mx = -INFINITY;
       const float* kv = stage + hh * m * 32;
-      for (int j0 = 0; j0 < m; j0 += 8) {
-        float s[8];
-        float cmax = mx;
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int j = j0 + jj;
-          s[jj] = -INFINITY;
-          if (j < m) {
-            const float4* kr = reinterpret_cast<const float4*>(kv + j * 32);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains instead of one of 16
-#pragma unroll
-            for (int d4 = 0; d4 < 4; ++d4) {
-              const float4 k4 = kr[d4];
-              acc[d4] = fmaf(q[4 * d4], k4.x, acc[d4]);
-              acc[d4] = fmaf(q[4 * d4 + 1], k4.y, acc[d4]);
-              acc[d4] = fmaf(q[4 * d4 + 2], k4.z, acc[d4]);
-              acc[d4] = fmaf(q[4 * d4 + 3], k4.w, acc[d4]);
-            }
-            s[jj] = fmaf(ubias(i, j, h), kLog2e, (acc[0] + acc[1]) + (acc[2] + acc[3]));
-            cmax = fmaxf(cmax, s[jj]);
-          }
-        }
-        const float corr = ex2(mx - cmax);
-        l *= corr;
-#pragma unroll
-        for (int d = 0; d < 16; ++d) o[d] *= corr;
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int j = j0 + jj;
-          if (j < m) {
-            const float pj = ex2(s[jj] - cmax);
-            l += pj;
-            const float4* vr = reinterpret_cast<const float4*>(kv + j * 32 + 16);
-#pragma unroll
-            for (int d4 = 0; d4 < 4; ++d4) {
-              const float4 v4 = vr[d4];
-              o[4 * d4] = fmaf(pj, v4.x, o[4 * d4]);
-              o[4 * d4 + 1] = fmaf(pj, v4.y, o[4 * d4 + 1]);
-              o[4 * d4 + 2] = fmaf(pj, v4.z, o[4 * d4 + 2]);
-              o[4 * d4 + 3] = fmaf(pj, v4.w, o[4 * d4 + 3]);
-            }
-          }
-        }
-        mx = cmax;
-      }
+      auto cur = ubias.row(i, h);
+      int j0 = 0;
+      for (; j0 + 8 <= m; j0 += 8) attention_chunk<false>(kv, j0, m, q, cur, o, l, mx);
+      if (j0 < m) attention_chunk<true>(kv, j0, m, q, cur, o, l, mx);
       const float inv = 1.0f / l;
 #pragma unroll
       for (int d = 0; d < 16; ++d) o[d] *= inv;
@@ -751,8 +759,14 @@ struct GlobalUBias {
   const Particles<PM>* S;
   const uint16_t* U;
   int n, P;
-  __device__ __forceinline__ float operator()(int i, int j, int h) const {
-    return bf16_to_f32(U[(((size_t)n * kH + h) * P + S->slot[i]) * P + S->slot[j]]);
+  struct Cursor {  // keys in compact order, read at their slots of row slot[i]
+    const uint16_t* row;
+    const int16_t* slot;
+    int j;
+    __device__ __forceinline__ float next() { return bf16_to_f32(row[slot[j++]]); }
+  };
+  __device__ __forceinline__ Cursor row(int i, int h) const {
+    return Cursor{U + (((size_t)n * kH + h) * P + S->slot[i]) * P, S->slot, 0};
   }
 };
 
@@ -807,20 +821,37 @@ struct SmemUSink {
   }
 };
 
-struct TriUBias {  // U of pair (i, j) at index max(i,j)(max(i,j)+1)/2 + min(i,j)
-  const __half* U;
-  __device__ __forceinline__ float operator()(int i, int j, int h) const {
-    const int hi = max(i, j), lo = min(i, j);
-    return __half2float(U[(hi * (hi + 1) / 2 + lo) * 8 + h]);
+// Row i of a triangle of 8-half records, pair (a, b) with a >= b at record
+// a (a + 1) / 2 + b: walking the keys j = 0, 1, ..., the record of key j + 1
+// follows that of key j by 1 record while j < i and by j + 1 records after.
+struct TriCursor {
+  const __half* p;
+  int i, j;
+  __device__ __forceinline__ float next() {
+    const float u = __half2float(*p);
+    p += (j < i ? 1 : j + 1) * 8;
+    ++j;
+    return u;
   }
 };
 
-struct RectUBias {  // U of (query i, key j) at index (i - i0) * m + j
+struct TriUBias {  // U of pair (i, j) at record max(i,j)(max(i,j)+1)/2 + min(i,j)
+  const __half* U;
+  __device__ __forceinline__ TriCursor row(int i, int h) const { return TriCursor{U + (i * (i + 1) / 2) * 8 + h, i, 0}; }
+};
+
+struct RectUBias {  // U of (query i, key j) at record (i - i0) * m + j
   const __half* U;
   int i0, m;
-  __device__ __forceinline__ float operator()(int i, int j, int h) const {
-    return __half2float(U[((i - i0) * m + j) * 8 + h]);
-  }
+  struct Cursor {
+    const __half* p;
+    __device__ __forceinline__ float next() {
+      const float u = __half2float(*p);
+      p += 8;
+      return u;
+    }
+  };
+  __device__ __forceinline__ Cursor row(int i, int h) const { return Cursor{U + ((i - i0) * m) * 8 + h}; }
 };
 
 template <int PM, int NG>
@@ -944,9 +975,8 @@ struct RecordSink {  // the 8 biases of a pair as 8 f16 in one 16-byte record
 
 struct RecordUBias {  // U[h, i, j] from the jet's records (unordered-pair index)
   const __half* rec;   // record 0 of the jet, as halves
-  __device__ __forceinline__ float operator()(int i, int j, int h) const {
-    const int hi = max(i, j), lo = min(i, j);
-    return __half2float(rec[(size_t)(hi * (hi + 1) / 2 + lo) * 8 + h]);
+  __device__ __forceinline__ TriCursor row(int i, int h) const {
+    return TriCursor{rec + (size_t)(i * (i + 1) / 2) * 8 + h, i, 0};
   }
 };
 
