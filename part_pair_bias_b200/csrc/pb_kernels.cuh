@@ -56,8 +56,80 @@ struct Particles {
   long long base;    // element index of slot 0 of this jet in the momentum arrays
 };
 
-// Block-wide; blockDim.x must be a multiple of 32 and >= J.P.
-template <int PM>
+// Stage jets into shared memory: the valid particles get compact indices in
+// slot order and, with kKin, their fp64 kinematics (the attention needs only
+// m, base and the slot map). Groups of ceil(P/32) warps take one jet each, as
+// many jets at a time as the block holds groups; jet_of(k) is the jet of ring
+// entry k. Block-wide; blockDim.x must be a multiple of 32 and >= J.P.
+template <int PM, bool kKin, class JetOf>
+__device__ void stage_jets(Particles<PM>* ring, const JetArgs& J, int K, const JetOf& jet_of) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wpj = (J.P + 31) >> 5;                   // warps per jet
+  const int per = (int)(blockDim.x >> 5) / wpj;      // jets staged at once
+  const int g = warp / wpj, lw = warp - g * wpj, t = lw * 32 + lane;
+  for (int k0 = 0; k0 < K; k0 += per) {
+    const int k = k0 + g;
+    const bool act = g < per && k < K;
+    Particles<PM>& S = ring[act ? k : 0];
+    long long base = 0;
+    int cnt = 0;
+    bool valid = false;
+    if (act) {
+      const int n = jet_of(k);
+      if (J.ptr) {
+        const long long lo = J.ptr[n], hi = J.ptr[n + 1];
+        if (lo < 0 || hi < lo || hi > J.tokens || hi - lo > J.P) {
+          if (t == 0) raise_status(kStBadPtr);
+        } else {
+          base = lo;
+          cnt = (int)(hi - lo);
+        }
+      } else {
+        base = (long long)n * J.P;
+        cnt = J.P;
+      }
+      if (t < J.P) valid = J.ptr ? (t < cnt) : (J.mask[base + t] != 0);
+    }
+    const unsigned ballot = __ballot_sync(0xffffffffu, valid);
+    if (act && lane == 0) S.warp_cnt[lw] = __popc(ballot);
+    __syncthreads();
+    if (act) {
+      int off = 0, total = 0;
+      for (int w = 0; w < wpj; ++w) {
+        const int c = S.warp_cnt[w];
+        off += (w < lw) ? c : 0;
+        total += c;
+      }
+      const int c = off + __popc(ballot & ((1u << lane) - 1u));
+      if (t < J.P) S.comp[t] = valid ? (int16_t)c : (int16_t)-1;
+      if (valid) {
+        S.slot[c] = (int16_t)t;
+        if (kKin) {
+          const long long e = base + t;
+          const double E = J.E[e], px = J.px[e], py = J.py[e], pz = J.pz[e];
+          const double wm = E - pz, wp = E + pz;  // exact: differences of fp32 values
+          const double pt = sqrt(px * px + py * py);
+          S.y[c] = 0.5 * log(wp / wm);
+          S.phi[c] = atan2(py, px);
+          S.wm[c] = wm;
+          S.wp[c] = wp;
+          S.px[c] = px;
+          S.py[c] = py;
+          S.pt[c] = (float)pt;
+          S.lnpt[c] = (float)log(pt);
+        }
+      }
+      if (t == 0) {
+        S.m = total;
+        S.base = base;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// One jet with the whole block (thread = slot); same result as stage_jets.
+template <int PM, bool kKin = true>
 __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   long long base;
@@ -90,19 +162,21 @@ __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
   const int c = off + __popc(ballot & ((1u << lane) - 1u));
   if (tid < J.P) S.comp[tid] = valid ? (int16_t)c : (int16_t)-1;
   if (valid) {
-    const long long e = base + tid;
-    const double E = J.E[e], px = J.px[e], py = J.py[e], pz = J.pz[e];
-    const double wm = E - pz, wp = E + pz;  // exact: differences of fp32 values
-    const double pt = sqrt(px * px + py * py);
-    S.y[c] = 0.5 * log(wp / wm);
-    S.phi[c] = atan2(py, px);
-    S.wm[c] = wm;
-    S.wp[c] = wp;
-    S.px[c] = px;
-    S.py[c] = py;
-    S.pt[c] = (float)pt;
-    S.lnpt[c] = (float)log(pt);
     S.slot[c] = (int16_t)tid;
+    if (kKin) {
+      const long long e = base + tid;
+      const double E = J.E[e], px = J.px[e], py = J.py[e], pz = J.pz[e];
+      const double wm = E - pz, wp = E + pz;  // exact: differences of fp32 values
+      const double pt = sqrt(px * px + py * py);
+      S.y[c] = 0.5 * log(wp / wm);
+      S.phi[c] = atan2(py, px);
+      S.wm[c] = wm;
+      S.wp[c] = wp;
+      S.px[c] = px;
+      S.py[c] = py;
+      S.pt[c] = (float)pt;
+      S.lnpt[c] = (float)log(pt);
+    }
   }
   if (tid == 0) {
     S.m = total;
@@ -678,6 +752,48 @@ __device__ __forceinline__ void attention_chunk(const float* kv, int j0, int m, 
   mx = cmax;
 }
 
+// K and V of heads [h0, h0 + hr) of the staged jet n into kv as fp32
+// [hr][m][32] (16 of K, then 16 of V, per key). Block-wide, no barrier.
+template <int PM>
+__device__ __forceinline__ void stage_kv(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int h0,
+                                         int hr, float* kv) {
+  const int m = S.m;
+  for (int idx = threadIdx.x; idx < hr * m * 4; idx += blockDim.x) {
+    const int part = idx & 3, j = (idx >> 2) % m, hh = (idx >> 2) / m;
+    const uint16_t* src = (part < 2 ? X.k : X.v) + qkv_off<PM>(S, J, n, h0 + hh, j) + (part & 1) * 8;
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(src), f);
+    float4* dst = reinterpret_cast<float4*>(kv + (hh * m + j) * 32 + (part >> 1) * 16 + (part & 1) * 8);
+    dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+    dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+// One (query, head): online softmax over the m staged keys of kv (one head)
+// with the bias from cur, in the log2 domain; writes the bf16 output row.
+template <class Cursor>
+__device__ __forceinline__ void attend_row(const float* kv, int m, uint4 qraw0, uint4 qraw1, Cursor cur,
+                                           uint16_t* op) {
+  const float qscale = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
+  float q[16];
+  bf16x8_to_f32(qraw0, q);
+  bf16x8_to_f32(qraw1, q + 8);
+#pragma unroll
+  for (int d = 0; d < 16; ++d) q[d] *= qscale;
+  float o[16];
+#pragma unroll
+  for (int d = 0; d < 16; ++d) o[d] = 0.f;
+  float l = 0.f, mx = -INFINITY;
+  int j0 = 0;
+  for (; j0 + 8 <= m; j0 += 8) attention_chunk<false>(kv, j0, m, q, cur, o, l, mx);
+  if (j0 < m) attention_chunk<true>(kv, j0, m, q, cur, o, l, mx);
+  const float inv = 1.0f / l;
+#pragma unroll
+  for (int d = 0; d < 16; ++d) o[d] *= inv;
+  *reinterpret_cast<uint4*>(op) = f32x8_to_bf16(o);
+  *reinterpret_cast<uint4*>(op + 8) = f32x8_to_bf16(o + 8);
+}
+
 template <int PM, class UBias>
 __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int i_lo,
                                 int i_hi, float* stage, int stage_floats, const UBias& ubias, int h_lo = 0,
@@ -687,7 +803,6 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
   const int tid = threadIdx.x, nthr = blockDim.x;
   if (m <= 0 || nq <= 0) return;
   const int HR = min(kH, stage_floats / (32 * m));
-  const float qscale = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
   for (int h0 = h_lo; h0 < h_hi; h0 += HR) {
     const int hr = min(HR, h_hi - h0);
     // this thread's first query row is fetched before the staging barrier so
@@ -698,43 +813,16 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
       qraw0 = *reinterpret_cast<const uint4*>(qp);
       qraw1 = *reinterpret_cast<const uint4*>(qp + 8);
     }
-    for (int idx = tid; idx < hr * m * 4; idx += nthr) {
-      const int part = idx & 3, j = (idx >> 2) % m, hh = (idx >> 2) / m;
-      const uint16_t* src = (part < 2 ? X.k : X.v) + qkv_off<PM>(S, J, n, h0 + hh, j) + (part & 1) * 8;
-      float f[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(src), f);
-      float4* dst = reinterpret_cast<float4*>(stage + (hh * m + j) * 32 + (part >> 1) * 16 + (part & 1) * 8);
-      dst[0] = make_float4(f[0], f[1], f[2], f[3]);
-      dst[1] = make_float4(f[4], f[5], f[6], f[7]);
-    }
+    stage_kv<PM>(S, J, X, n, h0, hr, stage);
     __syncthreads();
     for (int item = tid; item < hr * nq; item += nthr) {
       const int hh = item / nq, i = i_lo + item % nq, h = h0 + hh;
-      float q[16];
       if (item != tid) {
         const uint16_t* qp = X.q + qkv_off<PM>(S, J, n, h, i);
         qraw0 = *reinterpret_cast<const uint4*>(qp);
         qraw1 = *reinterpret_cast<const uint4*>(qp + 8);
       }
-      bf16x8_to_f32(qraw0, q);
-      bf16x8_to_f32(qraw1, q + 8);
-#pragma unroll
-      for (int d = 0; d < 16; ++d) q[d] *= qscale;
-      float o[16];
-#pragma unroll
-      for (int d = 0; d < 16; ++d) o[d] = 0.f;
-      float l = 0.f, mx = -INFINITY;
-      const float* kv = stage + hh * m * 32;
-      auto cur = ubias.row(i, h);
-      int j0 = 0;
-      for (; j0 + 8 <= m; j0 += 8) attention_chunk<false>(kv, j0, m, q, cur, o, l, mx);
-      if (j0 < m) attention_chunk<true>(kv, j0, m, q, cur, o, l, mx);
-      const float inv = 1.0f / l;
-#pragma unroll
-      for (int d = 0; d < 16; ++d) o[d] *= inv;
-      uint16_t* op = X.out + qkv_off<PM>(S, J, n, h, i);
-      *reinterpret_cast<uint4*>(op) = f32x8_to_bf16(o);
-      *reinterpret_cast<uint4*>(op + 8) = f32x8_to_bf16(o + 8);
+      attend_row(stage + hh * m * 32, m, qraw0, qraw1, ubias.row(i, h), X.out + qkv_off<PM>(S, J, n, h, i));
     }
     __syncthreads();
   }
@@ -783,7 +871,7 @@ __global__ void __launch_bounds__(256) k_attn_bias(JetArgs J, QkvArgs X, const u
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AttnSmem<PM>& S = *reinterpret_cast<AttnSmem<PM>*>(smem_raw);
   for (int n = blockIdx.x; n < J.N; n += gridDim.x) {
-    stage_jet<PM>(S.part, J, n);
+    stage_jet<PM, false>(S.part, J, n);
     GlobalUBias<PM> ub{&S.part, U, n, J.P};
     attention_block<PM>(S.part, J, X, n, 0, S.part.m, S.stage, kAttnStageFloats, ub);
     zero_masked_rows<PM>(S.part, J, X.out, n);
@@ -933,7 +1021,19 @@ struct BatchInfo {  // the jets of one phase-A batch
   int tbeg[GridCfg<PM>::kBatch + 1];      // prefix of their tiles within the batch
   int t_lo[GridCfg<PM>::kBatch];          // first tile of each jet taken by this CTA
   int npairs[GridCfg<PM>::kBatch];
+  int jet[GridCfg<PM>::kBatch];
   long long rowbase[GridCfg<PM>::kBatch]; // record index of the jet's pair 0
+};
+
+template <int PM>
+struct AttnBatch {  // the jets of one phase-B round, attended together
+  int K;                                  // jets gathered (and staged)
+  int Kf;                                 // leading jets whose data fit in the stage together
+  int next;                               // first jet of the next round
+  int jet[GridCfg<PM>::kBatch];
+  int hl[GridCfg<PM>::kBatch], hh[GridCfg<PM>::kBatch];   // head range of each jet
+  int uoff[GridCfg<PM>::kBatch], kvoff[GridCfg<PM>::kBatch];  // stage offsets (floats)
+  int ib[GridCfg<PM>::kBatch + 1];        // prefix of (head, query) items
 };
 
 template <int PM>
@@ -942,6 +1042,7 @@ struct FusedGridSmem {
   Particles<PM> ring[GridCfg<PM>::kBatch];
   int T[kGridMaxJets + 1];                 // exclusive prefix of tiles per jet
   BatchInfo<PM> batch;
+  AttnBatch<PM> ab;
   int warp_sums[32];
   int flag;
 };
@@ -1015,18 +1116,40 @@ __device__ bool grid_barrier(unsigned long long* ctr, unsigned nblk, int* smem_f
   return *smem_flag != 0;
 }
 
-// Valid particles of jet n without staging them (phase 0).
-__device__ __forceinline__ int jet_count(const JetArgs& J, int n, int lane) {
+// Nonzero bytes of a 32-bit word.
+__device__ __forceinline__ int nonzero_bytes(uint32_t w) { return __popc(__vcmpne4(w, 0u)) >> 3; }
+
+// Phase 0: the valid particles of every jet into T[1..N], all threads in
+// parallel (bounds of a packed jet as stage_jets checks them; a padded mask
+// read 16 bytes at a time when its rows allow it).
+__device__ void jet_counts(const JetArgs& J, int* T) {
+  const int tid = threadIdx.x, nthr = blockDim.x, N = J.N;
   if (J.ptr) {
-    const long long lo = J.ptr[n], hi = J.ptr[n + 1];
-    return (lo < 0 || hi < lo || hi > J.tokens || hi - lo > J.P) ? 0 : (int)(hi - lo);
+#pragma unroll 4
+    for (int n = tid; n < N; n += nthr) {
+      const long long lo = J.ptr[n], hi = J.ptr[n + 1];
+      T[n + 1] = (lo < 0 || hi < lo || hi > J.tokens || hi - lo > J.P) ? 0 : (int)(hi - lo);
+    }
+    return;
   }
-  int c = 0;
-  for (int s0 = 0; s0 < J.P; s0 += 32) {
-    const int sl = s0 + lane;
-    c += __popc(__ballot_sync(0xffffffffu, sl < J.P && J.mask[(long long)n * J.P + sl] != 0));
+  for (int n = tid; n < N; n += nthr) T[n + 1] = 0;
+  __syncthreads();
+  if ((J.P & 15) == 0 && (reinterpret_cast<uintptr_t>(J.mask) & 15) == 0) {
+    const int cpj = J.P >> 4;  // 16-byte chunks per jet
+    const uint4* mk = reinterpret_cast<const uint4*>(J.mask);
+    const int nc = N * cpj;
+#pragma unroll 4
+    for (int c = tid; c < nc; c += nthr) {
+      const uint4 w = mk[c];
+      const int k = nonzero_bytes(w.x) + nonzero_bytes(w.y) + nonzero_bytes(w.z) + nonzero_bytes(w.w);
+      if (k) atomicAdd(&T[c / cpj + 1], k);
+    }
+  } else {
+    const int ne = N * J.P;
+#pragma unroll 4
+    for (int e = tid; e < ne; e += nthr)
+      if (J.mask[e]) atomicAdd(&T[e / J.P + 1], 1);
   }
-  return c;
 }
 
 template <int PM>
@@ -1037,17 +1160,19 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
   unsigned long long* bar_ctr = reinterpret_cast<unsigned long long*>(ws);
   unsigned long long* exit_ctr = bar_ctr + 1;
   uint4* rec = reinterpret_cast<uint4*>(ws + kWsHeader);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, b = blockIdx.x;
   const int N = J.N;
 
   // ---------------------------------------------------------------- phase 0
-  // tiles per jet into T[n + 1] (one warp per jet), then an exclusive scan
-  for (int n = warp; n < N; n += nwarp) {
-    const int m = jet_count(J, n, lane);
-    if (lane == 0) S.T[n + 1] = (m * (m + 1) / 2 + kTileM - 1) / kTileM;
-  }
+  // multiplicities into T[n + 1], tiles per jet, then an exclusive scan
+  jet_counts(J, S.T);
   if (tid == 0) S.T[0] = 0;
+  __syncthreads();
+  for (int n = tid; n < N; n += blockDim.x) {
+    const int m = S.T[n + 1];
+    S.T[n + 1] = (m * (m + 1) / 2 + kTileM - 1) / kTileM;
+  }
   __syncthreads();
   {
     // each thread scans a contiguous chunk, warps then the block combine
@@ -1103,7 +1228,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
             S.batch.tbeg[K] = acc;
             S.batch.t_lo[K] = (int)(a0 - S.T[nn]);
             S.batch.rowbase[K] = (long long)S.T[nn] * kTileM;
-            S.batch.npairs[K] = nn;  // jet index for now; replaced after staging
+            S.batch.jet[K] = nn;
             acc += (int)(a1 - a0);
             ++K;
           }
@@ -1116,7 +1241,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
       __syncthreads();
       const int K = S.batch.K;
       const int n_next = S.flag;
-      for (int k = 0; k < K; ++k) stage_jet<PM>(S.ring[k], J, S.batch.npairs[k]);
+      stage_jets<PM, true>(S.ring, J, K, [&S](int k) { return S.batch.jet[k]; });
       if (tid == 0)
         for (int k = 0; k < K; ++k) S.batch.npairs[k] = S.ring[k].m * (S.ring[k].m + 1) / 2;
       __syncthreads();
@@ -1147,21 +1272,88 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
     }
     float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
     constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
-    for (; n < N && 8ll * ((long long)S.T[n] + n) < hi; ++n) {
-      const long long base = 8ll * ((long long)S.T[n] + n);
-      const long long c = (long long)(S.T[n + 1] - S.T[n]) + 1;
-      int h_lo = 0, h_hi = 0;
-      for (int h = 0; h < kH; ++h) {
-        const long long st = base + h * c;
-        if (st < lo) h_lo = h + 1;
-        if (st < hi) h_hi = h + 1;
+    AttnBatch<PM>& A = S.ab;
+    while (n < N && 8ll * ((long long)S.T[n] + n) < hi) {
+      // up to JB jets with heads in [lo, hi), staged (slots only) together
+      if (tid == 0) {
+        int K = 0, nn = n;
+        while (K < JB && nn < N && 8ll * ((long long)S.T[nn] + nn) < hi) {
+          const long long base = 8ll * ((long long)S.T[nn] + nn);
+          const long long c = (long long)(S.T[nn + 1] - S.T[nn]) + 1;
+          int h_lo = 0, h_hi = 0;
+          for (int h = 0; h < kH; ++h) {
+            const long long st = base + h * c;
+            if (st < lo) h_lo = h + 1;
+            if (st < hi) h_hi = h + 1;
+          }
+          if (h_lo < h_hi) {
+            A.jet[K] = nn;
+            A.hl[K] = h_lo;
+            A.hh[K] = h_hi;
+            ++K;
+          }
+          ++nn;
+        }
+        A.K = K;
+        A.next = nn;
       }
-      if (h_lo >= h_hi) continue;
-      stage_jet<PM>(S.ring[0], J, n);
-      RecordUBias ub{reinterpret_cast<const __half*>(rec + (size_t)S.T[n] * kTileM)};
-      attention_block<PM>(S.ring[0], J, X, n, 0, S.ring[0].m, stage, kStageFloats, ub, h_lo, h_hi);
-      if (h_lo == 0) zero_masked_rows<PM>(S.ring[0], J, X.out, n);
       __syncthreads();
+      const int K = A.K;
+      stage_jets<PM, false>(S.ring, J, K, [&A](int k) { return A.jet[k]; });
+      // the leading jets whose records and K/V fit in the stage together
+      if (tid == 0) {
+        int used = 0, items = 0, Kf = 0;
+        for (; Kf < K; ++Kf) {
+          const int m = S.ring[Kf].m, hr = A.hh[Kf] - A.hl[Kf];
+          const int need = m * (m + 1) / 2 * 4 + hr * m * 32;
+          if (used + need > kStageFloats) break;
+          A.uoff[Kf] = used;
+          A.kvoff[Kf] = used + m * (m + 1) / 2 * 4;
+          A.ib[Kf] = items;
+          used += need;
+          items += hr * m;
+        }
+        A.ib[Kf] = items;
+        A.Kf = Kf;
+        // jets that did not fit are staged again in the next round
+        if (Kf > 0 && Kf < K) A.next = A.jet[Kf];
+        else if (Kf == 0 && K > 1) A.next = A.jet[1];
+      }
+      __syncthreads();
+      const int Kf = A.Kf, n_next = A.next;
+      if (K == 0) {
+        // [lo, hi) lies inside one jet's head: nothing to do in this round
+      } else if (Kf == 0) {
+        // one jet too wide for the stage: its bias is read from the records
+        const int nj = A.jet[0];
+        RecordUBias ub{reinterpret_cast<const __half*>(rec + (size_t)S.T[nj] * kTileM)};
+        attention_block<PM>(S.ring[0], J, X, nj, 0, S.ring[0].m, stage, kStageFloats, ub, A.hl[0], A.hh[0]);
+        if (A.hl[0] == 0) zero_masked_rows<PM>(S.ring[0], J, X.out, nj);
+      } else {
+        for (int k = 0; k < Kf; ++k) {
+          const int nj = A.jet[k], m = S.ring[k].m, np = m * (m + 1) / 2;
+          const uint4* jrec = rec + (size_t)S.T[nj] * kTileM;
+          uint4* U8 = reinterpret_cast<uint4*>(stage + A.uoff[k]);
+          for (int r = tid; r < np; r += blockDim.x) U8[r] = __ldcg(jrec + r);
+          stage_kv<PM>(S.ring[k], J, X, nj, A.hl[k], A.hh[k] - A.hl[k], stage + A.kvoff[k]);
+        }
+        __syncthreads();
+        for (int item = tid; item < A.ib[Kf]; item += blockDim.x) {
+          int k = 0;
+#pragma unroll
+          for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= item) ? 1 : 0;
+          const Particles<PM>& P = S.ring[k];
+          const int m = P.m, loc = item - A.ib[k], hh = loc / m, i = loc % m, h = A.hl[k] + hh, nj = A.jet[k];
+          const uint16_t* qp = X.q + qkv_off<PM>(P, J, nj, h, i);
+          const uint4 q0 = *reinterpret_cast<const uint4*>(qp), q1 = *reinterpret_cast<const uint4*>(qp + 8);
+          TriUBias ub{reinterpret_cast<const __half*>(stage + A.uoff[k])};
+          attend_row(stage + A.kvoff[k] + hh * m * 32, m, q0, q1, ub.row(i, h), X.out + qkv_off<PM>(P, J, nj, h, i));
+        }
+        for (int k = 0; k < Kf; ++k)
+          if (A.hl[k] == 0) zero_masked_rows<PM>(S.ring[k], J, X.out, A.jet[k]);
+      }
+      __syncthreads();
+      n = n_next;
     }
   }
 
