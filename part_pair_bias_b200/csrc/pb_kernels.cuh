@@ -698,131 +698,263 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float* f) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Masked multi-head attention for queries [i_lo, i_hi) of the staged jet,
-// all valid keys, on CUDA cores: one thread per (query, head), keys streamed
-// from shared memory in chunks of 8 with an online (running-max) softmax in
-// the log2 domain, for heads [h_lo, h_hi). `ubias.row(i, h)` returns a cursor
-// whose next() yields U[h, i, 0], U[h, i, 1], ... in key order.
-// `stage` holds K and V of up to `stage_floats / (32 m)` heads at a time as fp32.
-// Full chunks run without predicates; only the last, partial chunk checks j < m.
-template <bool kTail, class Cursor>
-__device__ __forceinline__ void attention_chunk(const float* kv, int j0, int m, const float* q, Cursor& cur,
-                                                float* o, float& l, float& mx) {
-  float s[8];
-  float cmax = mx;
-#pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    s[jj] = -INFINITY;
-    if (!kTail || j0 + jj < m) {
-      const float4* kr = reinterpret_cast<const float4*>(kv + (j0 + jj) * 32);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four short chains instead of one of 16
-#pragma unroll
-      for (int d4 = 0; d4 < 4; ++d4) {
-        const float4 k4 = kr[d4];
-        acc[d4] = fmaf(q[4 * d4], k4.x, acc[d4]);
-        acc[d4] = fmaf(q[4 * d4 + 1], k4.y, acc[d4]);
-        acc[d4] = fmaf(q[4 * d4 + 2], k4.z, acc[d4]);
-        acc[d4] = fmaf(q[4 * d4 + 3], k4.w, acc[d4]);
-      }
-      s[jj] = fmaf(cur.next(), kLog2e, (acc[0] + acc[1]) + (acc[2] + acc[3]));
-      cmax = fmaxf(cmax, s[jj]);
-    }
-  }
-  // every chunk holds at least one valid key, so cmax is finite
-  const float corr = ex2(mx - cmax);
-  l *= corr;
-#pragma unroll
-  for (int d = 0; d < 16; ++d) o[d] *= corr;
-#pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    if (!kTail || j0 + jj < m) {
-      const float pj = ex2(s[jj] - cmax);
-      l += pj;
-      const float4* vr = reinterpret_cast<const float4*>(kv + (j0 + jj) * 32 + 16);
-#pragma unroll
-      for (int d4 = 0; d4 < 4; ++d4) {
-        const float4 v4 = vr[d4];
-        o[4 * d4] = fmaf(pj, v4.x, o[4 * d4]);
-        o[4 * d4 + 1] = fmaf(pj, v4.y, o[4 * d4 + 1]);
-        o[4 * d4 + 2] = fmaf(pj, v4.z, o[4 * d4 + 2]);
-        o[4 * d4 + 3] = fmaf(pj, v4.w, o[4 * d4 + 3]);
-      }
-    }
-  }
-  mx = cmax;
+// ---------------------------------------------------- attention on tensor cores
+//
+// Per (jet, head): S = Q K^T on m16n8k16 tensor-core tiles (bf16 operands,
+// fp32 accumulation) held in registers, the bias and the key mask added to S
+// there, an online softmax over blocks of 16 keys in the log2 domain, then
+// O += P V with P rounded to bf16 (P in [0, 1]: relative rounding 2^-9).
+// One warp owns 16 queries of one head. K and V of a head are staged in
+// shared memory as bf16, zero beyond m: K row-major [m16][kKStride] and V
+// transposed [16][m16 + 8]; both strides make the fragment loads of a warp
+// hit 32 distinct banks.
+
+constexpr int kKStride = 24;  // halves per staged K row (48 bytes)
+
+__host__ __device__ constexpr int round16(int m) { return (m + 15) & ~15; }
+
+// Bytes of the staged K and V of one head for m keys (a multiple of 16).
+__host__ __device__ constexpr int kv16_bytes(int m) {
+  return round16(m) * kKStride * 2 + 16 * (round16(m) + 8) * 2;
 }
 
-// K and V of heads [h0, h0 + hr) of the staged jet n into kv as fp32
-// [hr][m][32] (16 of K, then 16 of V, per key). Block-wide, no barrier.
+// K and V of heads [h0, h0 + hr) of the staged jet n into buf, one head
+// after another (kv16_bytes(m) each). Block-wide, no barrier.
 template <int PM>
-__device__ __forceinline__ void stage_kv(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int h0,
-                                         int hr, float* kv) {
-  const int m = S.m;
-  for (int idx = threadIdx.x; idx < hr * m * 4; idx += blockDim.x) {
-    const int part = idx & 3, j = (idx >> 2) % m, hh = (idx >> 2) / m;
-    const uint16_t* src = (part < 2 ? X.k : X.v) + qkv_off<PM>(S, J, n, h0 + hh, j) + (part & 1) * 8;
-    float f[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(src), f);
-    float4* dst = reinterpret_cast<float4*>(kv + (hh * m + j) * 32 + (part >> 1) * 16 + (part & 1) * 8);
-    dst[0] = make_float4(f[0], f[1], f[2], f[3]);
-    dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+__device__ void stage_kv16(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int h0, int hr,
+                           uint16_t* buf) {
+  const int m = S.m, m16 = round16(m), vts = m16 + 8, hb = kv16_bytes(m) / 2;
+  const int total = hr * m16 * 4, nthr = blockDim.x;
+  // four independent loads in flight per thread before any store
+  for (int base = threadIdx.x; base < total; base += 4 * nthr) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      const int part = idx & 3, j = (idx >> 2) % m16, hh = (idx >> 2) / m16;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (idx < total && j < m)
+        v[u] = *reinterpret_cast<const uint4*>((part < 2 ? X.k : X.v) + qkv_off<PM>(S, J, n, h0 + hh, j) +
+                                               (part & 1) * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      if (idx >= total) break;
+      const int part = idx & 3, j = (idx >> 2) % m16, hh = (idx >> 2) / m16;
+      uint16_t* kh = buf + hh * hb;
+      if (part < 2) {
+        *reinterpret_cast<uint4*>(kh + j * kKStride + (part & 1) * 8) = v[u];
+      } else {
+        uint16_t* vt = kh + m16 * kKStride + ((part & 1) * 8) * vts + j;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          vt[(2 * e) * vts] = (uint16_t)(w[e] & 0xffffu);
+          vt[(2 * e + 1) * vts] = (uint16_t)(w[e] >> 16);
+        }
+      }
+    }
   }
 }
 
-// One (query, head): online softmax over the m staged keys of kv (one head)
-// with the bias from cur, in the log2 domain; writes the bf16 output row.
-template <class Cursor>
-__device__ __forceinline__ void attend_row(const float* kv, int m, uint4 qraw0, uint4 qraw1, Cursor cur,
-                                           uint16_t* op) {
-  const float qscale = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
-  float q[16];
-  bf16x8_to_f32(qraw0, q);
-  bf16x8_to_f32(qraw1, q + 8);
-#pragma unroll
-  for (int d = 0; d < 16; ++d) q[d] *= qscale;
-  float o[16];
-#pragma unroll
-  for (int d = 0; d < 16; ++d) o[d] = 0.f;
-  float l = 0.f, mx = -INFINITY;
-  int j0 = 0;
-  for (; j0 + 8 <= m; j0 += 8) attention_chunk<false>(kv, j0, m, q, cur, o, l, mx);
-  if (j0 < m) attention_chunk<true>(kv, j0, m, q, cur, o, l, mx);
-  const float inv = 1.0f / l;
-#pragma unroll
-  for (int d = 0; d < 16; ++d) o[d] *= inv;
-  *reinterpret_cast<uint4*>(op) = f32x8_to_bf16(o);
-  *reinterpret_cast<uint4*>(op + 8) = f32x8_to_bf16(o + 8);
+__device__ __forceinline__ uint32_t lds_u32(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+// D += A B on one m16n8k16 tile: A 16x16 bf16 (row), B 16x8 bf16 (col), D fp32.
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Bias blocks: the 8 values of U[h, ., .] a lane needs for one key block
+// (see attend_tile16), from the storage layouts the kernels use.
+
+// Triangle of 8-half records, pair (a, b) with a >= b at record a(a+1)/2 + b;
+// U points at head h of record 0. Query tiles and key blocks are aligned to
+// 16, so a full key block lies wholly below the tile's rows (records
+// i(i+1)/2 + j, contiguous in j), wholly above them (records j(j+1)/2 + i),
+// or on the diagonal, which takes the general formula.
+struct TriBlock {
+  const __half* U;
+  __device__ __forceinline__ void operator()(int n0, int i0, int ia, int ib, int t, int m, float* u) const {
+    const int jb = n0 + 2 * t;
+    if (n0 + 16 <= m && n0 + 16 <= i0) {
+      const __half* ra = U + (ia * (ia + 1) / 2 + jb) * 8;
+      const __half* rb = U + (ib * (ib + 1) / 2 + jb) * 8;
+      u[0] = __half2float(ra[0]);
+      u[1] = __half2float(ra[8]);
+      u[4] = __half2float(ra[64]);
+      u[5] = __half2float(ra[72]);
+      u[2] = __half2float(rb[0]);
+      u[3] = __half2float(rb[8]);
+      u[6] = __half2float(rb[64]);
+      u[7] = __half2float(rb[72]);
+    } else if (n0 + 16 <= m && n0 >= i0 + 16) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = jb + (c & 1) + (c & 2) * 4, e = (c & 2) * 2 + (c & 1);
+        const __half* cj = U + (j * (j + 1) / 2) * 8;
+        u[e] = __half2float(cj[ia * 8]);
+        u[e + 2] = __half2float(cj[ib * 8]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int i = e & 2 ? ib : ia, j = min(m - 1, jb + (e & 4 ? 8 : 0) + (e & 1));
+        const int hi = max(i, j), lo = min(i, j);
+        u[e] = __half2float(U[(hi * (hi + 1) / 2 + lo) * 8]);
+      }
+    }
+  }
+};
+
+// Rectangle of 8-half records, (query i, key j) at record (i - r0) * m + j;
+// U points at head h of record 0.
+struct RectBlock {
+  const __half* U;
+  int r0, m;
+  __device__ __forceinline__ void operator()(int n0, int, int ia, int ib, int t, int, float* u) const {
+    const int jb = n0 + 2 * t;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = e & 2 ? ib : ia, j = min(m - 1, jb + (e & 4 ? 8 : 0) + (e & 1));
+      u[e] = __half2float(U[((i - r0) * m + j) * 8]);
+    }
+  }
+};
+
+// A fragment of the 16 queries [i0, i0 + nrows) (zero rows past nrows);
+// qrow(i) gives the bf16 row of query i. Warp-wide.
+template <class QRow>
+__device__ __forceinline__ void q_frag(int i0, int nrows, const QRow& qrow, uint32_t* a) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  a[0] = a[1] = a[2] = a[3] = 0u;
+  if (g < nrows) {
+    const uint16_t* q = qrow(i0 + g);
+    a[0] = *reinterpret_cast<const uint32_t*>(q + 2 * t);
+    a[2] = *reinterpret_cast<const uint32_t*>(q + 2 * t + 8);
+  }
+  if (g + 8 < nrows) {
+    const uint16_t* q = qrow(i0 + g + 8);
+    a[1] = *reinterpret_cast<const uint32_t*>(q + 2 * t);
+    a[3] = *reinterpret_cast<const uint32_t*>(q + 2 * t + 8);
+  }
+}
+
+// Queries [i0, i0 + nrows) (nrows <= 16, A fragment a from q_frag) of one
+// head against its m staged keys: kh = staged K, vth = staged V^T of that
+// head. orow(i) gives the bf16 output row of query i; ub(n0, i0, ia, ib, t,
+// m, u) fills the bias of the 8 score elements a lane holds for the key
+// block n0 (element e: row e & 2 ? ib : ia, key n0 + 8 (e >> 2) + 2 t +
+// (e & 1), keys past m clamped to m - 1). Warp-wide.
+template <class ORow, class UBlock>
+__device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t* vth, int m, int i0, int nrows,
+                                              const uint32_t* a, const ORow& orow, const UBlock& ub) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int vts = round16(m) + 8;
+  const bool va = g < nrows, vb = g + 8 < nrows;
+  const int ia = i0 + (va ? g : 0), ib = i0 + (vb ? g + 8 : 0);  // rows past the block alias row i0
+  const float qs = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
+  float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float mxa = -INFINITY, mxb = -INFINITY, la = 0.f, lb = 0.f;
+  for (int n0 = 0; n0 < m; n0 += 16) {
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint16_t* k0 = kh + (n0 + g) * kKStride + 2 * t;
+    mma_16816(s, a, lds_u32(k0), lds_u32(k0 + 8));
+    mma_16816(s + 4, a, lds_u32(k0 + 8 * kKStride), lds_u32(k0 + 8 * kKStride + 8));
+    float u[8];
+    ub(n0, i0, ia, ib, t, m, u);
+    if (n0 + 16 <= m) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[e] = fmaf(s[e], qs, u[e] * kLog2e);
+    } else {  // the last, partial block: keys past m are masked
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = n0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1);
+        s[e] = j < m ? fmaf(s[e], qs, u[e] * kLog2e) : -INFINITY;
+      }
+    }
+    float bma = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[4], s[5]));
+    float bmb = fmaxf(fmaxf(s[2], s[3]), fmaxf(s[6], s[7]));
+    bma = fmaxf(bma, __shfl_xor_sync(0xffffffffu, bma, 1));
+    bma = fmaxf(bma, __shfl_xor_sync(0xffffffffu, bma, 2));
+    bmb = fmaxf(bmb, __shfl_xor_sync(0xffffffffu, bmb, 1));
+    bmb = fmaxf(bmb, __shfl_xor_sync(0xffffffffu, bmb, 2));
+    // key n0 < m is valid for every row, so the new maxima are finite
+    const float nma = fmaxf(mxa, bma), nmb = fmaxf(mxb, bmb);
+    const float ca = ex2(mxa - nma), cb = ex2(mxb - nmb);
+    mxa = nma;
+    mxb = nmb;
+    float p[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) p[e] = ex2(s[e] - (e & 2 ? nmb : nma));
+    la = la * ca + ((p[0] + p[1]) + (p[4] + p[5]));
+    lb = lb * cb + ((p[2] + p[3]) + (p[6] + p[7]));
+    o[0] *= ca; o[1] *= ca; o[4] *= ca; o[5] *= ca;
+    o[2] *= cb; o[3] *= cb; o[6] *= cb; o[7] *= cb;
+    const uint32_t pa[4] = {cvt_bf16x2(p[0], p[1]), cvt_bf16x2(p[2], p[3]), cvt_bf16x2(p[4], p[5]),
+                            cvt_bf16x2(p[6], p[7])};
+    const uint16_t* v0 = vth + g * vts + n0 + 2 * t;  // V^T rows = dims g and 8 + g
+    mma_16816(o, pa, lds_u32(v0), lds_u32(v0 + 8));
+    mma_16816(o + 4, pa, lds_u32(v0 + 8 * vts), lds_u32(v0 + 8 * vts + 8));
+  }
+  la += __shfl_xor_sync(0xffffffffu, la, 1);
+  la += __shfl_xor_sync(0xffffffffu, la, 2);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+  if (va) {
+    const float r = 1.0f / la;
+    uint16_t* op = orow(ia);
+    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(o[0] * r, o[1] * r);
+    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(o[4] * r, o[5] * r);
+  }
+  if (vb) {
+    const float r = 1.0f / lb;
+    uint16_t* op = orow(ib);
+    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(o[2] * r, o[3] * r);
+    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(o[6] * r, o[7] * r);
+  }
+}
+
+// Masked multi-head attention for queries [i_lo, i_hi) of the staged jet
+// against all its valid keys, heads [h_lo, h_hi), on tensor cores: K and V of
+// as many heads as `stage` holds are staged at a time, then the warps take
+// (head, 16-query tile) items. ubias.head(h) gives the bias blocks of head h.
 template <int PM, class UBias>
 __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int i_lo,
                                 int i_hi, float* stage, int stage_floats, const UBias& ubias, int h_lo = 0,
                                 int h_hi = kH) {
   const int m = S.m;
   const int nq = i_hi - i_lo;
-  const int tid = threadIdx.x, nthr = blockDim.x;
   if (m <= 0 || nq <= 0) return;
-  const int HR = min(kH, stage_floats / (32 * m));
+  const int hb = kv16_bytes(m);
+  const int HR = max(1, min(kH, stage_floats * 4 / hb));
+  const int tiles = (nq + 15) >> 4;
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  uint16_t* buf = reinterpret_cast<uint16_t*>(stage);
   for (int h0 = h_lo; h0 < h_hi; h0 += HR) {
     const int hr = min(HR, h_hi - h0);
-    // this thread's first query row is fetched before the staging barrier so
-    // that its memory latency overlaps the K/V staging
-    uint4 qraw0 = make_uint4(0, 0, 0, 0), qraw1 = qraw0;
-    if (tid < hr * nq) {
-      const uint16_t* qp = X.q + qkv_off<PM>(S, J, n, h0 + tid / nq, i_lo + tid % nq);
-      qraw0 = *reinterpret_cast<const uint4*>(qp);
-      qraw1 = *reinterpret_cast<const uint4*>(qp + 8);
-    }
-    stage_kv<PM>(S, J, X, n, h0, hr, stage);
+    // the Q fragment of a warp's next item is loaded ahead: the first one
+    // before the staging barrier, the others while the previous item runs
+    uint32_t a[4] = {0u, 0u, 0u, 0u};
+    auto qload = [&](int it, uint32_t* f) {
+      const int h = h0 + it / tiles, i0 = i_lo + (it % tiles) * 16;
+      q_frag(i0, min(16, i_hi - i0), [&](int i) { return X.q + qkv_off<PM>(S, J, n, h, i); }, f);
+    };
+    if (warp < hr * tiles) qload(warp, a);
+    stage_kv16<PM>(S, J, X, n, h0, hr, buf);
     __syncthreads();
-    for (int item = tid; item < hr * nq; item += nthr) {
-      const int hh = item / nq, i = i_lo + item % nq, h = h0 + hh;
-      if (item != tid) {
-        const uint16_t* qp = X.q + qkv_off<PM>(S, J, n, h, i);
-        qraw0 = *reinterpret_cast<const uint4*>(qp);
-        qraw1 = *reinterpret_cast<const uint4*>(qp + 8);
-      }
-      attend_row(stage + hh * m * 32, m, qraw0, qraw1, ubias.row(i, h), X.out + qkv_off<PM>(S, J, n, h, i));
+    for (int it = warp; it < hr * tiles; it += nwarp) {
+      uint32_t an[4] = {0u, 0u, 0u, 0u};
+      if (it + nwarp < hr * tiles) qload(it + nwarp, an);
+      const int hh = it / tiles, i0 = i_lo + (it % tiles) * 16, h = h0 + hh;
+      const uint16_t* kh = buf + hh * (hb / 2);
+      attend_tile16(
+          kh, kh + round16(m) * kKStride, m, i0, min(16, i_hi - i0), a,
+          [&](int i) { return X.out + qkv_off<PM>(S, J, n, h, i); }, ubias.head(h));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] = an[e];
     }
     __syncthreads();
   }
@@ -843,19 +975,24 @@ __device__ void zero_masked_rows(const Particles<PM>& S, const JetArgs& J, uint1
 // ------------------------------------------- k_attn_bias (bias read from HBM)
 
 template <int PM>
-struct GlobalUBias {
+struct GlobalUBias {  // U[n, h, slot i, slot j] of a bf16 [N, 8, P, P] tensor
   const Particles<PM>* S;
   const uint16_t* U;
   int n, P;
-  struct Cursor {  // keys in compact order, read at their slots of row slot[i]
-    const uint16_t* row;
+  struct Block {
     const int16_t* slot;
-    int j;
-    __device__ __forceinline__ float next() { return bf16_to_f32(row[slot[j++]]); }
+    const uint16_t* Uh;  // U[n, h]
+    int P;
+    __device__ __forceinline__ void operator()(int n0, int, int ia, int ib, int t, int m, float* u) const {
+      const size_t ra = (size_t)slot[ia] * P, rb = (size_t)slot[ib] * P;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = min(m - 1, n0 + 2 * t + (e & 4 ? 8 : 0) + (e & 1));
+        u[e] = bf16_to_f32(Uh[(e & 2 ? rb : ra) + slot[j]]);
+      }
+    }
   };
-  __device__ __forceinline__ Cursor row(int i, int h) const {
-    return Cursor{U + (((size_t)n * kH + h) * P + S->slot[i]) * P, S->slot, 0};
-  }
+  __device__ __forceinline__ Block head(int h) const { return Block{S->slot, U + ((size_t)n * kH + h) * P * P, P}; }
 };
 
 constexpr int kAttnStageFloats = 16384;  // 64 KB of K/V staging
@@ -909,37 +1046,15 @@ struct SmemUSink {
   }
 };
 
-// Row i of a triangle of 8-half records, pair (a, b) with a >= b at record
-// a (a + 1) / 2 + b: walking the keys j = 0, 1, ..., the record of key j + 1
-// follows that of key j by 1 record while j < i and by j + 1 records after.
-struct TriCursor {
-  const __half* p;
-  int i, j;
-  __device__ __forceinline__ float next() {
-    const float u = __half2float(*p);
-    p += (j < i ? 1 : j + 1) * 8;
-    ++j;
-    return u;
-  }
-};
-
-struct TriUBias {  // U of pair (i, j) at record max(i,j)(max(i,j)+1)/2 + min(i,j)
+struct TriUBias {  // U of pair (i, j) at record max(i,j)(max(i,j)+1)/2 + min(i,j), 8 halves per record
   const __half* U;
-  __device__ __forceinline__ TriCursor row(int i, int h) const { return TriCursor{U + (i * (i + 1) / 2) * 8 + h, i, 0}; }
+  __device__ __forceinline__ TriBlock head(int h) const { return TriBlock{U + h}; }
 };
 
 struct RectUBias {  // U of (query i, key j) at record (i - i0) * m + j
   const __half* U;
   int i0, m;
-  struct Cursor {
-    const __half* p;
-    __device__ __forceinline__ float next() {
-      const float u = __half2float(*p);
-      p += 8;
-      return u;
-    }
-  };
-  __device__ __forceinline__ Cursor row(int i, int h) const { return Cursor{U + ((i - i0) * m) * 8 + h}; }
+  __device__ __forceinline__ RectBlock head(int h) const { return RectBlock{U + h, i0, m}; }
 };
 
 template <int PM, int NG>
@@ -1074,11 +1189,9 @@ struct RecordSink {  // the 8 biases of a pair as 8 f16 in one 16-byte record
   }
 };
 
-struct RecordUBias {  // U[h, i, j] from the jet's records (unordered-pair index)
+struct RecordUBias {  // U[h, i, j] from the jet's records in global memory (unordered-pair index)
   const __half* rec;   // record 0 of the jet, as halves
-  __device__ __forceinline__ TriCursor row(int i, int h) const {
-    return TriCursor{rec + (size_t)(i * (i + 1) / 2) * 8 + h, i, 0};
-  }
+  __device__ __forceinline__ TriBlock head(int h) const { return TriBlock{rec + h}; }
 };
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
@@ -1305,13 +1418,13 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
         int used = 0, items = 0, Kf = 0;
         for (; Kf < K; ++Kf) {
           const int m = S.ring[Kf].m, hr = A.hh[Kf] - A.hl[Kf];
-          const int need = m * (m + 1) / 2 * 4 + hr * m * 32;
+          const int need = m * (m + 1) / 2 * 4 + hr * (kv16_bytes(m) / 4);
           if (used + need > kStageFloats) break;
           A.uoff[Kf] = used;
           A.kvoff[Kf] = used + m * (m + 1) / 2 * 4;
           A.ib[Kf] = items;
           used += need;
-          items += hr * m;
+          items += hr * ((m + 15) >> 4);
         }
         A.ib[Kf] = items;
         A.Kf = Kf;
@@ -1330,24 +1443,53 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
         attention_block<PM>(S.ring[0], J, X, nj, 0, S.ring[0].m, stage, kStageFloats, ub, A.hl[0], A.hh[0]);
         if (A.hl[0] == 0) zero_masked_rows<PM>(S.ring[0], J, X.out, nj);
       } else {
+        // warp items: (jet, head, 16-query tile); Q fragments are loaded ahead
+        const int items = A.ib[Kf], nwarp = (int)(blockDim.x >> 5);
+        auto qload = [&](int it, uint32_t* f) {
+          int k = 0;
+#pragma unroll
+          for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= it) ? 1 : 0;
+          const Particles<PM>& P = S.ring[k];
+          const int m = P.m, tiles = (m + 15) >> 4, loc = it - A.ib[k];
+          const int h = A.hl[k] + loc / tiles, i0 = (loc % tiles) * 16, nj = A.jet[k];
+          q_frag(i0, min(16, m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, nj, h, i); }, f);
+        };
+        uint32_t a[4] = {0u, 0u, 0u, 0u};
+        if (warp < items) qload(warp, a);
         for (int k = 0; k < Kf; ++k) {
           const int nj = A.jet[k], m = S.ring[k].m, np = m * (m + 1) / 2;
           const uint4* jrec = rec + (size_t)S.T[nj] * kTileM;
           uint4* U8 = reinterpret_cast<uint4*>(stage + A.uoff[k]);
-          for (int r = tid; r < np; r += blockDim.x) U8[r] = __ldcg(jrec + r);
-          stage_kv<PM>(S.ring[k], J, X, nj, A.hl[k], A.hh[k] - A.hl[k], stage + A.kvoff[k]);
+          for (int r0 = tid; r0 < np; r0 += 4 * (int)blockDim.x) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int r = r0 + u * (int)blockDim.x;
+              v[u] = r < np ? __ldcg(jrec + r) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (r0 + u * (int)blockDim.x < np) U8[r0 + u * (int)blockDim.x] = v[u];
+          }
+          stage_kv16<PM>(S.ring[k], J, X, nj, A.hl[k], A.hh[k] - A.hl[k], reinterpret_cast<uint16_t*>(stage + A.kvoff[k]));
         }
         __syncthreads();
-        for (int item = tid; item < A.ib[Kf]; item += blockDim.x) {
+        for (int it = warp; it < items; it += nwarp) {
+          uint32_t an[4] = {0u, 0u, 0u, 0u};
+          if (it + nwarp < items) qload(it + nwarp, an);
           int k = 0;
 #pragma unroll
-          for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= item) ? 1 : 0;
+          for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= it) ? 1 : 0;
           const Particles<PM>& P = S.ring[k];
-          const int m = P.m, loc = item - A.ib[k], hh = loc / m, i = loc % m, h = A.hl[k] + hh, nj = A.jet[k];
-          const uint16_t* qp = X.q + qkv_off<PM>(P, J, nj, h, i);
-          const uint4 q0 = *reinterpret_cast<const uint4*>(qp), q1 = *reinterpret_cast<const uint4*>(qp + 8);
-          TriUBias ub{reinterpret_cast<const __half*>(stage + A.uoff[k])};
-          attend_row(stage + A.kvoff[k] + hh * m * 32, m, q0, q1, ub.row(i, h), X.out + qkv_off<PM>(P, J, nj, h, i));
+          const int m = P.m, tiles = (m + 15) >> 4, loc = it - A.ib[k];
+          const int hh = loc / tiles, i0 = (loc % tiles) * 16, h = A.hl[k] + hh, nj = A.jet[k];
+          const uint16_t* kh = reinterpret_cast<const uint16_t*>(stage + A.kvoff[k]) + hh * (kv16_bytes(m) / 2);
+          const TriBlock ub{reinterpret_cast<const __half*>(stage + A.uoff[k]) + h};
+          attend_tile16(
+              kh, kh + round16(m) * kKStride, m, i0, min(16, m - i0), a,
+              [&](int i) { return X.out + qkv_off<PM>(P, J, nj, h, i); }, ub);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) a[e] = an[e];
         }
         for (int k = 0; k < Kf; ++k)
           if (A.hl[k] == 0) zero_masked_rows<PM>(S.ring[k], J, X.out, A.jet[k]);
