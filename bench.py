@@ -32,7 +32,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from part_pair_bias_b200 import configs, synth  # noqa: E402
+from part_pair_bias_b200 import configs, shard, synth  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
 MLP_FLOP_PER_PAIR = 2 * (4 * 64 + 64 * 64 + 64 * 64 + 64 * 8)          # 17,920 (algorithmic)
@@ -183,7 +183,7 @@ def run_ours(args, world, rank, local):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wl = args.workload
-    b = synth.make_jets(**configs.workload(wl, seed=args.seed + rank))
+    b = synth.make_jets(**configs.workload(wl, seed=shard.rank_seed(args.seed, rank)))
     unordered, tiles, ordered = pair_counts(b)
     mlp = ops.folded_mlp(b.params, dev)
 
@@ -268,19 +268,16 @@ def run_ours(args, world, rank, local):
     e2e_ms = es.elapsed_time(ee)
     status |= ops.get_device_status()
 
-    t = torch.tensor([ms, e2e_ms, launch_ms, float(status)], dtype=torch.float64, device=dev)
+    ms, e2e_ms, launch_ms, status = shard.reduce_max([ms, e2e_ms, launch_ms, float(status)], device=dev)
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
         dist.destroy_process_group()
-    ms, e2e_ms, launch_ms, status = t.tolist()
     if rank != 0:
         return
     if status:
         raise RuntimeError(f"device status bits {int(status):#x} during the timed region")
 
-    jets_total = b.N * K * world
-    value = jets_total / (ms / 1e3)
+    value = shard.job_rate(b.N * K, world, ms / 1e3)
     peak_tf, hbm_gbs, peak_src = measured_peaks()
     alg_flop = unordered * MLP_FLOP_PER_PAIR
     achieved_tf = alg_flop / (launch_ms / 1e3) / 1e12
@@ -304,7 +301,7 @@ def run_ours(args, world, rank, local):
                    "mean_multiplicity": float(b.mult.mean()), "path": "fused (bias on chip)",
                    "l2": f"{R} rotating input sets of {set_bytes / 2**20:.1f} MiB (> 2x L2)",
                    "parallelism": f"data-parallel over jets x{world}, no collective"},
-        "pairs_per_s": ordered * K * world / (ms / 1e3),
+        "pairs_per_s": shard.job_rate(ordered * K, world, ms / 1e3),
         "gpu_launches": K,
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved_tf / peak_tf, "traffic": traffic,
@@ -314,7 +311,7 @@ def run_ours(args, world, rank, local):
                      "exec_tflops": exec_tf, "dense_equiv_tflops": dense_tf,
                      "peak_source": f"{peak_src} bf16 dense burst (f16 runs at the same tensor rate)"},
         "clocks": clocks,
-        "e2e": {"value": b.N * Ke * world / (e2e_ms / 1e3), "unit": "jets/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": shard.job_rate(b.N * Ke, world, e2e_ms / 1e3), "unit": "jets/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke},
     }
     if world == 1 and not args.no_cpu_baseline:
