@@ -54,19 +54,48 @@ pb_status device_sms(int* dev_out, int* sms_out) {
   return PB_OK;
 }
 
-// Raise the dynamic shared-memory limit of `kernel` (once per device) and
-// return the persistent grid size: SMs x resident CTAs, at most `work`.
+// Resident CTAs per SM of a kernel instance on a device, found once (the
+// shared-memory attribute is raised at the same time) and cached, so that a
+// launch costs no runtime queries after the first.
+constexpr int kMaxKernels = 32;
+struct KernelFacts {
+  const void* fn = nullptr;
+  int per_sm[kMaxDev] = {};
+};
+KernelFacts g_kernels[kMaxKernels];
+
+pb_status resident_per_sm(const void* fn, int dev, size_t smem, int threads, int* per_sm_out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int slot = -1;
+  for (int i = 0; i < kMaxKernels; ++i) {
+    if (g_kernels[i].fn == fn || g_kernels[i].fn == nullptr) {
+      slot = i;
+      break;
+    }
+  }
+  if (slot < 0) return fail(PB_ECUDA, "kernel cache full");
+  KernelFacts& f = g_kernels[slot];
+  if (f.fn == nullptr) f.fn = fn;
+  if (f.per_sm[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(%zu B smem): %s", smem, cudaGetErrorString(e));
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
+    if (e != cudaSuccess) return fail(PB_ECUDA, "occupancy query: %s", cudaGetErrorString(e));
+    if (per_sm < 1) return fail(PB_ECUDA, "kernel does not fit on an SM (%zu B smem)", smem);
+    f.per_sm[dev] = per_sm;
+  }
+  *per_sm_out = f.per_sm[dev];
+  return PB_OK;
+}
+
+// The persistent grid size of `kernel`: SMs x resident CTAs, at most `work`.
 template <class K>
 pb_status prepare(K kernel, size_t smem, int threads, int work, int* grid) {
-  int dev = 0, sms = 0;
+  int dev = 0, sms = 0, per_sm = 0;
   pb_status st = device_sms(&dev, &sms);
   if (st != PB_OK) return st;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(%zu B smem): %s", smem, cudaGetErrorString(e));
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
-  if (e != cudaSuccess) return fail(PB_ECUDA, "occupancy query: %s", cudaGetErrorString(e));
-  if (per_sm < 1) return fail(PB_ECUDA, "kernel does not fit on an SM (%zu B smem)", smem);
+  if ((st = resident_per_sm((const void*)kernel, dev, smem, threads, &per_sm)) != PB_OK) return st;
   long long g = (long long)sms * per_sm;
   if (g > work) g = work;
   *grid = (int)(g < 1 ? 1 : g);
@@ -166,19 +195,15 @@ pb_status run_fused_grid(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::Q
                          cudaStream_t s) {
   auto k = pb::k_fused_grid<PM>;
   const size_t smem = sizeof(pb::FusedGridSmem<PM>);
-  int dev = 0, sms = 0;
+  int dev = 0, sms = 0, per_sm = 0;
   pb_status st = device_sms(&dev, &sms);
   if (st != PB_OK) return st;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(%zu B smem): %s", smem, cudaGetErrorString(e));
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 512, smem);
-  if (e != cudaSuccess || per_sm < 1) return fail(PB_ECUDA, "k_fused_grid does not fit on an SM");
+  if ((st = resident_per_sm((const void*)k, dev, smem, 512, &per_sm)) != PB_OK) return st;
   long long g = sms;  // one CTA per SM, all resident
   if (g > 8ll * J.N) g = 8ll * J.N;
   unsigned char* wsb = static_cast<unsigned char*>(ws);
   void* args[] = {(void*)&J, (void*)&W, (void*)&X, (void*)&wsb};
-  e = cudaLaunchCooperativeKernel((const void*)k, dim3((unsigned)g), dim3(512), args, smem, s);
+  cudaError_t e = cudaLaunchCooperativeKernel((const void*)k, dim3((unsigned)g), dim3(512), args, smem, s);
   if (e != cudaSuccess) return fail(PB_ECUDA, "k_fused_grid cooperative launch: %s", cudaGetErrorString(e));
   return PB_OK;
 }

@@ -128,6 +128,24 @@ __device__ void stage_jets(Particles<PM>* ring, const JetArgs& J, int K, const J
   }
 }
 
+// Prefetch jet n's momenta (and mask) rows into L2 ahead of stage_jet. One
+// thread; only rows that are 16-byte aligned and whole (16-byte aligned
+// arrays, padded rows of P % 4 == 0 floats, masks of P % 16 == 0 bytes;
+// packed jets need their ptr entries, so they are left alone).
+__device__ __forceinline__ void prefetch_jet(const JetArgs& J, int n) {
+  if (J.ptr || n >= J.N || (J.P & 3) != 0) return;
+  if (((reinterpret_cast<uintptr_t>(J.E) | reinterpret_cast<uintptr_t>(J.px) | reinterpret_cast<uintptr_t>(J.py) |
+        reinterpret_cast<uintptr_t>(J.pz)) & 15) != 0)
+    return;
+  const size_t e = (size_t)n * J.P;
+  const uint32_t bytes = (uint32_t)J.P * 4;
+  prefetch_l2(J.E + e, bytes);
+  prefetch_l2(J.px + e, bytes);
+  prefetch_l2(J.py + e, bytes);
+  prefetch_l2(J.pz + e, bytes);
+  if ((J.P & 15) == 0 && (reinterpret_cast<uintptr_t>(J.mask) & 15) == 0) prefetch_l2(J.mask + e, (uint32_t)J.P);
+}
+
 // One jet with the whole block (thread = slot); same result as stage_jets.
 template <int PM, bool kKin = true>
 __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
@@ -682,6 +700,23 @@ __device__ __forceinline__ size_t qkv_off(const Particles<PM>& S, const JetArgs&
   return (((size_t)n * kH + h) * J.P + S.slot[c]) * kD;
 }
 
+// Prefetch the Q, K and V rows of the staged jet n into L2: per tensor and
+// head the slots [slot[0], slot[m-1]] (padded) or the jet's tokens (packed).
+// Threads 0..23 issue one bulk prefetch each; no barrier.
+template <int PM>
+__device__ __forceinline__ void prefetch_qkv(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n) {
+  const int t = threadIdx.x;
+  if (t >= 3 * kH || S.m <= 0) return;
+  const uint16_t* base = t < kH ? X.q : (t < 2 * kH ? X.k : X.v);
+  const int h = t % kH;
+  if (J.ptr) {
+    if (h == 0) prefetch_l2(base + (size_t)S.base * kH * kD, (uint32_t)S.m * kH * kD * 2);
+  } else {
+    const int s0 = S.slot[0], s1 = S.slot[S.m - 1];
+    prefetch_l2(base + (((size_t)n * kH + h) * J.P + s0) * kD, (uint32_t)(s1 - s0 + 1) * kD * 2);
+  }
+}
+
 __device__ __forceinline__ void bf16x8_to_f32(uint4 r, float* f) {
   const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
@@ -1069,6 +1104,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FusedSmem<PM, NG>& S = *reinterpret_cast<FusedSmem<PM, NG>*>(smem_raw);
   constexpr int SL = FusedLayout<PM, NG>::kSL;
+  if (threadIdx.x == 0) prefetch_jet(J, blockIdx.x);  // overlaps the weight loads
   mlp_setup<NG, SL>(S.mlp, W);
   // during attention the activation tiles hold K and V
   float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
@@ -1078,6 +1114,8 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
   bool aborted = false;
   for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
     stage_jet<PM>(S.part, J, n);
+    prefetch_qkv<PM>(S.part, J, X, n);  // read by the attention after the MLP
+    if (threadIdx.x == 32) prefetch_jet(J, n + gridDim.x);  // this CTA's next jet
     const int m = S.part.m;
     SmemUSink sink{S.U8};
     if (m * (m + 1) / 2 <= kUCap) {
@@ -1313,6 +1351,20 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
   __syncthreads();
   const long long Ttot = S.T[N];
 
+  // phase B's share of this CTA: item (n, h) costs tiles_n + 1 and starts at
+  // 8 (T[n] + n) + h (tiles_n + 1)
+  const long long CB = 8ll * (Ttot + N);
+  const long long loB = CB * b / G, hiB = CB * (b + 1) / G;
+  int nB = 0;
+  {
+    int l = 0, r = N;  // smallest n whose items end past loB
+    while (l < r) {
+      const int mid = (l + r) >> 1;
+      if (8ll * ((long long)S.T[mid + 1] + mid + 1) > loB) r = mid; else l = mid + 1;
+    }
+    nB = l;
+  }
+
   mlp_setup<NG, SL>(S.mlp, W);
   uint32_t phase = 0u;
   bool aborted = false;
@@ -1371,18 +1423,8 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
 
   // ---------------------------------------------------------------- phase B
   if (!aborted) {
-    // item (n, h) costs tiles_n + 1; its start is 8 (T[n] + n) + h (tiles_n + 1)
-    const long long C = 8ll * (Ttot + N);
-    const long long lo = C * b / G, hi = C * (b + 1) / G;
-    int n = 0;
-    {
-      int l = 0, r = N;  // smallest n whose items end past lo
-      while (l < r) {
-        const int mid = (l + r) >> 1;
-        if (8ll * ((long long)S.T[mid + 1] + mid + 1) > lo) r = mid; else l = mid + 1;
-      }
-      n = l;
-    }
+    const long long lo = loB, hi = hiB;
+    int n = nB;
     float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
     constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
     AttnBatch<PM>& A = S.ab;

@@ -93,8 +93,14 @@ def _check(st: int) -> None:
         raise PairBiasError(st, lib().pb_last_error().decode())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream) -> int:
+    """cudaStream_t of `stream`, or of torch's current stream on the current device."""
     if stream is None:
+        if _raw_stream is not None:
+            return int(_raw_stream(torch.cuda.current_device()))
         stream = torch.cuda.current_stream()
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
