@@ -166,3 +166,49 @@ def forward(b, params=None) -> np.ndarray:
                          _ptr(v, C.c_uint16), D, _ptr(out, C.c_double)) != 0:
         raise ValueError("oracle: invalid jet description")
     return out
+
+
+def _bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact widening of raw bf16 bit patterns."""
+    b = np.ascontiguousarray(bits, np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def block_forward(b, bi, params=None) -> np.ndarray:
+    """Multi-head attention with the pair bias and the projections either side
+    of it, in fp64 (the attention of page 1 "Fusion 3" inside a ParT block of
+    embedding 128 = 8 heads x 16): for each jet's valid particles X,
+    q, k, v = X Wqkv^T + bqkv split into 8 heads of 16, o_h = softmax(q_h k_h^T
+    / sqrt(16) + U_h) v_h over the jet's valid keys, y = concat_h(o_h) Wo^T +
+    bo. Rows of masked slots are 0. `bi` is a ``synth.BlockInputs``; the
+    result is float64 [rows, 128] in the layout of bi.x."""
+    U = pair_bias(b, params)
+    x = _bf16_bits_to_f64(bi.x)
+    Wqkv = _bf16_bits_to_f64(bi.Wqkv)
+    Wo = _bf16_bits_to_f64(bi.Wo)
+    bqkv = np.asarray(bi.bqkv, np.float64)
+    bo = np.asarray(bi.bo, np.float64)
+    y = np.zeros_like(x)
+    for n in range(b.N):
+        if b.layout == "padded":
+            slots = np.flatnonzero(b.mask[n * b.P:(n + 1) * b.P])
+            rows = n * b.P + slots
+            local = slots
+        else:
+            rows = np.arange(int(b.ptr[n]), int(b.ptr[n + 1]))
+            local = np.arange(len(rows))
+        m = len(rows)
+        if m == 0:
+            continue
+        qkv = x[rows] @ Wqkv.T + bqkv
+        o = np.zeros((m, H * D))
+        for h in range(H):
+            q = qkv[:, h * D:(h + 1) * D]
+            k = qkv[:, H * D + h * D:H * D + (h + 1) * D]
+            v = qkv[:, 2 * H * D + h * D:2 * H * D + (h + 1) * D]
+            s = q @ k.T / np.sqrt(D) + U[n, h][np.ix_(local, local)]
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            o[:, h * D:(h + 1) * D] = (p / p.sum(axis=1, keepdims=True)) @ v
+        y[rows] = o @ Wo.T + bo
+    return y

@@ -201,3 +201,51 @@ def slice_jets(b: JetBatch, lo: int, hi: int) -> JetBatch:
     return JetBatch("packed", hi - lo, b.P, b.mult[lo:hi].copy(), b.E[s].copy(), b.px[s].copy(),
                     b.py[s].copy(), b.pz[s].copy(), None, ptr,
                     b.q[s].copy(), b.k[s].copy(), b.v[s].copy(), b.params)
+
+
+# ------------------------------------------------ projections around the attention
+
+EMBED = H_HEADS * D_HEAD  # 128: the particle embedding width of a ParT block
+
+
+@dataclass
+class BlockInputs:
+    """Particle embeddings and the attention's in/out projections.
+
+    x: bf16 bits [rows, EMBED] with rows = N * P (padded, slot order) or
+    tokens (packed); Wqkv: bf16 bits [3 * EMBED, EMBED], rows 0..127 the
+    query, 128..255 the key and 256..383 the value projection (out x in);
+    bqkv: float32 [3 * EMBED]; Wo: bf16 bits [EMBED, EMBED]; bo: float32
+    [EMBED].
+    """
+
+    x: np.ndarray
+    Wqkv: np.ndarray
+    bqkv: np.ndarray
+    Wo: np.ndarray
+    bo: np.ndarray
+
+
+def make_block_inputs(b: JetBatch, seed: int) -> BlockInputs:
+    """Embeddings x ~ N(0, 1) for every slot or token, projection weights
+    N(0, 1/EMBED) (variance) and biases N(0, 0.1) (standard deviation), all
+    rounded like the model's bf16 tensors (biases stay fp32). Drawn from a
+    stream of their own, so a batch's other inputs do not change."""
+    rng = np.random.default_rng([int(seed), 0xB10C])
+    rows = b.N * b.P if b.layout == "padded" else int(b.ptr[-1])
+    x = f32_to_bf16_bits(rng.standard_normal((rows, EMBED)).astype(np.float32))
+    s = 1.0 / np.sqrt(EMBED)
+    Wqkv = f32_to_bf16_bits((rng.standard_normal((3 * EMBED, EMBED)) * s).astype(np.float32))
+    bqkv = (rng.standard_normal(3 * EMBED) * 0.1).astype(np.float32)
+    Wo = f32_to_bf16_bits((rng.standard_normal((EMBED, EMBED)) * s).astype(np.float32))
+    bo = (rng.standard_normal(EMBED) * 0.1).astype(np.float32)
+    return BlockInputs(x, Wqkv, bqkv, Wo, bo)
+
+
+def slice_block_inputs(b: JetBatch, bi: BlockInputs, lo: int, hi: int) -> BlockInputs:
+    """The embeddings of jets lo..hi-1 (same weights)."""
+    if b.layout == "padded":
+        x = bi.x[lo * b.P:hi * b.P].copy()
+    else:
+        x = bi.x[int(b.ptr[lo]):int(b.ptr[hi])].copy()
+    return BlockInputs(x, bi.Wqkv, bi.bqkv, bi.Wo, bi.bo)

@@ -12,6 +12,10 @@ affine or a dropped bias).
 Attention: the bias-free and the biased cases against torch's
 scaled_dot_product_attention in fp64, one-particle jets, constant keys, mask
 exclusion, and padded == packed.
+Block (attention with its in and out projections): against torch's
+multi_head_attention_forward in fp64 jet by jet, reduction to the pinned
+attention under identity projections, masked rows 0, and the output-bias
+shift.
 """
 import json
 import math
@@ -267,3 +271,67 @@ def test_forward_equals_bias_then_attention_and_packed_equals_padded(oracle_lib)
         t0 = pk.ptr[n]
         assert np.array_equal(f_pd[n, :m, :m], f_pk[n, :m, :m])
         assert np.array_equal(o_fwd[n, :, :m, :].transpose(1, 0, 2), o_pk[t0:t0 + m])
+
+
+# ---------------------------------------------------------------- block
+
+
+def _block_batch(layout="padded", seed=11):
+    b = synth.make_jets(N=6, P=24, layout=layout, dist="uniform", mult_lo=1, mult_hi=24,
+                        mask_mode="scrambled" if layout == "padded" else "prefix", seed=seed)
+    return b, synth.make_block_inputs(b, seed)
+
+
+def _jet_rows(b, n):
+    if b.layout == "padded":
+        slots = np.flatnonzero(b.mask[n * b.P:(n + 1) * b.P])
+        return n * b.P + slots, slots
+    rows = np.arange(int(b.ptr[n]), int(b.ptr[n + 1]))
+    return rows, np.arange(len(rows))
+
+
+@pytest.mark.parametrize("layout", ["padded", "packed"])
+def test_block_matches_torch_multi_head_attention(oracle_lib, layout):
+    """torch's own MHA (its in-projection, head split, scaling and out
+    projection) in fp64, with the pair bias as a per-head additive mask."""
+    b, bi = _block_batch(layout)
+    y = oracle_lib.block_forward(b, bi)
+    U = oracle_lib.pair_bias(b)
+    x = synth.bf16_bits_to_f64(bi.x)
+    for n in range(b.N):
+        rows, local = _jet_rows(b, n)
+        if len(rows) == 0:
+            continue
+        X = torch.from_numpy(x[rows]).unsqueeze(1)                       # (L, batch 1, E)
+        mask = torch.from_numpy(U[n][:, local][:, :, local].copy())       # (heads, L, L)
+        ref, _ = torch.nn.functional.multi_head_attention_forward(
+            X, X, X, 128, 8,
+            torch.from_numpy(synth.bf16_bits_to_f64(bi.Wqkv)), torch.from_numpy(bi.bqkv.astype(np.float64)),
+            None, None, False, 0.0,
+            torch.from_numpy(synth.bf16_bits_to_f64(bi.Wo)), torch.from_numpy(bi.bo.astype(np.float64)),
+            training=False, need_weights=False, attn_mask=mask)
+        np.testing.assert_allclose(y[rows], ref[:, 0].numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_block_with_identity_projections_is_the_pinned_attention(oracle_lib):
+    """q = k = v = x and y = o when every projection is the identity: the
+    block's attention must then equal the C attention pinned above."""
+    b, bi = _block_batch("padded", seed=12)
+    one = synth.f32_to_bf16_bits(np.eye(128, dtype=np.float32))
+    ident = synth.BlockInputs(bi.x, np.concatenate([one, one, one]), np.zeros(384, np.float32), one,
+                              np.zeros(128, np.float32))
+    y = oracle_lib.block_forward(b, ident)
+    qkv = bi.x.reshape(b.N, b.P, 8, 16).transpose(0, 2, 1, 3).copy()     # [N, H, P, D]
+    ref = oracle_lib.attention(b, oracle_lib.pair_bias(b), qkv, qkv, qkv)
+    np.testing.assert_allclose(y.reshape(b.N, b.P, 8, 16).transpose(0, 2, 1, 3), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_block_masked_rows_zero_and_output_bias_shift(oracle_lib):
+    b, bi = _block_batch("padded", seed=13)
+    y = oracle_lib.block_forward(b, bi)
+    valid = b.mask.astype(bool)
+    assert np.all(y[~valid] == 0.0)
+    shifted = synth.BlockInputs(bi.x, bi.Wqkv, bi.bqkv, bi.Wo, bi.bo + np.float32(0.5))
+    y2 = oracle_lib.block_forward(b, shifted)
+    np.testing.assert_allclose(y2[valid] - y[valid], 0.5, atol=1e-12)
+    assert np.all(y2[~valid] == 0.0)
