@@ -21,7 +21,8 @@
  *     pb_fold_affine (host). Nothing is allocated inside the library.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream), launches exactly one kernel (the
- *     balanced fused path as a cooperative launch) and does not synchronise.
+ *     balanced fused path as a cooperative launch; pair_block_forward three,
+ *     in order) and does not synchronise.
  *     Host-side argument errors return before any launch; device-side problems (an invalid ptr array, a bounded wait that
  *     ran out) set bits of a per-device status word, read with
  *     pb_get_device_status.
@@ -96,6 +97,17 @@ typedef struct pb_mlp_unfolded {
   const float *W4, *b4;              /* [8][64], [8]              */
 } pb_mlp_unfolded;
 
+/* Projections of the attention inside a ParT block (embedding E = H*D = 128):
+ * q, k, v = x Wq^T + bq, x Wk^T + bk, x Wv^T + bv and y = o Wo^T + bo, where
+ * o is the concatenation of the 8 heads' attention outputs. Device pointers,
+ * row-major (out x in); the bf16 matrices 16-byte aligned. */
+typedef struct {
+  const uint16_t *Wqkv;   /* bf16 [3*128][128]: rows 0..127 Wq, 128..255 Wk, 256..383 Wv */
+  const float *bqkv;      /* [3*128]                                                     */
+  const uint16_t *Wo;     /* bf16 [128][128]                                             */
+  const float *bo;        /* [128]                                                       */
+} pb_proj;
+
 /* Offsets (in floats) of the folded parameters inside the flat buffer that
  * pb_fold_affine writes; PB_FOLDED_FLOATS is its length. */
 enum {
@@ -150,6 +162,31 @@ pb_status pair_attention_forward(const pb_jets *jets, const pb_mlp *mlp, const u
  * again before reuse. Calls sharing one workspace must not overlap on the
  * device. */
 size_t pb_workspace_bytes(const pb_jets *jets);
+
+/* pair_block_forward -- the attention of a ParT block with its projections:
+ * from particle embeddings x to y = MHA(x; U) with the pair bias U of
+ * pairbias_mlp_forward (the projections either side of "Fusion 3", with the
+ * bias of "Fusion 2"; the ParT blocks of the same page use embedding 128 and
+ * 8 heads).
+ *   x, y: bf16 [N*P][128] (padded, slot order) or [tokens][128] (packed),
+ *         16-byte aligned; rows of masked slots of y are written as 0 and
+ *         those of x are never used for y.
+ *   proj: the projection weights (see pb_proj); H = 8, D = 16, E = 128.
+ *   workspace: device memory of at least pb_block_workspace_bytes(jets)
+ *         bytes, 256-byte aligned, for Q, K, V and O (bf16, the layout of
+ *         pair_attention_forward's q); its contents need no initialisation.
+ * Launches, in order on `stream`: the in-projection GEMM (tensor cores),
+ * the fused pair-bias attention (pair_attention_forward with mlp), and the
+ * output-projection GEMM. Calls that share a workspace must not overlap on
+ * the device. Errors as for pair_attention_forward. */
+pb_status pair_block_forward(const pb_jets *jets, const pb_mlp *mlp, const pb_proj *proj, int H, int D, int E,
+                             const uint16_t *x, uint16_t *y, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/* pb_block_workspace_bytes -- workspace size of pair_block_forward: four
+ * bf16 tensors of rows x 128 (rows = N*P padded, tokens packed), each
+ * rounded up to 256 bytes. 0 if `jets` is invalid. */
+size_t pb_block_workspace_bytes(const pb_jets *jets);
 
 /* PB_STATIC_SCRATCH_BYTES -- size of the library's static per-device scratch
  * array used by pair_attention_forward_noalloc (32 MiB). */

@@ -234,6 +234,21 @@ pb_status static_scratch(void** out) {
   return PB_OK;
 }
 
+template <int kNout, int kIn, int kOut>
+pb_status run_proj(const pb::JetArgs& J, const pb::ProjArgs& X, cudaStream_t s, const char* what) {
+  auto k = pb::k_proj<kNout, kIn, kOut>;
+  const size_t smem = sizeof(pb::ProjSmem<kNout>);
+  const long long rows = J.ptr ? J.tokens : (long long)J.N * J.P;
+  const long long tiles = (rows + pb::kTileM - 1) / pb::kTileM;
+  int grid = 0;
+  pb_status st = prepare(k, smem, 256, (int)(tiles < 1 ? 1 : (tiles > (1ll << 30) ? (1ll << 30) : tiles)), &grid);
+  if (st != PB_OK) return st;
+  k<<<grid, 256, smem, s>>>(J, X);
+  return launched(what);
+}
+
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
 }  // namespace
 
 extern "C" {
@@ -329,6 +344,50 @@ pb_status pair_attention_forward_noalloc(const pb_jets* jets, const pb_mlp* mlp,
   if (e != cudaSuccess) return fail(PB_ECUDA, "clearing the static scratch header: %s", cudaGetErrorString(e));
   const pb::QkvArgs X{q, k, v, out};
   return J.P <= 128 ? run_fused_grid<128>(J, W, X, ws, s) : run_fused_grid<256>(J, W, X, ws, s);
+}
+
+size_t pb_block_workspace_bytes(const pb_jets* jets) {
+  pb::JetArgs J;
+  if (check_jets(jets, &J) != PB_OK) return 0;
+  const long long rows = J.ptr ? J.tokens : (long long)J.N * J.P;
+  return 4 * round256((size_t)rows * pb::kEmbed * 2);
+}
+
+pb_status pair_block_forward(const pb_jets* jets, const pb_mlp* mlp, const pb_proj* proj, int H, int D, int E,
+                             const uint16_t* x, uint16_t* y, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  pb::JetArgs J;
+  pb::MlpArgs W;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK) return st;
+  if (H != pb::kH || D != pb::kD || E != pb::kEmbed)
+    return fail(PB_EUNSUPPORTED, "H = %d, D = %d, E = %d; only H = 8, D = 16, E = 128", H, D, E);
+  if ((st = check_mlp(mlp, &W)) != PB_OK) return st;
+  if (!proj) return fail(PB_EINVAL, "proj is NULL");
+  if (!proj->Wqkv || !proj->bqkv || !proj->Wo || !proj->bo) return fail(PB_EINVAL, "a projection pointer is NULL");
+  if (!aligned(proj->Wqkv, 16) || !aligned(proj->Wo, 16) || !aligned(proj->bqkv, 4) || !aligned(proj->bo, 4))
+    return fail(PB_EINVAL, "Wqkv and Wo must be 16-byte aligned, the biases 4-byte aligned");
+  if (J.N == 0) return PB_OK;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return fail(PB_EINVAL, "x and y must be non-NULL and 16-byte aligned");
+  const long long rows = J.ptr ? J.tokens : (long long)J.N * J.P;
+  const size_t tb = round256((size_t)rows * pb::kEmbed * 2);
+  if (!workspace || !aligned(workspace, 256)) return fail(PB_EINVAL, "workspace must be non-NULL and 256-byte aligned");
+  if (workspace_bytes < 4 * tb)
+    return fail(PB_EINVAL, "workspace of %zu bytes, %zu needed (pb_block_workspace_bytes)", workspace_bytes, 4 * tb);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  uint16_t* q = reinterpret_cast<uint16_t*>(ws);
+  uint16_t* k = reinterpret_cast<uint16_t*>(ws + tb);
+  uint16_t* v = reinterpret_cast<uint16_t*>(ws + 2 * tb);
+  uint16_t* o = reinterpret_cast<uint16_t*>(ws + 3 * tb);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rows == 0) return PB_OK;  // packed jets that are all empty: nothing to read or write
+  const pb::ProjArgs in{x, proj->Wqkv, proj->bqkv, q, k, v};
+  if ((st = run_proj<384, pb::kInRows, pb::kOutQKV>(J, in, s, "k_proj (in)")) != PB_OK) return st;
+  const pb::QkvArgs X{q, k, v, o};
+  st = J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
+  if (st != PB_OK) return st;
+  const pb::ProjArgs out{o, proj->Wo, proj->bo, y, nullptr, nullptr};
+  return run_proj<128, pb::kInHeads, pb::kOutRows>(J, out, s, "k_proj (out)");
 }
 
 pb_status pb_get_device_status(void* stream, uint32_t* bits) {

@@ -1566,4 +1566,187 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
   return kWsHeader + (size_t)rows * 16;
 }
 
+
+// ============================================ k_proj (projections either side)
+//
+// The in-projection of a ParT attention block (x -> Q, K, V) and its output
+// projection (O -> y) as one tensor-core GEMM kernel over particle rows:
+// out[r, :] = W in[r, :] + b for every row r of the padded slots (N * P) or
+// the packed tokens, with E = 128 input features. The whole weight matrix
+// (kNout x 128 bf16) stays in shared memory in the K-major layout of the MMA
+// operands; each CTA streams 128-row tiles of the input through a double
+// buffer, one thread issues 8 K steps x kNout/128 tcgen05 MMAs (bf16
+// operands, fp32 accumulation in TMEM), and 8 warps read the accumulator
+// back (TMEM lane = row), add the bias and store bf16.
+
+constexpr int kEmbed = kH * kD;  // 128
+
+enum ProjIn { kInRows = 0, kInHeads = 1 };     // [rows, 128] | attention layout [N, H, P, D]
+enum ProjOut { kOutQKV = 0, kOutRows = 1 };    // Q, K, V in attention layout | [rows, 128]
+
+struct ProjArgs {
+  const uint16_t* in;   // kInRows: x [rows, 128]; kInHeads: O in the layout of Q
+  const uint16_t* W;    // [kNout, 128] bf16, row-major (out x in)
+  const float* bias;    // [kNout]
+  uint16_t* out0;       // kOutQKV: Q; kOutRows: y [rows, 128]
+  uint16_t* out1;       // kOutQKV: K
+  uint16_t* out2;       // kOutQKV: V
+};
+
+template <int kNout>
+struct ProjSmem {
+  __nv_bfloat16 W[kNout * kEmbed];      // B operand, K-major, 8-row groups of 2,048 B
+  __nv_bfloat16 A[2][kTileM * kEmbed];  // A operand double buffer
+  float bias[kNout];
+  uint64_t mbar;
+  uint32_t tmem_base;
+};
+
+__host__ __device__ constexpr uint32_t proj_tmem_cols(int nout) { return nout <= 128 ? 128u : (nout <= 256 ? 256u : 512u); }
+
+// Rows of the GEMM: N * P padded slots or the packed tokens.
+__device__ __forceinline__ long long proj_rows(const JetArgs& J) { return J.ptr ? J.tokens : (long long)J.N * J.P; }
+
+// Row r of the output written? (the in-projection skips masked slots, whose
+// Q/K/V are never read; the out-projection writes 0 there)
+__device__ __forceinline__ bool proj_row_valid(const JetArgs& J, long long r) { return J.ptr || J.mask[r] != 0; }
+
+// Input tile t (rows t*128 ..) into A[buf]: 128 rows x 16 chunks of 8 bf16;
+// rows past the end are zero. Block-wide; no barrier.
+template <int kIn>
+__device__ __forceinline__ void proj_load_tile(__nv_bfloat16* A, const JetArgs& J, const ProjArgs& X, long long t,
+                                               long long R) {
+  constexpr int kPer = kTileM * (kEmbed / 8);  // 2048 16-byte chunks
+  uint4 v[kPer / 256];
+#pragma unroll
+  for (int u = 0; u < kPer / 256; ++u) {
+    const int idx = threadIdx.x + u * 256;
+    const int rr = idx >> 4, kc = idx & 15;
+    const long long r = t * kTileM + rr;
+    v[u] = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const uint16_t* src;
+      if (kIn == kInRows || J.ptr) {
+        src = X.in + r * kEmbed + kc * 8;
+      } else {  // O[n, h, slot, d] with column kc * 8 = h * 16 + (kc & 1) * 8
+        const long long n = r / J.P, slot = r % J.P;
+        src = X.in + ((n * kH + (kc >> 1)) * J.P + slot) * kD + (kc & 1) * 8;
+      }
+      v[u] = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPer / 256; ++u) {
+    const int idx = threadIdx.x + u * 256;
+    const int rr = idx >> 4, kc = idx & 15;
+    *reinterpret_cast<uint4*>(A + cofs(rr, kc * 8, kEmbed)) = v[u];
+  }
+}
+
+template <int kNout, int kIn, int kOut>
+__global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  ProjSmem<kNout>& S = *reinterpret_cast<ProjSmem<kNout>*>(smem_raw);
+  constexpr uint32_t kCols = proj_tmem_cols(kNout);
+  constexpr uint32_t kIdesc = idesc_bf16_m128(128);
+  constexpr uint32_t kSBO = kEmbed / 8 * 128;  // 2,048 B between 8-row groups
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long R = proj_rows(J);
+  const long long ntiles = (R + kTileM - 1) / kTileM;
+
+  // weights (K-major) and bias, once per CTA
+  for (int idx = tid; idx < kNout * (kEmbed / 8); idx += blockDim.x) {
+    const int n = idx >> 4, kc = idx & 15;
+    *reinterpret_cast<uint4*>(S.W + cofs(n, kc * 8, kEmbed)) =
+        *reinterpret_cast<const uint4*>(X.W + (size_t)n * kEmbed + kc * 8);
+  }
+  for (int i = tid; i < kNout; i += blockDim.x) S.bias[i] = X.bias[i];
+  if (tid == 0) {
+    mbar_init(&S.mbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
+  long long t = blockIdx.x;
+  if (t < ntiles) proj_load_tile<kIn>(S.A[0], J, X, t, R);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  uint32_t phase = 0;
+  bool ok = true;
+  int buf = 0;
+  for (; t < ntiles; t += gridDim.x, buf ^= 1) {
+    if (tid == 0) {
+      const uint32_t a0 = smem_u32(S.A[buf]), w0 = smem_u32(S.W);
+#pragma unroll 1
+      for (int c = 0; c < kNout / 128; ++c)
+#pragma unroll
+        for (int s = 0; s < kEmbed / 16; ++s)
+          mma_f16(tmem + 128u * c, smem_desc(a0 + 256u * s, 128, kSBO),
+                  smem_desc(w0 + (uint32_t)c * 128u * kSBO / 8u + 256u * s, 128, kSBO), kIdesc, s > 0 ? 1u : 0u);
+      mma_commit(&S.mbar);
+    }
+    // the next tile loads while the MMAs run
+    if (t + gridDim.x < ntiles) proj_load_tile<kIn>(S.A[buf ^ 1], J, X, t + gridDim.x, R);
+    const bool done = mbar_wait(&S.mbar, phase);
+    if (done) phase ^= 1u;  // on a timeout the teardown waits on the same phase once more
+    ok = __syncthreads_and(done && ok) != 0;
+    tc_fence_after();
+    if (!ok) break;
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. and half w / 4 of the columns
+    {
+      const int rr = (warp & 3) * 32 + lane;
+      const long long r = t * kTileM + rr;
+      const bool in_range = r < R;
+      const bool valid = in_range && proj_row_valid(J, r);
+      const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      constexpr int kHalf = kNout / 2;
+#pragma unroll 1
+      for (int c0 = (warp >> 2) * kHalf; c0 < (warp >> 2) * kHalf + kHalf; c0 += 32) {
+        float v[32];
+        tmem_ld32_wait(lane_base + (uint32_t)c0, v);  // warp-wide: every lane, in range or not
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = valid ? cvt_bf16x2(v[2 * i] + S.bias[c0 + 2 * i], v[2 * i + 1] + S.bias[c0 + 2 * i + 1]) : 0u;
+        if (kOut == kOutRows && in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(X.out0 + r * kEmbed + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        } else if (kOut == kOutQKV && valid) {
+          // columns c0 .. c0 + 31: two heads of one of Q, K, V
+          const int tensor = c0 / kEmbed, cc = c0 % kEmbed;
+          uint16_t* base = tensor == 0 ? X.out0 : (tensor == 1 ? X.out1 : X.out2);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = cc / kD + hh;
+            size_t off;
+            if (J.ptr) off = ((size_t)r * kH + h) * kD;
+            else off = (((size_t)(r / J.P) * kH + h) * J.P + (size_t)(r % J.P)) * kD;
+            uint4* dst = reinterpret_cast<uint4*>(base + off);
+            dst[0] = make_uint4(w[8 * hh], w[8 * hh + 1], w[8 * hh + 2], w[8 * hh + 3]);
+            dst[1] = make_uint4(w[8 * hh + 4], w[8 * hh + 5], w[8 * hh + 6], w[8 * hh + 7]);
+          }
+        }
+      }
+    }
+    // TMEM is read and the next A tile written before the next MMAs
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (!ok && tid == 0) raise_status(kStTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (!ok) {
+    // an MMA may still be in flight: wait once more (bounded) before freeing TMEM
+    if (tid == 0) (void)mbar_wait(&S.mbar, phase);
+    __syncthreads();
+  }
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kCols);
+}
+
 }  // namespace pb

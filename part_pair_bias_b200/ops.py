@@ -6,8 +6,8 @@ on first use and its absence is an error -- there is no fallback.
 
 Entry points mirror ``include/pairbias.h``: ``pairfeat_compute``,
 ``pairbias_mlp_forward``, ``pair_attention_forward``,
-``pair_attention_forward_noalloc``, ``get_device_status`` and the host
-helper ``fold_affine``.
+``pair_attention_forward_noalloc``, ``pair_block_forward``,
+``get_device_status`` and the host helper ``fold_affine``.
 """
 from __future__ import annotations
 
@@ -51,6 +51,10 @@ class _Mlp(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("W1", "b1", "W2", "b2", "W3", "b3", "W4", "b4")]
 
 
+class _Proj(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("Wqkv", "bqkv", "Wo", "bo")]
+
+
 class _MlpUnfolded(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("a0", "c0", "W1", "b1", "a1", "c1", "W2", "b2", "a2", "c2",
                                           "W3", "b3", "a3", "c3", "W4", "b4")]
@@ -75,6 +79,10 @@ def lib():
                                                  vp, vp, vp, vp, vp, C.c_size_t, vp]
             L.pair_attention_forward_noalloc.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.c_int, C.c_int,
                                                          vp, vp, vp, vp, vp]
+            L.pair_block_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.POINTER(_Proj), C.c_int, C.c_int,
+                                             C.c_int, vp, vp, vp, C.c_size_t, vp]
+            L.pb_block_workspace_bytes.argtypes = [C.POINTER(_Jets)]
+            L.pb_block_workspace_bytes.restype = C.c_size_t
             L.pb_workspace_bytes.argtypes = [C.POINTER(_Jets)]
             L.pb_workspace_bytes.restype = C.c_size_t
             L.pb_get_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
@@ -82,7 +90,8 @@ def lib():
             L.pb_last_error.restype = C.c_char_p
             L.pb_version.restype = C.c_char_p
             for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward,
-                      L.pair_attention_forward_noalloc, L.pb_get_device_status, L.pb_fold_affine):
+                      L.pair_attention_forward_noalloc, L.pair_block_forward, L.pb_get_device_status,
+                      L.pb_fold_affine):
                 f.restype = C.c_int
             _lib = L
         return _lib
@@ -222,6 +231,44 @@ def pair_attention_forward_noalloc(jets: Jets, mlp: FoldedMLP, q: torch.Tensor, 
     js, ms = jets.struct(), mlp.struct()
     _check(lib().pair_attention_forward_noalloc(C.byref(js), C.byref(ms), H, D, q.data_ptr(), k.data_ptr(),
                                                 v.data_ptr(), out.data_ptr(), _stream(stream)))
+
+
+@dataclass
+class Proj:
+    """Projection weights of the attention block (see pb_proj in the header):
+    bf16 Wqkv [384, 128] and Wo [128, 128], fp32 bqkv [384] and bo [128]."""
+
+    Wqkv: torch.Tensor
+    bqkv: torch.Tensor
+    Wo: torch.Tensor
+    bo: torch.Tensor
+
+    def struct(self) -> _Proj:
+        return _Proj(_dp(self.Wqkv), _dp(self.bqkv), _dp(self.Wo), _dp(self.bo))
+
+
+def proj_to_device(bi, device="cuda") -> Proj:
+    """The weights of a ``synth.BlockInputs`` as device tensors."""
+    f = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+    return Proj(bf16_to_device(bi.Wqkv, device), f(bi.bqkv), bf16_to_device(bi.Wo, device), f(bi.bo))
+
+
+def block_workspace_bytes(jets: Jets) -> int:
+    js = jets.struct()
+    return int(lib().pb_block_workspace_bytes(C.byref(js)))
+
+
+def pair_block_forward(jets: Jets, mlp: FoldedMLP, proj: Proj, x: torch.Tensor, y: torch.Tensor,
+                       workspace: torch.Tensor, stream=None) -> None:
+    """y = multi-head attention of x with the pair bias and its in/out
+    projections; x, y bf16 [rows, 128]; workspace uint8 of
+    ``block_workspace_bytes(jets)`` bytes."""
+    for t in (x, y):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    js, ms, ps = jets.struct(), mlp.struct(), proj.struct()
+    _check(lib().pair_block_forward(C.byref(js), C.byref(ms), C.byref(ps), H, D, H * D, x.data_ptr(), y.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)))
 
 
 def get_device_status(stream=None) -> int:

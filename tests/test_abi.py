@@ -139,3 +139,26 @@ def test_noalloc_host_rejections(L):
     assert L.pair_attention_forward_noalloc(C.byref(js), C.byref(mlp), 8, 16, d + 2, d, d, d, None) == ops.PB_EINVAL
     js.N = 0                          # nothing to do: no device needed
     assert L.pair_attention_forward_noalloc(C.byref(js), C.byref(mlp), 8, 16, d, d, d, d, None) == ops.PB_OK
+
+
+def test_block_host_validation_and_workspace(L):
+    js, keep = _jets(N=2, P=8)
+    d = np.zeros(64, np.float32).ctypes.data
+    mlp = ops._Mlp(*([d] * 8))
+    proj = ops._Proj(d, d, d, d)
+    need = 4 * ((2 * 8 * 128 * 2 + 255) // 256 * 256)
+    assert L.pb_block_workspace_bytes(C.byref(js)) == need
+    wbuf = np.zeros(need + 512, np.uint8)
+    ws = (wbuf.ctypes.data + 255) // 256 * 256
+    call = lambda **kw: L.pair_block_forward(C.byref(js), C.byref(mlp), kw.get("proj", C.byref(proj)), 8, 16,
+                                             kw.get("E", 128), kw.get("x", d), d, kw.get("ws", ws),
+                                             kw.get("wsb", need), None)
+    assert call(E=64) == ops.PB_EUNSUPPORTED
+    assert call(proj=None) == ops.PB_EINVAL
+    assert call(x=d + 8) == ops.PB_EINVAL                   # x not 16-byte aligned
+    assert call(wsb=need - 1) == ops.PB_EINVAL              # workspace too small
+    assert call(ws=ws + 16) == ops.PB_EINVAL                # workspace not 256-byte aligned
+    bad = ops._Proj(d, d, None, d)
+    assert call(proj=C.byref(bad)) == ops.PB_EINVAL
+    js.N = 0                                                # nothing to do, no device needed
+    assert call() == ops.PB_OK
