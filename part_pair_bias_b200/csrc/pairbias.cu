@@ -79,6 +79,10 @@ pb_status resident_per_sm(const void* fn, int dev, size_t smem, int threads, int
   if (f.per_sm[dev] == 0) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(%zu B smem): %s", smem, cudaGetErrorString(e));
+    // every kernel of the library asks for the same (maximal) shared-memory
+    // carveout, so that consecutive launches need no L1/shared repartition
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return fail(PB_ECUDA, "cudaFuncSetAttribute(carveout): %s", cudaGetErrorString(e));
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
     if (e != cudaSuccess) return fail(PB_ECUDA, "occupancy query: %s", cudaGetErrorString(e));

@@ -1611,17 +1611,28 @@ __device__ __forceinline__ long long proj_rows(const JetArgs& J) { return J.ptr 
 // Q/K/V are never read; the out-projection writes 0 there)
 __device__ __forceinline__ bool proj_row_valid(const JetArgs& J, long long r) { return J.ptr || J.mask[r] != 0; }
 
-// Input tile t (rows t*128 ..) into A[buf]: 128 rows x 16 chunks of 8 bf16;
-// rows past the end are zero. Block-wide; no barrier.
+// Input tile t (rows t*128 ..): 128 rows x 16 chunks of 8 bf16, loaded into
+// eight registers per thread (rows past the end are zero), then stored to
+// A in the operand layout. Block-wide (256 threads); no barrier.
+constexpr int kTileChunksPerThread = kTileM * (kEmbed / 8) / 256;  // 8
+
+// Chunk idx of a [rows][16 chunks] operand -> (row, chunk). A warp takes 8
+// rows x 4 chunks: the 16-byte bank group of a chunk in the operand layout
+// is its row mod 8, so each quarter-warp stores to 8 distinct bank groups,
+// and the warp still reads whole 32-byte sectors of every row.
+__device__ __forceinline__ void chunk_rc(int idx, int& r, int& kc) {
+  const int w = idx >> 5, l = idx & 31;
+  r = (w >> 2) * 8 + (l & 7);
+  kc = (w & 3) * 4 + (l >> 3);
+}
+
 template <int kIn>
-__device__ __forceinline__ void proj_load_tile(__nv_bfloat16* A, const JetArgs& J, const ProjArgs& X, long long t,
-                                               long long R) {
-  constexpr int kPer = kTileM * (kEmbed / 8);  // 2048 16-byte chunks
-  uint4 v[kPer / 256];
+__device__ __forceinline__ void proj_fetch_tile(uint4* v, const JetArgs& J, const ProjArgs& X, long long t,
+                                                long long R) {
 #pragma unroll
-  for (int u = 0; u < kPer / 256; ++u) {
-    const int idx = threadIdx.x + u * 256;
-    const int rr = idx >> 4, kc = idx & 15;
+  for (int u = 0; u < kTileChunksPerThread; ++u) {
+    int rr, kc;
+    chunk_rc(threadIdx.x + u * 256, rr, kc);
     const long long r = t * kTileM + rr;
     v[u] = make_uint4(0, 0, 0, 0);
     if (r < R) {
@@ -1635,12 +1646,23 @@ __device__ __forceinline__ void proj_load_tile(__nv_bfloat16* A, const JetArgs& 
       v[u] = *reinterpret_cast<const uint4*>(src);
     }
   }
+}
+
+__device__ __forceinline__ void proj_store_tile(__nv_bfloat16* A, const uint4* v) {
 #pragma unroll
-  for (int u = 0; u < kPer / 256; ++u) {
-    const int idx = threadIdx.x + u * 256;
-    const int rr = idx >> 4, kc = idx & 15;
+  for (int u = 0; u < kTileChunksPerThread; ++u) {
+    int rr, kc;
+    chunk_rc(threadIdx.x + u * 256, rr, kc);
     *reinterpret_cast<uint4*>(A + cofs(rr, kc * 8, kEmbed)) = v[u];
   }
+}
+
+template <int kIn>
+__device__ __forceinline__ void proj_load_tile(__nv_bfloat16* A, const JetArgs& J, const ProjArgs& X, long long t,
+                                               long long R) {
+  uint4 v[kTileChunksPerThread];
+  proj_fetch_tile<kIn>(v, J, X, t, R);
+  proj_store_tile(A, v);
 }
 
 template <int kNout, int kIn, int kOut>
@@ -1654,11 +1676,31 @@ __global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
   const long long R = proj_rows(J);
   const long long ntiles = (R + kTileM - 1) / kTileM;
 
-  // weights (K-major) and bias, once per CTA
-  for (int idx = tid; idx < kNout * (kEmbed / 8); idx += blockDim.x) {
-    const int n = idx >> 4, kc = idx & 15;
-    *reinterpret_cast<uint4*>(S.W + cofs(n, kc * 8, kEmbed)) =
-        *reinterpret_cast<const uint4*>(X.W + (size_t)n * kEmbed + kc * 8);
+  // the first input tile and the weights (K-major), once per CTA, with
+  // sixteen 16-byte loads per thread in flight before their stores
+  long long t = blockIdx.x;
+  {
+    uint4 a[kTileChunksPerThread];
+    if (t < ntiles) proj_fetch_tile<kIn>(a, J, X, t, R);
+    constexpr int kW = kNout * (kEmbed / 8) / 256;  // weight chunks per thread: 24 or 8
+    static_assert(kNout * (kEmbed / 8) % 256 == 0, "whole weight chunks per thread");
+#pragma unroll
+    for (int b0 = 0; b0 < kW; b0 += 16) {
+      uint4 w[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        int n, kc;
+        chunk_rc(tid + (b0 + u) * 256, n, kc);
+        if (b0 + u < kW) w[u] = *reinterpret_cast<const uint4*>(X.W + (size_t)n * kEmbed + kc * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        int n, kc;
+        chunk_rc(tid + (b0 + u) * 256, n, kc);
+        if (b0 + u < kW) *reinterpret_cast<uint4*>(S.W + cofs(n, kc * 8, kEmbed)) = w[u];
+      }
+    }
+    if (t < ntiles) proj_store_tile(S.A[0], a);
   }
   for (int i = tid; i < kNout; i += blockDim.x) S.bias[i] = X.bias[i];
   if (tid == 0) {
@@ -1666,8 +1708,6 @@ __global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
-  long long t = blockIdx.x;
-  if (t < ntiles) proj_load_tile<kIn>(S.A[0], J, X, t, R);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -1703,9 +1743,13 @@ __global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
       const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
       constexpr int kHalf = kNout / 2;
 #pragma unroll 1
-      for (int c0 = (warp >> 2) * kHalf; c0 < (warp >> 2) * kHalf + kHalf; c0 += 32) {
-        float v[32];
-        tmem_ld32_wait(lane_base + (uint32_t)c0, v);  // warp-wide: every lane, in range or not
+      for (int c64 = (warp >> 2) * kHalf; c64 < (warp >> 2) * kHalf + kHalf; c64 += 64) {
+        float v64[64];
+        tmem_ld64_wait(lane_base + (uint32_t)c64, v64);  // warp-wide: every lane, in range or not
+#pragma unroll
+       for (int half = 0; half < 2; ++half) {
+        const int c0 = c64 + 32 * half;
+        const float* v = v64 + 32 * half;
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -1729,6 +1773,7 @@ __global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
             dst[1] = make_uint4(w[8 * hh + 4], w[8 * hh + 5], w[8 * hh + 6], w[8 * hh + 7]);
           }
         }
+       }
       }
     }
     // TMEM is read and the next A tile written before the next MMAs
