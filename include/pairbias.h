@@ -221,6 +221,14 @@ pb_status pair_attention_forward_noalloc(const pb_jets *jets, const pb_mlp *mlp,
  * PB_ECUDA if the synchronisation itself failed. */
 pb_status pb_get_device_status(void *stream, uint32_t *bits);
 
+/* pb_selftest_wait_timeouts -- diagnostic of the failure path; no
+ * counterpart in the paper. Launches one small kernel whose two waits, an
+ * mbarrier that nothing completes and a grid barrier whose target nothing
+ * reaches, use the same bounded-wait code and limit (2 s) as the library's
+ * kernels. Both run out, PB_DEV_TIMEOUT is set, and the kernel ends
+ * normally, so the context stays usable. About 4 s of device time. */
+pb_status pb_selftest_wait_timeouts(void *stream);
+
 /* pb_fold_affine -- host helper, not on the GPU path: fold the batch-norm
  * affines of an unfolded MLP into Linear weights and biases (the eval-time
  * folding of "Fusion 2"), computing in double and rounding once to fp32.

@@ -394,6 +394,11 @@ pb_status pair_block_forward(const pb_jets* jets, const pb_mlp* mlp, const pb_pr
   return run_proj<128, pb::kInHeads, pb::kOutRows>(J, out, s, "k_proj (out)");
 }
 
+pb_status pb_selftest_wait_timeouts(void* stream) {
+  pb::k_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launched("k_wait_selftest");
+}
+
 pb_status pb_get_device_status(void* stream, uint32_t* bits) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(PB_ECUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));

@@ -1794,4 +1794,29 @@ __global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
   if (warp == 0) tmem_dealloc(tmem, kCols);
 }
 
+
+// ================================================= k_wait_selftest (diagnostic)
+//
+// Exercises the failure path of the library's bounded waits: an mbarrier
+// wait that nothing completes and a grid barrier whose target nothing
+// reaches, both with the library's own wait code and limit (2 s each). Each
+// runs out, raises kStTimeout and returns; the kernel then ends normally and
+// the context stays usable. One CTA of 32 threads.
+__device__ unsigned long long g_selftest_ctr[2];
+
+__global__ void k_wait_selftest() {
+  __shared__ uint64_t bar;
+  __shared__ int flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  (void)mbar_wait(&bar, 0);  // no arrival: runs out after the library's limit
+  __syncthreads();
+  // a grid barrier for two CTAs, launched as one: the target is never reached
+  (void)grid_barrier(&g_selftest_ctr[0], 2u, &flag);
+  if (threadIdx.x == 0) g_selftest_ctr[0] = 0;  // leave the counter as found
+}
+
 }  // namespace pb

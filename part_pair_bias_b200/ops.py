@@ -89,7 +89,8 @@ def lib():
             L.pb_fold_affine.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float)]
             L.pb_last_error.restype = C.c_char_p
             L.pb_version.restype = C.c_char_p
-            for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward,
+            L.pb_selftest_wait_timeouts.argtypes = [vp]
+            for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward, L.pb_selftest_wait_timeouts,
                       L.pair_attention_forward_noalloc, L.pair_block_forward, L.pb_get_device_status,
                       L.pb_fold_affine):
                 f.restype = C.c_int
@@ -269,6 +270,11 @@ def pair_block_forward(jets: Jets, mlp: FoldedMLP, proj: Proj, x: torch.Tensor, 
     _check(lib().pair_block_forward(C.byref(js), C.byref(ms), C.byref(ps), H, D, H * D, x.data_ptr(), y.data_ptr(),
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream)))
+
+
+def selftest_wait_timeouts(stream=None) -> None:
+    """Run the bounded-wait diagnostic (sets PB_DEV_TIMEOUT after ~4 s)."""
+    _check(lib().pb_selftest_wait_timeouts(_stream(stream)))
 
 
 def get_device_status(stream=None) -> int:

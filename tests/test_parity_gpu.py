@@ -188,3 +188,20 @@ def test_many_jets_per_cta(oracle_lib):
     pt.check_attention(pt.to_np(d.fused()), ref, b)
     pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
     assert ops.get_device_status() == 0
+
+
+@pytest.mark.parametrize("P", [2, 3, 5, 8])
+def test_tiny_jets_elementwise(oracle_lib, P):
+    """P = 2..8 with scrambled masks, empty and full jets: every entry point
+    against the oracle element by element."""
+    mults = [0, 1, P, max(1, P - 1), 2, P, 0, P // 2 + 1]
+    b = synth.make_jets(N=len(mults), P=P, mults=mults, mask_mode="scrambled", seed=30 + P)
+    d = pt.Device(b)
+    pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
+    pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
+    pt.check_bias(pt.to_np(d.bias(torch.bfloat16)), oracle_lib.pair_bias(b), b, bf16=True)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
+    pt.check_attention(pt.to_np(d.with_bias(d.bias(torch.bfloat16))), ref, b)
+    assert ops.get_device_status() == 0
