@@ -59,6 +59,10 @@ typedef enum { PB_BF16 = 0, PB_F32 = 1 } pb_dtype;
 #define PB_DEV_TIMEOUT 1u   /* a bounded wait inside a kernel ran out; outputs invalid */
 #define PB_DEV_BADPTR 2u    /* a packed jet had ptr[n] > ptr[n+1], more than P tokens,
                                or reached past `tokens`; that jet was skipped          */
+#define PB_DEV_BOUNDS 4u    /* only in a library built with PB_DEBUG_BOUNDS: a computed
+                               index (pair unpacking, bias slot or record, Q/K/V/out
+                               offset, attention staging) left its range; that access
+                               was skipped                                             */
 
 /* One batch of jets. Exactly one layout is used.
  * Padded (ptr == NULL): E, px, py, pz and mask are [N*P] (jet n, slot s at

@@ -10,22 +10,27 @@ SRC = os.path.join(_HERE, "csrc", "pairbias.cu")
 DEPS = [os.path.join(_HERE, "csrc", f) for f in ("pairbias.cu", "pb_device.cuh", "pb_kernels.cuh")] + [
     os.path.join(ROOT, "include", "pairbias.h")]
 OUT = os.path.join(_HERE, "libpairbias.so")
+# the same library with every computed-index check of PB_DEBUG_BOUNDS compiled in
+OUT_DEBUG = os.path.join(_HERE, "libpairbias_debug.so")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libpairbias.so if it is missing or older than a source file."""
-    stale = force or not os.path.exists(OUT) or any(os.path.getmtime(d) > os.path.getmtime(OUT) for d in DEPS)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile libpairbias.so (or, with debug, libpairbias_debug.so) if it is
+    missing or older than a source file."""
+    out = OUT_DEBUG if debug else OUT
+    stale = force or not os.path.exists(out) or any(os.path.getmtime(d) > os.path.getmtime(out) for d in DEPS)
     if stale:
         nvcc = os.environ.get("NVCC", "nvcc")
-        cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", OUT + ".tmp", SRC]
+        cmd = [nvcc, *NVCC_FLAGS, *(["-DPB_DEBUG_BOUNDS"] if debug else []), "-I", os.path.join(ROOT, "include"),
+               "-o", out + ".tmp", SRC]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)
-        os.replace(OUT + ".tmp", OUT)
-    return OUT
+        os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

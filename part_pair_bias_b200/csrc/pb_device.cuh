@@ -20,6 +20,7 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
 constexpr unsigned kStTimeout = 1u;  // == PB_DEV_TIMEOUT
 constexpr unsigned kStBadPtr = 2u;   // == PB_DEV_BADPTR
+constexpr unsigned kStBounds = 4u;   // == PB_DEV_BOUNDS (libraries built with PB_DEBUG_BOUNDS)
 
 __device__ unsigned int g_status;
 
@@ -28,6 +29,18 @@ __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// Computed-index check of debug builds (PB_DEBUG_BOUNDS): a failed check
+// raises kStBounds and the caller skips the access. Release builds compile
+// every check away.
+#ifdef PB_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok) {
+  if (!ok) raise_status(kStBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool) { return true; }
+#endif
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;

@@ -477,6 +477,7 @@ struct JetTiles {  // the pairs of one staged jet
     p = t * kTileM + r;
     if (p >= npairs) return false;
     pairs.map(p, a, b);
+    if (!in_bounds(a >= 0 && b >= 0 && a < P->m && b < P->m)) return false;
     pair_feat<PM, kFastLog>(*P, min(a, b), max(a, b), f);
     return true;
   }
@@ -636,6 +637,7 @@ struct GlobalUSink {
     const size_t plane = (size_t)P * P;
     const size_t base = (size_t)n * kH * plane;
     const int sa = S->slot[a], sb = S->slot[b];
+    if (!in_bounds(sa >= 0 && sb >= 0 && sa < P && sb < P)) return;
 #pragma unroll
     for (int h = 0; h < kH; ++h) {
       const size_t i0 = base + h * plane + (size_t)sa * P + sb;
@@ -696,6 +698,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_mlp_bias(JetArgs J, MlpArgs W, 
 // Element offset of (jet, head h, compact particle c) in Q/K/V/out.
 template <int PM>
 __device__ __forceinline__ size_t qkv_off(const Particles<PM>& S, const JetArgs& J, int n, int h, int c) {
+  if (!in_bounds(c >= 0 && c < S.m && h >= 0 && h < kH && n >= 0 && n < J.N)) return 0;
   if (J.ptr) return ((size_t)(S.base + c) * kH + h) * kD;
   return (((size_t)n * kH + h) * J.P + S.slot[c]) * kD;
 }
@@ -968,6 +971,7 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
   const int tiles = (nq + 15) >> 4;
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   uint16_t* buf = reinterpret_cast<uint16_t*>(stage);
+  if (!in_bounds(hb <= stage_floats * 4)) return;  // one head's K and V must fit
   for (int h0 = h_lo; h0 < h_hi; h0 += HR) {
     const int hr = min(HR, h_hi - h0);
     // the Q fragment of a warp's next item is loaded ahead: the first one
@@ -1075,7 +1079,9 @@ struct FusedLayout {
 
 struct SmemUSink {
   uint4* U8;
+  int cap;  // records the region holds
   __device__ __forceinline__ void operator()(int p, int, int, const float* u) const {
+    if (!in_bounds(p >= 0 && p < cap)) return;
     U8[p] = make_uint4(pack_half2(u[0], u[1]), pack_half2(u[2], u[3]), pack_half2(u[4], u[5]),
                        pack_half2(u[6], u[7]));
   }
@@ -1117,7 +1123,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
     prefetch_qkv<PM>(S.part, J, X, n);  // read by the attention after the MLP
     if (threadIdx.x == 32) prefetch_jet(J, n + gridDim.x);  // this CTA's next jet
     const int m = S.part.m;
-    SmemUSink sink{S.U8};
+    SmemUSink sink{S.U8, kUCap};
     if (m * (m + 1) / 2 <= kUCap) {
       const bool ok = mlp_pass<NG, SL>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, m * (m + 1) / 2, TriPairs{}}, sink, &phase);
       aborted = __syncthreads_or(!ok) != 0;
@@ -1213,6 +1219,7 @@ struct BatchTiles {
     const int pl = (B->t_lo[k] + bt - B->tbeg[k]) * kTileM + r;
     if (pl >= B->npairs[k]) return false;
     TriPairs{}.map(pl, a, b);
+    if (!in_bounds(a >= 0 && a <= b && b < ring[k].m)) return false;
     pair_feat<PM, true>(ring[k], min(a, b), max(a, b), f);
     p = (int)(B->rowbase[k] + pl);  // record index (fits: < 2^31 for N <= 8192, P <= 256)
     return true;
@@ -1221,7 +1228,9 @@ struct BatchTiles {
 
 struct RecordSink {  // the 8 biases of a pair as 8 f16 in one 16-byte record
   uint4* rec;
+  long long cap;  // records of this launch: 128 per MLP tile
   __device__ __forceinline__ void operator()(int p, int, int, const float* u) const {
+    if (!in_bounds(p >= 0 && p < cap)) return;
     rec[p] = make_uint4(pack_half2(u[0], u[1]), pack_half2(u[2], u[3]), pack_half2(u[4], u[5]),
                         pack_half2(u[6], u[7]));
   }
@@ -1410,7 +1419,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
       if (tid == 0)
         for (int k = 0; k < K; ++k) S.batch.npairs[k] = S.ring[k].m * (S.ring[k].m + 1) / 2;
       __syncthreads();
-      RecordSink sink{rec};
+      RecordSink sink{rec, Ttot * kTileM};
       const bool ok = mlp_pass<NG, SL>(S.mlp, BatchTiles<PM>{S.ring, &S.batch}, sink, &phase);
       aborted = __syncthreads_or(!ok) != 0;
       n = n_next;

@@ -60,6 +60,9 @@ class _MlpUnfolded(C.Structure):
                                           "W3", "b3", "a3", "c3", "W4", "b4")]
 
 
+DEBUG_LIB_PATH = os.path.join(_HERE, "libpairbias_debug.so")
+PB_DEV_BOUNDS = 4
+
 _lock = threading.Lock()
 _lib = None
 
@@ -69,33 +72,54 @@ def lib():
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build()")
-            L = C.CDLL(LIB_PATH)
-            vp = C.c_void_p
-            L.pairfeat_compute.argtypes = [C.POINTER(_Jets), vp, vp]
-            L.pairbias_mlp_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, vp]
-            L.pair_attention_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, C.c_int,
-                                                 vp, vp, vp, vp, vp, C.c_size_t, vp]
-            L.pair_attention_forward_noalloc.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.c_int, C.c_int,
-                                                         vp, vp, vp, vp, vp]
-            L.pair_block_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.POINTER(_Proj), C.c_int, C.c_int,
-                                             C.c_int, vp, vp, vp, C.c_size_t, vp]
-            L.pb_block_workspace_bytes.argtypes = [C.POINTER(_Jets)]
-            L.pb_block_workspace_bytes.restype = C.c_size_t
-            L.pb_workspace_bytes.argtypes = [C.POINTER(_Jets)]
-            L.pb_workspace_bytes.restype = C.c_size_t
-            L.pb_get_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
-            L.pb_fold_affine.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float)]
-            L.pb_last_error.restype = C.c_char_p
-            L.pb_version.restype = C.c_char_p
-            L.pb_selftest_wait_timeouts.argtypes = [vp]
-            for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward, L.pb_selftest_wait_timeouts,
-                      L.pair_attention_forward_noalloc, L.pair_block_forward, L.pb_get_device_status,
-                      L.pb_fold_affine):
-                f.restype = C.c_int
-            _lib = L
+            _lib = load(LIB_PATH)
         return _lib
+
+
+def use_library(path: str):
+    """Route every call of this module to the library at `path` (e.g. the
+    bounds-checking build); returns the previous one for restoring."""
+    global _lib
+    with _lock:
+        prev = _lib
+        _lib = load(path)
+        return prev
+
+
+def restore_library(prev) -> None:
+    global _lib
+    with _lock:
+        _lib = prev
+
+
+def load(path: str):
+    """Open one build of the library and declare its signatures."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with __graft_entry__.build()")
+    L = C.CDLL(path)
+    vp = C.c_void_p
+    L.pairfeat_compute.argtypes = [C.POINTER(_Jets), vp, vp]
+    L.pairbias_mlp_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, vp]
+    L.pair_attention_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), vp, C.c_int, C.c_int,
+                                         vp, vp, vp, vp, vp, C.c_size_t, vp]
+    L.pair_attention_forward_noalloc.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.c_int, C.c_int,
+                                                 vp, vp, vp, vp, vp]
+    L.pair_block_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.POINTER(_Proj), C.c_int, C.c_int,
+                                     C.c_int, vp, vp, vp, C.c_size_t, vp]
+    L.pb_block_workspace_bytes.argtypes = [C.POINTER(_Jets)]
+    L.pb_block_workspace_bytes.restype = C.c_size_t
+    L.pb_workspace_bytes.argtypes = [C.POINTER(_Jets)]
+    L.pb_workspace_bytes.restype = C.c_size_t
+    L.pb_get_device_status.argtypes = [vp, C.POINTER(C.c_uint32)]
+    L.pb_fold_affine.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float)]
+    L.pb_last_error.restype = C.c_char_p
+    L.pb_version.restype = C.c_char_p
+    L.pb_selftest_wait_timeouts.argtypes = [vp]
+    for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward, L.pb_selftest_wait_timeouts,
+              L.pair_attention_forward_noalloc, L.pair_block_forward, L.pb_get_device_status,
+              L.pb_fold_affine):
+        f.restype = C.c_int
+    return L
 
 
 def _check(st: int) -> None:

@@ -1,0 +1,69 @@
+"""The bounds-checking build (PB_DEBUG_BOUNDS) on the edge cases: every
+computed index it checks (pair unpacking, shared-memory bias slots, workspace
+records, global bias writes, Q/K/V/out offsets, the attention's staging)
+must stay in range, so no PB_DEV_BOUNDS bit may appear, and the results must
+still match the oracle. compute-sanitizer stands in for nothing here; this
+build records a failed check and skips the access instead of faulting."""
+import numpy as np
+import pytest
+import torch
+
+from part_pair_bias_b200 import build, ops, synth
+from tests import parity as pt
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _debug_library():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    torch.cuda.set_device(0)
+    build.build(debug=True)
+    prev = ops.use_library(ops.DEBUG_LIB_PATH)
+    assert ops.get_device_status() == 0
+    yield
+    ops.restore_library(prev)
+
+
+CASES = {
+    "odd_p_scrambled": dict(N=8, P=37, mults=[0, 1, 2, 37, 17, 36, 5, 33], mask_mode="scrambled", seed=3),
+    "wide_p256": dict(N=5, P=256, mults=[256, 200, 129, 128, 3], pt_lo=800, pt_hi=1000, prongs=3, seed=5),
+    "packed_empty": dict(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6),
+    "many_jets": dict(N=700, P=24, dist="uniform", mult_lo=1, mult_hi=24, mask_mode="scrambled", seed=8),
+    "tiny_p3": dict(N=8, P=3, mults=[0, 1, 3, 2, 2, 3, 0, 1], mask_mode="scrambled", seed=9),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_no_index_leaves_its_range(oracle_lib, case):
+    b = synth.make_jets(**CASES[case])
+    d = pt.Device(b)
+    pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
+    U = d.bias(torch.bfloat16)
+    ref_U = oracle_lib.pair_bias(b)
+    if b.layout == "padded":
+        pt.check_bias(pt.to_np(U), ref_U, b, bf16=True)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
+    if b.layout == "padded":
+        pt.check_attention(pt.to_np(d.with_bias(U)), ref, b)
+    bits = ops.get_device_status()
+    assert not bits & ops.PB_DEV_BOUNDS, f"a computed index left its range (status {bits:#x})"
+    assert bits == 0
+
+
+def test_block_path_indices(oracle_lib):
+    b = synth.make_jets(**CASES["odd_p_scrambled"])
+    bi = synth.make_block_inputs(b, 4)
+    d = pt.Device(b)
+    proj = ops.proj_to_device(bi)
+    x = ops.bf16_to_device(bi.x)
+    y = torch.full_like(x, float("nan"))
+    ws = torch.zeros(ops.block_workspace_bytes(d.jets), dtype=torch.uint8, device="cuda")
+    ops.pair_block_forward(d.jets, d.mlp, proj, x, y, ws)
+    assert ops.get_device_status() == 0
+    got, ref = pt.to_np(y), oracle_lib.block_forward(b, bi)
+    valid = b.mask.astype(bool)
+    assert np.linalg.norm(got[valid] - ref[valid]) / np.linalg.norm(ref[valid]) <= pt.ATT_RELL2
+    assert np.all(got[~valid] == 0.0)
