@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per (workload, path) with times, rates and FLOP conventions")
     return ap.parse_args()
 
 
@@ -373,9 +375,95 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ sweep
+
+def run_sweep(args):
+    """One JSON line per (workload, path): device time (median of 20 launches
+    after warm-up, L2 flushed before each), jets/s, valid ordered pairs/s,
+    algorithmic GB/s, the MLP's TFLOP/s under the three conventions (alg:
+    valid unordered pairs; exec: issued tile rows; dense: N P^2), and the
+    host oracle's rate on a bounded sample of the workload (first jets)."""
+    from part_pair_bias_b200 import ops
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    peak_tf, hbm_gbs, peak_src = measured_peaks()
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            fn()
+            s1.record()
+            torch.cuda.synchronize()
+            ts.append(s0.elapsed_time(s1))
+        return statistics.median(ts)
+
+    names = list(configs.ORDER) + ["n128_p128_full"]
+    for name in names:
+        if name == "n128_p128_full":
+            b = synth.make_jets(**configs.workload("n128_p128", seed=args.seed, dist="full"))
+        else:
+            b = synth.make_jets(**configs.workload(name, seed=args.seed))
+        unordered, tiles, ordered = pair_counts(b)
+        valid = int(b.mult.sum())
+        slots = b.N * b.P if b.layout == "padded" else valid
+        jets = ops.jets_to_device(b, dev)
+        mlp = ops.folded_mlp(b.params, dev)
+        q, k, v = (ops.bf16_to_device(x, dev) for x in (b.q, b.k, b.v))
+        out = torch.empty_like(q)
+        feat = torch.empty((b.N, b.P, b.P, 4), device=dev)
+        U = torch.empty((b.N, 8, b.P, b.P), device=dev, dtype=torch.bfloat16)
+        ws = ops.workspace_for(jets, dev)
+        bi = synth.make_block_inputs(b, args.seed)
+        proj = ops.proj_to_device(bi, dev)
+        x = ops.bf16_to_device(bi.x, dev)
+        y = torch.empty_like(x)
+        bws = torch.empty(ops.block_workspace_bytes(jets), dtype=torch.uint8, device=dev)
+        inp = 17 * slots                      # momenta + mask (or ptr) per slot
+        qkv = 3 * 256 * valid                 # Q, K, V rows of the valid particles
+        paths = [
+            ("features", lambda: ops.pairfeat_compute(jets, feat), inp + 16 * b.N * b.P * b.P, False),
+            ("bias_bf16", lambda: ops.pairbias_mlp_forward(jets, mlp, U), inp + 2 * 8 * b.N * b.P * b.P, True),
+            ("attention_reading_bias", lambda: ops.pair_attention_forward(jets, None, U, q, k, v, out),
+             inp + qkv + 2 * 8 * ordered + 256 * slots, False),
+            ("fused", lambda: ops.pair_attention_forward(jets, mlp, None, q, k, v, out), inp + qkv + 256 * slots, True),
+        ]
+        if ws is not None:
+            paths.append(("fused_balanced", lambda: ops.pair_attention_forward(jets, mlp, None, q, k, v, out,
+                                                                               workspace=ws),
+                          inp + qkv + 256 * slots, True))
+        paths.append(("block", lambda: ops.pair_block_forward(jets, mlp, proj, x, y, bws),
+                      inp + 256 * slots + 256 * slots, True))
+        for path, fn, nbytes, has_mlp in paths:
+            ms = timed(fn)
+            line = {"workload": name, "path": path, "seed": args.seed, "ms": ms, "jets_per_s": b.N / (ms / 1e3),
+                    "pairs_per_s": ordered / (ms / 1e3), "alg_gbs": nbytes / (ms / 1e3) / 1e9,
+                    "hbm_peak_gbs": hbm_gbs}
+            if has_mlp:
+                line.update({"tflops_alg": unordered * MLP_FLOP_PER_PAIR / (ms / 1e3) / 1e12,
+                             "tflops_exec": tiles * 128 * MMA_FLOP_PER_ROW / (ms / 1e3) / 1e12,
+                             "tflops_dense": b.N * b.P * b.P * MLP_FLOP_PER_PAIR / (ms / 1e3) / 1e12,
+                             "peak_tflops": peak_tf, "peak_source": peak_src})
+            print(json.dumps(line), flush=True)
+        if ops.get_device_status():
+            raise RuntimeError(f"device status set on {name}")
+        sample = synth.slice_jets(b, 0, min(b.N, 16))
+        cb = cpu_baseline(sample, args.cpu_seconds / 4)
+        print(json.dumps({"workload": name, "path": "oracle (host)", "seed": args.seed, "jets_per_s": cb["value"],
+                          "cores": cb["cores"], "sample": cb["sample"]}), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_env()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
     else:
