@@ -175,15 +175,16 @@ pb_status run_attn_bias(const pb::JetArgs& J, const pb::QkvArgs& X, const uint16
   return launched("k_attn_bias");
 }
 
-template <int PM>
-pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s) {
-  auto k = pb::k_fused<PM, kGroups>;
+template <int PM, bool kProj = false>
+pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s,
+                    const pb::ProjArgs& Pin = pb::ProjArgs{}, const pb::ProjArgs& Pout = pb::ProjArgs{}) {
+  auto k = pb::k_fused<PM, kGroups, kProj>;
   const size_t smem = sizeof(pb::FusedSmem<PM, kGroups>);
   int grid = 0;
   pb_status st = prepare(k, smem, kGroups * 128, J.N, &grid);
   if (st != PB_OK) return st;
-  k<<<grid, kGroups * 128, smem, s>>>(J, W, X);
-  return launched("k_fused");
+  k<<<grid, kGroups * 128, smem, s>>>(J, W, X, Pin, Pout);
+  return launched(kProj ? "k_fused (with projections)" : "k_fused");
 }
 
 constexpr long long kGridMaxMaskBytes = 1ll << 21;  // padded N*P scanned by every CTA in phase 0
@@ -386,11 +387,20 @@ pb_status pair_block_forward(const pb_jets* jets, const pb_mlp* mlp, const pb_pr
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (rows == 0) return PB_OK;  // packed jets that are all empty: nothing to read or write
   const pb::ProjArgs in{x, proj->Wqkv, proj->bqkv, q, k, v};
-  if ((st = run_proj<384, pb::kInRows, pb::kOutQKV>(J, in, s, "k_proj (in)")) != PB_OK) return st;
   const pb::QkvArgs X{q, k, v, o};
+  const pb::ProjArgs out{o, proj->Wo, proj->bo, y, nullptr, nullptr};
+  int dev = 0, sms = 0;
+  if ((st = device_sms(&dev, &sms)) != PB_OK) return st;
+  if (J.N <= sms) {
+    // at most one jet per CTA: the projections run inside the fused kernel,
+    // jet by jet, with Q, K, V and O kept in the (L2-resident) workspace
+    return J.P <= 128 ? run_fused<128, true>(J, W, X, s, in, out) : run_fused<256, true>(J, W, X, s, in, out);
+  }
+  // many jets per CTA: per-jet projection latency would add up, so the two
+  // projections run as GEMM kernels over all rows around the fused attention
+  if ((st = run_proj<384, pb::kInRows, pb::kOutQKV>(J, in, s, "k_proj (in)")) != PB_OK) return st;
   st = J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
   if (st != PB_OK) return st;
-  const pb::ProjArgs out{o, proj->Wo, proj->bo, y, nullptr, nullptr};
   return run_proj<128, pb::kInHeads, pb::kOutRows>(J, out, s, "k_proj (out)");
 }
 

@@ -1055,6 +1055,440 @@ __global__ void __launch_bounds__(256) k_attn_bias(JetArgs J, QkvArgs X, const u
   }
 }
 
+// ============================================ k_proj (projections either side)
+//
+// The in-projection of a ParT attention block (x -> Q, K, V) and its output
+// projection (O -> y) as one tensor-core GEMM kernel over particle rows:
+// out[r, :] = W in[r, :] + b for every row r of the padded slots (N * P) or
+// the packed tokens, with E = 128 input features. The whole weight matrix
+// (kNout x 128 bf16) stays in shared memory in the K-major layout of the MMA
+// operands; each CTA streams 128-row tiles of the input through a double
+// buffer, one thread issues 8 K steps x kNout/128 tcgen05 MMAs (bf16
+// operands, fp32 accumulation in TMEM), and 8 warps read the accumulator
+// back (TMEM lane = row), add the bias and store bf16.
+
+constexpr int kEmbed = kH * kD;  // 128
+
+enum ProjIn { kInRows = 0, kInHeads = 1 };     // [rows, 128] | attention layout [N, H, P, D]
+enum ProjOut { kOutQKV = 0, kOutRows = 1 };    // Q, K, V in attention layout | [rows, 128]
+
+struct ProjArgs {
+  const uint16_t* in;   // kInRows: x [rows, 128]; kInHeads: O in the layout of Q
+  const uint16_t* W;    // [kNout, 128] bf16, row-major (out x in)
+  const float* bias;    // [kNout]
+  uint16_t* out0;       // kOutQKV: Q; kOutRows: y [rows, 128]
+  uint16_t* out1;       // kOutQKV: K
+  uint16_t* out2;       // kOutQKV: V
+};
+
+template <int kNout>
+struct ProjSmem {
+  __nv_bfloat16 W[kNout * kEmbed];      // B operand, K-major, 8-row groups of 2,048 B
+  __nv_bfloat16 A[2][kTileM * kEmbed];  // A operand double buffer
+  float bias[kNout];
+  uint64_t mbar;
+  uint32_t tmem_base;
+};
+
+__host__ __device__ constexpr uint32_t proj_tmem_cols(int nout) { return nout <= 128 ? 128u : (nout <= 256 ? 256u : 512u); }
+
+// Rows of the GEMM: N * P padded slots or the packed tokens.
+__device__ __forceinline__ long long proj_rows(const JetArgs& J) { return J.ptr ? J.tokens : (long long)J.N * J.P; }
+
+// Row r of the output written? (the in-projection skips masked slots, whose
+// Q/K/V are never read; the out-projection writes 0 there)
+__device__ __forceinline__ bool proj_row_valid(const JetArgs& J, long long r) { return J.ptr || J.mask[r] != 0; }
+
+// Input tile t (rows t*128 ..): 128 rows x 16 chunks of 8 bf16, loaded into
+// eight registers per thread (rows past the end are zero), then stored to
+// A in the operand layout. Block-wide (256 threads); no barrier.
+constexpr int kTileChunksPerThread = kTileM * (kEmbed / 8) / 256;  // 8
+
+// Chunk idx of a [rows][16 chunks] operand -> (row, chunk). A warp takes 8
+// rows x 4 chunks: the 16-byte bank group of a chunk in the operand layout
+// is its row mod 8, so each quarter-warp stores to 8 distinct bank groups,
+// and the warp still reads whole 32-byte sectors of every row.
+__device__ __forceinline__ void chunk_rc(int idx, int& r, int& kc) {
+  const int w = idx >> 5, l = idx & 31;
+  r = (w >> 2) * 8 + (l & 7);
+  kc = (w & 3) * 4 + (l >> 3);
+}
+
+template <int kIn>
+__device__ __forceinline__ void proj_fetch_tile(uint4* v, const JetArgs& J, const ProjArgs& X, long long t,
+                                                long long R) {
+#pragma unroll
+  for (int u = 0; u < kTileChunksPerThread; ++u) {
+    int rr, kc;
+    chunk_rc(threadIdx.x + u * 256, rr, kc);
+    const long long r = t * kTileM + rr;
+    v[u] = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const uint16_t* src;
+      if (kIn == kInRows || J.ptr) {
+        src = X.in + r * kEmbed + kc * 8;
+      } else {  // O[n, h, slot, d] with column kc * 8 = h * 16 + (kc & 1) * 8
+        const long long n = r / J.P, slot = r % J.P;
+        src = X.in + ((n * kH + (kc >> 1)) * J.P + slot) * kD + (kc & 1) * 8;
+      }
+      v[u] = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+}
+
+__device__ __forceinline__ void proj_store_tile(__nv_bfloat16* A, const uint4* v) {
+#pragma unroll
+  for (int u = 0; u < kTileChunksPerThread; ++u) {
+    int rr, kc;
+    chunk_rc(threadIdx.x + u * 256, rr, kc);
+    *reinterpret_cast<uint4*>(A + cofs(rr, kc * 8, kEmbed)) = v[u];
+  }
+}
+
+template <int kIn>
+__device__ __forceinline__ void proj_load_tile(__nv_bfloat16* A, const JetArgs& J, const ProjArgs& X, long long t,
+                                               long long R) {
+  uint4 v[kTileChunksPerThread];
+  proj_fetch_tile<kIn>(v, J, X, t, R);
+  proj_store_tile(A, v);
+}
+
+template <int kNout, int kIn, int kOut>
+__global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  ProjSmem<kNout>& S = *reinterpret_cast<ProjSmem<kNout>*>(smem_raw);
+  constexpr uint32_t kCols = proj_tmem_cols(kNout);
+  constexpr uint32_t kIdesc = idesc_bf16_m128(128);
+  constexpr uint32_t kSBO = kEmbed / 8 * 128;  // 2,048 B between 8-row groups
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long R = proj_rows(J);
+  const long long ntiles = (R + kTileM - 1) / kTileM;
+
+  // the first input tile and the weights (K-major), once per CTA, with
+  // sixteen 16-byte loads per thread in flight before their stores
+  long long t = blockIdx.x;
+  {
+    uint4 a[kTileChunksPerThread];
+    if (t < ntiles) proj_fetch_tile<kIn>(a, J, X, t, R);
+    constexpr int kW = kNout * (kEmbed / 8) / 256;  // weight chunks per thread: 24 or 8
+    static_assert(kNout * (kEmbed / 8) % 256 == 0, "whole weight chunks per thread");
+#pragma unroll
+    for (int b0 = 0; b0 < kW; b0 += 16) {
+      uint4 w[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        int n, kc;
+        chunk_rc(tid + (b0 + u) * 256, n, kc);
+        if (b0 + u < kW) w[u] = *reinterpret_cast<const uint4*>(X.W + (size_t)n * kEmbed + kc * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        int n, kc;
+        chunk_rc(tid + (b0 + u) * 256, n, kc);
+        if (b0 + u < kW) *reinterpret_cast<uint4*>(S.W + cofs(n, kc * 8, kEmbed)) = w[u];
+      }
+    }
+    if (t < ntiles) proj_store_tile(S.A[0], a);
+  }
+  for (int i = tid; i < kNout; i += blockDim.x) S.bias[i] = X.bias[i];
+  if (tid == 0) {
+    mbar_init(&S.mbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  uint32_t phase = 0;
+  bool ok = true;
+  int buf = 0;
+  for (; t < ntiles; t += gridDim.x, buf ^= 1) {
+    if (tid == 0) {
+      const uint32_t a0 = smem_u32(S.A[buf]), w0 = smem_u32(S.W);
+#pragma unroll 1
+      for (int c = 0; c < kNout / 128; ++c)
+#pragma unroll
+        for (int s = 0; s < kEmbed / 16; ++s)
+          mma_f16(tmem + 128u * c, smem_desc(a0 + 256u * s, 128, kSBO),
+                  smem_desc(w0 + (uint32_t)c * 128u * kSBO / 8u + 256u * s, 128, kSBO), kIdesc, s > 0 ? 1u : 0u);
+      mma_commit(&S.mbar);
+    }
+    // the next tile loads while the MMAs run
+    if (t + gridDim.x < ntiles) proj_load_tile<kIn>(S.A[buf ^ 1], J, X, t + gridDim.x, R);
+    const bool done = mbar_wait(&S.mbar, phase);
+    if (done) phase ^= 1u;  // on a timeout the teardown waits on the same phase once more
+    ok = __syncthreads_and(done && ok) != 0;
+    tc_fence_after();
+    if (!ok) break;
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. and half w / 4 of the columns
+    {
+      const int rr = (warp & 3) * 32 + lane;
+      const long long r = t * kTileM + rr;
+      const bool in_range = r < R;
+      const bool valid = in_range && proj_row_valid(J, r);
+      const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      constexpr int kHalf = kNout / 2;
+#pragma unroll 1
+      for (int c64 = (warp >> 2) * kHalf; c64 < (warp >> 2) * kHalf + kHalf; c64 += 64) {
+        float v64[64];
+        tmem_ld64_wait(lane_base + (uint32_t)c64, v64);  // warp-wide: every lane, in range or not
+#pragma unroll
+       for (int half = 0; half < 2; ++half) {
+        const int c0 = c64 + 32 * half;
+        const float* v = v64 + 32 * half;
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = valid ? cvt_bf16x2(v[2 * i] + S.bias[c0 + 2 * i], v[2 * i + 1] + S.bias[c0 + 2 * i + 1]) : 0u;
+        if (kOut == kOutRows && in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(X.out0 + r * kEmbed + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        } else if (kOut == kOutQKV && valid) {
+          // columns c0 .. c0 + 31: two heads of one of Q, K, V
+          const int tensor = c0 / kEmbed, cc = c0 % kEmbed;
+          uint16_t* base = tensor == 0 ? X.out0 : (tensor == 1 ? X.out1 : X.out2);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int h = cc / kD + hh;
+            size_t off;
+            if (J.ptr) off = ((size_t)r * kH + h) * kD;
+            else off = (((size_t)(r / J.P) * kH + h) * J.P + (size_t)(r % J.P)) * kD;
+            uint4* dst = reinterpret_cast<uint4*>(base + off);
+            dst[0] = make_uint4(w[8 * hh], w[8 * hh + 1], w[8 * hh + 2], w[8 * hh + 3]);
+            dst[1] = make_uint4(w[8 * hh + 4], w[8 * hh + 5], w[8 * hh + 6], w[8 * hh + 7]);
+          }
+        }
+       }
+      }
+    }
+    // TMEM is read and the next A tile written before the next MMAs
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (!ok && tid == 0) raise_status(kStTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (!ok) {
+    // an MMA may still be in flight: wait once more (bounded) before freeing TMEM
+    if (tid == 0) (void)mbar_wait(&S.mbar, phase);
+    __syncthreads();
+  }
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kCols);
+}
+
+
+// ------------------------------------- per-jet projections inside k_fused
+//
+// With the projections fused, k_fused maps each jet's particle embeddings x
+// to Q, K, V before its MLP and its attention output O to y after it, on
+// the tensor cores, in the free activation tiles: a 128-row tile of input
+// rows and one 128-row chunk of the weights at a time (64 KB), 8 K steps of
+// M = 128, N = 128 into TMEM columns 0..127, then all 16 warps store the
+// chunk's 128 columns (bias added, bf16) for the valid rows. Q, K, V and O
+// live in the caller's workspace, in L2 for batches up to ~100 MB of them.
+
+// 128 rows of `in` from row r0 (rows >= r_end zero) into A, K-major operand
+// layout; 4 loads in flight per thread. Block-wide, no barrier.
+template <int kIn>
+__device__ void proj_stage_rows(__nv_bfloat16* A, const JetArgs& J, const uint16_t* in, long long r0,
+                                long long r_end) {
+  const int nthr = blockDim.x;
+  for (int base = threadIdx.x; base < kTileM * (kEmbed / 8); base += 4 * nthr) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (idx < kTileM * (kEmbed / 8)) {
+        int rr, kc;
+        chunk_rc(idx, rr, kc);
+        const long long r = r0 + rr;
+        if (r < r_end) {
+          const uint16_t* src;
+          if (kIn == kInRows || J.ptr) {
+            src = in + r * kEmbed + kc * 8;
+          } else {
+            const long long n = r / J.P, slot = r % J.P;
+            src = in + ((n * kH + (kc >> 1)) * J.P + slot) * kD + (kc & 1) * 8;
+          }
+          v[u] = *reinterpret_cast<const uint4*>(src);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      if (idx < kTileM * (kEmbed / 8)) {
+        int rr, kc;
+        chunk_rc(idx, rr, kc);
+        *reinterpret_cast<uint4*>(A + cofs(rr, kc * 8, kEmbed)) = v[u];
+      }
+    }
+  }
+}
+
+// Rows c*128 .. c*128+127 of a row-major [.][128] bf16 weight into Wsm.
+__device__ void proj_stage_w(__nv_bfloat16* Wsm, const uint16_t* W, int c) {
+  const int nthr = blockDim.x;
+  for (int base = threadIdx.x; base < kTileM * (kEmbed / 8); base += 4 * nthr) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      int n, kc;
+      chunk_rc(idx, n, kc);
+      if (idx < kTileM * (kEmbed / 8))
+        v[u] = *reinterpret_cast<const uint4*>(W + ((size_t)c * kTileM + n) * kEmbed + kc * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      int n, kc;
+      chunk_rc(idx, n, kc);
+      if (idx < kTileM * (kEmbed / 8)) *reinterpret_cast<uint4*>(Wsm + cofs(n, kc * 8, kEmbed)) = v[u];
+    }
+  }
+}
+
+// One row tile (rows r0 .., rows >= r_end zero) into A and weight chunks
+// 0 .. NW-1 (rows 128 c ..) into Wsm + c * 128 * 128, with every load of a
+// thread in flight before its stores (512 threads: 4 chunks per operand).
+// Block-wide, no barrier.
+template <int kIn, int NW>
+__device__ void proj_stage_tile_and_weights(__nv_bfloat16* A, __nv_bfloat16* Wsm, const JetArgs& J,
+                                            const uint16_t* in, long long r0, long long r_end, const uint16_t* W) {
+  constexpr int kChunks = kTileM * (kEmbed / 8);  // 2048 per operand
+  constexpr int kPer = kChunks / 512;             // 4
+  uint4 v[(1 + NW) * kPer];
+#pragma unroll
+  for (int o = 0; o <= NW; ++o)
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      int rr, kc;
+      chunk_rc(threadIdx.x + u * 512, rr, kc);
+      uint4 x = make_uint4(0, 0, 0, 0);
+      if (o == 0) {
+        const long long r = r0 + rr;
+        if (r < r_end) {
+          const uint16_t* src;
+          if (kIn == kInRows || J.ptr) {
+            src = in + r * kEmbed + kc * 8;
+          } else {
+            const long long n = r / J.P, slot = r % J.P;
+            src = in + ((n * kH + (kc >> 1)) * J.P + slot) * kD + (kc & 1) * 8;
+          }
+          x = *reinterpret_cast<const uint4*>(src);
+        }
+      } else {
+        x = *reinterpret_cast<const uint4*>(W + ((size_t)(o - 1) * kTileM + rr) * kEmbed + kc * 8);
+      }
+      v[o * kPer + u] = x;
+    }
+#pragma unroll
+  for (int o = 0; o <= NW; ++o)
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      int rr, kc;
+      chunk_rc(threadIdx.x + u * 512, rr, kc);
+      __nv_bfloat16* dst = o == 0 ? A : Wsm + (size_t)(o - 1) * kTileM * kEmbed;
+      *reinterpret_cast<uint4*>(dst + cofs(rr, kc * 8, kEmbed)) = v[o * kPer + u];
+    }
+}
+
+// NW products of A with weight chunks Wsm + c * 128 * 128 into TMEM columns
+// tmem + 128 c, one commit and one wait. Block-wide; false if the wait ran out.
+template <int NW>
+__device__ bool proj_mma_n(__nv_bfloat16* A, __nv_bfloat16* Wsm, uint32_t tmem, uint64_t* mbar, uint32_t* phase) {
+  constexpr uint32_t kSBO = kEmbed / 8 * 128;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) {
+    const uint32_t a0 = smem_u32(A), w0 = smem_u32(Wsm);
+#pragma unroll
+    for (int c = 0; c < NW; ++c)
+#pragma unroll
+      for (int s = 0; s < kEmbed / 16; ++s)
+        mma_f16(tmem + 128u * c, smem_desc(a0 + 256u * s, 128, kSBO),
+                smem_desc(w0 + (uint32_t)c * kTileM * kEmbed * 2u + 256u * s, 128, kSBO), idesc_bf16_m128(128),
+                s > 0 ? 1u : 0u);
+    mma_commit(mbar);
+  }
+  const bool done = mbar_wait(mbar, *phase & 1u);
+  if (done) *phase ^= 1u;
+  tc_fence_after();
+  return __syncthreads_and(done) != 0;
+}
+
+// One 128 x 128 x 128 product into TMEM columns tmem .. tmem+127 and its
+// wait: the operands were written by the block (generic proxy) before the
+// call. Block-wide; returns false if the wait ran out.
+__device__ bool proj_mma(__nv_bfloat16* A, __nv_bfloat16* Wsm, uint32_t tmem, uint64_t* mbar, uint32_t* phase) {
+  constexpr uint32_t kSBO = kEmbed / 8 * 128;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) {
+    const uint32_t a0 = smem_u32(A), w0 = smem_u32(Wsm);
+#pragma unroll
+    for (int s = 0; s < kEmbed / 16; ++s)
+      mma_f16(tmem, smem_desc(a0 + 256u * s, 128, kSBO), smem_desc(w0 + 256u * s, 128, kSBO),
+              idesc_bf16_m128(128), s > 0 ? 1u : 0u);
+    mma_commit(mbar);
+  }
+  const bool done = mbar_wait(mbar, *phase & 1u);
+  if (done) *phase ^= 1u;
+  tc_fence_after();
+  return __syncthreads_and(done) != 0;
+}
+
+// The 128 accumulator columns of rows r0 .. r0+127 (rows >= r_end skipped):
+// + bias, bf16, stored for valid rows either as tensor `tensor` (0 Q, 1 K,
+// 2 V) of the attention layout (kOutQKV, masked slots skipped) or as y rows
+// (kOutRows, masked slots written 0). 16 warps: warp w reads TMEM lanes
+// 32 (w % 4) and columns 32 (w / 4) ..
+template <int kOut>
+__device__ void proj_store(uint32_t tmem, const float* bias, const JetArgs& J, long long r0, long long r_end,
+                           uint16_t* out, int tensor) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rr = (warp & 3) * 32 + lane, c0 = (warp >> 2) * 32;
+  const long long r = r0 + rr;
+  float v[32];
+  tmem_ld32_wait(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c0, v);  // every lane of the warp
+  if (r >= r_end) return;
+  const bool valid = J.ptr || J.mask[r] != 0;
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    w[i] = valid ? cvt_bf16x2(v[2 * i] + __ldg(bias + tensor * kEmbed + c0 + 2 * i),
+                              v[2 * i + 1] + __ldg(bias + tensor * kEmbed + c0 + 2 * i + 1))
+                 : 0u;
+  if (kOut == kOutRows) {
+    uint4* dst = reinterpret_cast<uint4*>(out + r * kEmbed + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  } else if (valid) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = c0 / kD + hh;
+      size_t off;
+      if (J.ptr) off = ((size_t)r * kH + h) * kD;
+      else off = (((size_t)(r / J.P) * kH + h) * J.P + (size_t)(r % J.P)) * kD;
+      uint4* dst = reinterpret_cast<uint4*>(out + off);
+      dst[0] = make_uint4(w[8 * hh], w[8 * hh + 1], w[8 * hh + 2], w[8 * hh + 3]);
+      dst[1] = make_uint4(w[8 * hh + 4], w[8 * hh + 5], w[8 * hh + 6], w[8 * hh + 7]);
+    }
+  }
+}
+
 // ======================================================= k_fused (one pass)
 
 // The bias of the jet's pairs lives in shared memory as 8 f16 (one per head)
@@ -1103,25 +1537,76 @@ struct FusedSmem {
   MlpSmem<NG, FusedLayout<PM, NG>::kSL> mlp;
   Particles<PM> part;
   uint4 U8[FusedLayout<PM, NG>::kUCap];
+  uint64_t proj_mbar;  // completion of the projections' MMAs (kProj)
 };
 
-template <int PM, int NG>
-__global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, QkvArgs X) {
+// kProj: the jet's Q, K, V (X.q/k/v) are first computed from its embeddings
+// (Pin: x, Wqkv, bqkv) and its output O (X.out) is finally projected to y
+// (Pout: O, Wo, bo); see "per-jet projections inside k_fused" above.
+template <int PM, int NG, bool kProj>
+__global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, QkvArgs X, ProjArgs Pin,
+                                                       ProjArgs Pout) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FusedSmem<PM, NG>& S = *reinterpret_cast<FusedSmem<PM, NG>*>(smem_raw);
   constexpr int SL = FusedLayout<PM, NG>::kSL;
-  if (threadIdx.x == 0) prefetch_jet(J, blockIdx.x);  // overlaps the weight loads
+  if (threadIdx.x == 0) {
+    prefetch_jet(J, blockIdx.x);  // overlaps the weight loads
+    if (kProj) {
+      mbar_init(&S.proj_mbar, 1);
+      fence_mbar_init();  // made visible by the barrier at the end of mlp_setup
+    }
+  }
   mlp_setup<NG, SL>(S.mlp, W);
   // during attention the activation tiles hold K and V
   float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
   constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
   constexpr int kUCap = FusedLayout<PM, NG>::kUCap;
-  uint32_t phase = 0u;
-  bool aborted = false;
+  uint32_t phase = 0u, pphase = 0u;
+  bool aborted = false, proj_stuck = false;
+  __nv_bfloat16* const PA = reinterpret_cast<__nv_bfloat16*>(stage);  // projection operands: rows,
+  __nv_bfloat16* const PW = PA + kTileM * kEmbed;                     // then one weight chunk
   for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
     stage_jet<PM>(S.part, J, n);
-    prefetch_qkv<PM>(S.part, J, X, n);  // read by the attention after the MLP
     if (threadIdx.x == 32) prefetch_jet(J, n + gridDim.x);  // this CTA's next jet
+    // the jet's rows: padded slots n*P .. n*P+P-1, or its packed tokens
+    const long long r_lo = J.ptr ? S.part.base : (long long)n * J.P;
+    const long long r_hi = J.ptr ? r_lo + S.part.m : r_lo + J.P;
+    if (kProj) {
+      // Q, K, V of the jet's valid rows, one 128-row tile and one of the three weight chunks at a time
+      for (long long r0 = r_lo; r0 < r_hi && !aborted; r0 += kTileM) {
+        if (kStageFloats * 4 >= 4 * kTileM * kEmbed * 2) {
+          // the stage holds the row tile and all three weight chunks: one round of loads, one wait
+          proj_stage_tile_and_weights<kInRows, 3>(PA, PW, J, Pin.in, r0, r_hi, Pin.W);
+          if (!proj_mma_n<3>(PA, PW, S.mlp.tmem_base, &S.proj_mbar, &pphase)) {
+            aborted = proj_stuck = true;
+            break;
+          }
+#pragma unroll 1
+          for (int c = 0; c < 3; ++c)
+            proj_store<kOutQKV>(S.mlp.tmem_base + 128u * c, Pin.bias, J, r0, r_hi,
+                                c == 0 ? Pin.out0 : (c == 1 ? Pin.out1 : Pin.out2), c);
+          tc_fence_before();
+          __syncthreads();
+          tc_fence_after();
+          continue;
+        }
+        proj_stage_rows<kInRows>(PA, J, Pin.in, r0, r_hi);
+        for (int c = 0; c < 3; ++c) {
+          proj_stage_w(PW, Pin.W, c);
+          if (!proj_mma(PA, PW, S.mlp.tmem_base, &S.proj_mbar, &pphase)) {
+            aborted = proj_stuck = true;
+            break;
+          }
+          proj_store<kOutQKV>(S.mlp.tmem_base, Pin.bias, J, r0, r_hi, c == 0 ? Pin.out0 : (c == 1 ? Pin.out1 : Pin.out2), c);
+          tc_fence_before();  // TMEM read and the weight chunk consumed before the next one
+          __syncthreads();
+          tc_fence_after();
+        }
+      }
+      if (aborted) break;
+    } else {
+      prefetch_qkv<PM>(S.part, J, X, n);  // read by the attention after the MLP
+    }
     const int m = S.part.m;
     SmemUSink sink{S.U8, kUCap};
     if (m * (m + 1) / 2 <= kUCap) {
@@ -1144,7 +1629,22 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
     }
     zero_masked_rows<PM>(S.part, J, X.out, n);
     __syncthreads();
+    if (kProj) {
+      // y = O Wo^T + bo for the jet's rows (masked slots 0)
+      for (long long r0 = r_lo; r0 < r_hi && !aborted; r0 += kTileM) {
+        proj_stage_tile_and_weights<kInHeads, 1>(PA, PW, J, X.out, r0, r_hi, Pout.W);
+        if (!proj_mma_n<1>(PA, PW, S.mlp.tmem_base, &S.proj_mbar, &pphase)) {
+          aborted = proj_stuck = true;
+          break;
+        }
+        proj_store<kOutRows>(S.mlp.tmem_base, Pout.bias, J, r0, r_hi, Pout.out0, 0);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+      }
+    }
   }
+  if (kProj && proj_stuck && threadIdx.x == 0) (void)mbar_wait(&S.proj_mbar, pphase & 1u);  // bounded, before TMEM is freed
   mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
 }
 
@@ -1573,234 +2073,6 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
     rows = alt < rows ? alt : rows;
   }
   return kWsHeader + (size_t)rows * 16;
-}
-
-
-// ============================================ k_proj (projections either side)
-//
-// The in-projection of a ParT attention block (x -> Q, K, V) and its output
-// projection (O -> y) as one tensor-core GEMM kernel over particle rows:
-// out[r, :] = W in[r, :] + b for every row r of the padded slots (N * P) or
-// the packed tokens, with E = 128 input features. The whole weight matrix
-// (kNout x 128 bf16) stays in shared memory in the K-major layout of the MMA
-// operands; each CTA streams 128-row tiles of the input through a double
-// buffer, one thread issues 8 K steps x kNout/128 tcgen05 MMAs (bf16
-// operands, fp32 accumulation in TMEM), and 8 warps read the accumulator
-// back (TMEM lane = row), add the bias and store bf16.
-
-constexpr int kEmbed = kH * kD;  // 128
-
-enum ProjIn { kInRows = 0, kInHeads = 1 };     // [rows, 128] | attention layout [N, H, P, D]
-enum ProjOut { kOutQKV = 0, kOutRows = 1 };    // Q, K, V in attention layout | [rows, 128]
-
-struct ProjArgs {
-  const uint16_t* in;   // kInRows: x [rows, 128]; kInHeads: O in the layout of Q
-  const uint16_t* W;    // [kNout, 128] bf16, row-major (out x in)
-  const float* bias;    // [kNout]
-  uint16_t* out0;       // kOutQKV: Q; kOutRows: y [rows, 128]
-  uint16_t* out1;       // kOutQKV: K
-  uint16_t* out2;       // kOutQKV: V
-};
-
-template <int kNout>
-struct ProjSmem {
-  __nv_bfloat16 W[kNout * kEmbed];      // B operand, K-major, 8-row groups of 2,048 B
-  __nv_bfloat16 A[2][kTileM * kEmbed];  // A operand double buffer
-  float bias[kNout];
-  uint64_t mbar;
-  uint32_t tmem_base;
-};
-
-__host__ __device__ constexpr uint32_t proj_tmem_cols(int nout) { return nout <= 128 ? 128u : (nout <= 256 ? 256u : 512u); }
-
-// Rows of the GEMM: N * P padded slots or the packed tokens.
-__device__ __forceinline__ long long proj_rows(const JetArgs& J) { return J.ptr ? J.tokens : (long long)J.N * J.P; }
-
-// Row r of the output written? (the in-projection skips masked slots, whose
-// Q/K/V are never read; the out-projection writes 0 there)
-__device__ __forceinline__ bool proj_row_valid(const JetArgs& J, long long r) { return J.ptr || J.mask[r] != 0; }
-
-// Input tile t (rows t*128 ..): 128 rows x 16 chunks of 8 bf16, loaded into
-// eight registers per thread (rows past the end are zero), then stored to
-// A in the operand layout. Block-wide (256 threads); no barrier.
-constexpr int kTileChunksPerThread = kTileM * (kEmbed / 8) / 256;  // 8
-
-// Chunk idx of a [rows][16 chunks] operand -> (row, chunk). A warp takes 8
-// rows x 4 chunks: the 16-byte bank group of a chunk in the operand layout
-// is its row mod 8, so each quarter-warp stores to 8 distinct bank groups,
-// and the warp still reads whole 32-byte sectors of every row.
-__device__ __forceinline__ void chunk_rc(int idx, int& r, int& kc) {
-  const int w = idx >> 5, l = idx & 31;
-  r = (w >> 2) * 8 + (l & 7);
-  kc = (w & 3) * 4 + (l >> 3);
-}
-
-template <int kIn>
-__device__ __forceinline__ void proj_fetch_tile(uint4* v, const JetArgs& J, const ProjArgs& X, long long t,
-                                                long long R) {
-#pragma unroll
-  for (int u = 0; u < kTileChunksPerThread; ++u) {
-    int rr, kc;
-    chunk_rc(threadIdx.x + u * 256, rr, kc);
-    const long long r = t * kTileM + rr;
-    v[u] = make_uint4(0, 0, 0, 0);
-    if (r < R) {
-      const uint16_t* src;
-      if (kIn == kInRows || J.ptr) {
-        src = X.in + r * kEmbed + kc * 8;
-      } else {  // O[n, h, slot, d] with column kc * 8 = h * 16 + (kc & 1) * 8
-        const long long n = r / J.P, slot = r % J.P;
-        src = X.in + ((n * kH + (kc >> 1)) * J.P + slot) * kD + (kc & 1) * 8;
-      }
-      v[u] = *reinterpret_cast<const uint4*>(src);
-    }
-  }
-}
-
-__device__ __forceinline__ void proj_store_tile(__nv_bfloat16* A, const uint4* v) {
-#pragma unroll
-  for (int u = 0; u < kTileChunksPerThread; ++u) {
-    int rr, kc;
-    chunk_rc(threadIdx.x + u * 256, rr, kc);
-    *reinterpret_cast<uint4*>(A + cofs(rr, kc * 8, kEmbed)) = v[u];
-  }
-}
-
-template <int kIn>
-__device__ __forceinline__ void proj_load_tile(__nv_bfloat16* A, const JetArgs& J, const ProjArgs& X, long long t,
-                                               long long R) {
-  uint4 v[kTileChunksPerThread];
-  proj_fetch_tile<kIn>(v, J, X, t, R);
-  proj_store_tile(A, v);
-}
-
-template <int kNout, int kIn, int kOut>
-__global__ void __launch_bounds__(256, 1) k_proj(JetArgs J, ProjArgs X) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  ProjSmem<kNout>& S = *reinterpret_cast<ProjSmem<kNout>*>(smem_raw);
-  constexpr uint32_t kCols = proj_tmem_cols(kNout);
-  constexpr uint32_t kIdesc = idesc_bf16_m128(128);
-  constexpr uint32_t kSBO = kEmbed / 8 * 128;  // 2,048 B between 8-row groups
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long R = proj_rows(J);
-  const long long ntiles = (R + kTileM - 1) / kTileM;
-
-  // the first input tile and the weights (K-major), once per CTA, with
-  // sixteen 16-byte loads per thread in flight before their stores
-  long long t = blockIdx.x;
-  {
-    uint4 a[kTileChunksPerThread];
-    if (t < ntiles) proj_fetch_tile<kIn>(a, J, X, t, R);
-    constexpr int kW = kNout * (kEmbed / 8) / 256;  // weight chunks per thread: 24 or 8
-    static_assert(kNout * (kEmbed / 8) % 256 == 0, "whole weight chunks per thread");
-#pragma unroll
-    for (int b0 = 0; b0 < kW; b0 += 16) {
-      uint4 w[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        int n, kc;
-        chunk_rc(tid + (b0 + u) * 256, n, kc);
-        if (b0 + u < kW) w[u] = *reinterpret_cast<const uint4*>(X.W + (size_t)n * kEmbed + kc * 8);
-      }
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        int n, kc;
-        chunk_rc(tid + (b0 + u) * 256, n, kc);
-        if (b0 + u < kW) *reinterpret_cast<uint4*>(S.W + cofs(n, kc * 8, kEmbed)) = w[u];
-      }
-    }
-    if (t < ntiles) proj_store_tile(S.A[0], a);
-  }
-  for (int i = tid; i < kNout; i += blockDim.x) S.bias[i] = X.bias[i];
-  if (tid == 0) {
-    mbar_init(&S.mbar, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(&S.tmem_base, kCols);
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
-  uint32_t phase = 0;
-  bool ok = true;
-  int buf = 0;
-  for (; t < ntiles; t += gridDim.x, buf ^= 1) {
-    if (tid == 0) {
-      const uint32_t a0 = smem_u32(S.A[buf]), w0 = smem_u32(S.W);
-#pragma unroll 1
-      for (int c = 0; c < kNout / 128; ++c)
-#pragma unroll
-        for (int s = 0; s < kEmbed / 16; ++s)
-          mma_f16(tmem + 128u * c, smem_desc(a0 + 256u * s, 128, kSBO),
-                  smem_desc(w0 + (uint32_t)c * 128u * kSBO / 8u + 256u * s, 128, kSBO), kIdesc, s > 0 ? 1u : 0u);
-      mma_commit(&S.mbar);
-    }
-    // the next tile loads while the MMAs run
-    if (t + gridDim.x < ntiles) proj_load_tile<kIn>(S.A[buf ^ 1], J, X, t + gridDim.x, R);
-    const bool done = mbar_wait(&S.mbar, phase);
-    if (done) phase ^= 1u;  // on a timeout the teardown waits on the same phase once more
-    ok = __syncthreads_and(done && ok) != 0;
-    tc_fence_after();
-    if (!ok) break;
-    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. and half w / 4 of the columns
-    {
-      const int rr = (warp & 3) * 32 + lane;
-      const long long r = t * kTileM + rr;
-      const bool in_range = r < R;
-      const bool valid = in_range && proj_row_valid(J, r);
-      const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-      constexpr int kHalf = kNout / 2;
-#pragma unroll 1
-      for (int c64 = (warp >> 2) * kHalf; c64 < (warp >> 2) * kHalf + kHalf; c64 += 64) {
-        float v64[64];
-        tmem_ld64_wait(lane_base + (uint32_t)c64, v64);  // warp-wide: every lane, in range or not
-#pragma unroll
-       for (int half = 0; half < 2; ++half) {
-        const int c0 = c64 + 32 * half;
-        const float* v = v64 + 32 * half;
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = valid ? cvt_bf16x2(v[2 * i] + S.bias[c0 + 2 * i], v[2 * i + 1] + S.bias[c0 + 2 * i + 1]) : 0u;
-        if (kOut == kOutRows && in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(X.out0 + r * kEmbed + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        } else if (kOut == kOutQKV && valid) {
-          // columns c0 .. c0 + 31: two heads of one of Q, K, V
-          const int tensor = c0 / kEmbed, cc = c0 % kEmbed;
-          uint16_t* base = tensor == 0 ? X.out0 : (tensor == 1 ? X.out1 : X.out2);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int h = cc / kD + hh;
-            size_t off;
-            if (J.ptr) off = ((size_t)r * kH + h) * kD;
-            else off = (((size_t)(r / J.P) * kH + h) * J.P + (size_t)(r % J.P)) * kD;
-            uint4* dst = reinterpret_cast<uint4*>(base + off);
-            dst[0] = make_uint4(w[8 * hh], w[8 * hh + 1], w[8 * hh + 2], w[8 * hh + 3]);
-            dst[1] = make_uint4(w[8 * hh + 4], w[8 * hh + 5], w[8 * hh + 6], w[8 * hh + 7]);
-          }
-        }
-       }
-      }
-    }
-    // TMEM is read and the next A tile written before the next MMAs
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
-  if (!ok && tid == 0) raise_status(kStTimeout);
-  tc_fence_before();
-  __syncthreads();
-  if (!ok) {
-    // an MMA may still be in flight: wait once more (bounded) before freeing TMEM
-    if (tid == 0) (void)mbar_wait(&S.mbar, phase);
-    __syncthreads();
-  }
-  tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, kCols);
 }
 
 
