@@ -18,11 +18,12 @@
  *
  * Conventions for every entry point:
  *   - All array arguments are DEVICE pointers owned by the caller, except in
- *     pb_fold_affine (host). Nothing is allocated inside the library.
+ *     pb_fold_affine and pb_unfold_grad (host). Nothing is allocated inside
+ *     the library.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream), launches exactly one kernel (the
- *     balanced fused path as a cooperative launch; pair_block_forward three,
- *     in order) and does not synchronise.
+ *     balanced fused path as a cooperative launch; pair_block_forward three
+ *     and pair_attention_backward four, in order) and does not synchronise.
  *     Host-side argument errors return before any launch; device-side problems (an invalid ptr array, a bounded wait that
  *     ran out) set bits of a per-device status word, read with
  *     pb_get_device_status.
@@ -119,6 +120,26 @@ enum {
   PB_OFF_W3 = 4480, PB_OFF_B3 = 8576, PB_OFF_W4 = 8640, PB_OFF_B4 = 9152,
   PB_FOLDED_FLOATS = 9160
 };
+
+/* Offsets (in floats) of the unfolded parameters' gradients inside the flat
+ * buffer that pb_unfold_grad writes (the order of pb_mlp_unfolded);
+ * PB_UNFOLDED_FLOATS is its length. */
+enum {
+  PB_UOFF_A0 = 0, PB_UOFF_C0 = 4, PB_UOFF_W1 = 8, PB_UOFF_B1 = 264, PB_UOFF_A1 = 328,
+  PB_UOFF_C1 = 392, PB_UOFF_W2 = 456, PB_UOFF_B2 = 4552, PB_UOFF_A2 = 4616, PB_UOFF_C2 = 4680,
+  PB_UOFF_W3 = 4744, PB_UOFF_B3 = 8840, PB_UOFF_A3 = 8904, PB_UOFF_C3 = 8968, PB_UOFF_W4 = 9032,
+  PB_UOFF_B4 = 9544, PB_UNFOLDED_FLOATS = 9552
+};
+
+/* Gradients with respect to the folded MLP parameters (the pb_mlp that the
+ * forward consumed): fp32 device buffers with pb_mlp's shapes, row-major
+ * [out][in]; every element is overwritten. */
+typedef struct {
+  float *W1, *b1;  /* [64][4], [64]   */
+  float *W2, *b2;  /* [64][64], [64]  */
+  float *W3, *b3;  /* [64][64], [64]  */
+  float *W4, *b4;  /* [8][64], [8]    */
+} pb_mlp_grad;
 
 /* pairfeat_compute -- the four pair features of every slot pair.
  * feat: fp32 [N, P, P, 4], channel order (ln kT, ln z, ln dR, ln m^2);
@@ -218,6 +239,54 @@ size_t pb_block_workspace_bytes(const pb_jets *jets);
 pb_status pair_attention_forward_noalloc(const pb_jets *jets, const pb_mlp *mlp, int H, int D,
                                          const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                          uint16_t *out, void *stream);
+
+/* pair_attention_backward -- gradients of the fused path of
+ * pair_attention_forward (mlp given): for an upstream gradient dout of out,
+ * dq, dk, dv and the gradients of the folded MLP parameters. The section
+ * "Fusion 3" ships its biased attention with a backward kernel; the MLP
+ * gradients are the chain rule of the "Fusion 2" MLP, each unordered pair's
+ * bias row receiving dL/dU[h,i,j] + dL/dU[h,j,i]. The pair features are not
+ * differentiated (the momenta are data).
+ *   q, k, v, dout: bf16 inputs, dq, dk, dv: bf16 outputs, all in the layout
+ *     of `jets` (as pair_attention_forward's q), 16-byte aligned; masked rows
+ *     of dq, dk, dv are written as 0.
+ *   dmlp: device gradient buffers (see pb_mlp_grad), overwritten, also when
+ *     N = 0 (zeros).
+ *   workspace: device memory of at least pb_backward_workspace_bytes(jets)
+ *     bytes, 256-byte aligned, no initialisation needed; calls sharing one
+ *     workspace must not overlap on the device.
+ * Arithmetic: the bias is recomputed by the forward MLP kernel and kept in
+ * the workspace as bf16; attention gradients use bf16 tensor-core operands
+ * with fp32 accumulation and fp32 softmax statistics, dL/dU is kept as bf16;
+ * the MLP is recomputed with bf16 operands (hi + lo terms for the first
+ * layer), fp32 accumulation and the erf form of GELU; the weight gradients
+ * accumulate in fp32 per CTA and are summed over CTAs in a fixed order, so
+ * the result does not depend on timing.
+ * Launches, in order on `stream`: the bias kernel of pairbias_mlp_forward,
+ * the attention backward, the MLP backward and a gradient-sum kernel (with
+ * N = 0 only the last, writing zeros). Errors as for
+ * pair_attention_forward; PB_EINVAL also for a missing or small workspace
+ * or a NULL gradient buffer. */
+pb_status pair_attention_backward(const pb_jets *jets, const pb_mlp *mlp, int H, int D,
+                                  const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  const uint16_t *dout, uint16_t *dq, uint16_t *dk, uint16_t *dv,
+                                  const pb_mlp_grad *dmlp, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/* pb_backward_workspace_bytes -- workspace size of pair_attention_backward:
+ * N*8*P*P bf16 values (the bias, then dL/dU) plus min(N, 256) partial
+ * gradients of PB_FOLDED_FLOATS floats, each part rounded up to 256 bytes.
+ * 0 if `jets` is invalid. */
+size_t pb_backward_workspace_bytes(const pb_jets *jets);
+
+/* pb_unfold_grad -- host helper, not on the GPU path: gradients of the
+ * unfolded parameters (a0, c0, W1, b1, a1, c1, ... as in pb_mlp_unfolded)
+ * from those of the folded ones, by the chain rule of pb_fold_affine's
+ * folding (computed in double, rounded once to fp32).
+ * folded_grad: host buffer of PB_FOLDED_FLOATS floats (PB_OFF_* layout);
+ * out: host buffer of PB_UNFOLDED_FLOATS floats (PB_UOFF_* layout).
+ * Returns PB_EINVAL for a NULL pointer. */
+pb_status pb_unfold_grad(const pb_mlp_unfolded *in, const float *folded_grad, float *out);
 
 /* pb_get_device_status -- synchronise `stream`, then read and clear the
  * status word of the current device. *bits (may be NULL) receives the

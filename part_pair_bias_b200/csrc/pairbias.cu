@@ -2,8 +2,9 @@
 //
 // Host side only validates arguments, picks the template instance for P
 // (<= 128 or <= 256), sizes a persistent grid from the SM count and the
-// occupancy of that instance, and launches exactly one kernel on the caller's
-// stream. Nothing is allocated and nothing is synchronised here.
+// occupancy of that instance, and launches the entry point's kernels (one;
+// three for pair_block_forward, four for pair_attention_backward) on the
+// caller's stream. Nothing is allocated and nothing is synchronised here.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdarg.h>
@@ -13,6 +14,7 @@
 #include <mutex>
 
 #include "pairbias.h"
+#include "pb_backward.cuh"
 #include "pb_kernels.cuh"
 
 namespace {
@@ -254,6 +256,39 @@ pb_status run_proj(const pb::JetArgs& J, const pb::ProjArgs& X, cudaStream_t s, 
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+// Backward workspace: the bf16 bias / dL/dU planes [N, 8, P, P], then one
+// partial of the folded weight gradients per k_mlp_bwd CTA.
+size_t bwd_u_bytes(const pb::JetArgs& J) { return round256((size_t)J.N * pb::kH * J.P * J.P * 2); }
+int bwd_parts(const pb::JetArgs& J) { return J.N < pb::kBwdMaxCtas ? J.N : pb::kBwdMaxCtas; }
+size_t bwd_workspace_bytes(const pb::JetArgs& J) {
+  return bwd_u_bytes(J) + round256((size_t)bwd_parts(J) * pb::kFoldedFloats * sizeof(float));
+}
+
+template <int PM>
+pb_status run_backward(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::BwdArgs& X, const pb::GradArgs& G,
+                       float* partials, cudaStream_t s) {
+  pb_status st = run_mlp_bias<PM, false>(J, W, X.U, s);
+  if (st != PB_OK) return st;
+  {
+    auto k = pb::k_attn_bwd<PM>;
+    const size_t smem = sizeof(pb::AttnBwdSmem<PM>);
+    int grid = 0;
+    if ((st = prepare(k, smem, 256, J.N, &grid)) != PB_OK) return st;
+    k<<<grid, 256, smem, s>>>(J, X);
+    if ((st = launched("k_attn_bwd")) != PB_OK) return st;
+  }
+  int parts = 0;
+  {
+    auto k = pb::k_mlp_bwd<PM>;
+    const size_t smem = sizeof(pb::MlpBwdSmem<PM>);
+    if ((st = prepare(k, smem, 512, bwd_parts(J), &parts)) != PB_OK) return st;
+    k<<<parts, 512, smem, s>>>(J, W, X.U, partials);
+    if ((st = launched("k_mlp_bwd")) != PB_OK) return st;
+  }
+  pb::k_grad_reduce<<<(pb::kFoldedFloats + 255) / 256, 256, 0, s>>>(partials, parts, G);
+  return launched("k_grad_reduce");
+}
+
 }  // namespace
 
 extern "C" {
@@ -402,6 +437,102 @@ pb_status pair_block_forward(const pb_jets* jets, const pb_mlp* mlp, const pb_pr
   st = J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
   if (st != PB_OK) return st;
   return run_proj<128, pb::kInHeads, pb::kOutRows>(J, out, s, "k_proj (out)");
+}
+
+size_t pb_backward_workspace_bytes(const pb_jets* jets) {
+  pb::JetArgs J;
+  if (check_jets(jets, &J) != PB_OK) return 0;
+  return bwd_workspace_bytes(J);
+}
+
+pb_status pair_attention_backward(const pb_jets* jets, const pb_mlp* mlp, int H, int D, const uint16_t* q,
+                                  const uint16_t* k, const uint16_t* v, const uint16_t* dout, uint16_t* dq,
+                                  uint16_t* dk, uint16_t* dv, const pb_mlp_grad* dmlp, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  pb::JetArgs J;
+  pb::MlpArgs W;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK) return st;
+  if (H != pb::kH || D != pb::kD) return fail(PB_EUNSUPPORTED, "H = %d, D = %d; only H = 8, D = 16", H, D);
+  if ((st = check_mlp(mlp, &W)) != PB_OK) return st;
+  if (!dmlp) return fail(PB_EINVAL, "dmlp is NULL");
+  float* gp[8] = {dmlp->W1, dmlp->b1, dmlp->W2, dmlp->b2, dmlp->W3, dmlp->b3, dmlp->W4, dmlp->b4};
+  for (float* p : gp)
+    if (!p || !aligned(p, 4)) return fail(PB_EINVAL, "the gradient buffers of dmlp must be non-NULL and 4-byte aligned");
+  const pb::GradArgs G{gp[0], gp[1], gp[2], gp[3], gp[4], gp[5], gp[6], gp[7]};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (J.N == 0) {  // no pairs: the weight gradients are zero
+    pb::k_grad_reduce<<<(pb::kFoldedFloats + 255) / 256, 256, 0, s>>>(nullptr, 0, G);
+    return launched("k_grad_reduce");
+  }
+  if (!q || !k || !v || !dout || !dq || !dk || !dv) return fail(PB_EINVAL, "q, k, v, dout, dq, dk and dv must be non-NULL");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dq, 16) ||
+      !aligned(dk, 16) || !aligned(dv, 16))
+    return fail(PB_EINVAL, "q, k, v, dout, dq, dk and dv must be 16-byte aligned");
+  const size_t need = bwd_workspace_bytes(J);
+  if (!workspace || !aligned(workspace, 256)) return fail(PB_EINVAL, "workspace must be non-NULL and 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(PB_EINVAL, "workspace of %zu bytes, %zu needed (pb_backward_workspace_bytes)", workspace_bytes, need);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const pb::BwdArgs X{q, k, v, dout, dq, dk, dv, reinterpret_cast<uint16_t*>(ws)};
+  float* partials = reinterpret_cast<float*>(ws + bwd_u_bytes(J));
+  return J.P <= 128 ? run_backward<128>(J, W, X, G, partials, s) : run_backward<256>(J, W, X, G, partials, s);
+}
+
+pb_status pb_unfold_grad(const pb_mlp_unfolded* in, const float* folded_grad, float* out) {
+  if (!in || !folded_grad || !out) return fail(PB_EINVAL, "NULL argument");
+  const float* need[] = {in->a0, in->c0, in->W1, in->b1, in->a1, in->c1, in->W2, in->b2,
+                         in->a2, in->c2, in->W3, in->b3, in->a3, in->c3, in->W4, in->b4};
+  for (const float* p : need)
+    if (!p) return fail(PB_EINVAL, "an unfolded parameter pointer is NULL");
+  const float* g = folded_grad;
+  // layer 1: W1' = a1 W1 a0 (per row and column), b1' = a1 (W1 c0 + b1) + c1
+  for (int j = 0; j < 4; ++j) {
+    double da0 = 0.0, dc0 = 0.0;
+    for (int o = 0; o < 64; ++o) {
+      const double aw = (double)in->a1[o] * (double)in->W1[o * 4 + j];
+      da0 += aw * (double)g[PB_OFF_W1 + o * 4 + j];
+      dc0 += aw * (double)g[PB_OFF_B1 + o];
+    }
+    out[PB_UOFF_A0 + j] = (float)da0;
+    out[PB_UOFF_C0 + j] = (float)dc0;
+  }
+  for (int o = 0; o < 64; ++o) {
+    const double a1 = in->a1[o], gb = g[PB_OFF_B1 + o];
+    double t = in->b1[o], da1 = 0.0;
+    for (int j = 0; j < 4; ++j) {
+      const double w = in->W1[o * 4 + j], gw = g[PB_OFF_W1 + o * 4 + j];
+      out[PB_UOFF_W1 + o * 4 + j] = (float)(a1 * ((double)in->a0[j] * gw + (double)in->c0[j] * gb));
+      da1 += w * (double)in->a0[j] * gw;
+      t += w * (double)in->c0[j];
+    }
+    out[PB_UOFF_B1 + o] = (float)(a1 * gb);
+    out[PB_UOFF_A1 + o] = (float)(da1 + t * gb);
+    out[PB_UOFF_C1 + o] = (float)gb;
+  }
+  // layers 2, 3: W' = a W, b' = a b + c
+  const float* Ws[2] = {in->W2, in->W3};
+  const float* bs[2] = {in->b2, in->b3};
+  const float* as[2] = {in->a2, in->a3};
+  const int gW[2] = {PB_OFF_W2, PB_OFF_W3}, gB[2] = {PB_OFF_B2, PB_OFF_B3};
+  const int uW[2] = {PB_UOFF_W2, PB_UOFF_W3}, uB[2] = {PB_UOFF_B2, PB_UOFF_B3};
+  const int uA[2] = {PB_UOFF_A2, PB_UOFF_A3}, uC[2] = {PB_UOFF_C2, PB_UOFF_C3};
+  for (int L = 0; L < 2; ++L)
+    for (int o = 0; o < 64; ++o) {
+      const double a = as[L][o], gb = g[gB[L] + o];
+      double da = (double)bs[L][o] * gb;
+      for (int i = 0; i < 64; ++i) {
+        const double gw = g[gW[L] + o * 64 + i];
+        out[uW[L] + o * 64 + i] = (float)(a * gw);
+        da += (double)Ws[L][o * 64 + i] * gw;
+      }
+      out[uB[L] + o] = (float)(a * gb);
+      out[uA[L] + o] = (float)da;
+      out[uC[L] + o] = (float)gb;
+    }
+  memcpy(out + PB_UOFF_W4, g + PB_OFF_W4, sizeof(float) * 8 * 64);
+  memcpy(out + PB_UOFF_B4, g + PB_OFF_B4, sizeof(float) * 8);
+  return PB_OK;
 }
 
 pb_status pb_selftest_wait_timeouts(void* stream) {

@@ -1,0 +1,761 @@
+// pb_backward.cuh -- gradients of the fused pair-bias attention for sm_100a.
+//
+// pair_attention_backward launches, in order:
+//   k_mlp_bias     (forward kernel) the bias U of every pair into the workspace
+//   k_attn_bwd     per jet: softmax statistics, dQ, dK, dV on m16n8k16 tensor
+//                  cores; dL/dU overwrites U in place (transposed, bf16)
+//   k_mlp_bwd      per 128-pair tile: the MLP recomputed on tcgen05 (the
+//                  pre-activations stay in TMEM), the backward through it on
+//                  tcgen05, the weight gradients on m16n8k16 tensor cores in
+//                  registers that persist over all the CTA's tiles
+//   k_grad_reduce  the per-CTA weight-gradient partials summed in CTA order
+//
+// Source: "Event Classification with Masked Transformer Autoencoders",
+// section "Fusion 3 -- Self-Attention + Additive Bias -> Fused Triton
+// Attention" (forward and backward kernels of the biased attention), with the
+// pair-MLP bias of "Fusion 2 -- Pairwise Features + Conv1d MLP ->
+// FusedPairMLP".
+#pragma once
+
+#include "pb_kernels.cuh"
+
+namespace pb {
+
+struct BwdArgs {
+  const uint16_t *q, *k, *v, *dout;  // bf16, layout of the jets (padded [N,H,P,D], packed [tokens,H,D])
+  uint16_t *dq, *dk, *dv;
+  uint16_t* U;                       // [N, 8, P, P] bf16: the bias in, dL/dU (transposed) out
+};
+
+// ------------------------------------------------------------ ldmatrix
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ============================================== attention backward (k_attn_bwd)
+//
+// Per (jet, head), over the jet's m valid particles, with s = q.k/4 + U in
+// log2 units (x log2 e):
+//   query pass (warp = 16 queries): the row maximum and sum of exp2 give
+//     lse_i; O_i = sum_j p_ij v_j (p split into two bf16 terms so that O is
+//     accurate to ~2^-17) gives D_i = dO_i . O_i; a second sweep over the keys
+//     recomputes p_ij = exp2(s_ij - lse_i), dP_ij = dO_i . v_j,
+//     dS_ij = p_ij (dP_ij - D_i) and accumulates dQ_i = 1/4 sum_j dS_ij k_j;
+//   key pass (warp = 16 keys): the transposed tiles S^T = K Q^T, dP^T = V dO^T
+//     give p_ij and dS_ij again, accumulated into dV_j = sum_i p_ij dO_i and
+//     dK_j = 1/4 sum_i dS_ij q_i; dS_ij is stored (bf16) over U at [j][i].
+// The query pass of a head finishes before its key pass starts, and the key
+// pass of key block J reads and writes only rows J of the U plane, so the
+// in-place update never overwrites a bias still to be read.
+//
+// Each staged head holds Q, K, V and dO of its rows as bf16 [m16][kKStride]
+// (zero rows past m), then lse and D as fp32 [m16]. Every operand fragment
+// comes from these row-major tiles through ldmatrix (.trans for the
+// operands whose K dimension runs along the rows).
+
+__host__ __device__ constexpr int bwd_tensor_bytes(int m) { return round16(m) * kKStride * 2; }
+__host__ __device__ constexpr int bwd_head_bytes(int m) { return 4 * bwd_tensor_bytes(m) + 8 * round16(m); }
+
+template <int PM>
+__device__ void stage_bwd(const Particles<PM>& S, const JetArgs& J, const BwdArgs& X, int n, int h0, int hr,
+                          unsigned char* buf) {
+  const int m = S.m, m16 = round16(m), hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m);
+  const int total = hr * m16 * 8, nthr = blockDim.x;
+  for (int base = threadIdx.x; base < total; base += 4 * nthr) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      const int part = idx & 7, j = (idx >> 3) % m16, hh = (idx >> 3) / m16;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (idx < total && j < m) {
+        const uint16_t* src = part < 2 ? X.q : (part < 4 ? X.k : (part < 6 ? X.v : X.dout));
+        v[u] = *reinterpret_cast<const uint4*>(src + qkv_off<PM>(S, J, n, h0 + hh, j) + (part & 1) * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nthr;
+      if (idx >= total) break;
+      const int part = idx & 7, j = (idx >> 3) % m16, hh = (idx >> 3) / m16;
+      *reinterpret_cast<uint4*>(buf + hh * hb + (part >> 1) * tb + j * kKStride * 2 + (part & 1) * 16) = v[u];
+    }
+  }
+  // lse and D of rows m .. m16-1 (read, masked, by the key pass) are 0
+  for (int idx = threadIdx.x; idx < hr * 2 * m16; idx += nthr) {
+    const int hh = idx / (2 * m16), r = idx % (2 * m16);
+    reinterpret_cast<float*>(buf + hh * hb + 4 * tb)[r] = 0.f;
+  }
+}
+
+// Byte offsets, inside a staged tensor, of this lane's ldmatrix row for the
+// three fragment shapes used (add the tile's first row times the row pitch):
+//   A  (16 rows x 16 cols, x4):            rows 0-7 | 8-15, cols 0-7 | 8-15
+//   Bn (two n8 blocks of rows, d = K, x4):  b0,b1 of rows 0-7, then of rows 8-15
+//   Bt (rows = K, d = N, x4.trans):         b0,b1 of d 0-7, then of d 8-15
+__device__ __forceinline__ uint32_t frag_a_off(int lane) {
+  return (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kKStride * 2 + (lane >> 4) * 16);
+}
+__device__ __forceinline__ uint32_t frag_bn_off(int lane) {
+  return (uint32_t)(((lane & 7) + ((lane >> 4) & 1) * 8) * kKStride * 2 + ((lane >> 3) & 1) * 16);
+}
+__device__ __forceinline__ uint32_t frag_bt_off(int lane) {
+  return (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kKStride * 2 + ((lane >> 4) & 1) * 16);
+}
+
+// p (fp32) as the A fragment of a k16 step, split into hi + lo bf16 terms.
+__device__ __forceinline__ void split_bf16_frag(const float* p, uint32_t* hi, uint32_t* lo) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hi[i] = cvt_bf16x2(p[2 * i], p[2 * i + 1]);
+    lo[i] = cvt_bf16x2(p[2 * i] - bf16lo(hi[i]), p[2 * i + 1] - bf16hi(hi[i]));
+  }
+}
+
+__device__ __forceinline__ void pack_bf16_frag(const float* p, uint32_t* a) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = cvt_bf16x2(p[2 * i], p[2 * i + 1]);
+}
+
+// Scores of one 16 x 16 block in log2 units: s = acc / 4 + u, -inf where the
+// column index (cols(e)) is >= m.
+template <class Col>
+__device__ __forceinline__ void bwd_scores(float* s, const float* u, int m, const Col& col) {
+  const float qs = 0.25f * kLog2e;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s[e] = col(e) < m ? fmaf(s[e], qs, u[e] * kLog2e) : -INFINITY;
+}
+
+// Query pass for queries [i0, i0 + 16) of one staged head at shared address
+// hs: writes lse (log2 units) and D of its valid rows and dQ through dqrow(i).
+// Warp-wide.
+template <class UBlock, class ORow>
+__device__ void bwd_query_tile(uint32_t hs, int m, int i0, const UBlock& ub, float* lse, float* dd,
+                               const ORow& dqrow) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint32_t pitch = kKStride * 2, tb = (uint32_t)bwd_tensor_bytes(m);
+  const uint32_t Qs = hs, Ks = hs + tb, Vs = hs + 2 * tb, Os = hs + 3 * tb;
+  const int nrows = min(16, m - i0);
+  const bool va = g < nrows, vb = g + 8 < nrows;
+  const int ia = i0 + (va ? g : 0), ib = i0 + (vb ? g + 8 : 0);  // rows past the block alias row i0
+  const uint32_t fa = frag_a_off(lane), fbn = frag_bn_off(lane), fbt = frag_bt_off(lane);
+  uint32_t aq[4], ado[4];
+  ldsm_x4(Qs + i0 * pitch + fa, aq);
+  ldsm_x4(Os + i0 * pitch + fa, ado);
+
+  // sweep 1: statistics and O
+  float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float mxa = -INFINITY, mxb = -INFINITY, la = 0.f, lb = 0.f;
+  for (int n0 = 0; n0 < m; n0 += 16) {
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t bk[4];
+    ldsm_x4(Ks + n0 * pitch + fbn, bk);
+    mma_16816(s, aq, bk[0], bk[1]);
+    mma_16816(s + 4, aq, bk[2], bk[3]);
+    float u[8];
+    ub(n0, i0, ia, ib, t, m, u);
+    bwd_scores(s, u, m, [&](int e) { return n0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1); });
+    float bma = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[4], s[5]));
+    float bmb = fmaxf(fmaxf(s[2], s[3]), fmaxf(s[6], s[7]));
+    bma = fmaxf(bma, __shfl_xor_sync(0xffffffffu, bma, 1));
+    bma = fmaxf(bma, __shfl_xor_sync(0xffffffffu, bma, 2));
+    bmb = fmaxf(bmb, __shfl_xor_sync(0xffffffffu, bmb, 1));
+    bmb = fmaxf(bmb, __shfl_xor_sync(0xffffffffu, bmb, 2));
+    const float nma = fmaxf(mxa, bma), nmb = fmaxf(mxb, bmb);  // finite: key n0 < m is valid
+    const float ca = ex2(mxa - nma), cb = ex2(mxb - nmb);
+    mxa = nma;
+    mxb = nmb;
+    float p[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) p[e] = ex2(s[e] - (e & 2 ? nmb : nma));
+    la = la * ca + ((p[0] + p[1]) + (p[4] + p[5]));
+    lb = lb * cb + ((p[2] + p[3]) + (p[6] + p[7]));
+    o[0] *= ca; o[1] *= ca; o[4] *= ca; o[5] *= ca;
+    o[2] *= cb; o[3] *= cb; o[6] *= cb; o[7] *= cb;
+    uint32_t ph[4], pl[4], bv[4];
+    split_bf16_frag(p, ph, pl);
+    ldsm_x4_t(Vs + n0 * pitch + fbt, bv);
+    mma_16816(o, ph, bv[0], bv[1]);
+    mma_16816(o + 4, ph, bv[2], bv[3]);
+    mma_16816(o, pl, bv[0], bv[1]);
+    mma_16816(o + 4, pl, bv[2], bv[3]);
+  }
+  la += __shfl_xor_sync(0xffffffffu, la, 1);
+  la += __shfl_xor_sync(0xffffffffu, la, 2);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+  const float lse_a = mxa + __log2f(la), lse_b = mxb + __log2f(lb);
+  // D = dO . O: the lane's O elements sit at the positions of its dO fragment
+  float da = bf16lo(ado[0]) * o[0] + bf16hi(ado[0]) * o[1] + bf16lo(ado[2]) * o[4] + bf16hi(ado[2]) * o[5];
+  float db = bf16lo(ado[1]) * o[2] + bf16hi(ado[1]) * o[3] + bf16lo(ado[3]) * o[6] + bf16hi(ado[3]) * o[7];
+  da += __shfl_xor_sync(0xffffffffu, da, 1);
+  da += __shfl_xor_sync(0xffffffffu, da, 2);
+  db += __shfl_xor_sync(0xffffffffu, db, 1);
+  db += __shfl_xor_sync(0xffffffffu, db, 2);
+  da /= la;
+  db /= lb;
+  if (t == 0) {
+    if (va) {
+      lse[ia] = lse_a;
+      dd[ia] = da;
+    }
+    if (vb) {
+      lse[ib] = lse_b;
+      dd[ib] = db;
+    }
+  }
+
+  // sweep 2: dS and dQ
+  float dq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int n0 = 0; n0 < m; n0 += 16) {
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t bk[4];
+    ldsm_x4(Ks + n0 * pitch + fbn, bk);
+    mma_16816(s, aq, bk[0], bk[1]);
+    mma_16816(s + 4, aq, bk[2], bk[3]);
+    float u[8];
+    ub(n0, i0, ia, ib, t, m, u);
+    bwd_scores(s, u, m, [&](int e) { return n0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1); });
+    float dp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t bv[4];
+    ldsm_x4(Vs + n0 * pitch + fbn, bv);
+    mma_16816(dp, ado, bv[0], bv[1]);
+    mma_16816(dp + 4, ado, bv[2], bv[3]);
+    float ds[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ds[e] = ex2(s[e] - (e & 2 ? lse_b : lse_a)) * (dp[e] - (e & 2 ? db : da));
+    uint32_t pd[4], bkt[4];
+    pack_bf16_frag(ds, pd);
+    ldsm_x4_t(Ks + n0 * pitch + fbt, bkt);
+    mma_16816(dq, pd, bkt[0], bkt[1]);
+    mma_16816(dq + 4, pd, bkt[2], bkt[3]);
+  }
+  if (va) {
+    uint16_t* op = dqrow(ia);
+    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(0.25f * dq[0], 0.25f * dq[1]);
+    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(0.25f * dq[4], 0.25f * dq[5]);
+  }
+  if (vb) {
+    uint16_t* op = dqrow(ib);
+    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(0.25f * dq[2], 0.25f * dq[3]);
+    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(0.25f * dq[6], 0.25f * dq[7]);
+  }
+}
+
+// Key pass for keys [j0, j0 + 16) of one staged head: dK, dV through
+// dkrow(j), dvrow(j), and dS_ij (bf16) into the head's U plane at
+// Uh[slot[j] * P + slot[i]] (the positions its bias was read from). Warp-wide.
+template <int PM, class UBlock, class KRow, class VRow>
+__device__ void bwd_key_tile(uint32_t hs, const Particles<PM>& S, int j0, const UBlock& ub, const float* lse,
+                             const float* dd, uint16_t* Uh, int P, const KRow& dkrow, const VRow& dvrow) {
+  const int m = S.m;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint32_t pitch = kKStride * 2, tb = (uint32_t)bwd_tensor_bytes(m);
+  const uint32_t Qs = hs, Ks = hs + tb, Vs = hs + 2 * tb, Os = hs + 3 * tb;
+  const int nrows = min(16, m - j0);
+  const bool va = g < nrows, vb = g + 8 < nrows;
+  const int ja = j0 + (va ? g : 0), jb = j0 + (vb ? g + 8 : 0);
+  const uint32_t fa = frag_a_off(lane), fbn = frag_bn_off(lane), fbt = frag_bt_off(lane);
+  uint32_t ak[4], av[4];
+  ldsm_x4(Ks + j0 * pitch + fa, ak);
+  ldsm_x4(Vs + j0 * pitch + fa, av);
+  const size_t ra = (size_t)S.slot[ja] * P, rb = (size_t)S.slot[jb] * P;
+  float dk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float dv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int i0 = 0; i0 < m; i0 += 16) {
+    auto col = [&](int e) { return i0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1); };
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t bq[4];
+    ldsm_x4(Qs + i0 * pitch + fbn, bq);
+    mma_16816(s, ak, bq[0], bq[1]);
+    mma_16816(s + 4, ak, bq[2], bq[3]);
+    float u[8];
+    ub(i0, j0, ja, jb, t, m, u);  // U[j][i] = U[i][j]
+    bwd_scores(s, u, m, col);
+    const float2 l0 = *reinterpret_cast<const float2*>(lse + i0 + 2 * t);
+    const float2 l1 = *reinterpret_cast<const float2*>(lse + i0 + 8 + 2 * t);
+    const float2 d0 = *reinterpret_cast<const float2*>(dd + i0 + 2 * t);
+    const float2 d1 = *reinterpret_cast<const float2*>(dd + i0 + 8 + 2 * t);
+    const float lsev[4] = {l0.x, l0.y, l1.x, l1.y}, ddv[4] = {d0.x, d0.y, d1.x, d1.y};
+    float dp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint32_t bo[4];
+    ldsm_x4(Os + i0 * pitch + fbn, bo);
+    mma_16816(dp, av, bo[0], bo[1]);
+    mma_16816(dp + 4, av, bo[2], bo[3]);
+    float p[8], ds[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = (e & 1) + ((e >> 1) & 2);  // column slot of element e: 2t + (e & 1) + 8 (e >> 2)
+      p[e] = ex2(s[e] - lsev[c]);
+      ds[e] = p[e] * (dp[e] - ddv[c]);
+    }
+    uint32_t pp[4], pd[4], bot[4], bqt[4];
+    pack_bf16_frag(p, pp);
+    pack_bf16_frag(ds, pd);
+    ldsm_x4_t(Os + i0 * pitch + fbt, bot);
+    mma_16816(dv, pp, bot[0], bot[1]);
+    mma_16816(dv + 4, pp, bot[2], bot[3]);
+    ldsm_x4_t(Qs + i0 * pitch + fbt, bqt);
+    mma_16816(dk, pd, bqt[0], bqt[1]);
+    mma_16816(dk + 4, pd, bqt[2], bqt[3]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = col(e);
+      const bool row_ok = e & 2 ? vb : va;
+      if (row_ok && i < m && in_bounds(i >= 0)) Uh[(e & 2 ? rb : ra) + S.slot[i]] = f32_to_bf16(ds[e]);
+    }
+  }
+  if (va) {
+    uint16_t* kp = dkrow(ja);
+    uint16_t* vp = dvrow(ja);
+    *reinterpret_cast<uint32_t*>(kp + 2 * t) = cvt_bf16x2(0.25f * dk[0], 0.25f * dk[1]);
+    *reinterpret_cast<uint32_t*>(kp + 8 + 2 * t) = cvt_bf16x2(0.25f * dk[4], 0.25f * dk[5]);
+    *reinterpret_cast<uint32_t*>(vp + 2 * t) = cvt_bf16x2(dv[0], dv[1]);
+    *reinterpret_cast<uint32_t*>(vp + 8 + 2 * t) = cvt_bf16x2(dv[4], dv[5]);
+  }
+  if (vb) {
+    uint16_t* kp = dkrow(jb);
+    uint16_t* vp = dvrow(jb);
+    *reinterpret_cast<uint32_t*>(kp + 2 * t) = cvt_bf16x2(0.25f * dk[2], 0.25f * dk[3]);
+    *reinterpret_cast<uint32_t*>(kp + 8 + 2 * t) = cvt_bf16x2(0.25f * dk[6], 0.25f * dk[7]);
+    *reinterpret_cast<uint32_t*>(vp + 2 * t) = cvt_bf16x2(dv[2], dv[3]);
+    *reinterpret_cast<uint32_t*>(vp + 8 + 2 * t) = cvt_bf16x2(dv[6], dv[7]);
+  }
+}
+
+constexpr int kBwdStageBytes = 100 * 1024;  // staged heads of the attention backward
+
+template <int PM>
+struct AttnBwdSmem {
+  unsigned char stage[kBwdStageBytes];
+  Particles<PM> part;
+};
+
+template <int PM>
+__global__ void __launch_bounds__(256) k_attn_bwd(JetArgs J, BwdArgs X) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  AttnBwdSmem<PM>& S = *reinterpret_cast<AttnBwdSmem<PM>*>(smem_raw);
+  const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  for (int n = blockIdx.x; n < J.N; n += gridDim.x) {
+    stage_jet<PM, false>(S.part, J, n);
+    const int m = S.part.m;
+    if (m > 0) {
+      const int hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m), m16 = round16(m);
+      const int HR = max(1, min(kH, kBwdStageBytes / hb));
+      const int tiles = (m + 15) >> 4;
+      const GlobalUBias<PM> ub{&S.part, X.U, n, J.P};
+      if (in_bounds(hb <= kBwdStageBytes)) {
+        for (int h0 = 0; h0 < kH; h0 += HR) {
+          const int hr = min(HR, kH - h0);
+          stage_bwd<PM>(S.part, J, X, n, h0, hr, S.stage);
+          __syncthreads();
+          for (int it = warp; it < hr * tiles; it += nwarp) {
+            const int hh = it / tiles, h = h0 + hh;
+            unsigned char* hbuf = S.stage + hh * hb;
+            float* lse = reinterpret_cast<float*>(hbuf + 4 * tb);
+            bwd_query_tile(smem_u32(hbuf), m, (it % tiles) * 16, ub.head(h), lse, lse + m16,
+                           [&](int i) { return X.dq + qkv_off<PM>(S.part, J, n, h, i); });
+          }
+          __syncthreads();
+          for (int it = warp; it < hr * tiles; it += nwarp) {
+            const int hh = it / tiles, h = h0 + hh;
+            unsigned char* hbuf = S.stage + hh * hb;
+            const float* lse = reinterpret_cast<const float*>(hbuf + 4 * tb);
+            uint16_t* Uh = X.U + ((size_t)n * kH + h) * J.P * J.P;
+            bwd_key_tile<PM>(smem_u32(hbuf), S.part, (it % tiles) * 16, ub.head(h), lse, lse + m16, Uh, J.P,
+                             [&](int j) { return X.dk + qkv_off<PM>(S.part, J, n, h, j); },
+                             [&](int j) { return X.dv + qkv_off<PM>(S.part, J, n, h, j); });
+          }
+          __syncthreads();
+        }
+      }
+    }
+    zero_masked_rows<PM>(S.part, J, X.dq, n);
+    zero_masked_rows<PM>(S.part, J, X.dk, n);
+    zero_masked_rows<PM>(S.part, J, X.dv, n);
+    __syncthreads();
+  }
+}
+
+// ==================================================== MLP backward (k_mlp_bwd)
+//
+// For the unordered pair (a, b) of a jet, the bias row u = MLP(f(a, b)) feeds
+// both U[h, a, b] and U[h, b, a], so its upstream gradient is
+// g_h = dS_h[a, b] + dS_h[b, a] (a != b) or dS_h[a, a]. Per tile of 128 such
+// rows (one CTA, 512 threads; thread (row r, quarter c) owns TMEM lane r and
+// columns 16c .. 16c + 15 of each 64-wide accumulator):
+//   z1 = W1' f + b1', h1 = GELU(z1), z2 = W2' h1 + b2', ... h3   (tcgen05, z in TMEM)
+//   e3 = g W4 (issued with z1), d3 = e3 * GELU'(z3), e2 = d3 W3', d2, e1 = d2 W2', d1
+//   dW4 += g^T h3, dWk' += dk^T h(k-1) (h0 = f), dbk' += column sums of dk
+// with bf16 operands and fp32 accumulation; the folded layer-1 weights and
+// the features enter as bf16 hi + lo terms. GELU is the erf form (normcdff).
+// The weight gradients are 31 (layer, 16-row block, up to three 8-column
+// blocks) parts spread over the 16 warps as m16n8k16 MMAs whose A operand
+// (d^T) and B operand (h) come from the row-major tiles through
+// ldmatrix.trans; a column block of ones gives the bias gradients.
+
+constexpr int kBwdMaxCtas = 256;     // partial-gradient slots in the workspace
+constexpr int kFoldedFloats = 9160;  // W1 b1 W2 b2 W3 b3 W4 b4, as pb_fold_affine lays them out
+constexpr int kOffW1 = 0, kOffB1 = 256, kOffW2 = 320, kOffB2 = 4416, kOffW3 = 4480, kOffB3 = 8576,
+              kOffW4 = 8640, kOffB4 = 9152;
+
+struct GradArgs {
+  float *W1, *b1, *W2, *b2, *W3, *b3, *W4, *b4;
+};
+
+template <int PM>
+struct MlpBwdSmem {
+  __nv_bfloat16 A0[kTileM * 16];     // [hi(f) | lo(f) | hi(f) | 0]
+  __nv_bfloat16 G4[kTileM * 16];     // [g (8 heads) | 0]
+  __nv_bfloat16 Hs[3][kTileM * 64];  // h1, h2, h3
+  __nv_bfloat16 Ds[3][kTileM * 64];  // d1, d2, d3 = dL/dz
+  __nv_bfloat16 W1f[64 * 16];        // [hi(W1') | hi(W1') | lo(W1') | 0] per output row
+  __nv_bfloat16 Wf[2][64 * 64];      // W2', W3' as [out][in]
+  __nv_bfloat16 Wt[2][64 * 64];      // W2'^T, W3'^T as [in][out]
+  __nv_bfloat16 W4t[64 * 16];        // W4^T as [in][out], out 8..15 zero
+  float bias[3][64];                 // b1', b2', b3'
+  uint64_t mbar;
+  uint32_t tmem_base;
+  Particles<PM> part;
+};
+
+// Weights in the canonical K-major layouts of their MMA roles.
+template <int PM>
+__device__ void bwd_load_weights(MlpBwdSmem<PM>& S, const MlpArgs& W) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  for (int e = tid; e < 64 * 64; e += nthr) {
+    const int o = e >> 6, i = e & 63;
+    const float w2 = W.W2[e], w3 = W.W3[e];
+    S.Wf[0][cofs(o, i, 64)] = __float2bfloat16_rn(w2);
+    S.Wf[1][cofs(o, i, 64)] = __float2bfloat16_rn(w3);
+    S.Wt[0][cofs(i, o, 64)] = __float2bfloat16_rn(w2);
+    S.Wt[1][cofs(i, o, 64)] = __float2bfloat16_rn(w3);
+  }
+  for (int e = tid; e < 64 * 16; e += nthr) {
+    const int r = e >> 4, k = e & 15;  // W1f row = output r, W4t row = input r
+    const float w1 = k < 12 ? W.W1[r * 4 + (k & 3)] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w1);
+    S.W1f[cofs(r, k, 16)] = (k >= 8 && k < 12) ? __float2bfloat16_rn(w1 - __bfloat162float(hi)) : hi;
+    S.W4t[cofs(r, k, 16)] = __float2bfloat16_rn(k < 8 ? W.W4[k * 64 + r] : 0.f);
+  }
+  for (int e = tid; e < 3 * 64; e += nthr) S.bias[e >> 6][e & 63] = (e < 64 ? W.b1 : (e < 128 ? W.b2 : W.b3))[e & 63];
+}
+
+__device__ __forceinline__ float gelu_erf(float z) { return z * normcdff(z); }
+__device__ __forceinline__ float gelu_erf_grad(float z) {
+  return normcdff(z) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+}
+
+// One weight-gradient part: layer L (1..4), 16-row block mb of dW, column
+// blocks nb0 .. nb0 + nc - 1 (the last block index of a layer is the ones
+// column: 8 for L = 2..4, 1 for L = 1).
+struct GradPart {
+  int L, mb, nb0, nc;
+};
+
+__device__ __forceinline__ GradPart grad_part(int q) {
+  if (q < 3) return GradPart{4, 0, 3 * q, 3};
+  if (q < 15) return GradPart{3, (q - 3) / 3, 3 * ((q - 3) % 3), 3};
+  if (q < 27) return GradPart{2, (q - 15) / 3, 3 * ((q - 15) % 3), 3};
+  return GradPart{1, q - 27, 0, 2};
+}
+constexpr int kGradParts = 31;
+
+template <int PM>
+__device__ __forceinline__ void grad_tiles(const MlpBwdSmem<PM>& S, const GradPart& gp, const __nv_bfloat16*& Dt,
+                                           int& Kd, const __nv_bfloat16*& Bt, int& Kb, int& ones) {
+  Dt = gp.L == 4 ? S.G4 : S.Ds[gp.L - 1];
+  Kd = gp.L == 4 ? 16 : 64;
+  Bt = gp.L == 1 ? S.A0 : S.Hs[gp.L - 2];
+  Kb = gp.L == 1 ? 16 : 64;
+  ones = gp.L == 1 ? 1 : 8;
+}
+
+// acc[j] += d^T h over the tile's 128 rows for the part's column blocks.
+template <int PM>
+__device__ __forceinline__ void grad_mma(const MlpBwdSmem<PM>& S, const GradPart& gp, float (*acc)[4]) {
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16 *Dt, *Bt;
+  int Kd, Kb, ones;
+  grad_tiles(S, gp, Dt, Kd, Bt, Kb, ones);
+  const int mi = lane >> 3;
+  const uint32_t d_base = smem_u32(Dt), b_base = smem_u32(Bt);
+#pragma unroll 1
+  for (int k0 = 0; k0 < kTileM; k0 += 16) {
+    uint32_t a[4];
+    ldsm_x4_t(d_base + 2u * cofs(k0 + (lane & 7) + (mi >> 1) * 8, gp.mb * 16 + (mi & 1) * 8, Kd), a);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      if (j >= gp.nc) break;
+      const int nb = gp.nb0 + j;
+      uint32_t b[2];
+      if (nb == ones) {
+        b[0] = b[1] = 0x3F803F80u;  // bf16 1.0 in both halves
+      } else {
+        ldsm_x2_t(b_base + 2u * cofs(k0 + (lane & 7) + ((lane >> 3) & 1) * 8, nb * 8, Kb), b);
+      }
+      mma_16816(acc[j], a, b[0], b[1]);
+    }
+  }
+}
+
+// The part's accumulators into the CTA's partial (folded layout).
+__device__ void grad_store(const GradPart& gp, float (*acc)[4], float* part) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int oa = gp.mb * 16 + g, ob = oa + 8;
+  for (int j = 0; j < gp.nc; ++j) {
+    const int nb = gp.nb0 + j;
+    const float* c = acc[j];
+    if (gp.L == 1) {
+      // columns 0..3 hold sum d hi(f), 4..7 sum d lo(f)
+      const float p0 = __shfl_down_sync(0xffffffffu, c[0], 2), p1 = __shfl_down_sync(0xffffffffu, c[1], 2);
+      const float p2 = __shfl_down_sync(0xffffffffu, c[2], 2), p3 = __shfl_down_sync(0xffffffffu, c[3], 2);
+      if (nb == 0) {
+        if (t < 2) {
+          part[kOffW1 + oa * 4 + 2 * t] = c[0] + p0;
+          part[kOffW1 + oa * 4 + 2 * t + 1] = c[1] + p1;
+          part[kOffW1 + ob * 4 + 2 * t] = c[2] + p2;
+          part[kOffW1 + ob * 4 + 2 * t + 1] = c[3] + p3;
+        }
+      } else if (t == 0) {
+        part[kOffB1 + oa] = c[0];
+        part[kOffB1 + ob] = c[2];
+      }
+    } else if (gp.L == 4) {  // output rows 8..15 are padding
+      if (nb < 8) {
+        part[kOffW4 + g * 64 + nb * 8 + 2 * t] = c[0];
+        part[kOffW4 + g * 64 + nb * 8 + 2 * t + 1] = c[1];
+      } else if (t == 0) {
+        part[kOffB4 + g] = c[0];
+      }
+    } else {
+      const int offW = gp.L == 2 ? kOffW2 : kOffW3, offB = gp.L == 2 ? kOffB2 : kOffB3;
+      if (nb < 8) {
+        part[offW + oa * 64 + nb * 8 + 2 * t] = c[0];
+        part[offW + oa * 64 + nb * 8 + 2 * t + 1] = c[1];
+        part[offW + ob * 64 + nb * 8 + 2 * t] = c[2];
+        part[offW + ob * 64 + nb * 8 + 2 * t + 1] = c[3];
+      } else if (t == 0) {
+        part[offB + oa] = c[0];
+        part[offB + ob] = c[2];
+      }
+    }
+  }
+}
+
+template <int PM>
+__global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, const uint16_t* __restrict__ dU,
+                                                    float* __restrict__ partials) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  MlpBwdSmem<PM>& S = *reinterpret_cast<MlpBwdSmem<PM>*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = tid & 127, c = tid >> 7;  // tile row (TMEM lane) and column quarter
+  bwd_load_weights<PM>(S, W);
+  if (tid == 0) {
+    mbar_init(&S.mbar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&S.tmem_base, 256);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192), e3 / e2 / e1 [192, 256)
+  const uint32_t tm = S.tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  constexpr uint32_t kId = idesc_bf16_m128(64);
+  const uint32_t a0 = smem_u32(S.A0), g4 = smem_u32(S.G4), w1f = smem_u32(S.W1f), w4t = smem_u32(S.W4t);
+  uint32_t phase = 0u;
+  bool ok = true, aborted = false;
+
+  const GradPart gp0 = grad_part(warp), gp1 = grad_part(min(warp + 16, kGradParts - 1));
+  const bool has1 = warp + 16 < kGradParts;
+  float acc0[3][4], acc1[3][4];
+#pragma unroll
+  for (int j = 0; j < 3; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc0[j][e] = acc1[j][e] = 0.f;
+
+  // operand writes published, then thread 0 issues `body` and commits
+  auto issue = [&](auto&& body) -> bool {
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (__syncthreads_or(!ok)) return false;
+    if (tid == 0) {
+      tc_fence_after();
+      body();
+      mma_commit(&S.mbar);
+    }
+    return true;
+  };
+  auto wait = [&]() {
+    const bool done = mbar_wait(&S.mbar, phase);
+    phase ^= 1u;
+    ok = ok && done;
+    tc_fence_after();
+  };
+  auto gemm64 = [&](uint32_t d, const __nv_bfloat16* A, const __nv_bfloat16* B) {
+    const uint32_t aa = smem_u32(A), bb = smem_u32(B);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      mma_f16(d, smem_desc(aa + 256u * k, 128, 1024), smem_desc(bb + 256u * k, 128, 1024), kId, k > 0 ? 1u : 0u);
+  };
+  auto store16 = [&](__nv_bfloat16* T, const float* v) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = cvt_bf16x2(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4*>(T + cofs(r, 16 * c, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(T + cofs(r, 16 * c + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
+  };
+  // h_k = GELU(z_k + b_k) (k = 0..2) of this thread's 16 columns
+  auto hidden = [&](int k) {
+    float z[16];
+    tmem_ld16_wait(tm + lane_off + 64u * k + 16u * c, z);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z[i] = gelu_erf(z[i] + S.bias[k][16 * c + i]);
+    store16(S.Hs[k], z);
+  };
+  // d_k = e * GELU'(z_k + b_k)
+  auto delta = [&](int k) {
+    float z[16], e[16];
+    tmem_ld16_wait(tm + lane_off + 64u * k + 16u * c, z);
+    tmem_ld16_wait(tm + lane_off + 192u + 16u * c, e);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) e[i] *= gelu_erf_grad(z[i] + S.bias[k][16 * c + i]);
+    store16(S.Ds[k], e);
+  };
+
+  for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
+    stage_jet<PM>(S.part, J, n);
+    const int m = S.part.m, P = J.P;
+    const int npairs = m * (m + 1) / 2, ntiles = (npairs + kTileM - 1) / kTileM;
+    const uint16_t* Un = dU + (size_t)n * kH * P * P;
+    for (int t = 0; t < ntiles; ++t) {
+      // row r: the unordered pair p = b(b+1)/2 + a; features (c = 0) and g (c = 1)
+      const int p = t * kTileM + r;
+      int a = 0, b = 0;
+      bool valid = p < npairs;
+      if (valid && c < 2) {
+        TriPairs{}.map(p, a, b);
+        valid = in_bounds(a >= 0 && a <= b && b < m);
+      }
+      if (c == 0) {
+        float f[4] = {0.f, 0.f, 0.f, 0.f};
+        if (valid) pair_feat<PM, false>(S.part, a, b, f);
+        uint32_t hl[4], lh[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const uint32_t hi = cvt_bf16x2(f[2 * i], f[2 * i + 1]);
+          hl[i] = hi;
+          lh[i] = cvt_bf16x2(f[2 * i] - bf16lo(hi), f[2 * i + 1] - bf16hi(hi));
+        }
+        hl[2] = lh[0];
+        hl[3] = lh[1];
+        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 0, 16)) = make_uint4(hl[0], hl[1], hl[2], hl[3]);
+        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 8, 16)) = make_uint4(hl[0], hl[1], 0u, 0u);
+      } else if (c == 1) {
+        float gv[8];
+        const int sa = S.part.slot[a], sb = S.part.slot[b];
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
+          const uint16_t* Uh = Un + (size_t)h * P * P;
+          gv[h] = valid ? bf16_to_f32(Uh[(size_t)sa * P + sb]) + (a != b ? bf16_to_f32(Uh[(size_t)sb * P + sa]) : 0.f)
+                        : 0.f;
+        }
+        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 0, 16)) =
+            make_uint4(cvt_bf16x2(gv[0], gv[1]), cvt_bf16x2(gv[2], gv[3]), cvt_bf16x2(gv[4], gv[5]),
+                       cvt_bf16x2(gv[6], gv[7]));
+        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 8, 16)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      // forward: z1 (and e3 = g W4, which needs nothing else), z2, z3
+      if (!issue([&] {
+            mma_f16(tm, smem_desc(a0, 128, 256), smem_desc(w1f, 128, 256), kId, 0u);
+            mma_f16(tm + 192u, smem_desc(g4, 128, 256), smem_desc(w4t, 128, 256), kId, 0u);
+          })) {
+        aborted = true;
+        break;
+      }
+      wait();
+      hidden(0);
+      if (!issue([&] { gemm64(tm + 64u, S.Hs[0], S.Wf[0]); })) {
+        aborted = true;
+        break;
+      }
+      wait();
+      hidden(1);
+      if (!issue([&] { gemm64(tm + 128u, S.Hs[1], S.Wf[1]); })) {
+        aborted = true;
+        break;
+      }
+      wait();
+      hidden(2);
+      delta(2);
+      // backward: e2 = d3 W3', e1 = d2 W2'
+      if (!issue([&] { gemm64(tm + 192u, S.Ds[2], S.Wt[1]); })) {
+        aborted = true;
+        break;
+      }
+      wait();
+      delta(1);
+      if (!issue([&] { gemm64(tm + 192u, S.Ds[1], S.Wt[0]); })) {
+        aborted = true;
+        break;
+      }
+      wait();
+      delta(0);
+      __syncthreads();  // every tile row written before the weight-gradient MMAs read them
+      grad_mma(S, gp0, acc0);
+      if (has1) grad_mma(S, gp1, acc1);
+      tc_fence_before();
+      __syncthreads();  // operands and TMEM free for the next tile
+      tc_fence_after();
+    }
+    aborted = __syncthreads_or(aborted || !ok) != 0;
+  }
+  float* part = partials + (size_t)blockIdx.x * kFoldedFloats;
+  grad_store(gp0, acc0, part);
+  if (has1) grad_store(gp1, acc1, part);
+  tc_fence_before();
+  __syncthreads();
+  if (aborted && tid == 0) (void)mbar_wait(&S.mbar, phase ^ 1u);  // bounded: the last commit before TMEM is freed
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(S.tmem_base, 256);
+}
+
+// Weight gradients: the sum over the CTAs' partials, in CTA order.
+__global__ void __launch_bounds__(256) k_grad_reduce(const float* __restrict__ partials, int nparts, GradArgs G) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= kFoldedFloats) return;
+  float s = 0.f;
+  for (int c = 0; c < nparts; ++c) s += partials[(size_t)c * kFoldedFloats + e];
+  if (e < kOffB1) G.W1[e - kOffW1] = s;
+  else if (e < kOffW2) G.b1[e - kOffB1] = s;
+  else if (e < kOffB2) G.W2[e - kOffW2] = s;
+  else if (e < kOffW3) G.b2[e - kOffB2] = s;
+  else if (e < kOffB3) G.W3[e - kOffW3] = s;
+  else if (e < kOffW4) G.b3[e - kOffB3] = s;
+  else if (e < kOffB4) G.W4[e - kOffW4] = s;
+  else G.b4[e - kOffB4] = s;
+}
+
+}  // namespace pb

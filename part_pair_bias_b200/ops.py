@@ -7,7 +7,8 @@ on first use and its absence is an error -- there is no fallback.
 Entry points mirror ``include/pairbias.h``: ``pairfeat_compute``,
 ``pairbias_mlp_forward``, ``pair_attention_forward``,
 ``pair_attention_forward_noalloc``, ``pair_block_forward``,
-``get_device_status`` and the host helper ``fold_affine``.
+``pair_attention_backward``, ``get_device_status`` and the host helpers
+``fold_affine`` and ``unfold_grad``.
 """
 from __future__ import annotations
 
@@ -33,6 +34,12 @@ H, D = 8, 16
 FOLDED_OFFSETS = dict(W1=(0, (64, 4)), b1=(256, (64,)), W2=(320, (64, 64)), b2=(4416, (64,)),
                       W3=(4480, (64, 64)), b3=(8576, (64,)), W4=(8640, (8, 64)), b4=(9152, (8,)))
 FOLDED_FLOATS = 9160
+# offsets of the unfolded parameters' gradients (PB_UOFF_* in the header)
+UNFOLDED_OFFSETS = dict(a0=(0, (4,)), c0=(4, (4,)), W1=(8, (64, 4)), b1=(264, (64,)), a1=(328, (64,)),
+                        c1=(392, (64,)), W2=(456, (64, 64)), b2=(4552, (64,)), a2=(4616, (64,)),
+                        c2=(4680, (64,)), W3=(4744, (64, 64)), b3=(8840, (64,)), a3=(8904, (64,)),
+                        c3=(8968, (64,)), W4=(9032, (8, 64)), b4=(9544, (8,)))
+UNFOLDED_FLOATS = 9552
 
 
 class PairBiasError(RuntimeError):
@@ -115,9 +122,14 @@ def load(path: str):
     L.pb_last_error.restype = C.c_char_p
     L.pb_version.restype = C.c_char_p
     L.pb_selftest_wait_timeouts.argtypes = [vp]
+    L.pair_attention_backward.argtypes = [C.POINTER(_Jets), C.POINTER(_Mlp), C.c_int, C.c_int, vp, vp, vp, vp,
+                                          vp, vp, vp, C.POINTER(_Mlp), vp, C.c_size_t, vp]
+    L.pb_backward_workspace_bytes.argtypes = [C.POINTER(_Jets)]
+    L.pb_backward_workspace_bytes.restype = C.c_size_t
+    L.pb_unfold_grad.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float), C.POINTER(C.c_float)]
     for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward, L.pb_selftest_wait_timeouts,
               L.pair_attention_forward_noalloc, L.pair_block_forward, L.pb_get_device_status,
-              L.pb_fold_affine):
+              L.pb_fold_affine, L.pair_attention_backward, L.pb_unfold_grad):
         f.restype = C.c_int
     return L
 
@@ -174,6 +186,19 @@ class FoldedMLP:
     def struct(self) -> _Mlp:
         base = self.flat.data_ptr()
         return _Mlp(**{k: base + 4 * off for k, (off, _s) in FOLDED_OFFSETS.items()})
+
+
+def unfold_grad(params: Dict[str, np.ndarray], folded_grad: np.ndarray) -> Dict[str, np.ndarray]:
+    """Gradients of the unfolded parameters from those of the folded ones
+    (host, C library): a dict keyed like ``params``."""
+    arrs = {k: np.ascontiguousarray(v, np.float32) for k, v in params.items()}
+    st = _MlpUnfolded(**{n: arrs[n].ctypes.data for n, _t in _MlpUnfolded._fields_})
+    g = np.ascontiguousarray(folded_grad, np.float32)
+    assert g.size == FOLDED_FLOATS
+    out = np.zeros(UNFOLDED_FLOATS, np.float32)
+    fp = C.POINTER(C.c_float)
+    _check(lib().pb_unfold_grad(C.byref(st), g.ctypes.data_as(fp), out.ctypes.data_as(fp)))
+    return {k: out[off:off + int(np.prod(shape))].reshape(shape) for k, (off, shape) in UNFOLDED_OFFSETS.items()}
 
 
 def fold_affine(params: Dict[str, np.ndarray]) -> np.ndarray:
@@ -294,6 +319,42 @@ def pair_block_forward(jets: Jets, mlp: FoldedMLP, proj: Proj, x: torch.Tensor, 
     _check(lib().pair_block_forward(C.byref(js), C.byref(ms), C.byref(ps), H, D, H * D, x.data_ptr(), y.data_ptr(),
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream)))
+
+
+class MlpGrad:
+    """Gradients of the folded MLP parameters in one flat fp32 device buffer
+    (PB_OFF_* layout, the layout of ``FoldedMLP.flat``)."""
+
+    def __init__(self, device="cuda"):
+        self.flat = torch.empty(FOLDED_FLOATS, dtype=torch.float32, device=device)
+
+    def struct(self) -> _Mlp:
+        base = self.flat.data_ptr()
+        return _Mlp(**{k: base + 4 * off for k, (off, _s) in FOLDED_OFFSETS.items()})
+
+    def as_dict(self) -> Dict[str, np.ndarray]:
+        f = self.flat.cpu().numpy()
+        return {k: f[off:off + int(np.prod(shape))].reshape(shape) for k, (off, shape) in FOLDED_OFFSETS.items()}
+
+
+def backward_workspace_bytes(jets: Jets) -> int:
+    js = jets.struct()
+    return int(lib().pb_backward_workspace_bytes(C.byref(js)))
+
+
+def pair_attention_backward(jets: Jets, mlp: FoldedMLP, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            dout: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor,
+                            dmlp: MlpGrad, workspace: torch.Tensor, stream=None) -> None:
+    """Gradients of the fused forward for the upstream gradient `dout`: dq,
+    dk, dv (bf16, layout of q) and the folded MLP's parameter gradients into
+    `dmlp`; workspace uint8 of ``backward_workspace_bytes(jets)`` bytes."""
+    for t in (q, k, v, dout, dq, dk, dv):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    js, ms, gs = jets.struct(), mlp.struct(), dmlp.struct()
+    _check(lib().pair_attention_backward(C.byref(js), C.byref(ms), H, D, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), C.byref(gs),
+                                         _dp(workspace), 0 if workspace is None else workspace.numel(),
+                                         _stream(stream)))
 
 
 def selftest_wait_timeouts(stream=None) -> None:

@@ -249,3 +249,19 @@ def slice_block_inputs(b: JetBatch, bi: BlockInputs, lo: int, hi: int) -> BlockI
     else:
         x = bi.x[int(b.ptr[lo]):int(b.ptr[hi])].copy()
     return BlockInputs(x, bi.Wqkv, bi.bqkv, bi.Wo, bi.bo)
+
+
+def make_upstream(b: JetBatch, seed: int) -> np.ndarray:
+    """An upstream gradient dL/dout for the backward pass: N(0, 1) values
+    rounded to bf16 (raw bits), in the layout of b.q, from a stream of its
+    own. Masked rows hold values too; the forward output there is constant 0,
+    so they carry no gradient."""
+    rng = np.random.default_rng([int(seed), 0xD0])
+    return f32_to_bf16_bits(rng.standard_normal(b.q.shape).astype(np.float32))
+
+
+def slice_rows(b: JetBatch, x: np.ndarray, lo: int, hi: int) -> np.ndarray:
+    """The rows of jets lo..hi-1 of an array in the layout of b.q."""
+    if b.layout == "padded":
+        return x[lo:hi].copy()
+    return x[int(b.ptr[lo]):int(b.ptr[hi])].copy()

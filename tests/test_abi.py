@@ -32,7 +32,8 @@ def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
     assert {"pairfeat_compute", "pairbias_mlp_forward", "pair_attention_forward",
             "pb_get_device_status", "pb_fold_affine", "pb_last_error", "pb_version",
-            "pb_workspace_bytes", "pair_attention_forward_noalloc"} <= set(names)
+            "pb_workspace_bytes", "pair_attention_forward_noalloc", "pair_attention_backward",
+            "pb_backward_workspace_bytes", "pb_unfold_grad"} <= set(names)
     for n in names:
         assert hasattr(L, n), f"{n} declared in pairbias.h but not exported"
     assert ops.version().startswith("pairbias-b200")
@@ -162,3 +163,60 @@ def test_block_host_validation_and_workspace(L):
     assert call(proj=C.byref(bad)) == ops.PB_EINVAL
     js.N = 0                                                # nothing to do, no device needed
     assert call() == ops.PB_OK
+
+
+def _r256(b):
+    return (b + 255) // 256 * 256
+
+
+def test_backward_workspace_size(L):
+    """bf16 bias planes [N, 8, P, P] plus min(N, 256) fp32 gradient partials."""
+    for N, P in ((2, 8), (128, 128), (300, 37)):
+        js, keep = _jets(N=N, P=P)
+        want = _r256(N * 8 * P * P * 2) + _r256(min(N, 256) * ops.FOLDED_FLOATS * 4)
+        assert L.pb_backward_workspace_bytes(C.byref(js)) == want
+    js.P = 300
+    assert L.pb_backward_workspace_bytes(C.byref(js)) == 0
+
+
+def test_backward_host_rejections(L):
+    """Argument errors of pair_attention_backward return before any launch."""
+    js, keep = _jets(N=2, P=8)
+    buf = np.zeros(1 << 16, np.uint8)
+    d = (buf.ctypes.data + 255) // 256 * 256
+    mlp = ops._Mlp(*([d] * 8))
+    grad = ops._Mlp(*([d] * 8))
+    need = L.pb_backward_workspace_bytes(C.byref(js))
+    call = lambda H=8, D=16, m=mlp, q=d, dout=d, g=grad, ws=d, wsb=need: L.pair_attention_backward(
+        C.byref(js), None if m is None else C.byref(m), H, D, q, d, d, dout, d, d, d,
+        None if g is None else C.byref(g), ws, wsb, None)
+    assert call(H=4) == ops.PB_EUNSUPPORTED
+    assert call(D=32) == ops.PB_EUNSUPPORTED
+    assert call(m=None) == ops.PB_EINVAL
+    assert call(g=None) == ops.PB_EINVAL
+    assert call(g=ops._Mlp(*([d] * 7 + [0]))) == ops.PB_EINVAL
+    assert call(g=ops._Mlp(*([d] * 7 + [d + 2]))) == ops.PB_EINVAL       # misaligned gradient buffer
+    assert call(q=None) == ops.PB_EINVAL
+    assert call(dout=d + 2) == ops.PB_EINVAL                            # misaligned upstream gradient
+    assert call(ws=None) == ops.PB_EINVAL
+    assert call(ws=d + 16) == ops.PB_EINVAL                             # workspace not 256-byte aligned
+    assert call(wsb=need - 1) == ops.PB_EINVAL
+    assert "pb_backward_workspace_bytes" in L.pb_last_error().decode()
+
+
+def test_unfold_grad_matches_oracle(L, oracle_lib):
+    """The host helper's chain rule through the folding reproduces the
+    oracle's directly computed gradients of the unfolded parameters."""
+    from oracle import backward as bw
+    for seed in range(3):
+        b = synth.make_jets(N=3, P=8, mults=[5, 8, 3], mask_mode="scrambled", seed=40 + seed)
+        dO = np.random.default_rng(seed).standard_normal(b.q.shape)
+        r = bw.backward(b, dO)
+        flat = np.zeros(ops.FOLDED_FLOATS)
+        for name, (off, shape) in ops.FOLDED_OFFSETS.items():
+            flat[off:off + int(np.prod(shape))] = r["folded"][name].reshape(-1)
+        got = ops.unfold_grad(b.params, flat)
+        for name, ref in r["unfolded"].items():
+            scale = max(np.max(np.abs(ref)), 1e-30)
+            assert np.max(np.abs(got[name] - ref)) <= 1e-5 * scale, name
+    assert L.pb_unfold_grad(None, None, None) == ops.PB_EINVAL

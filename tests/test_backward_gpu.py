@@ -1,0 +1,153 @@
+"""GPU parity of pair_attention_backward (through the C ABI) against the fp64
+backward oracle.
+
+Tolerances (no bar is stated for gradients; these follow from the
+arithmetic of the forward bars and the backward's own roundings):
+  dq, dk, dv      relative L2 over valid rows <= 2e-2, masked rows exactly 0.
+                  The bias enters through the forward MLP kernel (bias bar:
+                  rel L2 1e-2), the softmax gradient dS = P (dP - D) loses
+                  relative accuracy where dP ~ D, and dq, dk, dv are bf16.
+  MLP gradients   relative L2 per folded tensor <= 3e-2. dL/dU is stored as
+                  bf16 and the MLP is recomputed with bf16 operands; each
+                  gradient is a sum of many such terms.
+  db4             zero in exact arithmetic (rows of dS sum to 0); bounded by
+                  the same relative error of the sum of |dL/dU|, here taken
+                  as 3e-2 times the largest dW4 row norm.
+"""
+import numpy as np
+import pytest
+import torch
+
+from part_pair_bias_b200 import configs, ops, synth
+from tests import parity as pt
+
+pytestmark = pytest.mark.gpu
+
+QKV_RELL2 = 2e-2
+GRAD_RELL2 = 3e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    torch.cuda.set_device(0)
+    ops.lib()
+    yield
+    assert ops.get_device_status() == 0
+
+
+@pytest.fixture(scope="module")
+def bw(oracle_lib):
+    from oracle import backward
+    return backward
+
+
+class Bwd:
+    def __init__(self, b, seed=0):
+        self.b = b
+        self.d = pt.Device(b)
+        self.dout_bits = synth.make_upstream(b, seed)
+        self.dout = ops.bf16_to_device(self.dout_bits)
+        self.ws = torch.empty(ops.backward_workspace_bytes(self.d.jets), dtype=torch.uint8, device="cuda")
+
+    def run(self):
+        d = self.d
+        dq, dk, dv = (torch.full_like(d.q, float("nan")) for _ in range(3))
+        g = ops.MlpGrad()
+        g.flat.fill_(float("nan"))
+        ops.pair_attention_backward(d.jets, d.mlp, d.q, d.k, d.v, self.dout, dq, dk, dv, g, self.ws)
+        return dq, dk, dv, g
+
+
+def rel_l2(got, ref):
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def check_qkv(got, ref, b):
+    vr = pt.valid_rows(b, got.shape)
+    rel = rel_l2(got[vr], ref[vr])
+    assert rel <= QKV_RELL2, f"rel L2 {rel:.3e}"
+    assert np.all(got[~vr] == 0.0), "masked rows must be 0"
+    return rel
+
+
+def check_grads(g, ref):
+    errs = {}
+    for name in ("W1", "b1", "W2", "b2", "W3", "b3", "W4"):
+        errs[name] = rel_l2(g[name], ref[name])
+        assert errs[name] <= GRAD_RELL2, f"d{name} rel L2 {errs[name]:.3e}"
+    w4_row = np.linalg.norm(ref["W4"], axis=1).max()
+    errs["b4_abs"] = float(np.abs(g["b4"] - ref["b4"]).max() / max(w4_row, 1e-300))
+    assert errs["b4_abs"] <= GRAD_RELL2, f"db4 {g['b4']} vs {ref['b4']}"
+    return errs
+
+
+def compare(b, seed=0, bw=None):
+    x = Bwd(b, seed)
+    dq, dk, dv, g = x.run()
+    assert ops.get_device_status() == 0
+    r = bw.backward(b, x.dout_bits)
+    out = {n: check_qkv(pt.to_np(t), r[n], b) for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+    out.update(check_grads(g.as_dict(), r["folded"]))
+    print(f"\n{b.layout} N={b.N} P={b.P}: " + ", ".join(f"{k} {v:.2e}" for k, v in out.items()))
+    return out
+
+
+CASES = {
+    "odd_p_scrambled": dict(N=8, P=37, mults=[0, 1, 2, 37, 17, 36, 5, 33], mask_mode="scrambled", seed=3),
+    "packed_empty": dict(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6),
+    "tiny_p3": dict(N=8, P=3, mults=[0, 1, 3, 2, 2, 3, 0, 1], mask_mode="scrambled", seed=9),
+    "wide_p256": dict(N=3, P=256, mults=[256, 130, 17], pt_lo=800, pt_hi=1000, prongs=3, seed=5),
+    "many_jets": dict(N=300, P=24, dist="uniform", mult_lo=1, mult_hi=24, mask_mode="scrambled", seed=8),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_backward_edge_cases(bw, case):
+    compare(synth.make_jets(**CASES[case]), seed=1, bw=bw)
+
+
+@pytest.mark.parametrize("name", ["pr1_n8_p32", "n128_p128"])
+def test_backward_workloads(bw, name):
+    compare(synth.make_jets(**configs.workload(name, seed=0)), seed=0, bw=bw)
+
+
+@pytest.mark.parametrize("name", ["packed_8192", "n256_p256_3prong"])
+def test_backward_large_workloads_sampled(bw, name):
+    """Full-size batches: dq, dk, dv of sampled jets against the oracle on
+    those jets alone (each jet's gradients depend on that jet only); the
+    MLP gradients of the whole batch against the sum of the slices' oracle
+    gradients over the whole batch would take minutes, so they are checked on
+    a 64-jet slice run by itself."""
+    b = synth.make_jets(**configs.workload(name, seed=0))
+    x = Bwd(b, 0)
+    dq, dk, dv, _g = x.run()
+    assert ops.get_device_status() == 0
+    for lo in (0, b.N // 2, b.N - 4):
+        s = synth.slice_jets(b, lo, lo + 4)
+        r = bw.backward(s, synth.slice_rows(b, x.dout_bits, lo, lo + 4))
+        for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+            got = synth.slice_rows(b, pt.to_np(t), lo, lo + 4)
+            check_qkv(got, r[n], s)
+    s = synth.slice_jets(b, 0, 64)
+    compare(s, seed=2, bw=bw)
+
+
+def test_backward_empty_batch_zero_gradients():
+    b = synth.make_jets(N=2, P=8, mults=[0, 0], seed=1)
+    x = Bwd(b, 0)
+    dq, dk, dv, g = x.run()
+    assert ops.get_device_status() == 0
+    for t in (dq, dk, dv):
+        assert torch.all(t == 0)
+    assert torch.all(g.flat == 0)
+
+
+def test_backward_deterministic():
+    b = synth.make_jets(**configs.workload("n128_p128", seed=1))
+    x = Bwd(b, 1)
+    r1 = x.run()
+    r2 = x.run()
+    for a, c in zip(r1[:3], r2[:3]):
+        assert torch.equal(a, c)
+    assert torch.equal(r1[3].flat, r2[3].flat)
