@@ -209,7 +209,8 @@ pb_status run_fused_grid(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::Q
   long long g = sms;  // one CTA per SM, all resident
   if (g > 8ll * J.N) g = 8ll * J.N;
   unsigned char* wsb = static_cast<unsigned char*>(ws);
-  void* args[] = {(void*)&J, (void*)&W, (void*)&X, (void*)&wsb};
+  int* no_table = nullptr;
+  void* args[] = {(void*)&J, (void*)&W, (void*)&X, (void*)&wsb, (void*)&no_table};
   cudaError_t e = cudaLaunchCooperativeKernel((const void*)k, dim3((unsigned)g), dim3(512), args, smem, s);
   if (e != cudaSuccess) return fail(PB_ECUDA, "k_fused_grid cooperative launch: %s", cudaGetErrorString(e));
   return PB_OK;
@@ -256,36 +257,95 @@ pb_status run_proj(const pb::JetArgs& J, const pb::ProjArgs& X, cudaStream_t s, 
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-// Backward workspace: the bf16 bias / dL/dU planes [N, 8, P, P], then one
-// partial of the folded weight gradients per k_mlp_bwd CTA.
-size_t bwd_u_bytes(const pb::JetArgs& J) { return round256((size_t)J.N * pb::kH * J.P * J.P * 2); }
-int bwd_parts(const pb::JetArgs& J) { return J.N < pb::kBwdMaxCtas ? J.N : pb::kBwdMaxCtas; }
-size_t bwd_workspace_bytes(const pb::JetArgs& J) {
-  return bwd_u_bytes(J) + round256((size_t)bwd_parts(J) * pb::kFoldedFloats * sizeof(float));
+// Backward: jets are processed in chunks that the balanced bias kernel
+// accepts (at most kGridMaxJets jets and, padded, N*P <= kGridMaxMaskBytes).
+// Workspace: the 256-byte header of the bias kernel, the bias records (16
+// bytes per row), the gradient records (32 bytes per row), the tile prefix of
+// a chunk, then kBwdMaxCtas weight-gradient partials. Record rows are bounded
+// for a chunk as for the balanced forward path.
+int bwd_chunk_jets(const pb::JetArgs& J) {
+  long long c = pb::kGridMaxJets;
+  if (!J.ptr && (long long)c * J.P > kGridMaxMaskBytes) c = kGridMaxMaskBytes / J.P;
+  return (int)(J.N < c ? J.N : c);
 }
 
+struct BwdLayout {
+  size_t urec, grec, table, partials, total;
+};
+
+BwdLayout bwd_layout(const pb::JetArgs& J) {
+  const int nc = bwd_chunk_jets(J);
+  const size_t rows = (pb::grid_workspace_bytes(nc, J.P, J.tokens, J.ptr != nullptr) - pb::kWsHeader) / 16;
+  BwdLayout L;
+  L.urec = pb::kWsHeader;
+  L.grec = round256(L.urec + rows * 16);
+  L.table = round256(L.grec + rows * 32);
+  L.partials = round256(L.table + (size_t)(nc + 1) * sizeof(int));
+  L.total = round256(L.partials + (size_t)pb::kBwdMaxCtas * pb::kFoldedFloats * sizeof(float));
+  return L;
+}
+
+// One chunk of jets: bias records, attention backward, MLP backward.
 template <int PM>
-pb_status run_backward(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::BwdArgs& X, const pb::GradArgs& G,
-                       float* partials, cudaStream_t s) {
-  pb_status st = run_mlp_bias<PM, false>(J, W, X.U, s);
+pb_status run_backward_chunk(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::BwdArgs& X, unsigned char* ws,
+                             int* table, float* partials, int mlp_grid, bool accumulate, cudaStream_t s) {
+  int dev = 0, sms = 0, per_sm = 0;
+  pb_status st = device_sms(&dev, &sms);
   if (st != PB_OK) return st;
+  {
+    auto k = pb::k_fused_grid<PM, true>;
+    const size_t smem = sizeof(pb::FusedGridSmem<PM>);
+    if ((st = resident_per_sm((const void*)k, dev, smem, 512, &per_sm)) != PB_OK) return st;
+    long long g = sms;
+    if (g > 8ll * J.N) g = 8ll * J.N;
+    k<<<(unsigned)g, 512, smem, s>>>(J, W, pb::QkvArgs{nullptr, nullptr, nullptr, nullptr}, ws, table);
+    if ((st = launched("k_fused_grid (bias records)")) != PB_OK) return st;
+  }
   {
     auto k = pb::k_attn_bwd<PM>;
     const size_t smem = sizeof(pb::AttnBwdSmem<PM>);
     int grid = 0;
-    if ((st = prepare(k, smem, 256, J.N, &grid)) != PB_OK) return st;
-    k<<<grid, 256, smem, s>>>(J, X);
+    if ((st = prepare(k, smem, 512, J.N, &grid)) != PB_OK) return st;
+    k<<<grid, 512, smem, s>>>(J, X);
     if ((st = launched("k_attn_bwd")) != PB_OK) return st;
   }
-  int parts = 0;
-  {
-    auto k = pb::k_mlp_bwd<PM>;
-    const size_t smem = sizeof(pb::MlpBwdSmem<PM>);
-    if ((st = prepare(k, smem, 512, bwd_parts(J), &parts)) != PB_OK) return st;
-    k<<<parts, 512, smem, s>>>(J, W, X.U, partials);
-    if ((st = launched("k_mlp_bwd")) != PB_OK) return st;
+  auto k = pb::k_mlp_bwd<PM>;
+  k<<<mlp_grid, 512, sizeof(pb::MlpBwdSmem<PM>), s>>>(J, W, X, partials, accumulate ? 1 : 0);
+  return launched("k_mlp_bwd");
+}
+
+template <int PM>
+pb_status run_backward(const pb::JetArgs& J, const pb::MlpArgs& W, pb::BwdArgs X, const pb::GradArgs& G,
+                       unsigned char* ws, cudaStream_t s) {
+  const BwdLayout L = bwd_layout(J);
+  int* table = reinterpret_cast<int*>(ws + L.table);
+  float* partials = reinterpret_cast<float*>(ws + L.partials);
+  X.urec = reinterpret_cast<const uint4*>(ws + L.urec);
+  X.grec = reinterpret_cast<float*>(ws + L.grec);
+  X.T = table;
+  // the MLP backward's grid is fixed (one partial slot per CTA for all chunks)
+  int dev = 0, sms = 0, per_sm = 0;
+  pb_status st = device_sms(&dev, &sms);
+  if (st != PB_OK) return st;
+  auto kb = pb::k_mlp_bwd<PM>;
+  if ((st = resident_per_sm((const void*)kb, dev, sizeof(pb::MlpBwdSmem<PM>), 512, &per_sm)) != PB_OK) return st;
+  const int mlp_grid = sms * per_sm < pb::kBwdMaxCtas ? sms * per_sm : pb::kBwdMaxCtas;
+  const int nc = bwd_chunk_jets(J);
+  for (int c0 = 0; c0 < J.N; c0 += nc) {
+    const int cn = J.N - c0 < nc ? J.N - c0 : nc;
+    pb::JetArgs Jc = J;
+    pb::BwdArgs Xc = X;
+    Jc.N = cn;
+    if (J.ptr) {
+      Jc.ptr = J.ptr + c0;  // token indices stay global: momenta and q/k/v rows are shared
+    } else {
+      const size_t e = (size_t)c0 * J.P, r = e * pb::kH * pb::kD;
+      Jc.E += e; Jc.px += e; Jc.py += e; Jc.pz += e; Jc.mask += e;
+      Xc.q += r; Xc.k += r; Xc.v += r; Xc.dout += r; Xc.dq += r; Xc.dk += r; Xc.dv += r;
+    }
+    if ((st = run_backward_chunk<PM>(Jc, W, Xc, ws, table, partials, mlp_grid, c0 > 0, s)) != PB_OK) return st;
   }
-  pb::k_grad_reduce<<<(pb::kFoldedFloats + 255) / 256, 256, 0, s>>>(partials, parts, G);
+  pb::k_grad_reduce<<<(pb::kFoldedFloats + 255) / 256, 256, 0, s>>>(partials, mlp_grid, G);
   return launched("k_grad_reduce");
 }
 
@@ -441,8 +501,8 @@ pb_status pair_block_forward(const pb_jets* jets, const pb_mlp* mlp, const pb_pr
 
 size_t pb_backward_workspace_bytes(const pb_jets* jets) {
   pb::JetArgs J;
-  if (check_jets(jets, &J) != PB_OK) return 0;
-  return bwd_workspace_bytes(J);
+  if (check_jets(jets, &J) != PB_OK || J.N == 0) return 0;
+  return bwd_layout(J).total;
 }
 
 pb_status pair_attention_backward(const pb_jets* jets, const pb_mlp* mlp, int H, int D, const uint16_t* q,
@@ -469,14 +529,13 @@ pb_status pair_attention_backward(const pb_jets* jets, const pb_mlp* mlp, int H,
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) || !aligned(dq, 16) ||
       !aligned(dk, 16) || !aligned(dv, 16))
     return fail(PB_EINVAL, "q, k, v, dout, dq, dk and dv must be 16-byte aligned");
-  const size_t need = bwd_workspace_bytes(J);
+  const size_t need = bwd_layout(J).total;
   if (!workspace || !aligned(workspace, 256)) return fail(PB_EINVAL, "workspace must be non-NULL and 256-byte aligned");
   if (workspace_bytes < need)
     return fail(PB_EINVAL, "workspace of %zu bytes, %zu needed (pb_backward_workspace_bytes)", workspace_bytes, need);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  const pb::BwdArgs X{q, k, v, dout, dq, dk, dv, reinterpret_cast<uint16_t*>(ws)};
-  float* partials = reinterpret_cast<float*>(ws + bwd_u_bytes(J));
-  return J.P <= 128 ? run_backward<128>(J, W, X, G, partials, s) : run_backward<256>(J, W, X, G, partials, s);
+  const pb::BwdArgs X{q, k, v, dout, dq, dk, dv, nullptr, nullptr, nullptr};
+  return J.P <= 128 ? run_backward<128>(J, W, X, G, ws, s) : run_backward<256>(J, W, X, G, ws, s);
 }
 
 pb_status pb_unfold_grad(const pb_mlp_unfolded* in, const float* folded_grad, float* out) {

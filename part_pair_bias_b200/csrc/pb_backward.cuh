@@ -1,14 +1,19 @@
 // pb_backward.cuh -- gradients of the fused pair-bias attention for sm_100a.
 //
-// pair_attention_backward launches, in order:
-//   k_mlp_bias     (forward kernel) the bias U of every pair into the workspace
+// pair_attention_backward launches, in order (per chunk of at most 8192 jets):
+//   k_fused_grid<PM, true>  the bias of every unordered pair, 8 f16 in one
+//                  16-byte record (the forward's balanced MLP phase over all
+//                  SMs, the same values as the forward's fused paths), and
+//                  the tile prefix T of the jets
 //   k_attn_bwd     per jet: softmax statistics, dQ, dK, dV on m16n8k16 tensor
-//                  cores; dL/dU overwrites U in place (transposed, bf16)
-//   k_mlp_bwd      per 128-pair tile: the MLP recomputed on tcgen05 (the
-//                  pre-activations stay in TMEM), the backward through it on
-//                  tcgen05, the weight gradients on m16n8k16 tensor cores in
-//                  registers that persist over all the CTA's tiles
-//   k_grad_reduce  the per-CTA weight-gradient partials summed in CTA order
+//                  cores; dL/dU[h,i,j] + dL/dU[h,j,i] accumulated into one
+//                  fp32 record per unordered pair
+//   k_mlp_bwd      the pairs' 128-row tiles split evenly over the CTAs: the
+//                  MLP recomputed on tcgen05 (GELU' kept in TMEM), the
+//                  backward through it on tcgen05, the weight gradients on
+//                  m16n8k16 tensor cores in registers that persist over all
+//                  the CTA's tiles (and chunks)
+// then, once, k_grad_reduce: the per-CTA partials summed in CTA order.
 //
 // Source: "Event Classification with Masked Transformer Autoencoders",
 // section "Fusion 3 -- Self-Attention + Additive Bias -> Fused Triton
@@ -21,10 +26,15 @@
 
 namespace pb {
 
+// Records of jet n's unordered pair p = b(b+1)/2 + a (a <= b) sit at row
+// T[n] * 128 + p of the record arrays (rows of a jet's last tile past its
+// pairs are unused).
 struct BwdArgs {
   const uint16_t *q, *k, *v, *dout;  // bf16, layout of the jets (padded [N,H,P,D], packed [tokens,H,D])
   uint16_t *dq, *dk, *dv;
-  uint16_t* U;                       // [N, 8, P, P] bf16: the bias in, dL/dU (transposed) out
+  const uint4* urec;                 // bias: 8 f16 per pair
+  float* grec;                       // upstream gradient of the pair's bias row: 8 fp32 per pair
+  const int* T;                      // tile prefix [N + 1]
 };
 
 // ------------------------------------------------------------ ldmatrix
@@ -64,10 +74,11 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 //     dS_ij = p_ij (dP_ij - D_i) and accumulates dQ_i = 1/4 sum_j dS_ij k_j;
 //   key pass (warp = 16 keys): the transposed tiles S^T = K Q^T, dP^T = V dO^T
 //     give p_ij and dS_ij again, accumulated into dV_j = sum_i p_ij dO_i and
-//     dK_j = 1/4 sum_i dS_ij q_i; dS_ij is stored (bf16) over U at [j][i].
-// The query pass of a head finishes before its key pass starts, and the key
-// pass of key block J reads and writes only rows J of the U plane, so the
-// in-place update never overwrites a bias still to be read.
+//     dK_j = 1/4 sum_i dS_ij q_i; dS_ij is added (fp32) to the record of the
+//     unordered pair {i, j}. Each off-diagonal record receives exactly two
+//     additions onto zero (dS_ij and dS_ji) and a diagonal one one, so the
+//     order of the atomic adds cannot change the result.
+// The query pass of a head finishes before its key pass reads lse and D.
 //
 // Each staged head holds Q, K, V and dO of its rows as bf16 [m16][kKStride]
 // (zero rows past m), then lse and D as fp32 [m16]. Every operand fragment
@@ -264,12 +275,11 @@ __device__ void bwd_query_tile(uint32_t hs, int m, int i0, const UBlock& ub, flo
 }
 
 // Key pass for keys [j0, j0 + 16) of one staged head: dK, dV through
-// dkrow(j), dvrow(j), and dS_ij (bf16) into the head's U plane at
-// Uh[slot[j] * P + slot[i]] (the positions its bias was read from). Warp-wide.
-template <int PM, class UBlock, class KRow, class VRow>
-__device__ void bwd_key_tile(uint32_t hs, const Particles<PM>& S, int j0, const UBlock& ub, const float* lse,
-                             const float* dd, uint16_t* Uh, int P, const KRow& dkrow, const VRow& dvrow) {
-  const int m = S.m;
+// dkrow(j), dvrow(j), and dS_ij added to gh[8 r] of the pair's record r
+// (gh = the jet's first record, at head h). Warp-wide.
+template <class UBlock, class KRow, class VRow>
+__device__ void bwd_key_tile(uint32_t hs, int m, int j0, const UBlock& ub, const float* lse, const float* dd,
+                             float* gh, const KRow& dkrow, const VRow& dvrow) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const uint32_t pitch = kKStride * 2, tb = (uint32_t)bwd_tensor_bytes(m);
   const uint32_t Qs = hs, Ks = hs + tb, Vs = hs + 2 * tb, Os = hs + 3 * tb;
@@ -280,7 +290,6 @@ __device__ void bwd_key_tile(uint32_t hs, const Particles<PM>& S, int j0, const 
   uint32_t ak[4], av[4];
   ldsm_x4(Ks + j0 * pitch + fa, ak);
   ldsm_x4(Vs + j0 * pitch + fa, av);
-  const size_t ra = (size_t)S.slot[ja] * P, rb = (size_t)S.slot[jb] * P;
   float dk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float dv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int i0 = 0; i0 < m; i0 += 16) {
@@ -321,9 +330,12 @@ __device__ void bwd_key_tile(uint32_t hs, const Particles<PM>& S, int j0, const 
     mma_16816(dk + 4, pd, bqt[2], bqt[3]);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const int i = col(e);
+      const int i = col(e), j = e & 2 ? jb : ja;
       const bool row_ok = e & 2 ? vb : va;
-      if (row_ok && i < m && in_bounds(i >= 0)) Uh[(e & 2 ? rb : ra) + S.slot[i]] = f32_to_bf16(ds[e]);
+      if (row_ok && i < m && in_bounds(i >= 0)) {
+        const int hi = max(i, j), lo = min(i, j);
+        atomicAdd(gh + 8 * (hi * (hi + 1) / 2 + lo), ds[e]);
+      }
     }
   }
   if (va) {
@@ -344,7 +356,7 @@ __device__ void bwd_key_tile(uint32_t hs, const Particles<PM>& S, int j0, const 
   }
 }
 
-constexpr int kBwdStageBytes = 100 * 1024;  // staged heads of the attention backward
+constexpr int kBwdStageBytes = 192 * 1024;  // staged heads of the attention backward
 
 template <int PM>
 struct AttnBwdSmem {
@@ -353,18 +365,23 @@ struct AttnBwdSmem {
 };
 
 template <int PM>
-__global__ void __launch_bounds__(256) k_attn_bwd(JetArgs J, BwdArgs X) {
+__global__ void __launch_bounds__(512, 1) k_attn_bwd(JetArgs J, BwdArgs X) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AttnBwdSmem<PM>& S = *reinterpret_cast<AttnBwdSmem<PM>*>(smem_raw);
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
   for (int n = blockIdx.x; n < J.N; n += gridDim.x) {
     stage_jet<PM, false>(S.part, J, n);
     const int m = S.part.m;
+    const size_t rowbase = (size_t)X.T[n] * kTileM;
     if (m > 0) {
+      // the jet's gradient records start at zero
+      const int np = m * (m + 1) / 2;
+      float4* g4 = reinterpret_cast<float4*>(X.grec + rowbase * 8);
+      for (int e = threadIdx.x; e < 2 * np; e += blockDim.x) g4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
       const int hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m), m16 = round16(m);
       const int HR = max(1, min(kH, kBwdStageBytes / hb));
       const int tiles = (m + 15) >> 4;
-      const GlobalUBias<PM> ub{&S.part, X.U, n, J.P};
+      const RecordUBias ub{reinterpret_cast<const __half*>(X.urec + rowbase)};
       if (in_bounds(hb <= kBwdStageBytes)) {
         for (int h0 = 0; h0 < kH; h0 += HR) {
           const int hr = min(HR, kH - h0);
@@ -382,10 +399,9 @@ __global__ void __launch_bounds__(256) k_attn_bwd(JetArgs J, BwdArgs X) {
             const int hh = it / tiles, h = h0 + hh;
             unsigned char* hbuf = S.stage + hh * hb;
             const float* lse = reinterpret_cast<const float*>(hbuf + 4 * tb);
-            uint16_t* Uh = X.U + ((size_t)n * kH + h) * J.P * J.P;
-            bwd_key_tile<PM>(smem_u32(hbuf), S.part, (it % tiles) * 16, ub.head(h), lse, lse + m16, Uh, J.P,
-                             [&](int j) { return X.dk + qkv_off<PM>(S.part, J, n, h, j); },
-                             [&](int j) { return X.dv + qkv_off<PM>(S.part, J, n, h, j); });
+            bwd_key_tile(smem_u32(hbuf), m, (it % tiles) * 16, ub.head(h), lse, lse + m16, X.grec + rowbase * 8 + h,
+                         [&](int j) { return X.dk + qkv_off<PM>(S.part, J, n, h, j); },
+                         [&](int j) { return X.dv + qkv_off<PM>(S.part, J, n, h, j); });
           }
           __syncthreads();
         }
@@ -402,18 +418,21 @@ __global__ void __launch_bounds__(256) k_attn_bwd(JetArgs J, BwdArgs X) {
 //
 // For the unordered pair (a, b) of a jet, the bias row u = MLP(f(a, b)) feeds
 // both U[h, a, b] and U[h, b, a], so its upstream gradient is
-// g_h = dS_h[a, b] + dS_h[b, a] (a != b) or dS_h[a, a]. Per tile of 128 such
-// rows (one CTA, 512 threads; thread (row r, quarter c) owns TMEM lane r and
-// columns 16c .. 16c + 15 of each 64-wide accumulator):
-//   z1 = W1' f + b1', h1 = GELU(z1), z2 = W2' h1 + b2', ... h3   (tcgen05, z in TMEM)
+// g_h = dS_h[a, b] + dS_h[b, a] (a != b) or dS_h[a, a], the record that the
+// attention backward accumulated. Per tile of 128 such rows (one CTA, 512
+// threads; thread (row r, quarter c) owns TMEM lane r and columns 16c ..
+// 16c + 15 of each 64-wide accumulator):
+//   z1 = W1' f + b1', h1 = GELU(z1), z2 = W2' h1 + b2', ... h3   (tcgen05)
 //   e3 = g W4 (issued with z1), d3 = e3 * GELU'(z3), e2 = d3 W3', d2, e1 = d2 W2', d1
 //   dW4 += g^T h3, dWk' += dk^T h(k-1) (h0 = f), dbk' += column sums of dk
-// with bf16 operands and fp32 accumulation; the folded layer-1 weights and
-// the features enter as bf16 hi + lo terms. GELU is the erf form (normcdff).
-// The weight gradients are 31 (layer, 16-row block, up to three 8-column
-// blocks) parts spread over the 16 warps as m16n8k16 MMAs whose A operand
-// (d^T) and B operand (h) come from the row-major tiles through
-// ldmatrix.trans; a column block of ones gives the bias gradients.
+// with bf16 operands and fp32 accumulation; f, g and the folded layer-1
+// weights enter as bf16 hi + lo terms. GELU is the tanh form the forward
+// kernels use (tanh.approx); GELU'(z) is computed with h and parked in TMEM
+// over z until the backward step needs it. The weight gradients are 31
+// (layer, 16-row block, up to three 8-column blocks) parts spread over the
+// 16 warps as m16n8k16 MMAs whose A operand (d^T) and B operand (h) come
+// from the row-major tiles through ldmatrix.trans; a column block of ones
+// gives the bias gradients.
 
 constexpr int kBwdMaxCtas = 256;     // partial-gradient slots in the workspace
 constexpr int kFoldedFloats = 9160;  // W1 b1 W2 b2 W3 b3 W4 b4, as pb_fold_affine lays them out
@@ -427,13 +446,13 @@ struct GradArgs {
 template <int PM>
 struct MlpBwdSmem {
   __nv_bfloat16 A0[kTileM * 16];     // [hi(f) | lo(f) | hi(f) | 0]
-  __nv_bfloat16 G4[kTileM * 16];     // [g (8 heads) | 0]
+  __nv_bfloat16 G4[kTileM * 16];     // [hi(g) | lo(g)] (8 heads each)
   __nv_bfloat16 Hs[3][kTileM * 64];  // h1, h2, h3
   __nv_bfloat16 Ds[3][kTileM * 64];  // d1, d2, d3 = dL/dz
   __nv_bfloat16 W1f[64 * 16];        // [hi(W1') | hi(W1') | lo(W1') | 0] per output row
   __nv_bfloat16 Wf[2][64 * 64];      // W2', W3' as [out][in]
   __nv_bfloat16 Wt[2][64 * 64];      // W2'^T, W3'^T as [in][out]
-  __nv_bfloat16 W4t[64 * 16];        // W4^T as [in][out], out 8..15 zero
+  __nv_bfloat16 W4t[64 * 16];        // [W4^T | W4^T] as [in][out]
   float bias[3][64];                 // b1', b2', b3'
   uint64_t mbar;
   uint32_t tmem_base;
@@ -457,14 +476,40 @@ __device__ void bwd_load_weights(MlpBwdSmem<PM>& S, const MlpArgs& W) {
     const float w1 = k < 12 ? W.W1[r * 4 + (k & 3)] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(w1);
     S.W1f[cofs(r, k, 16)] = (k >= 8 && k < 12) ? __float2bfloat16_rn(w1 - __bfloat162float(hi)) : hi;
-    S.W4t[cofs(r, k, 16)] = __float2bfloat16_rn(k < 8 ? W.W4[k * 64 + r] : 0.f);
+    S.W4t[cofs(r, k, 16)] = __float2bfloat16_rn(W.W4[(k & 7) * 64 + r]);
   }
   for (int e = tid; e < 3 * 64; e += nthr) S.bias[e >> 6][e & 63] = (e < 64 ? W.b1 : (e < 128 ? W.b2 : W.b3))[e & 63];
 }
 
-__device__ __forceinline__ float gelu_erf(float z) { return z * normcdff(z); }
-__device__ __forceinline__ float gelu_erf_grad(float z) {
-  return normcdff(z) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GELU(z) = z/2 (1 + tanh(u)), u = sqrt(2/pi) (z + 0.044715 z^3), and its derivative.
+__device__ __forceinline__ void gelu_tanh_and_grad(float z, float& h, float& dh) {
+  constexpr float kC0 = 0.7978845608028654f, kC1 = 0.044715f;
+  const float z2 = z * z;
+  const float t = tanh_approx(kC0 * fmaf(kC1 * z2, z, z));
+  const float half_z = 0.5f * z;
+  h = fmaf(half_z, t, half_z);
+  dh = fmaf(0.5f, t, 0.5f) + half_z * fmaf(-t, t, 1.f) * kC0 * fmaf(3.f * kC1, z2, 1.f);
+}
+
+// TMEM <- registers, 32 lanes x 16 columns (thread t of the warp writes lane
+// quadrant base + t), then wait for the stores.
+__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
 }
 
 // One weight-gradient part: layer L (1..4), 16-row block mb of dW, column
@@ -520,10 +565,12 @@ __device__ __forceinline__ void grad_mma(const MlpBwdSmem<PM>& S, const GradPart
   }
 }
 
-// The part's accumulators into the CTA's partial (folded layout).
-__device__ void grad_store(const GradPart& gp, float (*acc)[4], float* part) {
+// The part's accumulators into the CTA's partial (folded layout), added to
+// what the slot holds when `accumulate`.
+__device__ void grad_store(const GradPart& gp, float (*acc)[4], float* part, bool accumulate) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int oa = gp.mb * 16 + g, ob = oa + 8;
+  auto put = [&](int idx, float v) { part[idx] = accumulate ? part[idx] + v : v; };
   for (int j = 0; j < gp.nc; ++j) {
     const int nb = gp.nb0 + j;
     const float* c = acc[j];
@@ -533,40 +580,43 @@ __device__ void grad_store(const GradPart& gp, float (*acc)[4], float* part) {
       const float p2 = __shfl_down_sync(0xffffffffu, c[2], 2), p3 = __shfl_down_sync(0xffffffffu, c[3], 2);
       if (nb == 0) {
         if (t < 2) {
-          part[kOffW1 + oa * 4 + 2 * t] = c[0] + p0;
-          part[kOffW1 + oa * 4 + 2 * t + 1] = c[1] + p1;
-          part[kOffW1 + ob * 4 + 2 * t] = c[2] + p2;
-          part[kOffW1 + ob * 4 + 2 * t + 1] = c[3] + p3;
+          put(kOffW1 + oa * 4 + 2 * t, c[0] + p0);
+          put(kOffW1 + oa * 4 + 2 * t + 1, c[1] + p1);
+          put(kOffW1 + ob * 4 + 2 * t, c[2] + p2);
+          put(kOffW1 + ob * 4 + 2 * t + 1, c[3] + p3);
         }
       } else if (t == 0) {
-        part[kOffB1 + oa] = c[0];
-        part[kOffB1 + ob] = c[2];
+        put(kOffB1 + oa, c[0]);
+        put(kOffB1 + ob, c[2]);
       }
-    } else if (gp.L == 4) {  // output rows 8..15 are padding
+    } else if (gp.L == 4) {  // rows g: sum hi(g) h3, rows g + 8: sum lo(g) h3
       if (nb < 8) {
-        part[kOffW4 + g * 64 + nb * 8 + 2 * t] = c[0];
-        part[kOffW4 + g * 64 + nb * 8 + 2 * t + 1] = c[1];
+        put(kOffW4 + g * 64 + nb * 8 + 2 * t, c[0] + c[2]);
+        put(kOffW4 + g * 64 + nb * 8 + 2 * t + 1, c[1] + c[3]);
       } else if (t == 0) {
-        part[kOffB4 + g] = c[0];
+        put(kOffB4 + g, c[0] + c[2]);
       }
     } else {
       const int offW = gp.L == 2 ? kOffW2 : kOffW3, offB = gp.L == 2 ? kOffB2 : kOffB3;
       if (nb < 8) {
-        part[offW + oa * 64 + nb * 8 + 2 * t] = c[0];
-        part[offW + oa * 64 + nb * 8 + 2 * t + 1] = c[1];
-        part[offW + ob * 64 + nb * 8 + 2 * t] = c[2];
-        part[offW + ob * 64 + nb * 8 + 2 * t + 1] = c[3];
+        put(offW + oa * 64 + nb * 8 + 2 * t, c[0]);
+        put(offW + oa * 64 + nb * 8 + 2 * t + 1, c[1]);
+        put(offW + ob * 64 + nb * 8 + 2 * t, c[2]);
+        put(offW + ob * 64 + nb * 8 + 2 * t + 1, c[3]);
       } else if (t == 0) {
-        part[offB + oa] = c[0];
-        part[offB + ob] = c[2];
+        put(offB + oa, c[0]);
+        put(offB + ob, c[2]);
       }
     }
   }
 }
 
+// The T[N] tiles are split evenly over the CTAs (a CTA's range may start and
+// end inside a jet); the CTA's weight-gradient partial goes to slot
+// blockIdx.x, added to it when `accumulate` (later chunks of a batch).
 template <int PM>
-__global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, const uint16_t* __restrict__ dU,
-                                                    float* __restrict__ partials) {
+__global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArgs X, float* __restrict__ partials,
+                                                    int accumulate) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   MlpBwdSmem<PM>& S = *reinterpret_cast<MlpBwdSmem<PM>*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -581,7 +631,7 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, const 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192), e3 / e2 / e1 [192, 256)
+  // TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192) (then GELU'), e3 / e2 / e1 [192, 256)
   const uint32_t tm = S.tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
   constexpr uint32_t kId = idesc_bf16_m128(64);
   const uint32_t a0 = smem_u32(S.A0), g4 = smem_u32(S.G4), w1f = smem_u32(S.W1f), w4t = smem_u32(S.W4t);
@@ -627,65 +677,78 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, const 
     *reinterpret_cast<uint4*>(T + cofs(r, 16 * c, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
     *reinterpret_cast<uint4*>(T + cofs(r, 16 * c + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
   };
-  // h_k = GELU(z_k + b_k) (k = 0..2) of this thread's 16 columns
+  // h_k = GELU(z_k + b_k) to the operand tile, GELU'(z_k + b_k) back over z_k in TMEM
   auto hidden = [&](int k) {
-    float z[16];
-    tmem_ld16_wait(tm + lane_off + 64u * k + 16u * c, z);
+    float z[16], h[16];
+    const uint32_t ta = tm + lane_off + 64u * k + 16u * c;
+    tmem_ld16_wait(ta, z);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) z[i] = gelu_erf(z[i] + S.bias[k][16 * c + i]);
-    store16(S.Hs[k], z);
+    for (int i = 0; i < 16; ++i) gelu_tanh_and_grad(z[i] + S.bias[k][16 * c + i], h[i], z[i]);
+    store16(S.Hs[k], h);
+    tmem_st16_wait(ta, z);
   };
   // d_k = e * GELU'(z_k + b_k)
   auto delta = [&](int k) {
-    float z[16], e[16];
-    tmem_ld16_wait(tm + lane_off + 64u * k + 16u * c, z);
+    float gp[16], e[16];
+    tmem_ld16_wait(tm + lane_off + 64u * k + 16u * c, gp);
     tmem_ld16_wait(tm + lane_off + 192u + 16u * c, e);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) e[i] *= gelu_erf_grad(z[i] + S.bias[k][16 * c + i]);
+    for (int i = 0; i < 16; ++i) e[i] *= gp[i];
     store16(S.Ds[k], e);
   };
 
-  for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
+  const long long Ttot = X.T[J.N];
+  const long long lo = Ttot * blockIdx.x / gridDim.x, hi = Ttot * (blockIdx.x + 1) / gridDim.x;
+  int n = 0;
+  {
+    int l = 0, rr = J.N;  // first jet whose tiles reach past lo
+    while (l < rr) {
+      const int mid = (l + rr) >> 1;
+      if (X.T[mid + 1] > lo) rr = mid; else l = mid + 1;
+    }
+    n = l;
+  }
+  for (; n < J.N && X.T[n] < hi && !aborted; ++n) {
+    const long long tj0 = X.T[n], tj1 = X.T[n + 1];
+    if (tj1 <= tj0) continue;  // no pairs
     stage_jet<PM>(S.part, J, n);
-    const int m = S.part.m, P = J.P;
-    const int npairs = m * (m + 1) / 2, ntiles = (npairs + kTileM - 1) / kTileM;
-    const uint16_t* Un = dU + (size_t)n * kH * P * P;
-    for (int t = 0; t < ntiles; ++t) {
+    const int m = S.part.m;
+    const int npairs = m * (m + 1) / 2;
+    const float* gjet = X.grec + (size_t)tj0 * kTileM * 8;
+    const int t_first = (int)(max(lo, tj0) - tj0), t_last = (int)(min(hi, tj1) - tj0);
+    for (int t = t_first; t < t_last; ++t) {
       // row r: the unordered pair p = b(b+1)/2 + a; features (c = 0) and g (c = 1)
       const int p = t * kTileM + r;
       int a = 0, b = 0;
       bool valid = p < npairs;
-      if (valid && c < 2) {
+      if (valid && c == 0) {
         TriPairs{}.map(p, a, b);
         valid = in_bounds(a >= 0 && a <= b && b < m);
       }
       if (c == 0) {
         float f[4] = {0.f, 0.f, 0.f, 0.f};
         if (valid) pair_feat<PM, false>(S.part, a, b, f);
-        uint32_t hl[4], lh[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const uint32_t hi = cvt_bf16x2(f[2 * i], f[2 * i + 1]);
-          hl[i] = hi;
-          lh[i] = cvt_bf16x2(f[2 * i] - bf16lo(hi), f[2 * i + 1] - bf16hi(hi));
-        }
-        hl[2] = lh[0];
-        hl[3] = lh[1];
-        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 0, 16)) = make_uint4(hl[0], hl[1], hl[2], hl[3]);
-        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 8, 16)) = make_uint4(hl[0], hl[1], 0u, 0u);
+        const uint32_t h01 = cvt_bf16x2(f[0], f[1]), h23 = cvt_bf16x2(f[2], f[3]);
+        const uint32_t l01 = cvt_bf16x2(f[0] - bf16lo(h01), f[1] - bf16hi(h01));
+        const uint32_t l23 = cvt_bf16x2(f[2] - bf16lo(h23), f[3] - bf16hi(h23));
+        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 0, 16)) = make_uint4(h01, h23, l01, l23);
+        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 8, 16)) = make_uint4(h01, h23, 0u, 0u);
       } else if (c == 1) {
-        float gv[8];
-        const int sa = S.part.slot[a], sb = S.part.slot[b];
-#pragma unroll
-        for (int h = 0; h < kH; ++h) {
-          const uint16_t* Uh = Un + (size_t)h * P * P;
-          gv[h] = valid ? bf16_to_f32(Uh[(size_t)sa * P + sb]) + (a != b ? bf16_to_f32(Uh[(size_t)sb * P + sa]) : 0.f)
-                        : 0.f;
+        float gv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (valid) {
+          const float4 u0 = *reinterpret_cast<const float4*>(gjet + (size_t)p * 8);
+          const float4 u1 = *reinterpret_cast<const float4*>(gjet + (size_t)p * 8 + 4);
+          gv[0] = u0.x; gv[1] = u0.y; gv[2] = u0.z; gv[3] = u0.w;
+          gv[4] = u1.x; gv[5] = u1.y; gv[6] = u1.z; gv[7] = u1.w;
         }
-        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 0, 16)) =
-            make_uint4(cvt_bf16x2(gv[0], gv[1]), cvt_bf16x2(gv[2], gv[3]), cvt_bf16x2(gv[4], gv[5]),
-                       cvt_bf16x2(gv[6], gv[7]));
-        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 8, 16)) = make_uint4(0u, 0u, 0u, 0u);
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          hw[i] = cvt_bf16x2(gv[2 * i], gv[2 * i + 1]);
+          lw[i] = cvt_bf16x2(gv[2 * i] - bf16lo(hw[i]), gv[2 * i + 1] - bf16hi(hw[i]));
+        }
+        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 0, 16)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 8, 16)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       // forward: z1 (and e3 = g W4, which needs nothing else), z2, z3
       if (!issue([&] {
@@ -733,8 +796,8 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, const 
     aborted = __syncthreads_or(aborted || !ok) != 0;
   }
   float* part = partials + (size_t)blockIdx.x * kFoldedFloats;
-  grad_store(gp0, acc0, part);
-  if (has1) grad_store(gp1, acc1, part);
+  grad_store(gp0, acc0, part, accumulate != 0);
+  if (has1) grad_store(gp1, acc1, part, accumulate != 0);
   tc_fence_before();
   __syncthreads();
   if (aborted && tid == 0) (void)mbar_wait(&S.mbar, phase ^ 1u);  // bounded: the last commit before TMEM is freed

@@ -1812,8 +1812,12 @@ __device__ void jet_counts(const JetArgs& J, int* T) {
   }
 }
 
-template <int PM>
-__global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, QkvArgs X, unsigned char* ws) {
+// kBiasOnly: phase 0 and phase A only (no barrier, no attention, counters
+// untouched); CTA 0 also writes the tile prefix T[0..N] to Tout. The bias
+// records then serve the backward pass.
+template <int PM, bool kBiasOnly = false>
+__global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, QkvArgs X, unsigned char* ws,
+                                                       int* Tout) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FusedGridSmem<PM>& S = *reinterpret_cast<FusedGridSmem<PM>*>(smem_raw);
   constexpr int NG = 4, SL = 2, JB = GridCfg<PM>::kBatch;
@@ -1924,6 +1928,13 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
       aborted = __syncthreads_or(!ok) != 0;
       n = n_next;
     }
+  }
+
+  if (kBiasOnly) {
+    if (b == 0)
+      for (int n = tid; n <= N; n += blockDim.x) Tout[n] = S.T[n];
+    mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
+    return;
   }
 
   // --------------------------------------------------------------- barrier

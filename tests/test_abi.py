@@ -170,11 +170,24 @@ def _r256(b):
 
 
 def test_backward_workspace_size(L):
-    """bf16 bias planes [N, 8, P, P] plus min(N, 256) fp32 gradient partials."""
-    for N, P in ((2, 8), (128, 128), (300, 37)):
+    """Header, 16-byte bias and 32-byte gradient records for the rows of a
+    chunk's tiles (at most 8192 jets, padded N*P <= 2^21), the chunk's tile
+    prefix and 256 fp32 partials of the folded weight gradients."""
+    def want(N, P, tokens=None):
+        nc = min(N, 8192 if tokens is not None else min(8192, (1 << 21) // P))
+        rows = nc * ((P * (P + 1) // 2 + 127) // 128) * 128
+        if tokens is not None:
+            rows = min(rows, tokens * (P + 1) // 2 + 127 * nc + 128)
+        grec = _r256(256 + rows * 16)
+        table = _r256(grec + rows * 32)
+        part = _r256(table + (nc + 1) * 4)
+        return _r256(part + 256 * ops.FOLDED_FLOATS * 4)
+    for N, P in ((2, 8), (128, 128), (300, 37), (20000, 256)):
         js, keep = _jets(N=N, P=P)
-        want = _r256(N * 8 * P * P * 2) + _r256(min(N, 256) * ops.FOLDED_FLOATS * 4)
-        assert L.pb_backward_workspace_bytes(C.byref(js)) == want
+        assert L.pb_backward_workspace_bytes(C.byref(js)) == want(N, P)
+    js, keep = _jets(N=8192, P=128, ptr=True)
+    js.tokens = 327680
+    assert L.pb_backward_workspace_bytes(C.byref(js)) == want(8192, 128, 327680)
     js.P = 300
     assert L.pb_backward_workspace_bytes(C.byref(js)) == 0
 

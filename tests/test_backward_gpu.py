@@ -7,12 +7,16 @@ arithmetic of the forward bars and the backward's own roundings):
                   The bias enters through the forward MLP kernel (bias bar:
                   rel L2 1e-2), the softmax gradient dS = P (dP - D) loses
                   relative accuracy where dP ~ D, and dq, dk, dv are bf16.
-  MLP gradients   relative L2 per folded tensor <= 3e-2. dL/dU is stored as
-                  bf16 and the MLP is recomputed with bf16 operands; each
-                  gradient is a sum of many such terms.
-  db4             zero in exact arithmetic (rows of dS sum to 0); bounded by
-                  the same relative error of the sum of |dL/dU|, here taken
-                  as 3e-2 times the largest dW4 row norm.
+  MLP gradients   relative L2 per folded tensor <= 4e-2. These sums of
+                  g * h over the pairs cancel heavily (each row of dS sums to
+                  0), so an error in the bias U reaches them amplified:
+                  perturbing U in the fp64 oracle by noise of 5e-3 (2e-2)
+                  moves them by up to 1e-2 (4e-2), a gain of up to 2-4 on the
+                  bias bar (rel L2 1e-2). The bias here is the forward
+                  kernel's (f16 records); dL/dU accumulates in fp32; the MLP
+                  is recomputed with bf16 operands (f and g as hi + lo).
+  db4             zero in exact arithmetic (rows of dS sum to 0): at most
+                  4e-2 times the largest dW4 row norm.
 """
 import numpy as np
 import pytest
@@ -24,7 +28,7 @@ from tests import parity as pt
 pytestmark = pytest.mark.gpu
 
 QKV_RELL2 = 2e-2
-GRAD_RELL2 = 3e-2
+GRAD_RELL2 = 4e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -131,6 +135,13 @@ def test_backward_large_workloads_sampled(bw, name):
             check_qkv(got, r[n], s)
     s = synth.slice_jets(b, 0, 64)
     compare(s, seed=2, bw=bw)
+
+
+def test_backward_in_chunks(bw):
+    """More jets than one pass of the bias kernel takes (8192): the batch runs
+    in two chunks whose weight gradients add up in the same partial slots."""
+    compare(synth.make_jets(N=8300, P=8, dist="uniform", mult_lo=1, mult_hi=8, mask_mode="scrambled", seed=12),
+            seed=3, bw=bw)
 
 
 def test_backward_empty_batch_zero_gradients():
