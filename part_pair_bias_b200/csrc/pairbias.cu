@@ -345,7 +345,7 @@ pb_status run_backward(const pb::JetArgs& J, const pb::MlpArgs& W, pb::BwdArgs X
     }
     if ((st = run_backward_chunk<PM>(Jc, W, Xc, ws, table, partials, mlp_grid, c0 > 0, s)) != PB_OK) return st;
   }
-  pb::k_grad_reduce<<<(pb::kFoldedFloats + 255) / 256, 256, 0, s>>>(partials, mlp_grid, G);
+  pb::k_grad_reduce<<<pb::kReduceCtas, 256, 0, s>>>(partials, mlp_grid, G);
   return launched("k_grad_reduce");
 }
 
@@ -522,7 +522,7 @@ pb_status pair_attention_backward(const pb_jets* jets, const pb_mlp* mlp, int H,
   const pb::GradArgs G{gp[0], gp[1], gp[2], gp[3], gp[4], gp[5], gp[6], gp[7]};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (J.N == 0) {  // no pairs: the weight gradients are zero
-    pb::k_grad_reduce<<<(pb::kFoldedFloats + 255) / 256, 256, 0, s>>>(nullptr, 0, G);
+    pb::k_grad_reduce<<<pb::kReduceCtas, 256, 0, s>>>(nullptr, 0, G);
     return launched("k_grad_reduce");
   }
   if (!q || !k || !v || !dout || !dq || !dk || !dv) return fail(PB_EINVAL, "q, k, v, dout, dq, dk and dv must be non-NULL");

@@ -66,19 +66,21 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 // ============================================== attention backward (k_attn_bwd)
 //
 // Per (jet, head), over the jet's m valid particles, with s = q.k/4 + U in
-// log2 units (x log2 e):
-//   query pass (warp = 16 queries): the row maximum and sum of exp2 give
-//     lse_i; O_i = sum_j p_ij v_j (p split into two bf16 terms so that O is
-//     accurate to ~2^-17) gives D_i = dO_i . O_i; a second sweep over the keys
-//     recomputes p_ij = exp2(s_ij - lse_i), dP_ij = dO_i . v_j,
-//     dS_ij = p_ij (dP_ij - D_i) and accumulates dQ_i = 1/4 sum_j dS_ij k_j;
-//   key pass (warp = 16 keys): the transposed tiles S^T = K Q^T, dP^T = V dO^T
-//     give p_ij and dS_ij again, accumulated into dV_j = sum_i p_ij dO_i and
-//     dK_j = 1/4 sum_i dS_ij q_i; dS_ij is added (fp32) to the record of the
-//     unordered pair {i, j}. Each off-diagonal record receives exactly two
-//     additions onto zero (dS_ij and dS_ji) and a diagonal one one, so the
-//     order of the atomic adds cannot change the result.
-// The query pass of a head finishes before its key pass reads lse and D.
+// log2 units (x log2 e) and 16-particle tiles I, J:
+//   statistics (warp = tile I as queries): the row maximum and sum of exp2
+//     give lse_i; O_i = sum_j p_ij v_j (p split into two bf16 terms so that O
+//     is accurate to ~2^-17) gives D_i = dO_i . O_i;
+//   gradients (warp = tile I, both as queries and as keys), for every tile J:
+//     as queries  p_ij = exp2(s_ij - lse_i), dS_ij = p_ij (dO_i.v_j - D_i),
+//                 dQ_i += 1/4 dS_ij k_j;
+//     as keys     p_ji, dS_ji from the transposed tiles K_I Q_J^T, V_I dO_J^T
+//                 (the bias U_ji = U_ij is the same element), dV_i += p_ji dO_j,
+//                 dK_i += 1/4 dS_ji q_j;
+//     both dS_ij and dS_ji then sit at the same fragment position, and the
+//     pair's bias row gets g = dS_ij + dS_ji (dS_ii on the diagonal), written
+//     once, by the tile of its smaller particle index, to the pair's fp32
+//     record: no atomics and no zero-fill.
+// Every statistics item finishes before any gradient item reads lse and D.
 //
 // Each staged head holds Q, K, V and dO of its rows as bf16 [m16][kKStride]
 // (zero rows past m), then lse and D as fp32 [m16]. Every operand fragment
@@ -158,12 +160,10 @@ __device__ __forceinline__ void bwd_scores(float* s, const float* u, int m, cons
   for (int e = 0; e < 8; ++e) s[e] = col(e) < m ? fmaf(s[e], qs, u[e] * kLog2e) : -INFINITY;
 }
 
-// Query pass for queries [i0, i0 + 16) of one staged head at shared address
-// hs: writes lse (log2 units) and D of its valid rows and dQ through dqrow(i).
-// Warp-wide.
-template <class UBlock, class ORow>
-__device__ void bwd_query_tile(uint32_t hs, int m, int i0, const UBlock& ub, float* lse, float* dd,
-                               const ORow& dqrow) {
+// Statistics of the queries [i0, i0 + 16) of one staged head at shared
+// address hs: lse (log2 units) and D of its valid rows. Warp-wide.
+template <class UBlock>
+__device__ void bwd_stats_tile(uint32_t hs, int m, int i0, const UBlock& ub, float* lse, float* dd) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const uint32_t pitch = kKStride * 2, tb = (uint32_t)bwd_tensor_bytes(m);
   const uint32_t Qs = hs, Ks = hs + tb, Vs = hs + 2 * tb, Os = hs + 3 * tb;
@@ -174,8 +174,6 @@ __device__ void bwd_query_tile(uint32_t hs, int m, int i0, const UBlock& ub, flo
   uint32_t aq[4], ado[4];
   ldsm_x4(Qs + i0 * pitch + fa, aq);
   ldsm_x4(Os + i0 * pitch + fa, ado);
-
-  // sweep 1: statistics and O
   float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float mxa = -INFINITY, mxb = -INFINITY, la = 0.f, lb = 0.f;
   for (int n0 = 0; n0 < m; n0 += 16) {
@@ -216,7 +214,6 @@ __device__ void bwd_query_tile(uint32_t hs, int m, int i0, const UBlock& ub, flo
   la += __shfl_xor_sync(0xffffffffu, la, 2);
   lb += __shfl_xor_sync(0xffffffffu, lb, 1);
   lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-  const float lse_a = mxa + __log2f(la), lse_b = mxb + __log2f(lb);
   // D = dO . O: the lane's O elements sit at the positions of its dO fragment
   float da = bf16lo(ado[0]) * o[0] + bf16hi(ado[0]) * o[1] + bf16lo(ado[2]) * o[4] + bf16hi(ado[2]) * o[5];
   float db = bf16lo(ado[1]) * o[2] + bf16hi(ado[1]) * o[3] + bf16lo(ado[3]) * o[6] + bf16hi(ado[3]) * o[7];
@@ -224,135 +221,111 @@ __device__ void bwd_query_tile(uint32_t hs, int m, int i0, const UBlock& ub, flo
   da += __shfl_xor_sync(0xffffffffu, da, 2);
   db += __shfl_xor_sync(0xffffffffu, db, 1);
   db += __shfl_xor_sync(0xffffffffu, db, 2);
-  da /= la;
-  db /= lb;
   if (t == 0) {
     if (va) {
-      lse[ia] = lse_a;
-      dd[ia] = da;
+      lse[ia] = mxa + __log2f(la);
+      dd[ia] = da / la;
     }
     if (vb) {
-      lse[ib] = lse_b;
-      dd[ib] = db;
+      lse[ib] = mxb + __log2f(lb);
+      dd[ib] = db / lb;
     }
-  }
-
-  // sweep 2: dS and dQ
-  float dq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int n0 = 0; n0 < m; n0 += 16) {
-    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint32_t bk[4];
-    ldsm_x4(Ks + n0 * pitch + fbn, bk);
-    mma_16816(s, aq, bk[0], bk[1]);
-    mma_16816(s + 4, aq, bk[2], bk[3]);
-    float u[8];
-    ub(n0, i0, ia, ib, t, m, u);
-    bwd_scores(s, u, m, [&](int e) { return n0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1); });
-    float dp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint32_t bv[4];
-    ldsm_x4(Vs + n0 * pitch + fbn, bv);
-    mma_16816(dp, ado, bv[0], bv[1]);
-    mma_16816(dp + 4, ado, bv[2], bv[3]);
-    float ds[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ds[e] = ex2(s[e] - (e & 2 ? lse_b : lse_a)) * (dp[e] - (e & 2 ? db : da));
-    uint32_t pd[4], bkt[4];
-    pack_bf16_frag(ds, pd);
-    ldsm_x4_t(Ks + n0 * pitch + fbt, bkt);
-    mma_16816(dq, pd, bkt[0], bkt[1]);
-    mma_16816(dq + 4, pd, bkt[2], bkt[3]);
-  }
-  if (va) {
-    uint16_t* op = dqrow(ia);
-    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(0.25f * dq[0], 0.25f * dq[1]);
-    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(0.25f * dq[4], 0.25f * dq[5]);
-  }
-  if (vb) {
-    uint16_t* op = dqrow(ib);
-    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(0.25f * dq[2], 0.25f * dq[3]);
-    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(0.25f * dq[6], 0.25f * dq[7]);
   }
 }
 
-// Key pass for keys [j0, j0 + 16) of one staged head: dK, dV through
-// dkrow(j), dvrow(j), and dS_ij added to gh[8 r] of the pair's record r
-// (gh = the jet's first record, at head h). Warp-wide.
-template <class UBlock, class KRow, class VRow>
-__device__ void bwd_key_tile(uint32_t hs, int m, int j0, const UBlock& ub, const float* lse, const float* dd,
-                             float* gh, const KRow& dkrow, const VRow& dvrow) {
+// Gradients of tile [i0, i0 + 16) of one staged head: dQ (its particles as
+// queries), dK and dV (as keys) through dqrow / dkrow / dvrow, and the
+// pairs' bias-row gradients g into gh[8 r] (gh = the jet's first record at
+// head h, r = j(j+1)/2 + i for i <= j). Warp-wide.
+template <class UBlock, class QRow, class KRow, class VRow>
+__device__ void bwd_pair_tile(uint32_t hs, int m, int i0, const UBlock& ub, const float* lse, const float* dd,
+                              float* gh, const QRow& dqrow, const KRow& dkrow, const VRow& dvrow) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const uint32_t pitch = kKStride * 2, tb = (uint32_t)bwd_tensor_bytes(m);
   const uint32_t Qs = hs, Ks = hs + tb, Vs = hs + 2 * tb, Os = hs + 3 * tb;
-  const int nrows = min(16, m - j0);
+  const int nrows = min(16, m - i0);
   const bool va = g < nrows, vb = g + 8 < nrows;
-  const int ja = j0 + (va ? g : 0), jb = j0 + (vb ? g + 8 : 0);
+  const int ia = i0 + (va ? g : 0), ib = i0 + (vb ? g + 8 : 0);
   const uint32_t fa = frag_a_off(lane), fbn = frag_bn_off(lane), fbt = frag_bt_off(lane);
-  uint32_t ak[4], av[4];
-  ldsm_x4(Ks + j0 * pitch + fa, ak);
-  ldsm_x4(Vs + j0 * pitch + fa, av);
+  uint32_t aq[4], ado[4], ak[4], av[4];
+  ldsm_x4(Qs + i0 * pitch + fa, aq);
+  ldsm_x4(Os + i0 * pitch + fa, ado);
+  ldsm_x4(Ks + i0 * pitch + fa, ak);
+  ldsm_x4(Vs + i0 * pitch + fa, av);
+  const float lse_a = lse[ia], lse_b = lse[ib], d_a = dd[ia], d_b = dd[ib];
+  float dq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float dk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float dv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int i0 = 0; i0 < m; i0 += 16) {
-    auto col = [&](int e) { return i0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1); };
-    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint32_t bq[4];
-    ldsm_x4(Qs + i0 * pitch + fbn, bq);
-    mma_16816(s, ak, bq[0], bq[1]);
-    mma_16816(s + 4, ak, bq[2], bq[3]);
+  for (int n0 = 0; n0 < m; n0 += 16) {
+    auto col = [&](int e) { return n0 + (e & 4 ? 8 : 0) + 2 * t + (e & 1); };
     float u[8];
-    ub(i0, j0, ja, jb, t, m, u);  // U[j][i] = U[i][j]
-    bwd_scores(s, u, m, col);
-    const float2 l0 = *reinterpret_cast<const float2*>(lse + i0 + 2 * t);
-    const float2 l1 = *reinterpret_cast<const float2*>(lse + i0 + 8 + 2 * t);
-    const float2 d0 = *reinterpret_cast<const float2*>(dd + i0 + 2 * t);
-    const float2 d1 = *reinterpret_cast<const float2*>(dd + i0 + 8 + 2 * t);
-    const float lsev[4] = {l0.x, l0.y, l1.x, l1.y}, ddv[4] = {d0.x, d0.y, d1.x, d1.y};
-    float dp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    uint32_t bo[4];
-    ldsm_x4(Os + i0 * pitch + fbn, bo);
-    mma_16816(dp, av, bo[0], bo[1]);
-    mma_16816(dp + 4, av, bo[2], bo[3]);
-    float p[8], ds[8];
+    ub(n0, i0, ia, ib, t, m, u);  // U_ij = U_ji
+    uint32_t bk[4], bq[4], bv[4], bo[4];
+    ldsm_x4(Ks + n0 * pitch + fbn, bk);
+    ldsm_x4(Qs + n0 * pitch + fbn, bq);
+    ldsm_x4(Vs + n0 * pitch + fbn, bv);
+    ldsm_x4(Os + n0 * pitch + fbn, bo);
+    // rows of the tile as queries: S = Q_I K_J^T, dP = dO_I V_J^T
+    float sq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, dpq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    mma_16816(sq, aq, bk[0], bk[1]);
+    mma_16816(sq + 4, aq, bk[2], bk[3]);
+    mma_16816(dpq, ado, bv[0], bv[1]);
+    mma_16816(dpq + 4, ado, bv[2], bv[3]);
+    // as keys: S^T = K_I Q_J^T, dP^T = V_I dO_J^T
+    float sk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, dpk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    mma_16816(sk, ak, bq[0], bq[1]);
+    mma_16816(sk + 4, ak, bq[2], bq[3]);
+    mma_16816(dpk, av, bo[0], bo[1]);
+    mma_16816(dpk + 4, av, bo[2], bo[3]);
+    bwd_scores(sq, u, m, col);
+    bwd_scores(sk, u, m, col);
+    const float2 l0 = *reinterpret_cast<const float2*>(lse + n0 + 2 * t);
+    const float2 l1 = *reinterpret_cast<const float2*>(lse + n0 + 8 + 2 * t);
+    const float2 d0 = *reinterpret_cast<const float2*>(dd + n0 + 2 * t);
+    const float2 d1 = *reinterpret_cast<const float2*>(dd + n0 + 8 + 2 * t);
+    const float lcol[4] = {l0.x, l0.y, l1.x, l1.y}, dcol[4] = {d0.x, d0.y, d1.x, d1.y};
+    float dsq[8], pk[8], dsk[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const int c = (e & 1) + ((e >> 1) & 2);  // column slot of element e: 2t + (e & 1) + 8 (e >> 2)
-      p[e] = ex2(s[e] - lsev[c]);
-      ds[e] = p[e] * (dp[e] - ddv[c]);
+      const int cidx = (e & 1) + ((e >> 1) & 2);  // column slot of element e: 2t + (e & 1) + 8 (e >> 2)
+      const float pq = ex2(sq[e] - (e & 2 ? lse_b : lse_a));
+      dsq[e] = pq * (dpq[e] - (e & 2 ? d_b : d_a));
+      pk[e] = ex2(sk[e] - lcol[cidx]);
+      dsk[e] = pk[e] * (dpk[e] - dcol[cidx]);
     }
-    uint32_t pp[4], pd[4], bot[4], bqt[4];
-    pack_bf16_frag(p, pp);
-    pack_bf16_frag(ds, pd);
-    ldsm_x4_t(Os + i0 * pitch + fbt, bot);
-    mma_16816(dv, pp, bot[0], bot[1]);
-    mma_16816(dv + 4, pp, bot[2], bot[3]);
-    ldsm_x4_t(Qs + i0 * pitch + fbt, bqt);
-    mma_16816(dk, pd, bqt[0], bqt[1]);
-    mma_16816(dk + 4, pd, bqt[2], bqt[3]);
+    uint32_t pa[4], bkt[4], bot[4], bqt[4];
+    pack_bf16_frag(dsq, pa);
+    ldsm_x4_t(Ks + n0 * pitch + fbt, bkt);
+    mma_16816(dq, pa, bkt[0], bkt[1]);
+    mma_16816(dq + 4, pa, bkt[2], bkt[3]);
+    pack_bf16_frag(pk, pa);
+    ldsm_x4_t(Os + n0 * pitch + fbt, bot);
+    mma_16816(dv, pa, bot[0], bot[1]);
+    mma_16816(dv + 4, pa, bot[2], bot[3]);
+    pack_bf16_frag(dsk, pa);
+    ldsm_x4_t(Qs + n0 * pitch + fbt, bqt);
+    mma_16816(dk, pa, bqt[0], bqt[1]);
+    mma_16816(dk + 4, pa, bqt[2], bqt[3]);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const int i = col(e), j = e & 2 ? jb : ja;
+      const int i = e & 2 ? ib : ia, j = col(e);
       const bool row_ok = e & 2 ? vb : va;
-      if (row_ok && i < m && in_bounds(i >= 0)) {
-        const int hi = max(i, j), lo = min(i, j);
-        atomicAdd(gh + 8 * (hi * (hi + 1) / 2 + lo), ds[e]);
-      }
+      if (row_ok && j < m && i <= j) gh[8 * (j * (j + 1) / 2 + i)] = i == j ? dsq[e] : dsq[e] + dsk[e];
     }
   }
+  auto put = [&](uint16_t* row, const float* x, int o, float sc) {
+    *reinterpret_cast<uint32_t*>(row + 2 * t) = cvt_bf16x2(sc * x[o], sc * x[o + 1]);
+    *reinterpret_cast<uint32_t*>(row + 8 + 2 * t) = cvt_bf16x2(sc * x[o + 4], sc * x[o + 5]);
+  };
   if (va) {
-    uint16_t* kp = dkrow(ja);
-    uint16_t* vp = dvrow(ja);
-    *reinterpret_cast<uint32_t*>(kp + 2 * t) = cvt_bf16x2(0.25f * dk[0], 0.25f * dk[1]);
-    *reinterpret_cast<uint32_t*>(kp + 8 + 2 * t) = cvt_bf16x2(0.25f * dk[4], 0.25f * dk[5]);
-    *reinterpret_cast<uint32_t*>(vp + 2 * t) = cvt_bf16x2(dv[0], dv[1]);
-    *reinterpret_cast<uint32_t*>(vp + 8 + 2 * t) = cvt_bf16x2(dv[4], dv[5]);
+    put(dqrow(ia), dq, 0, 0.25f);
+    put(dkrow(ia), dk, 0, 0.25f);
+    put(dvrow(ia), dv, 0, 1.f);
   }
   if (vb) {
-    uint16_t* kp = dkrow(jb);
-    uint16_t* vp = dvrow(jb);
-    *reinterpret_cast<uint32_t*>(kp + 2 * t) = cvt_bf16x2(0.25f * dk[2], 0.25f * dk[3]);
-    *reinterpret_cast<uint32_t*>(kp + 8 + 2 * t) = cvt_bf16x2(0.25f * dk[6], 0.25f * dk[7]);
-    *reinterpret_cast<uint32_t*>(vp + 2 * t) = cvt_bf16x2(dv[2], dv[3]);
-    *reinterpret_cast<uint32_t*>(vp + 8 + 2 * t) = cvt_bf16x2(dv[6], dv[7]);
+    put(dqrow(ib), dq, 2, 0.25f);
+    put(dkrow(ib), dk, 2, 0.25f);
+    put(dvrow(ib), dv, 2, 1.f);
   }
 }
 
@@ -374,10 +347,6 @@ __global__ void __launch_bounds__(512, 1) k_attn_bwd(JetArgs J, BwdArgs X) {
     const int m = S.part.m;
     const size_t rowbase = (size_t)X.T[n] * kTileM;
     if (m > 0) {
-      // the jet's gradient records start at zero
-      const int np = m * (m + 1) / 2;
-      float4* g4 = reinterpret_cast<float4*>(X.grec + rowbase * 8);
-      for (int e = threadIdx.x; e < 2 * np; e += blockDim.x) g4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
       const int hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m), m16 = round16(m);
       const int HR = max(1, min(kH, kBwdStageBytes / hb));
       const int tiles = (m + 15) >> 4;
@@ -391,17 +360,17 @@ __global__ void __launch_bounds__(512, 1) k_attn_bwd(JetArgs J, BwdArgs X) {
             const int hh = it / tiles, h = h0 + hh;
             unsigned char* hbuf = S.stage + hh * hb;
             float* lse = reinterpret_cast<float*>(hbuf + 4 * tb);
-            bwd_query_tile(smem_u32(hbuf), m, (it % tiles) * 16, ub.head(h), lse, lse + m16,
-                           [&](int i) { return X.dq + qkv_off<PM>(S.part, J, n, h, i); });
+            bwd_stats_tile(smem_u32(hbuf), m, (it % tiles) * 16, ub.head(h), lse, lse + m16);
           }
           __syncthreads();
           for (int it = warp; it < hr * tiles; it += nwarp) {
             const int hh = it / tiles, h = h0 + hh;
             unsigned char* hbuf = S.stage + hh * hb;
             const float* lse = reinterpret_cast<const float*>(hbuf + 4 * tb);
-            bwd_key_tile(smem_u32(hbuf), m, (it % tiles) * 16, ub.head(h), lse, lse + m16, X.grec + rowbase * 8 + h,
-                         [&](int j) { return X.dk + qkv_off<PM>(S.part, J, n, h, j); },
-                         [&](int j) { return X.dv + qkv_off<PM>(S.part, J, n, h, j); });
+            bwd_pair_tile(smem_u32(hbuf), m, (it % tiles) * 16, ub.head(h), lse, lse + m16, X.grec + rowbase * 8 + h,
+                          [&](int i) { return X.dq + qkv_off<PM>(S.part, J, n, h, i); },
+                          [&](int i) { return X.dk + qkv_off<PM>(S.part, J, n, h, i); },
+                          [&](int i) { return X.dv + qkv_off<PM>(S.part, J, n, h, i); });
           }
           __syncthreads();
         }
@@ -805,20 +774,34 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
   if (warp == 0) tmem_dealloc(S.tmem_base, 256);
 }
 
-// Weight gradients: the sum over the CTAs' partials, in CTA order.
+// Weight gradients: the sum over the CTAs' partials in a fixed order. CTA
+// x owns 32 consecutive elements; warp w sums the slots w, w + 8, ... in
+// order, then the eight warp sums are added in warp order.
+constexpr int kReduceCtas = (kFoldedFloats + 31) / 32;
+
 __global__ void __launch_bounds__(256) k_grad_reduce(const float* __restrict__ partials, int nparts, GradArgs G) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= kFoldedFloats) return;
+  __shared__ float wsum[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
   float s = 0.f;
-  for (int c = 0; c < nparts; ++c) s += partials[(size_t)c * kFoldedFloats + e];
-  if (e < kOffB1) G.W1[e - kOffW1] = s;
-  else if (e < kOffW2) G.b1[e - kOffB1] = s;
-  else if (e < kOffB2) G.W2[e - kOffW2] = s;
-  else if (e < kOffW3) G.b2[e - kOffB2] = s;
-  else if (e < kOffB3) G.W3[e - kOffW3] = s;
-  else if (e < kOffW4) G.b3[e - kOffB3] = s;
-  else if (e < kOffB4) G.W4[e - kOffW4] = s;
-  else G.b4[e - kOffB4] = s;
+  if (e < kFoldedFloats) {
+#pragma unroll 4
+    for (int c = w; c < nparts; c += 8) s += partials[(size_t)c * kFoldedFloats + e];
+  }
+  wsum[w][lane] = s;
+  __syncthreads();
+  if (w != 0 || e >= kFoldedFloats) return;
+  float t = 0.f;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) t += wsum[q][lane];
+  if (e < kOffB1) G.W1[e - kOffW1] = t;
+  else if (e < kOffW2) G.b1[e - kOffB1] = t;
+  else if (e < kOffB2) G.W2[e - kOffW2] = t;
+  else if (e < kOffW3) G.b2[e - kOffB2] = t;
+  else if (e < kOffB3) G.W3[e - kOffW3] = t;
+  else if (e < kOffW4) G.b3[e - kOffB3] = t;
+  else if (e < kOffB4) G.W4[e - kOffW4] = t;
+  else G.b4[e - kOffB4] = t;
 }
 
 }  // namespace pb
