@@ -305,8 +305,8 @@ pb_status run_backward_chunk(const pb::JetArgs& J, const pb::MlpArgs& W, const p
     auto k = pb::k_attn_bwd<PM>;
     const size_t smem = sizeof(pb::AttnBwdSmem<PM>);
     int grid = 0;
-    if ((st = prepare(k, smem, 512, J.N, &grid)) != PB_OK) return st;
-    k<<<grid, 512, smem, s>>>(J, X);
+    if ((st = prepare(k, smem, 256, J.N * pb::kBwdHeadGroups, &grid)) != PB_OK) return st;
+    k<<<grid, 256, smem, s>>>(J, X);
     if ((st = launched("k_attn_bwd")) != PB_OK) return st;
   }
   auto k = pb::k_mlp_bwd<PM>;

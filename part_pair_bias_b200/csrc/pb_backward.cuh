@@ -329,7 +329,8 @@ __device__ void bwd_pair_tile(uint32_t hs, int m, int i0, const UBlock& ub, cons
   }
 }
 
-constexpr int kBwdStageBytes = 192 * 1024;  // staged heads of the attention backward
+constexpr int kBwdStageBytes = 96 * 1024;  // staged heads of the attention backward (two CTAs per SM)
+constexpr int kBwdHeadGroups = 2;          // CTA items: (jet, half of the heads)
 
 template <int PM>
 struct AttnBwdSmem {
@@ -338,22 +339,24 @@ struct AttnBwdSmem {
 };
 
 template <int PM>
-__global__ void __launch_bounds__(512, 1) k_attn_bwd(JetArgs J, BwdArgs X) {
+__global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   AttnBwdSmem<PM>& S = *reinterpret_cast<AttnBwdSmem<PM>*>(smem_raw);
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  for (int n = blockIdx.x; n < J.N; n += gridDim.x) {
+  constexpr int kHG = kH / kBwdHeadGroups;
+  for (int item = blockIdx.x; item < J.N * kBwdHeadGroups; item += gridDim.x) {
+    const int n = item / kBwdHeadGroups, hg = item % kBwdHeadGroups;
     stage_jet<PM, false>(S.part, J, n);
     const int m = S.part.m;
     const size_t rowbase = (size_t)X.T[n] * kTileM;
     if (m > 0) {
       const int hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m), m16 = round16(m);
-      const int HR = max(1, min(kH, kBwdStageBytes / hb));
+      const int HR = max(1, min(kHG, kBwdStageBytes / hb));
       const int tiles = (m + 15) >> 4;
       const RecordUBias ub{reinterpret_cast<const __half*>(X.urec + rowbase)};
       if (in_bounds(hb <= kBwdStageBytes)) {
-        for (int h0 = 0; h0 < kH; h0 += HR) {
-          const int hr = min(HR, kH - h0);
+        for (int h0 = hg * kHG; h0 < (hg + 1) * kHG; h0 += HR) {
+          const int hr = min(HR, (hg + 1) * kHG - h0);
           stage_bwd<PM>(S.part, J, X, n, h0, hr, S.stage);
           __syncthreads();
           for (int it = warp; it < hr * tiles; it += nwarp) {
@@ -376,9 +379,11 @@ __global__ void __launch_bounds__(512, 1) k_attn_bwd(JetArgs J, BwdArgs X) {
         }
       }
     }
-    zero_masked_rows<PM>(S.part, J, X.dq, n);
-    zero_masked_rows<PM>(S.part, J, X.dk, n);
-    zero_masked_rows<PM>(S.part, J, X.dv, n);
+    if (hg == 0) {  // masked rows of every head
+      zero_masked_rows<PM>(S.part, J, X.dq, n);
+      zero_masked_rows<PM>(S.part, J, X.dk, n);
+      zero_masked_rows<PM>(S.part, J, X.dv, n);
+    }
     __syncthreads();
   }
 }
@@ -456,14 +461,16 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
-// GELU(z) = z/2 (1 + tanh(u)), u = sqrt(2/pi) (z + 0.044715 z^3), and its derivative.
+// GELU(z) = z/2 (1 + tanh(u)), u = sqrt(2/pi) (z + 0.044715 z^3), and its
+// derivative Phi + z/2 (1 - tanh^2 u) sqrt(2/pi) (1 + 3 0.044715 z^2), where
+// Phi = (1 + tanh u) / 2.
 __device__ __forceinline__ void gelu_tanh_and_grad(float z, float& h, float& dh) {
   constexpr float kC0 = 0.7978845608028654f, kC1 = 0.044715f;
-  const float z2 = z * z;
-  const float t = tanh_approx(kC0 * fmaf(kC1 * z2, z, z));
-  const float half_z = 0.5f * z;
-  h = fmaf(half_z, t, half_z);
-  dh = fmaf(0.5f, t, 0.5f) + half_z * fmaf(-t, t, 1.f) * kC0 * fmaf(3.f * kC1, z2, 1.f);
+  const float z2 = z * z, c0z = kC0 * z;
+  const float t = tanh_approx(c0z * fmaf(kC1, z2, 1.f));
+  const float phi = fmaf(0.5f, t, 0.5f);
+  h = z * phi;
+  dh = fmaf(0.5f * fmaf(-t, t, 1.f), c0z * fmaf(3.f * kC1, z2, 1.f), phi);
 }
 
 // TMEM <- registers, 32 lanes x 16 columns (thread t of the warp writes lane
@@ -507,6 +514,8 @@ __device__ __forceinline__ void grad_tiles(const MlpBwdSmem<PM>& S, const GradPa
 }
 
 // acc[j] += d^T h over the tile's 128 rows for the part's column blocks.
+// Lane addresses are formed once; each 16-row step moves both operands by
+// two 8-row core groups.
 template <int PM>
 __device__ __forceinline__ void grad_mma(const MlpBwdSmem<PM>& S, const GradPart& gp, float (*acc)[4]) {
   const int lane = threadIdx.x & 31;
@@ -514,20 +523,29 @@ __device__ __forceinline__ void grad_mma(const MlpBwdSmem<PM>& S, const GradPart
   int Kd, Kb, ones;
   grad_tiles(S, gp, Dt, Kd, Bt, Kb, ones);
   const int mi = lane >> 3;
-  const uint32_t d_base = smem_u32(Dt), b_base = smem_u32(Bt);
-#pragma unroll 1
-  for (int k0 = 0; k0 < kTileM; k0 += 16) {
+  const uint32_t a_addr = smem_u32(Dt) + 2u * cofs((lane & 7) + (mi >> 1) * 8, gp.mb * 16 + (mi & 1) * 8, Kd);
+  const uint32_t b_row = smem_u32(Bt) + 2u * cofs((lane & 7) + ((lane >> 3) & 1) * 8, 0, Kb);
+  const uint32_t a_step = (uint32_t)Kd * 32u, b_step = (uint32_t)Kb * 32u;  // 16 rows
+  uint32_t b_addr[3];
+  bool is_one[3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int nb = gp.nb0 + j;
+    is_one[j] = nb == ones;
+    b_addr[j] = b_row + 128u * (uint32_t)(is_one[j] ? 0 : nb);
+  }
+#pragma unroll 2
+  for (int k = 0; k < kTileM / 16; ++k) {
     uint32_t a[4];
-    ldsm_x4_t(d_base + 2u * cofs(k0 + (lane & 7) + (mi >> 1) * 8, gp.mb * 16 + (mi & 1) * 8, Kd), a);
+    ldsm_x4_t(a_addr + a_step * k, a);
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       if (j >= gp.nc) break;
-      const int nb = gp.nb0 + j;
       uint32_t b[2];
-      if (nb == ones) {
+      if (is_one[j]) {
         b[0] = b[1] = 0x3F803F80u;  // bf16 1.0 in both halves
       } else {
-        ldsm_x2_t(b_base + 2u * cofs(k0 + (lane & 7) + ((lane >> 3) & 1) * 8, nb * 8, Kb), b);
+        ldsm_x2_t(b_addr[j] + b_step * k, b);
       }
       mma_16816(acc[j], a, b[0], b[1]);
     }
@@ -651,8 +669,17 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
     float z[16], h[16];
     const uint32_t ta = tm + lane_off + 64u * k + 16u * c;
     tmem_ld16_wait(ta, z);
+    const float4* bq = reinterpret_cast<const float4*>(&S.bias[k][16 * c]);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) gelu_tanh_and_grad(z[i] + S.bias[k][16 * c + i], h[i], z[i]);
+    for (int i = 0; i < 4; ++i) {
+      const float4 bb = bq[i];
+      z[4 * i] += bb.x;
+      z[4 * i + 1] += bb.y;
+      z[4 * i + 2] += bb.z;
+      z[4 * i + 3] += bb.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) gelu_tanh_and_grad(z[i], h[i], z[i]);
     store16(S.Hs[k], h);
     tmem_st16_wait(ta, z);
   };
@@ -696,7 +723,7 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
       }
       if (c == 0) {
         float f[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) pair_feat<PM, false>(S.part, a, b, f);
+        if (valid) pair_feat<PM, true>(S.part, a, b, f);  // the forward MLP's features
         const uint32_t h01 = cvt_bf16x2(f[0], f[1]), h23 = cvt_bf16x2(f[2], f[3]);
         const uint32_t l01 = cvt_bf16x2(f[0] - bf16lo(h01), f[1] - bf16hi(h01));
         const uint32_t l23 = cvt_bf16x2(f[2] - bf16lo(h23), f[3] - bf16hi(h23));
