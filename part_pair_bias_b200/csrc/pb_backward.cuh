@@ -37,32 +37,6 @@ struct BwdArgs {
   const int* T;                      // tile prefix [N + 1]
 };
 
-// ------------------------------------------------------------ ldmatrix
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t* r) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(addr)
-               : "memory");
-}
-
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
 // ============================================== attention backward (k_attn_bwd)
 //
 // Per (jet, head), over the jet's m valid particles, with s = q.k/4 + U in
@@ -120,21 +94,6 @@ __device__ void stage_bwd(const Particles<PM>& S, const JetArgs& J, const BwdArg
     const int hh = idx / (2 * m16), r = idx % (2 * m16);
     reinterpret_cast<float*>(buf + hh * hb + 4 * tb)[r] = 0.f;
   }
-}
-
-// Byte offsets, inside a staged tensor, of this lane's ldmatrix row for the
-// three fragment shapes used (add the tile's first row times the row pitch):
-//   A  (16 rows x 16 cols, x4):            rows 0-7 | 8-15, cols 0-7 | 8-15
-//   Bn (two n8 blocks of rows, d = K, x4):  b0,b1 of rows 0-7, then of rows 8-15
-//   Bt (rows = K, d = N, x4.trans):         b0,b1 of d 0-7, then of d 8-15
-__device__ __forceinline__ uint32_t frag_a_off(int lane) {
-  return (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kKStride * 2 + (lane >> 4) * 16);
-}
-__device__ __forceinline__ uint32_t frag_bn_off(int lane) {
-  return (uint32_t)(((lane & 7) + ((lane >> 4) & 1) * 8) * kKStride * 2 + ((lane >> 3) & 1) * 16);
-}
-__device__ __forceinline__ uint32_t frag_bt_off(int lane) {
-  return (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kKStride * 2 + ((lane >> 4) & 1) * 16);
 }
 
 // p (fp32) as the A fragment of a k16 step, split into hi + lo bf16 terms.

@@ -747,53 +747,81 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float* f) {
 // transposed [16][m16 + 8]; both strides make the fragment loads of a warp
 // hit 32 distinct banks.
 
-constexpr int kKStride = 24;  // halves per staged K row (48 bytes)
+constexpr int kKStride = 24;  // halves per staged K or V row (48 bytes)
 
 __host__ __device__ constexpr int round16(int m) { return (m + 15) & ~15; }
 
-// Bytes of the staged K and V of one head for m keys (a multiple of 16).
-__host__ __device__ constexpr int kv16_bytes(int m) {
-  return round16(m) * kKStride * 2 + 16 * (round16(m) + 8) * 2;
+// Bytes of the staged K and V of one head for m keys: K rows, then V rows.
+__host__ __device__ constexpr int kv16_bytes(int m) { return 2 * round16(m) * kKStride * 2; }
+
+// ldmatrix: four (or two) 8x8 b16 matrices from shared memory into the
+// fragment layout of mma.sync; .trans delivers each matrix transposed.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
 
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Byte offsets, inside a staged [rows][kKStride] tensor, of this lane's
+// ldmatrix row for the three fragment shapes used (add the tile's first row
+// times the row pitch):
+//   A  (16 rows x 16 cols, x4):            rows 0-7 | 8-15, cols 0-7 | 8-15
+//   Bn (two n8 blocks of rows, d = K, x4):  b0,b1 of rows 0-7, then of rows 8-15
+//   Bt (rows = K, d = N, x4.trans):         b0,b1 of d 0-7, then of d 8-15
+__device__ __forceinline__ uint32_t frag_a_off(int lane) {
+  return (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kKStride * 2 + (lane >> 4) * 16);
+}
+__device__ __forceinline__ uint32_t frag_bn_off(int lane) {
+  return (uint32_t)(((lane & 7) + ((lane >> 4) & 1) * 8) * kKStride * 2 + ((lane >> 3) & 1) * 16);
+}
+__device__ __forceinline__ uint32_t frag_bt_off(int lane) {
+  return (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kKStride * 2 + ((lane >> 4) & 1) * 16);
+}
+
+// 16-byte global -> shared copy that bypasses the registers; with
+// src_bytes = 0 nothing is read and the destination is zero-filled.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // K and V of heads [h0, h0 + hr) of the staged jet n into buf, one head
-// after another (kv16_bytes(m) each). Block-wide, no barrier.
+// after another (kv16_bytes(m) each): K rows then V rows, bf16 [m16][kKStride],
+// zero rows past m. Asynchronous 16-byte copies, committed as one group: the
+// caller waits with cp_async_wait_all() and a barrier. Block-wide.
 template <int PM>
 __device__ void stage_kv16(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int h0, int hr,
                            uint16_t* buf) {
-  const int m = S.m, m16 = round16(m), vts = m16 + 8, hb = kv16_bytes(m) / 2;
+  const int m = S.m, m16 = round16(m), hb = kv16_bytes(m) / 2;
   const int total = hr * m16 * 4, nthr = blockDim.x;
-  // four independent loads in flight per thread before any store
-  for (int base = threadIdx.x; base < total; base += 4 * nthr) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int idx = base + u * nthr;
-      const int part = idx & 3, j = (idx >> 2) % m16, hh = (idx >> 2) / m16;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (idx < total && j < m)
-        v[u] = *reinterpret_cast<const uint4*>((part < 2 ? X.k : X.v) + qkv_off<PM>(S, J, n, h0 + hh, j) +
-                                               (part & 1) * 8);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int idx = base + u * nthr;
-      if (idx >= total) break;
-      const int part = idx & 3, j = (idx >> 2) % m16, hh = (idx >> 2) / m16;
-      uint16_t* kh = buf + hh * hb;
-      if (part < 2) {
-        *reinterpret_cast<uint4*>(kh + j * kKStride + (part & 1) * 8) = v[u];
-      } else {
-        uint16_t* vt = kh + m16 * kKStride + ((part & 1) * 8) * vts + j;
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          vt[(2 * e) * vts] = (uint16_t)(w[e] & 0xffffu);
-          vt[(2 * e + 1) * vts] = (uint16_t)(w[e] >> 16);
-        }
-      }
-    }
+  for (int idx = threadIdx.x; idx < total; idx += nthr) {
+    const int part = idx & 3, j = (idx >> 2) % m16, hh = (idx >> 2) / m16;
+    const uint16_t* base = part < 2 ? X.k : X.v;
+    const bool valid = j < m;
+    const uint16_t* src = base + (valid ? qkv_off<PM>(S, J, n, h0 + hh, j) : 0) + (part & 1) * 8;
+    cp_async16(buf + hh * hb + (part >> 1) * m16 * kKStride + j * kKStride + (part & 1) * 8, src, valid ? 16u : 0u);
   }
+  cp_async_commit();
 }
 
 __device__ __forceinline__ uint32_t lds_u32(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
@@ -881,16 +909,16 @@ __device__ __forceinline__ void q_frag(int i0, int nrows, const QRow& qrow, uint
 }
 
 // Queries [i0, i0 + nrows) (nrows <= 16, A fragment a from q_frag) of one
-// head against its m staged keys: kh = staged K, vth = staged V^T of that
-// head. orow(i) gives the bf16 output row of query i; ub(n0, i0, ia, ib, t,
+// head against its m staged keys: kh = staged K, vh = staged V of that head
+// (row-major; its P V operand comes through ldmatrix.trans). orow(i) gives the bf16 output row of query i; ub(n0, i0, ia, ib, t,
 // m, u) fills the bias of the 8 score elements a lane holds for the key
 // block n0 (element e: row e & 2 ? ib : ia, key n0 + 8 (e >> 2) + 2 t +
 // (e & 1), keys past m clamped to m - 1). Warp-wide.
 template <class ORow, class UBlock>
-__device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t* vth, int m, int i0, int nrows,
+__device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t* vh, int m, int i0, int nrows,
                                               const uint32_t* a, const ORow& orow, const UBlock& ub) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int vts = round16(m) + 8;
+  const uint32_t v_base = smem_u32(vh) + frag_bt_off(lane);
   const bool va = g < nrows, vb = g + 8 < nrows;
   const int ia = i0 + (va ? g : 0), ib = i0 + (vb ? g + 8 : 0);  // rows past the block alias row i0
   const float qs = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
@@ -933,9 +961,10 @@ __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t
     o[2] *= cb; o[3] *= cb; o[6] *= cb; o[7] *= cb;
     const uint32_t pa[4] = {cvt_bf16x2(p[0], p[1]), cvt_bf16x2(p[2], p[3]), cvt_bf16x2(p[4], p[5]),
                             cvt_bf16x2(p[6], p[7])};
-    const uint16_t* v0 = vth + g * vts + n0 + 2 * t;  // V^T rows = dims g and 8 + g
-    mma_16816(o, pa, lds_u32(v0), lds_u32(v0 + 8));
-    mma_16816(o + 4, pa, lds_u32(v0 + 8 * vts), lds_u32(v0 + 8 * vts + 8));
+    uint32_t bv[4];
+    ldsm_x4_t(v_base + (uint32_t)n0 * (kKStride * 2), bv);
+    mma_16816(o, pa, bv[0], bv[1]);
+    mma_16816(o + 4, pa, bv[2], bv[3]);
   }
   la += __shfl_xor_sync(0xffffffffu, la, 1);
   la += __shfl_xor_sync(0xffffffffu, la, 2);
@@ -983,6 +1012,7 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
     };
     if (warp < hr * tiles) qload(warp, a);
     stage_kv16<PM>(S, J, X, n, h0, hr, buf);
+    cp_async_wait_all();
     __syncthreads();
     for (int it = warp; it < hr * tiles; it += nwarp) {
       uint32_t an[4] = {0u, 0u, 0u, 0u};
@@ -2035,6 +2065,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
           }
           stage_kv16<PM>(S.ring[k], J, X, nj, A.hl[k], A.hh[k] - A.hl[k], reinterpret_cast<uint16_t*>(stage + A.kvoff[k]));
         }
+        cp_async_wait_all();
         __syncthreads();
         for (int it = warp; it < items; it += nwarp) {
           uint32_t an[4] = {0u, 0u, 0u, 0u};
