@@ -751,8 +751,11 @@ constexpr int kKStride = 24;  // halves per staged K or V row (48 bytes)
 
 __host__ __device__ constexpr int round16(int m) { return (m + 15) & ~15; }
 
-// Bytes of the staged K and V of one head for m keys: K rows, then V rows.
-__host__ __device__ constexpr int kv16_bytes(int m) { return 2 * round16(m) * kKStride * 2; }
+// The forward attention stages K and V rows unpadded (32 bytes, two 16-byte
+// chunks) with chunk c of row r at chunk c ^ ((r >> 2) & 1): the 8 rows of an
+// ldmatrix phase then cover all 32 banks once.
+__host__ __device__ constexpr int kv16_bytes(int m) { return 2 * round16(m) * 32; }
+__device__ __forceinline__ uint32_t kv_off(int r, int c) { return (uint32_t)(r * 32 + ((c ^ ((r >> 2) & 1)) << 4)); }
 
 // ldmatrix: four (or two) 8x8 b16 matrices from shared memory into the
 // fragment layout of mma.sync; .trans delivers each matrix transposed.
@@ -806,8 +809,8 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // K and V of heads [h0, h0 + hr) of the staged jet n into buf, one head
-// after another (kv16_bytes(m) each): K rows then V rows, bf16 [m16][kKStride],
-// zero rows past m. Asynchronous 16-byte copies, committed as one group: the
+// after another (kv16_bytes(m) each): K rows then V rows, bf16 [m16][16] in
+// the swizzled chunk order of kv_off, zero rows past m. Asynchronous 16-byte copies, committed as one group: the
 // caller waits with cp_async_wait_all() and a barrier. Block-wide.
 template <int PM>
 __device__ void stage_kv16(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int h0, int hr,
@@ -819,12 +822,10 @@ __device__ void stage_kv16(const Particles<PM>& S, const JetArgs& J, const QkvAr
     const uint16_t* base = part < 2 ? X.k : X.v;
     const bool valid = j < m;
     const uint16_t* src = base + (valid ? qkv_off<PM>(S, J, n, h0 + hh, j) : 0) + (part & 1) * 8;
-    cp_async16(buf + hh * hb + (part >> 1) * m16 * kKStride + j * kKStride + (part & 1) * 8, src, valid ? 16u : 0u);
+    cp_async16(buf + hh * hb + (part >> 1) * m16 * 16 + kv_off(j, part & 1) / 2, src, valid ? 16u : 0u);
   }
   cp_async_commit();
 }
-
-__device__ __forceinline__ uint32_t lds_u32(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
 // D += A B on one m16n8k16 tile: A 16x16 bf16 (row), B 16x8 bf16 (col), D fp32.
 __device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
@@ -910,7 +911,8 @@ __device__ __forceinline__ void q_frag(int i0, int nrows, const QRow& qrow, uint
 
 // Queries [i0, i0 + nrows) (nrows <= 16, A fragment a from q_frag) of one
 // head against its m staged keys: kh = staged K, vh = staged V of that head
-// (row-major; its P V operand comes through ldmatrix.trans). orow(i) gives the bf16 output row of query i; ub(n0, i0, ia, ib, t,
+// (rows in kv_off order; the Q K^T operand comes through ldmatrix, the P V
+// operand through ldmatrix.trans). orow(i) gives the bf16 output row of query i; ub(n0, i0, ia, ib, t,
 // m, u) fills the bias of the 8 score elements a lane holds for the key
 // block n0 (element e: row e & 2 ? ib : ia, key n0 + 8 (e >> 2) + 2 t +
 // (e & 1), keys past m clamped to m - 1). Warp-wide.
@@ -918,7 +920,10 @@ template <class ORow, class UBlock>
 __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t* vh, int m, int i0, int nrows,
                                               const uint32_t* a, const ORow& orow, const UBlock& ub) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const uint32_t v_base = smem_u32(vh) + frag_bt_off(lane);
+  // lane rows of the two fragment shapes (see frag_bn_off / frag_bt_off); a
+  // 16-row step keeps the swizzle phase
+  const uint32_t k_base = smem_u32(kh) + kv_off((lane & 7) + ((lane >> 4) & 1) * 8, (lane >> 3) & 1);
+  const uint32_t v_base = smem_u32(vh) + kv_off((lane & 7) + ((lane >> 3) & 1) * 8, (lane >> 4) & 1);
   const bool va = g < nrows, vb = g + 8 < nrows;
   const int ia = i0 + (va ? g : 0), ib = i0 + (vb ? g + 8 : 0);  // rows past the block alias row i0
   const float qs = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
@@ -926,9 +931,10 @@ __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t
   float mxa = -INFINITY, mxb = -INFINITY, la = 0.f, lb = 0.f;
   for (int n0 = 0; n0 < m; n0 += 16) {
     float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const uint16_t* k0 = kh + (n0 + g) * kKStride + 2 * t;
-    mma_16816(s, a, lds_u32(k0), lds_u32(k0 + 8));
-    mma_16816(s + 4, a, lds_u32(k0 + 8 * kKStride), lds_u32(k0 + 8 * kKStride + 8));
+    uint32_t bk[4];
+    ldsm_x4(k_base + (uint32_t)n0 * 32u, bk);
+    mma_16816(s, a, bk[0], bk[1]);
+    mma_16816(s + 4, a, bk[2], bk[3]);
     float u[8];
     ub(n0, i0, ia, ib, t, m, u);
     if (n0 + 16 <= m) {
@@ -962,7 +968,7 @@ __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t
     const uint32_t pa[4] = {cvt_bf16x2(p[0], p[1]), cvt_bf16x2(p[2], p[3]), cvt_bf16x2(p[4], p[5]),
                             cvt_bf16x2(p[6], p[7])};
     uint32_t bv[4];
-    ldsm_x4_t(v_base + (uint32_t)n0 * (kKStride * 2), bv);
+    ldsm_x4_t(v_base + (uint32_t)n0 * 32u, bv);
     mma_16816(o, pa, bv[0], bv[1]);
     mma_16816(o + 4, pa, bv[2], bv[3]);
   }
@@ -988,19 +994,25 @@ __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t
 // against all its valid keys, heads [h_lo, h_hi), on tensor cores: K and V of
 // as many heads as `stage` holds are staged at a time, then the warps take
 // (head, 16-query tile) items. ubias.head(h) gives the bias blocks of head h.
+// With `prestaged`, the K and V of all heads [h_lo, h_hi) were already
+// issued there by this block (stage_kv16, one group per thread): the copies
+// are awaited and `stage` is not used.
 template <int PM, class UBias>
 __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const QkvArgs& X, int n, int i_lo,
                                 int i_hi, float* stage, int stage_floats, const UBias& ubias, int h_lo = 0,
-                                int h_hi = kH) {
+                                int h_hi = kH, uint16_t* prestaged = nullptr) {
   const int m = S.m;
   const int nq = i_hi - i_lo;
-  if (m <= 0 || nq <= 0) return;
+  if (m <= 0 || nq <= 0) {
+    if (prestaged) cp_async_wait_all();
+    return;
+  }
   const int hb = kv16_bytes(m);
-  const int HR = max(1, min(kH, stage_floats * 4 / hb));
+  const int HR = prestaged ? h_hi - h_lo : max(1, min(kH, stage_floats * 4 / hb));
   const int tiles = (nq + 15) >> 4;
   const int warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  uint16_t* buf = reinterpret_cast<uint16_t*>(stage);
-  if (!in_bounds(hb <= stage_floats * 4)) return;  // one head's K and V must fit
+  uint16_t* buf = prestaged ? prestaged : reinterpret_cast<uint16_t*>(stage);
+  if (!prestaged && !in_bounds(hb <= stage_floats * 4)) return;  // one head's K and V must fit
   for (int h0 = h_lo; h0 < h_hi; h0 += HR) {
     const int hr = min(HR, h_hi - h0);
     // the Q fragment of a warp's next item is loaded ahead: the first one
@@ -1011,7 +1023,7 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
       q_frag(i0, min(16, i_hi - i0), [&](int i) { return X.q + qkv_off<PM>(S, J, n, h, i); }, f);
     };
     if (warp < hr * tiles) qload(warp, a);
-    stage_kv16<PM>(S, J, X, n, h0, hr, buf);
+    if (!prestaged) stage_kv16<PM>(S, J, X, n, h0, hr, buf);
     cp_async_wait_all();
     __syncthreads();
     for (int it = warp; it < hr * tiles; it += nwarp) {
@@ -1020,7 +1032,7 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
       const int hh = it / tiles, i0 = i_lo + (it % tiles) * 16, h = h0 + hh;
       const uint16_t* kh = buf + hh * (hb / 2);
       attend_tile16(
-          kh, kh + round16(m) * kKStride, m, i0, min(16, i_hi - i0), a,
+          kh, kh + round16(m) * 16, m, i0, min(16, i_hi - i0), a,
           [&](int i) { return X.out + qkv_off<PM>(S, J, n, h, i); }, ubias.head(h));
 #pragma unroll
       for (int e = 0; e < 4; ++e) a[e] = an[e];
@@ -1639,12 +1651,23 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
     }
     const int m = S.part.m;
     SmemUSink sink{S.U8, kUCap};
-    if (m * (m + 1) / 2 <= kUCap) {
-      const bool ok = mlp_pass<NG, SL>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, m * (m + 1) / 2, TriPairs{}}, sink, &phase);
+    const int np = m * (m + 1) / 2;
+    if (np <= kUCap) {
+      // when the bias triangle leaves room, the K and V of all heads are
+      // copied in behind it while the MLP runs
+      uint16_t* early = nullptr;
+      if (m > 0 && np + kH * kv16_bytes(m) / 16 <= kUCap) {
+        early = reinterpret_cast<uint16_t*>(S.U8 + np);
+        stage_kv16<PM>(S.part, J, X, n, 0, kH, early);
+      }
+      const bool ok = mlp_pass<NG, SL>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, np, TriPairs{}}, sink, &phase);
       aborted = __syncthreads_or(!ok) != 0;
-      if (aborted) break;
+      if (aborted) {
+        if (early) cp_async_wait_all();
+        break;
+      }
       TriUBias ub{reinterpret_cast<const __half*>(S.U8)};
-      attention_block<PM>(S.part, J, X, n, 0, m, stage, kStageFloats, ub);
+      attention_block<PM>(S.part, J, X, n, 0, m, stage, kStageFloats, ub, 0, kH, early);
     } else {
       const int qb = kUCap / m;
       for (int i0 = 0; i0 < m; i0 += qb) {
@@ -2079,7 +2102,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
           const uint16_t* kh = reinterpret_cast<const uint16_t*>(stage + A.kvoff[k]) + hh * (kv16_bytes(m) / 2);
           const TriBlock ub{reinterpret_cast<const __half*>(stage + A.uoff[k]) + h};
           attend_tile16(
-              kh, kh + round16(m) * kKStride, m, i0, min(16, m - i0), a,
+              kh, kh + round16(m) * 16, m, i0, min(16, m - i0), a,
               [&](int i) { return X.out + qkv_off<PM>(P, J, nj, h, i); }, ub);
 #pragma unroll
           for (int e = 0; e < 4; ++e) a[e] = an[e];
