@@ -74,6 +74,7 @@ __device__ void stage_jets(Particles<PM>* ring, const JetArgs& J, int K, const J
     long long base = 0;
     int cnt = 0;
     bool valid = false;
+    float fE = 0.f, fx = 0.f, fy = 0.f, fz = 0.f;  // loaded with the mask: one round trip
     if (act) {
       const int n = jet_of(k);
       if (J.ptr) {
@@ -88,7 +89,16 @@ __device__ void stage_jets(Particles<PM>* ring, const JetArgs& J, int K, const J
         base = (long long)n * J.P;
         cnt = J.P;
       }
-      if (t < J.P) valid = J.ptr ? (t < cnt) : (J.mask[base + t] != 0);
+      if (t < J.P) {
+        valid = J.ptr ? (t < cnt) : (J.mask[base + t] != 0);
+        if (kKin && t < cnt) {
+          const long long e = base + t;
+          fE = J.E[e];
+          fx = J.px[e];
+          fy = J.py[e];
+          fz = J.pz[e];
+        }
+      }
     }
     const unsigned ballot = __ballot_sync(0xffffffffu, valid);
     if (act && lane == 0) S.warp_cnt[lw] = __popc(ballot);
@@ -105,8 +115,7 @@ __device__ void stage_jets(Particles<PM>* ring, const JetArgs& J, int K, const J
       if (valid) {
         S.slot[c] = (int16_t)t;
         if (kKin) {
-          const long long e = base + t;
-          const double E = J.E[e], px = J.px[e], py = J.py[e], pz = J.pz[e];
+          const double E = fE, px = fx, py = fy, pz = fz;
           const double wm = E - pz, wp = E + pz;  // exact: differences of fp32 values
           const double pt = sqrt(px * px + py * py);
           S.y[c] = 0.5 * log(wp / wm);
@@ -167,7 +176,17 @@ __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
     cnt = J.P;
   }
   bool valid = false;
-  if (tid < J.P) valid = J.ptr ? (tid < cnt) : (J.mask[base + tid] != 0);
+  float fE = 0.f, fx = 0.f, fy = 0.f, fz = 0.f;  // loaded with the mask: one round trip
+  if (tid < J.P) {
+    valid = J.ptr ? (tid < cnt) : (J.mask[base + tid] != 0);
+    if (kKin && tid < cnt) {
+      const long long e = base + tid;
+      fE = J.E[e];
+      fx = J.px[e];
+      fy = J.py[e];
+      fz = J.pz[e];
+    }
+  }
   const unsigned ballot = __ballot_sync(0xffffffffu, valid);
   if (lane == 0) S.warp_cnt[warp] = __popc(ballot);
   __syncthreads();
@@ -182,8 +201,7 @@ __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
   if (valid) {
     S.slot[c] = (int16_t)tid;
     if (kKin) {
-      const long long e = base + tid;
-      const double E = J.E[e], px = J.px[e], py = J.py[e], pz = J.pz[e];
+      const double E = fE, px = fx, py = fy, pz = fz;
       const double wm = E - pz, wp = E + pz;  // exact: differences of fp32 values
       const double pt = sqrt(px * px + py * py);
       S.y[c] = 0.5 * log(wp / wm);
