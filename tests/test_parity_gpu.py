@@ -143,6 +143,20 @@ def test_wide_jets_query_block_path(oracle_lib):
     assert ops.get_device_status() == 0
 
 
+@pytest.mark.parametrize("P,mults", [(128, [61, 62, 88, 89, 1]), (256, [94, 95, 122, 123, 2])])
+def test_staging_path_boundaries(oracle_lib, P, mults):
+    """Jets on either side of the per-CTA kernel's layout limits: K and V
+    copied in behind the bias triangle during the MLP (up to m = 61 at
+    P = 128, 94 at P = 256), staged after it (triangle up to m = 88 / 122),
+    and the query-block path beyond."""
+    b = synth.make_jets(N=len(mults), P=P, mults=mults, mask_mode="scrambled", seed=31)
+    d = pt.Device(b)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
+    assert ops.get_device_status() == 0
+
+
 def test_packed_with_empty_jets(oracle_lib):
     b = synth.make_jets(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6)
     d = pt.Device(b)
