@@ -333,65 +333,74 @@ __device__ __forceinline__ uint32_t h2bits(__half lo, __half hi) {
 // Scale of input column k of layers 2..4: the tanh columns hold 2 GELU.
 __device__ __forceinline__ float act_scale(int k) { return (k >> 3) < kTanhChunks ? 0.5f : 1.0f; }
 
-// Weight tiles in the canonical layout. All global loads of a thread are
-// issued before any conversion so that their latencies overlap.
-template <int NG, int SL>
-__device__ void load_weights(MlpSmem<NG, SL>& S, const MlpArgs& W) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  constexpr int kPer = (2 * 1024 + 255) / 256;  // float4 loads of W2 and W3 per thread (>= 256 threads)
-  float4 w[kPer];
+// The folded weights of one thread's share, held in registers between the
+// global loads and the shared-memory stores, so that other latency (the
+// first jet's staging, the jet table) can overlap the loads.
+struct WeightRegs {
+  static constexpr int kPer = (2 * 1024 + 255) / 256;  // float4 loads of W2 and W3 per thread (>= 256 threads)
+  float4 w[kPer], w4, w1;
+  float bias1, bias2, bias3, bias4;
+  __device__ void load(const MlpArgs& W) {
+    const int tid = threadIdx.x, nthr = blockDim.x;
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int q = tid + j * nthr;
-    w[j] = q < 2048 ? reinterpret_cast<const float4*>(q < 1024 ? W.W2 : W.W3)[q & 1023] : make_float4(0, 0, 0, 0);
+    for (int j = 0; j < kPer; ++j) {
+      const int q = tid + j * nthr;
+      w[j] = q < 2048 ? reinterpret_cast<const float4*>(q < 1024 ? W.W2 : W.W3)[q & 1023] : make_float4(0, 0, 0, 0);
+    }
+    w4 = tid < 128 ? reinterpret_cast<const float4*>(W.W4)[tid] : make_float4(0, 0, 0, 0);
+    w1 = tid < 64 ? reinterpret_cast<const float4*>(W.W1)[tid] : make_float4(0, 0, 0, 0);
+    bias1 = tid < 64 ? W.b1[tid] : 0.f;
+    bias2 = tid < 64 ? W.b2[tid] : 0.f;
+    bias3 = tid < 64 ? W.b3[tid] : 0.f;
+    bias4 = tid < 8 ? W.b4[tid] : 0.f;
   }
-  const float4 w4 = tid < 128 ? reinterpret_cast<const float4*>(W.W4)[tid] : make_float4(0, 0, 0, 0);
-  const float4 w1 = tid < 64 ? reinterpret_cast<const float4*>(W.W1)[tid] : make_float4(0, 0, 0, 0);
-  const float bias1 = tid < 64 ? W.b1[tid] : 0.f;
-  const float bias2 = tid < 64 ? W.b2[tid] : 0.f;
-  const float bias3 = tid < 64 ? W.b3[tid] : 0.f;
-  const float bias4 = tid < 8 ? W.b4[tid] : 0.f;
+};
+
+// Weight tiles in the canonical layout, from the registers of WeightRegs.
+template <int NG, int SL>
+__device__ void store_weights(MlpSmem<NG, SL>& S, const WeightRegs& R) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) {
+  for (int j = 0; j < WeightRegs::kPer; ++j) {
     const int q = tid + j * nthr;
     if (q < 2048) {
       const int e = (q & 1023) * 4, n = e >> 6, k = e & 63;  // 4 consecutive k of one chunk
       const float sc = act_scale(k);
       __half* dst = (q < 1024 ? S.W2 : S.W3) + cofs(n, k, kWK);
       reinterpret_cast<uint2*>(dst)[0] =
-          make_uint2(h2bits(__float2half_rn(sc * w[j].x), __float2half_rn(sc * w[j].y)),
-                     h2bits(__float2half_rn(sc * w[j].z), __float2half_rn(sc * w[j].w)));
+          make_uint2(h2bits(__float2half_rn(sc * R.w[j].x), __float2half_rn(sc * R.w[j].y)),
+                     h2bits(__float2half_rn(sc * R.w[j].z), __float2half_rn(sc * R.w[j].w)));
     }
   }
   if (tid < 128) {  // W4 rows 0..7, zero rows 8..15
     const int e = tid * 4, n = e >> 6, k = e & 63;
     const float sc = act_scale(k);
     reinterpret_cast<uint2*>(S.W4 + cofs(n, k, kWK))[0] =
-        make_uint2(h2bits(__float2half_rn(sc * w4.x), __float2half_rn(sc * w4.y)),
-                   h2bits(__float2half_rn(sc * w4.z), __float2half_rn(sc * w4.w)));
+        make_uint2(h2bits(__float2half_rn(sc * R.w4.x), __float2half_rn(sc * R.w4.y)),
+                   h2bits(__float2half_rn(sc * R.w4.z), __float2half_rn(sc * R.w4.w)));
     reinterpret_cast<uint2*>(S.W4 + cofs(8 + n, k, kWK))[0] = make_uint2(0u, 0u);
   }
   if (tid < 64) {  // layer-1 row n = tid, and the bias columns of W2, W3, W4
     const int n = tid;
     __half h[4], l[4], bh, bl;
-    split_half(w1.x, h[0], l[0]);
-    split_half(w1.y, h[1], l[1]);
-    split_half(w1.z, h[2], l[2]);
-    split_half(w1.w, h[3], l[3]);
-    split_half(bias1, bh, bl);
+    split_half(R.w1.x, h[0], l[0]);
+    split_half(R.w1.y, h[1], l[1]);
+    split_half(R.w1.z, h[2], l[2]);
+    split_half(R.w1.w, h[3], l[3]);
+    split_half(R.bias1, bh, bl);
     const __half z = __float2half_rn(0.f);
     *reinterpret_cast<uint4*>(S.W1 + cofs(n, 0, 16)) =
         make_uint4(h2bits(h[0], h[1]), h2bits(h[2], h[3]), h2bits(l[0], l[1]), h2bits(l[2], l[3]));
     *reinterpret_cast<uint4*>(S.W1 + cofs(n, 8, 16)) =
         make_uint4(h2bits(h[0], h[1]), h2bits(h[2], h[3]), h2bits(bh, bl), h2bits(z, z));
-    split_half(bias2, bh, bl);
+    split_half(R.bias2, bh, bl);
     *reinterpret_cast<uint4*>(S.W2 + cofs(n, 64, kWK)) = make_uint4(h2bits(bh, bl), 0u, 0u, 0u);
     *reinterpret_cast<uint4*>(S.W2 + cofs(n, 72, kWK)) = make_uint4(0u, 0u, 0u, 0u);
-    split_half(bias3, bh, bl);
+    split_half(R.bias3, bh, bl);
     *reinterpret_cast<uint4*>(S.W3 + cofs(n, 64, kWK)) = make_uint4(h2bits(bh, bl), 0u, 0u, 0u);
     *reinterpret_cast<uint4*>(S.W3 + cofs(n, 72, kWK)) = make_uint4(0u, 0u, 0u, 0u);
     if (n < 16) {  // thread n < 8 holds b4[n]; rows 8..15 get zeros
-      split_half(n < 8 ? bias4 : 0.f, bh, bl);
+      split_half(n < 8 ? R.bias4 : 0.f, bh, bl);
       *reinterpret_cast<uint4*>(S.W4 + cofs(n, 64, kWK)) = make_uint4(h2bits(bh, bl), 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(S.W4 + cofs(n, 72, kWK)) = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -402,10 +411,11 @@ __device__ void load_weights(MlpSmem<NG, SL>& S, const MlpArgs& W) {
   }
 }
 
-// Once per CTA: weights, mbarriers, TMEM (warp 0 allocates NG*SL*64 columns).
+// Once per CTA: weights (loaded into R beforehand), mbarriers, TMEM (warp 0
+// allocates NG*SL*64 columns).
 template <int NG, int SL>
-__device__ void mlp_setup(MlpSmem<NG, SL>& S, const MlpArgs& W) {
-  load_weights<NG, SL>(S, W);
+__device__ void mlp_setup(MlpSmem<NG, SL>& S, const WeightRegs& R) {
+  store_weights<NG, SL>(S, R);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NG * SL; ++i) mbar_init(&S.mbar[i], 1);
     fence_mbar_init();
@@ -415,6 +425,13 @@ __device__ void mlp_setup(MlpSmem<NG, SL>& S, const MlpArgs& W) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+}
+
+template <int NG, int SL>
+__device__ void mlp_setup(MlpSmem<NG, SL>& S, const MlpArgs& W) {
+  WeightRegs R;
+  R.load(W);
+  mlp_setup<NG, SL>(S, R);
 }
 
 template <int NG, int SL>
@@ -1616,7 +1633,11 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
       fence_mbar_init();  // made visible by the barrier at the end of mlp_setup
     }
   }
-  mlp_setup<NG, SL>(S.mlp, W);
+  // the weights' loads are in flight while the first jet is staged
+  WeightRegs wr;
+  wr.load(W);
+  if (blockIdx.x < J.N) stage_jet<PM>(S.part, J, blockIdx.x);
+  mlp_setup<NG, SL>(S.mlp, wr);
   // during attention the activation tiles hold K and V
   float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
   constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
@@ -1626,7 +1647,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
   __nv_bfloat16* const PA = reinterpret_cast<__nv_bfloat16*>(stage);  // projection operands: rows,
   __nv_bfloat16* const PW = PA + kTileM * kEmbed;                     // then one weight chunk
   for (int n = blockIdx.x; n < J.N && !aborted; n += gridDim.x) {
-    stage_jet<PM>(S.part, J, n);
+    if (n != (int)blockIdx.x) stage_jet<PM>(S.part, J, n);
     if (threadIdx.x == 32) prefetch_jet(J, n + gridDim.x);  // this CTA's next jet
     // the jet's rows: padded slots n*P .. n*P+P-1, or its packed tokens
     const long long r_lo = J.ptr ? S.part.base : (long long)n * J.P;
@@ -1899,6 +1920,10 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
   const int G = gridDim.x, b = blockIdx.x;
   const int N = J.N;
 
+  // the weights' loads are in flight during phase 0
+  WeightRegs wr;
+  wr.load(W);
+
   // ---------------------------------------------------------------- phase 0
   // multiplicities into T[n + 1], tiles per jet, then an exclusive scan
   jet_counts(J, S.T);
@@ -1949,7 +1974,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
     nB = l;
   }
 
-  mlp_setup<NG, SL>(S.mlp, W);
+  mlp_setup<NG, SL>(S.mlp, wr);
   uint32_t phase = 0u;
   bool aborted = false;
 
