@@ -103,6 +103,7 @@ CASES = {
     "tiny_p3": dict(N=8, P=3, mults=[0, 1, 3, 2, 2, 3, 0, 1], mask_mode="scrambled", seed=9),
     "wide_p256": dict(N=3, P=256, mults=[256, 130, 17], pt_lo=800, pt_hi=1000, prongs=3, seed=5),
     "many_jets": dict(N=300, P=24, dist="uniform", mult_lo=1, mult_hi=24, mask_mode="scrambled", seed=8),
+    "packed_wide": dict(N=4, P=200, layout="packed", mults=[200, 150, 0, 7], pt_lo=800, pt_hi=1000, prongs=3, seed=10),
 }
 
 

@@ -157,6 +157,19 @@ def test_staging_path_boundaries(oracle_lib, P, mults):
     assert ops.get_device_status() == 0
 
 
+def test_packed_wide_jets(oracle_lib):
+    """Packed jets of up to 200 particles (the P = 256 kernels): triangle,
+    query-block and balanced paths against the oracle."""
+    b = synth.make_jets(N=4, P=200, layout="packed", mults=[200, 150, 0, 7], pt_lo=800, pt_hi=1000, prongs=3,
+                        seed=10)
+    d = pt.Device(b)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
+    pt.check_features(pt.to_np(d.features()), oracle_lib.features(b), b)
+    assert ops.get_device_status() == 0
+
+
 def test_packed_with_empty_jets(oracle_lib):
     b = synth.make_jets(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6)
     d = pt.Device(b)
