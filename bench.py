@@ -37,6 +37,13 @@ from part_pair_bias_b200 import configs, shard, synth  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 MLP_FLOP_PER_PAIR = 2 * (4 * 64 + 64 * 64 + 64 * 64 + 64 * 8)          # 17,920 (algorithmic)
 MMA_FLOP_PER_ROW = 2 * (16 * 64 + 64 * 64 + 64 * 64 + 64 * 16)         # 20,480 (issued per tile row)
+# backward MLP per unordered pair: recompute of layers 1-3, dL/dh3..dL/dh1
+# (g W4, d3 W3, d2 W2) and the weight gradients dW4, dW3, dW2, dW1
+BWD_FLOP_PER_PAIR = 2 * (4 * 64 + 2 * 64 * 64) + 2 * (8 * 64 + 2 * 64 * 64) + 2 * (8 * 64 + 2 * 64 * 64 + 64 * 4)
+# issued per tile row by the MLP backward kernel: z1 and g W4 (K = 16), four
+# 64 x 64 GEMMs, and the weight-gradient MMAs (dW4: 16 x 72, dW3, dW2: 64 x 72,
+# dW1: 64 x 16 with the bias columns)
+BWD_MMA_FLOP_PER_ROW = 2 * (2 * 16 * 64 + 4 * 64 * 64) + 2 * (16 * 72 + 2 * 64 * 72 + 64 * 16)
 PROFILE = os.path.join(ROOT, "profiles", "k_fused_n128_p128.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "part_pair_bias_b200", "csrc", f)
                   for f in ("pb_kernels.cuh", "pb_device.cuh", "pairbias.cu")]
@@ -54,6 +61,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per (workload, path) with times, rates and FLOP conventions")
+    ap.add_argument("--sweep-workloads", default=None, help="comma list restricting --sweep's workloads")
+    ap.add_argument("--sweep-paths", default=None, help="comma list restricting --sweep's paths")
     return ap.parse_args()
 
 
@@ -156,11 +165,21 @@ class ClockSampler:
         return out
 
 
-def cpu_baseline(b, seconds):
-    """The fp64 oracle, as it stands, on the host cores: full batches until
-    `seconds` have passed (at least one)."""
+def cpu_baseline(b, seconds, threads=None):
+    """The fp64 oracle, as it stands, on the host cores (all of them, or
+    `threads`): full batches until `seconds` have passed (at least one)."""
     import oracle
     oracle.build()
+    prev = oracle.threads()
+    if threads is not None:
+        oracle.set_threads(threads)
+    try:
+        return _time_oracle(oracle, b, seconds)
+    finally:
+        oracle.set_threads(prev if threads is not None else 0)
+
+
+def _time_oracle(oracle, b, seconds):
     t0 = time.perf_counter()
     passes = 0
     while True:
@@ -404,6 +423,9 @@ def run_sweep(args):
         return statistics.median(ts)
 
     names = list(configs.ORDER) + ["n128_p128_full"]
+    if args.sweep_workloads:
+        names = [n for n in names if n in args.sweep_workloads.split(",")]
+    only = set(args.sweep_paths.split(",")) if args.sweep_paths else None
     for name in names:
         if name == "n128_p128_full":
             b = synth.make_jets(**configs.workload("n128_p128", seed=args.seed, dist="full"))
@@ -439,12 +461,28 @@ def run_sweep(args):
                           inp + qkv + 256 * slots, True))
         paths.append(("block", lambda: ops.pair_block_forward(jets, mlp, proj, x, y, bws),
                       inp + 256 * slots + 256 * slots, True))
+        dout = ops.bf16_to_device(synth.make_upstream(b, args.seed), dev)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        grad = ops.MlpGrad(dev)
+        gws = torch.empty(ops.backward_workspace_bytes(jets), dtype=torch.uint8, device=dev)
+        # bytes: inputs twice (bias kernel, MLP backward), q/k/v/dout read, dq/dk/dv written,
+        # the bf16 bias planes written, read and overwritten, dL/dU read per pair
+        plane = 2 * 8 * b.N * b.P * b.P
+        paths.append(("backward", lambda: ops.pair_attention_backward(jets, mlp, q, k, v, dout, dq, dk, dv, grad, gws),
+                      2 * inp + 4 * 256 * valid + 3 * 256 * slots + 3 * plane + 2 * 8 * ordered, "bwd"))
         for path, fn, nbytes, has_mlp in paths:
+            if only is not None and path not in only:
+                continue
             ms = timed(fn)
             line = {"workload": name, "path": path, "seed": args.seed, "ms": ms, "jets_per_s": b.N / (ms / 1e3),
                     "pairs_per_s": ordered / (ms / 1e3), "alg_gbs": nbytes / (ms / 1e3) / 1e9,
                     "hbm_peak_gbs": hbm_gbs}
-            if has_mlp:
+            if has_mlp == "bwd":
+                line.update({"tflops_alg": unordered * (MLP_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR) / (ms / 1e3) / 1e12,
+                             "tflops_exec": tiles * 128 * (MMA_FLOP_PER_ROW + BWD_MMA_FLOP_PER_ROW) / (ms / 1e3) / 1e12,
+                             "flop_convention": "alg: bias recompute 17,920 + backward 52,224 per valid unordered pair",
+                             "peak_tflops": peak_tf, "peak_source": peak_src})
+            elif has_mlp:
                 line.update({"tflops_alg": unordered * MLP_FLOP_PER_PAIR / (ms / 1e3) / 1e12,
                              "tflops_exec": tiles * 128 * MMA_FLOP_PER_ROW / (ms / 1e3) / 1e12,
                              "tflops_dense": b.N * b.P * b.P * MLP_FLOP_PER_PAIR / (ms / 1e3) / 1e12,
@@ -452,10 +490,14 @@ def run_sweep(args):
             print(json.dumps(line), flush=True)
         if ops.get_device_status():
             raise RuntimeError(f"device status set on {name}")
+        if args.no_cpu_baseline:
+            continue
         sample = synth.slice_jets(b, 0, min(b.N, 16))
-        cb = cpu_baseline(sample, args.cpu_seconds / 4)
-        print(json.dumps({"workload": name, "path": "oracle (host)", "seed": args.seed, "jets_per_s": cb["value"],
-                          "cores": cb["cores"], "sample": cb["sample"]}), flush=True)
+        for threads in (None, 1):
+            cb = cpu_baseline(sample, args.cpu_seconds / 4, threads)
+            print(json.dumps({"workload": name, "path": "oracle (host)" if threads is None else "oracle (1 thread)",
+                              "seed": args.seed, "jets_per_s": cb["value"], "cores": cb["cores"],
+                              "sample": cb["sample"]}), flush=True)
 
 
 def main():
