@@ -380,12 +380,13 @@ template <int PM>
 struct MlpBwdSmem {
   __nv_bfloat16 A0[kTileM * 16];     // [hi(f) | lo(f) | hi(f) | 0]
   __nv_bfloat16 G4[kTileM * 16];     // [hi(g) | lo(g)] (8 heads each)
-  __nv_bfloat16 Hs[3][kTileM * 64];  // h1, h2, h3
+  __half Hf[2][kTileM * 64];         // h1, h2 in f16: operands of z2, z3
+  __nv_bfloat16 Hs[3][kTileM * 64];  // h1, h2, h3 in bf16: operands of the weight gradients
   __nv_bfloat16 Ds[3][kTileM * 64];  // d1, d2, d3 = dL/dz
   __nv_bfloat16 W1f[64 * 16];        // [hi(W1') | hi(W1') | lo(W1') | 0] per output row
-  __nv_bfloat16 Wf[2][64 * 64];      // W2', W3' as [out][in]
-  __nv_bfloat16 Wt[2][64 * 64];      // W2'^T, W3'^T as [in][out]
-  __nv_bfloat16 W4t[64 * 16];        // [W4^T | W4^T] as [in][out]
+  __half Wf[2][2][64 * 64];          // W2', W3' as [out][in], f16: hi, lo
+  __nv_bfloat16 Wt[2][2][64 * 64];   // W2'^T, W3'^T as [in][out]: hi, lo
+  __nv_bfloat16 W4t[2][64 * 16];     // [W4^T | W4^T] as [in][out]: hi, lo
   float bias[3][64];                 // b1', b2', b3'
   uint64_t mbar;
   uint32_t tmem_base;
@@ -398,38 +399,46 @@ __device__ void bwd_load_weights(MlpBwdSmem<PM>& S, const MlpArgs& W) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   for (int e = tid; e < 64 * 64; e += nthr) {
     const int o = e >> 6, i = e & 63;
-    const float w2 = W.W2[e], w3 = W.W3[e];
-    S.Wf[0][cofs(o, i, 64)] = __float2bfloat16_rn(w2);
-    S.Wf[1][cofs(o, i, 64)] = __float2bfloat16_rn(w3);
-    S.Wt[0][cofs(i, o, 64)] = __float2bfloat16_rn(w2);
-    S.Wt[1][cofs(i, o, 64)] = __float2bfloat16_rn(w3);
+    const float w[2] = {W.W2[e], W.W3[e]};
+#pragma unroll
+    for (int L = 0; L < 2; ++L) {
+      const __half fh = __float2half_rn(w[L]), fl = __float2half_rn(w[L] - __half2float(fh));
+      S.Wf[L][0][cofs(o, i, 64)] = fh;
+      S.Wf[L][1][cofs(o, i, 64)] = fl;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(w[L]), lo = __float2bfloat16_rn(w[L] - __bfloat162float(hi));
+      S.Wt[L][0][cofs(i, o, 64)] = hi;
+      S.Wt[L][1][cofs(i, o, 64)] = lo;
+    }
   }
   for (int e = tid; e < 64 * 16; e += nthr) {
     const int r = e >> 4, k = e & 15;  // W1f row = output r, W4t row = input r
     const float w1 = k < 12 ? W.W1[r * 4 + (k & 3)] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(w1);
     S.W1f[cofs(r, k, 16)] = (k >= 8 && k < 12) ? __float2bfloat16_rn(w1 - __bfloat162float(hi)) : hi;
-    S.W4t[cofs(r, k, 16)] = __float2bfloat16_rn(W.W4[(k & 7) * 64 + r]);
+    const float w4 = W.W4[(k & 7) * 64 + r];
+    const __nv_bfloat16 h4 = __float2bfloat16_rn(w4);
+    S.W4t[0][cofs(r, k, 16)] = h4;
+    S.W4t[1][cofs(r, k, 16)] = __float2bfloat16_rn(w4 - __bfloat162float(h4));
   }
   for (int e = tid; e < 3 * 64; e += nthr) S.bias[e >> 6][e & 63] = (e < 64 ? W.b1 : (e < 128 ? W.b2 : W.b3))[e & 63];
 }
 
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // GELU(z) = z/2 (1 + tanh(u)), u = sqrt(2/pi) (z + 0.044715 z^3), and its
-// derivative Phi + z/2 (1 - tanh^2 u) sqrt(2/pi) (1 + 3 0.044715 z^2), where
-// Phi = (1 + tanh u) / 2.
+// derivative Phi + z/2 sech^2(u) sqrt(2/pi) (1 + 3 0.044715 z^2), where
+// Phi = (1 + tanh u) / 2. Both come from w = exp(-2|u|): Phi = 1 / (1 + w)
+// (u >= 0) or w / (1 + w), sech^2 u = 4 w / (1 + w)^2, which stay accurate
+// where tanh saturates (1 - tanh^2 from an approximate tanh would not, and
+// its error there is the same for every pair with large |u|).
 __device__ __forceinline__ void gelu_tanh_and_grad(float z, float& h, float& dh) {
   constexpr float kC0 = 0.7978845608028654f, kC1 = 0.044715f;
   const float z2 = z * z, c0z = kC0 * z;
-  const float t = tanh_approx(c0z * fmaf(kC1, z2, 1.f));
-  const float phi = fmaf(0.5f, t, 0.5f);
+  const float u = c0z * fmaf(kC1, z2, 1.f);
+  const float w = ex2(-2.f * kLog2e * fabsf(u));
+  const float r = __fdividef(1.f, 1.f + w);
+  const float phi = u >= 0.f ? r : w * r;
   h = z * phi;
-  dh = fmaf(0.5f * fmaf(-t, t, 1.f), c0z * fmaf(3.f * kC1, z2, 1.f), phi);
+  const float sech2 = 4.f * w * r * r;
+  dh = fmaf(0.5f * sech2, c0z * fmaf(3.f * kC1, z2, 1.f), phi);
 }
 
 // TMEM <- registers, 32 lanes x 16 columns (thread t of the warp writes lane
@@ -580,7 +589,8 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
   // TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192) (then GELU'), e3 / e2 / e1 [192, 256)
   const uint32_t tm = S.tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
   constexpr uint32_t kId = idesc_bf16_m128(64);
-  const uint32_t a0 = smem_u32(S.A0), g4 = smem_u32(S.G4), w1f = smem_u32(S.W1f), w4t = smem_u32(S.W4t);
+  const uint32_t a0 = smem_u32(S.A0), g4 = smem_u32(S.G4), w1f = smem_u32(S.W1f);
+  const uint32_t w4t_hi = smem_u32(S.W4t[0]), w4t_lo = smem_u32(S.W4t[1]);
   uint32_t phase = 0u;
   bool ok = true, aborted = false;
 
@@ -610,18 +620,28 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
     ok = ok && done;
     tc_fence_after();
   };
-  auto gemm64 = [&](uint32_t d, const __nv_bfloat16* A, const __nv_bfloat16* B) {
-    const uint32_t aa = smem_u32(A), bb = smem_u32(B);
+  // D = A (W_hi + W_lo): the weights' rounding error is the same for every
+  // pair row and would not average out of the gradient sums, so they enter as
+  // two terms. The recompute's products (A = h, f16) use kind::f16 with f16
+  // operands, the backward's (A = d, bf16) bf16 operands.
+  auto gemm64 = [&](uint32_t d, uint32_t aa, uint32_t b_hi, uint32_t b_lo, uint32_t id) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      mma_f16(d, smem_desc(aa + 256u * k, 128, 1024), smem_desc(bb + 256u * k, 128, 1024), kId, k > 0 ? 1u : 0u);
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t bb = part ? b_lo : b_hi;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_f16(d, smem_desc(aa + 256u * k, 128, 1024), smem_desc(bb + 256u * k, 128, 1024), id,
+                (part | k) != 0 ? 1u : 0u);
+    }
   };
-  auto store16 = [&](__nv_bfloat16* T, const float* v) {
+  constexpr uint32_t kIdF16 = idesc_f16_m128(64);
+  auto store16 = [&](void* T, const float* v, bool f16) {
     uint32_t w[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = cvt_bf16x2(v[2 * i], v[2 * i + 1]);
-    *reinterpret_cast<uint4*>(T + cofs(r, 16 * c, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(T + cofs(r, 16 * c + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
+    for (int i = 0; i < 8; ++i) w[i] = f16 ? cvt_f16x2(v[2 * i], v[2 * i + 1]) : cvt_bf16x2(v[2 * i], v[2 * i + 1]);
+    uint16_t* T16 = static_cast<uint16_t*>(T);
+    *reinterpret_cast<uint4*>(T16 + cofs(r, 16 * c, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(T16 + cofs(r, 16 * c + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
   };
   // h_k = GELU(z_k + b_k) to the operand tile, GELU'(z_k + b_k) back over z_k in TMEM
   auto hidden = [&](int k) {
@@ -639,7 +659,8 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) gelu_tanh_and_grad(z[i], h[i], z[i]);
-    store16(S.Hs[k], h);
+    if (k < 2) store16(S.Hf[k], h, true);  // the next layer's operand
+    store16(S.Hs[k], h, false);
     tmem_st16_wait(ta, z);
   };
   // d_k = e * GELU'(z_k + b_k)
@@ -649,7 +670,7 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
     tmem_ld16_wait(tm + lane_off + 192u + 16u * c, e);
 #pragma unroll
     for (int i = 0; i < 16; ++i) e[i] *= gp[i];
-    store16(S.Ds[k], e);
+    store16(S.Ds[k], e, false);
   };
 
   const long long Ttot = X.T[J.N];
@@ -708,20 +729,21 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
       // forward: z1 (and e3 = g W4, which needs nothing else), z2, z3
       if (!issue([&] {
             mma_f16(tm, smem_desc(a0, 128, 256), smem_desc(w1f, 128, 256), kId, 0u);
-            mma_f16(tm + 192u, smem_desc(g4, 128, 256), smem_desc(w4t, 128, 256), kId, 0u);
+            mma_f16(tm + 192u, smem_desc(g4, 128, 256), smem_desc(w4t_hi, 128, 256), kId, 0u);
+            mma_f16(tm + 192u, smem_desc(g4, 128, 256), smem_desc(w4t_lo, 128, 256), kId, 1u);
           })) {
         aborted = true;
         break;
       }
       wait();
       hidden(0);
-      if (!issue([&] { gemm64(tm + 64u, S.Hs[0], S.Wf[0]); })) {
+      if (!issue([&] { gemm64(tm + 64u, smem_u32(S.Hf[0]), smem_u32(S.Wf[0][0]), smem_u32(S.Wf[0][1]), kIdF16); })) {
         aborted = true;
         break;
       }
       wait();
       hidden(1);
-      if (!issue([&] { gemm64(tm + 128u, S.Hs[1], S.Wf[1]); })) {
+      if (!issue([&] { gemm64(tm + 128u, smem_u32(S.Hf[1]), smem_u32(S.Wf[1][0]), smem_u32(S.Wf[1][1]), kIdF16); })) {
         aborted = true;
         break;
       }
@@ -729,13 +751,13 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
       hidden(2);
       delta(2);
       // backward: e2 = d3 W3', e1 = d2 W2'
-      if (!issue([&] { gemm64(tm + 192u, S.Ds[2], S.Wt[1]); })) {
+      if (!issue([&] { gemm64(tm + 192u, smem_u32(S.Ds[2]), smem_u32(S.Wt[1][0]), smem_u32(S.Wt[1][1]), kId); })) {
         aborted = true;
         break;
       }
       wait();
       delta(1);
-      if (!issue([&] { gemm64(tm + 192u, S.Ds[1], S.Wt[0]); })) {
+      if (!issue([&] { gemm64(tm + 192u, smem_u32(S.Ds[1]), smem_u32(S.Wt[0][0]), smem_u32(S.Wt[0][1]), kId); })) {
         aborted = true;
         break;
       }

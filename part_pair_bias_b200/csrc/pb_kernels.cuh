@@ -956,6 +956,86 @@ __device__ __forceinline__ void q_frag(int i0, int nrows, const QRow& qrow, uint
 // m, u) fills the bias of the 8 score elements a lane holds for the key
 // block n0 (element e: row e & 2 ? ib : ia, key n0 + 8 (e >> 2) + 2 t +
 // (e & 1), keys past m clamped to m - 1). Warp-wide.
+// Normalise and store the two output rows of a lane (o as accumulated, la /
+// lb the lane's partial row sums of p).
+template <class ORow>
+__device__ __forceinline__ void store_out16(const float* o, float la, float lb, bool va, bool vb, int ia, int ib,
+                                            int t, const ORow& orow) {
+  la += __shfl_xor_sync(0xffffffffu, la, 1);
+  la += __shfl_xor_sync(0xffffffffu, la, 2);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+  if (va) {
+    const float r = 1.0f / la;
+    uint16_t* op = orow(ia);
+    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(o[0] * r, o[1] * r);
+    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(o[4] * r, o[5] * r);
+  }
+  if (vb) {
+    const float r = 1.0f / lb;
+    uint16_t* op = orow(ib);
+    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(o[2] * r, o[3] * r);
+    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(o[6] * r, o[7] * r);
+  }
+}
+
+// Jets of at most 16 NKB keys: every block's scores stay in registers, so the
+// softmax takes two passes (one row maximum, then the exponentials and P V)
+// and the blocks' products and exponentials are independent of each other,
+// with no rescaling chain between blocks.
+template <int NKB, class ORow, class UBlock>
+__device__ __forceinline__ void attend_tile16_short(uint32_t k_base, uint32_t v_base, int m, int i0, int ia, int ib,
+                                                    bool va, bool vb, const uint32_t* a, const ORow& orow,
+                                                    const UBlock& ub) {
+  const int t = threadIdx.x & 3;
+  const float qs = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
+  float s[NKB][8];
+#pragma unroll
+  for (int kb = 0; kb < NKB; ++kb) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[kb][e] = 0.f;
+    uint32_t bk[4];
+    ldsm_x4(k_base + (uint32_t)kb * 512u, bk);
+    mma_16816(s[kb], a, bk[0], bk[1]);
+    mma_16816(s[kb] + 4, a, bk[2], bk[3]);
+  }
+  float mxa = -INFINITY, mxb = -INFINITY;
+#pragma unroll
+  for (int kb = 0; kb < NKB; ++kb) {
+    float u[8];
+    ub(16 * kb, i0, ia, ib, t, m, u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = 16 * kb + (e & 4 ? 8 : 0) + 2 * t + (e & 1);
+      s[kb][e] = j < m ? fmaf(s[kb][e], qs, u[e] * kLog2e) : -INFINITY;
+    }
+    mxa = fmaxf(mxa, fmaxf(fmaxf(s[kb][0], s[kb][1]), fmaxf(s[kb][4], s[kb][5])));
+    mxb = fmaxf(mxb, fmaxf(fmaxf(s[kb][2], s[kb][3]), fmaxf(s[kb][6], s[kb][7])));
+  }
+  // key 0 < m is valid for every row, so the maxima are finite
+  mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+  mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+  mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+  mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+  float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float la = 0.f, lb = 0.f;
+#pragma unroll
+  for (int kb = 0; kb < NKB; ++kb) {
+    float p[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) p[e] = ex2(s[kb][e] - (e & 2 ? mxb : mxa));
+    la += (p[0] + p[1]) + (p[4] + p[5]);
+    lb += (p[2] + p[3]) + (p[6] + p[7]);
+    const uint32_t pa[4] = {cvt_bf16x2(p[0], p[1]), cvt_bf16x2(p[2], p[3]), cvt_bf16x2(p[4], p[5]),
+                            cvt_bf16x2(p[6], p[7])};
+    uint32_t bv[4];
+    ldsm_x4_t(v_base + (uint32_t)kb * 512u, bv);
+    mma_16816(o, pa, bv[0], bv[1]);
+    mma_16816(o + 4, pa, bv[2], bv[3]);
+  }
+  store_out16(o, la, lb, va, vb, ia, ib, t, orow);
+}
+
 template <class ORow, class UBlock>
 __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t* vh, int m, int i0, int nrows,
                                               const uint32_t* a, const ORow& orow, const UBlock& ub) {
@@ -966,6 +1046,13 @@ __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t
   const uint32_t v_base = smem_u32(vh) + kv_off((lane & 7) + ((lane >> 3) & 1) * 8, (lane >> 4) & 1);
   const bool va = g < nrows, vb = g + 8 < nrows;
   const int ia = i0 + (va ? g : 0), ib = i0 + (vb ? g + 8 : 0);  // rows past the block alias row i0
+  switch ((m + 15) >> 4) {
+    case 1: attend_tile16_short<1>(k_base, v_base, m, i0, ia, ib, va, vb, a, orow, ub); return;
+    case 2: attend_tile16_short<2>(k_base, v_base, m, i0, ia, ib, va, vb, a, orow, ub); return;
+    case 3: attend_tile16_short<3>(k_base, v_base, m, i0, ia, ib, va, vb, a, orow, ub); return;
+    case 4: attend_tile16_short<4>(k_base, v_base, m, i0, ia, ib, va, vb, a, orow, ub); return;
+    default: break;
+  }
   const float qs = 0.25f * kLog2e;  // 1/sqrt(D) with D = 16, in log2 units
   float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float mxa = -INFINITY, mxb = -INFINITY, la = 0.f, lb = 0.f;
@@ -1012,22 +1099,7 @@ __device__ __forceinline__ void attend_tile16(const uint16_t* kh, const uint16_t
     mma_16816(o, pa, bv[0], bv[1]);
     mma_16816(o + 4, pa, bv[2], bv[3]);
   }
-  la += __shfl_xor_sync(0xffffffffu, la, 1);
-  la += __shfl_xor_sync(0xffffffffu, la, 2);
-  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
-  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-  if (va) {
-    const float r = 1.0f / la;
-    uint16_t* op = orow(ia);
-    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(o[0] * r, o[1] * r);
-    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(o[4] * r, o[5] * r);
-  }
-  if (vb) {
-    const float r = 1.0f / lb;
-    uint16_t* op = orow(ib);
-    *reinterpret_cast<uint32_t*>(op + 2 * t) = cvt_bf16x2(o[2] * r, o[3] * r);
-    *reinterpret_cast<uint32_t*>(op + 8 + 2 * t) = cvt_bf16x2(o[6] * r, o[7] * r);
-  }
+  store_out16(o, la, lb, va, vb, ia, ib, t, orow);
 }
 
 // Masked multi-head attention for queries [i_lo, i_hi) of the staged jet

@@ -7,16 +7,17 @@ arithmetic of the forward bars and the backward's own roundings):
                   The bias enters through the forward MLP kernel (bias bar:
                   rel L2 1e-2), the softmax gradient dS = P (dP - D) loses
                   relative accuracy where dP ~ D, and dq, dk, dv are bf16.
-  MLP gradients   relative L2 per folded tensor <= 4e-2. These sums of
-                  g * h over the pairs cancel heavily (each row of dS sums to
-                  0), so an error in the bias U reaches them amplified:
-                  perturbing U in the fp64 oracle by noise of 5e-3 (2e-2)
-                  moves them by up to 1e-2 (4e-2), a gain of up to 2-4 on the
-                  bias bar (rel L2 1e-2). The bias here is the forward
-                  kernel's (f16 records); dL/dU accumulates in fp32; the MLP
-                  is recomputed with bf16 operands (f and g as hi + lo).
+  MLP gradients   relative L2 per folded tensor <= 3e-2. These sums of
+                  d * h over the pairs cancel heavily (each row of dS sums
+                  to 0), so operand roundings reach them amplified. An fp64
+                  emulation of the kernel's rounding points reproduces the
+                  measured errors: with bf16 activations feeding the next
+                  layer, dW1 was off by 2.5 %; the recompute now keeps them
+                  in f16 (and the weights as hi + lo pairs), which leaves
+                  0.3-1.5 % (bf16 operands in the weight products, f16 in
+                  the recompute, the forward kernel's own bias).
   db4             zero in exact arithmetic (rows of dS sum to 0): at most
-                  4e-2 times the largest dW4 row norm.
+                  3e-2 times the largest dW4 row norm.
 """
 import numpy as np
 import pytest
@@ -28,7 +29,7 @@ from tests import parity as pt
 pytestmark = pytest.mark.gpu
 
 QKV_RELL2 = 2e-2
-GRAD_RELL2 = 4e-2
+GRAD_RELL2 = 3e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
