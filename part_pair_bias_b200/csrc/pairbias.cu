@@ -189,6 +189,41 @@ pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArg
   return launched(kProj ? "k_fused (with projections)" : "k_fused");
 }
 
+// The 4-CTA cluster kernel takes batches of at most this many jets per SM
+// (one jet per CTA); larger batches already balance over the persistent CTAs.
+constexpr int kClusterJetsPerSm = 1;
+
+template <int PM>
+pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s) {
+  auto k = pb::k_fused_cluster<PM>;
+  const size_t smem = sizeof(pb::ClusterSmem<PM>);
+  int dev = 0, sms = 0, per_sm = 0;
+  pb_status st = device_sms(&dev, &sms);
+  if (st != PB_OK) return st;
+  if ((st = resident_per_sm((const void*)k, dev, smem, 512, &per_sm)) != PB_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((J.N + pb::kCJ - 1) / pb::kCJ * pb::kCJ));
+  cfg.blockDim = dim3(512);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pb::kCJ;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k, J, W, X);
+  if (e != cudaSuccess) return fail(PB_ECUDA, "k_fused_cluster launch: %s", cudaGetErrorString(e));
+  return PB_OK;
+}
+
+bool cluster_applies(const pb::JetArgs& J) {
+  int dev = 0, sms = 0;
+  if (device_sms(&dev, &sms) != PB_OK) return false;
+  return J.P <= 128 && J.N >= 1 && J.N <= kClusterJetsPerSm * sms;
+}
+
 constexpr long long kGridMaxMaskBytes = 1ll << 21;  // padded N*P scanned by every CTA in phase 0
 
 bool grid_applies(const pb::JetArgs& J) {
@@ -412,6 +447,7 @@ pb_status pair_attention_forward(const pb_jets* jets, const pb_mlp* mlp, const u
           workspace_bytes >= pb::grid_workspace_bytes(J.N, J.P, J.tokens, J.ptr != nullptr))
         return J.P <= 128 ? run_fused_grid<128>(J, W, X, workspace, s) : run_fused_grid<256>(J, W, X, workspace, s);
     }
+    if (cluster_applies(J)) return run_fused_cluster<128>(J, W, X, s);
     return J.P <= 128 ? run_fused<128>(J, W, X, s) : run_fused<256>(J, W, X, s);
   }
   return J.P <= 128 ? run_attn_bias<128>(J, X, U, s) : run_attn_bias<256>(J, X, U, s);

@@ -877,44 +877,47 @@ __device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t 
 // Bias blocks: the 8 values of U[h, ., .] a lane needs for one key block
 // (see attend_tile16), from the storage layouts the kernels use.
 
-// Triangle of 8-half records, pair (a, b) with a >= b at record a(a+1)/2 + b;
+// Triangle of records of RS halves (one per head: 8 for all heads, 2 where
+// a CTA holds two heads), pair (a, b) with a >= b at record a(a+1)/2 + b;
 // U points at head h of record 0. Query tiles and key blocks are aligned to
 // 16, so a full key block lies wholly below the tile's rows (records
 // i(i+1)/2 + j, contiguous in j), wholly above them (records j(j+1)/2 + i),
 // or on the diagonal, which takes the general formula.
-struct TriBlock {
+template <int RS>
+struct TriBlockS {
   const __half* U;
   __device__ __forceinline__ void operator()(int n0, int i0, int ia, int ib, int t, int m, float* u) const {
     const int jb = n0 + 2 * t;
     if (n0 + 16 <= m && n0 + 16 <= i0) {
-      const __half* ra = U + (ia * (ia + 1) / 2 + jb) * 8;
-      const __half* rb = U + (ib * (ib + 1) / 2 + jb) * 8;
+      const __half* ra = U + (ia * (ia + 1) / 2 + jb) * RS;
+      const __half* rb = U + (ib * (ib + 1) / 2 + jb) * RS;
       u[0] = __half2float(ra[0]);
-      u[1] = __half2float(ra[8]);
-      u[4] = __half2float(ra[64]);
-      u[5] = __half2float(ra[72]);
+      u[1] = __half2float(ra[RS]);
+      u[4] = __half2float(ra[8 * RS]);
+      u[5] = __half2float(ra[9 * RS]);
       u[2] = __half2float(rb[0]);
-      u[3] = __half2float(rb[8]);
-      u[6] = __half2float(rb[64]);
-      u[7] = __half2float(rb[72]);
+      u[3] = __half2float(rb[RS]);
+      u[6] = __half2float(rb[8 * RS]);
+      u[7] = __half2float(rb[9 * RS]);
     } else if (n0 + 16 <= m && n0 >= i0 + 16) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int j = jb + (c & 1) + (c & 2) * 4, e = (c & 2) * 2 + (c & 1);
-        const __half* cj = U + (j * (j + 1) / 2) * 8;
-        u[e] = __half2float(cj[ia * 8]);
-        u[e + 2] = __half2float(cj[ib * 8]);
+        const __half* cj = U + (j * (j + 1) / 2) * RS;
+        u[e] = __half2float(cj[ia * RS]);
+        u[e + 2] = __half2float(cj[ib * RS]);
       }
     } else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int i = e & 2 ? ib : ia, j = min(m - 1, jb + (e & 4 ? 8 : 0) + (e & 1));
         const int hi = max(i, j), lo = min(i, j);
-        u[e] = __half2float(U[(hi * (hi + 1) / 2 + lo) * 8]);
+        u[e] = __half2float(U[(hi * (hi + 1) / 2 + lo) * RS]);
       }
     }
   }
 };
+using TriBlock = TriBlockS<8>;
 
 // Rectangle of 8-half records, (query i, key j) at record (i - r0) * m + j;
 // U points at head h of record 0.
@@ -2260,6 +2263,221 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
   return kWsHeader + (size_t)rows * 16;
 }
 
+
+// ============================================== k_fused_cluster (4-CTA jets)
+//
+// The fused path for batches of few jets, where one CTA per jet would wait
+// for the widest one: a thread-block cluster of 4 CTAs takes 4 jets.
+//   - every CTA stages all 4 jets; the MLP tiles of the 4 jets are split
+//     evenly over the 4 CTAs (contiguous ranges of the cluster's tile list);
+//   - a tile row's 8 biases go straight to the CTA that owns their heads:
+//     CTA q keeps heads 2q, 2q + 1 of every pair of the 4 jets, 4 bytes per
+//     pair, written through distributed shared memory (st.shared::cluster);
+//   - a cluster barrier publishes them; CTA q then attends heads 2q, 2q + 1
+//     of each jet from its own shared memory.
+// When the 4 jets' pairs do not fit (kClusterUCap pairs), each CTA runs one
+// of the jets alone on query blocks (8-head records in the same space).
+// Cluster barriers are hardware barriers that every CTA reaches on every
+// path; the first one makes sure all 4 CTAs run before any remote store.
+
+constexpr int kCJ = 4;  // jets and CTAs per cluster
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+
+template <int PM>
+struct ClusterHead {
+  MlpSmem<4, 2> mlp;  // activation tiles double as the attention stage
+  Particles<PM> ring[kCJ];
+  int tbeg[kCJ + 1];     // prefix of the jets' MLP tiles
+  int tri_off[kCJ + 1];  // prefix of the jets' pairs
+  int lo, hi;            // this CTA's tiles of the cluster's list
+  int fits;
+  int kvoff[kCJ + 1];    // staged K/V of each jet (halves) in the attention
+  int ib[kCJ + 1];       // prefix of each jet's (head, query tile) items
+};
+
+template <int PM>
+struct ClusterSmem {
+  static constexpr int kHead = ((int)sizeof(ClusterHead<PM>) + 15) & ~15;
+  static constexpr int kUCap = (kSmemLimit - kHead - 1024) / 16 * 4;
+  ClusterHead<PM> h;
+  alignas(16) uint32_t U[kUCap];  // heads 2q, 2q + 1 of every pair (f16x2), jet after jet; or 16-byte 8-head records
+};
+
+// The rows of this CTA's tiles of the cluster's 4 jets; the sink key is the
+// pair's index in the cluster's triangles.
+template <int PM>
+struct ClusterTiles {
+  const ClusterHead<PM>* H;
+  __device__ __forceinline__ int ntiles() const { return H->hi - H->lo; }
+  __device__ __forceinline__ bool row(int t, int r, int& p, int& a, int& b, float f[4]) const {
+    const int gt = H->lo + t;
+    int k = 0;
+#pragma unroll
+    for (int q = 1; q < kCJ; ++q) k += H->tbeg[q] <= gt ? 1 : 0;
+    const int pl = (gt - H->tbeg[k]) * kTileM + r;
+    const int m = H->ring[k].m;
+    if (pl >= m * (m + 1) / 2) return false;
+    TriPairs{}.map(pl, a, b);
+    if (!in_bounds(a >= 0 && a <= b && b < m)) return false;
+    pair_feat<PM, true>(H->ring[k], a, b, f);
+    p = H->tri_off[k] + pl;
+    return true;
+  }
+};
+
+struct ClusterUSink {  // pair p's heads 2q, 2q + 1 to CTA q's entry p
+  uint32_t base[kCJ];  // shared::cluster address of U in each CTA
+  int cap;
+  __device__ __forceinline__ void operator()(int p, int, int, const float* u) const {
+    if (!in_bounds(p >= 0 && p < cap)) return;
+#pragma unroll
+    for (int q = 0; q < kCJ; ++q) st_cluster_u32(base[q] + 4u * (uint32_t)p, pack_half2(u[2 * q], u[2 * q + 1]));
+  }
+};
+
+struct ClusterUBias {  // heads h0, h0 + 1 of one jet's triangle, 2 halves per pair
+  const __half* U;
+  int h0;
+  __device__ __forceinline__ TriBlockS<2> head(int h) const { return TriBlockS<2>{U + (h - h0)}; }
+};
+
+template <int PM>
+__global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, QkvArgs X) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  ClusterSmem<PM>& S = *reinterpret_cast<ClusterSmem<PM>*>(smem_raw);
+  ClusterHead<PM>& H = S.h;
+  constexpr int NG = 4, SL = 2;
+  constexpr int kUCap = ClusterSmem<PM>::kUCap;
+  const int q = (int)cluster_ctarank();
+  const int n0 = (blockIdx.x / kCJ) * kCJ;
+  const int K = min(kCJ, J.N - n0);  // >= 1: the grid covers the jets
+  WeightRegs wr;
+  wr.load(W);
+  stage_jets<PM, true>(H.ring, J, K, [n0](int k) { return n0 + k; });
+  mlp_setup<NG, SL>(H.mlp, wr);
+  if (threadIdx.x == 0) {
+    int pairs = 0, tiles = 0;
+    for (int k = 0; k < kCJ; ++k) {
+      const int m = k < K ? H.ring[k].m : 0;
+      H.tri_off[k] = pairs;
+      H.tbeg[k] = tiles;
+      pairs += m * (m + 1) / 2;
+      tiles += (m * (m + 1) / 2 + kTileM - 1) / kTileM;
+    }
+    H.tri_off[kCJ] = pairs;
+    H.tbeg[kCJ] = tiles;
+    H.kvoff[0] = 0;
+    H.ib[0] = 0;
+    for (int k = 0; k < kCJ; ++k) {
+      const int m = k < K ? H.ring[k].m : 0;
+      H.kvoff[k + 1] = H.kvoff[k] + (m > 0 ? kv16_bytes(m) : 0);  // two heads of kv16_bytes / 2 halves
+      H.ib[k + 1] = H.ib[k] + (m > 0 ? 2 * ((m + 15) >> 4) : 0);
+    }
+    H.lo = tiles * q / kCJ;
+    H.hi = tiles * (q + 1) / kCJ;
+    H.fits = pairs <= kUCap ? 1 : 0;
+  }
+  __syncthreads();
+  cluster_sync_all();  // all 4 CTAs run: their shared memory may be written
+  float* stage = reinterpret_cast<float*>(&H.mlp.A[0][0]);
+  constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
+  uint32_t phase = 0u;
+  bool aborted = false;
+  if (H.fits) {
+    ClusterUSink sink;
+    const uint32_t local = smem_u32(S.U);
+#pragma unroll
+    for (int c = 0; c < kCJ; ++c) sink.base[c] = map_shared_rank(local, (uint32_t)c);
+    sink.cap = kUCap;
+    const bool ok = mlp_pass<NG, SL>(H.mlp, ClusterTiles<PM>{&H}, sink, &phase);
+    aborted = __syncthreads_or(!ok) != 0;
+    cluster_sync_all();  // every CTA's stores into this one are visible
+    if (!aborted) {
+      // heads 2q, 2q + 1 of all the cluster's jets at once: K and V of every
+      // (jet, head) staged together, then the warps take (jet, head, 16-query
+      // tile) items, the next item's Q fragment loaded ahead
+      uint16_t* kv = reinterpret_cast<uint16_t*>(stage);
+      const int* kvoff = H.kvoff;
+      const int* ib = H.ib;
+      for (int k = 0; k < K; ++k)
+        if (H.ring[k].m > 0) stage_kv16<PM>(H.ring[k], J, X, n0 + k, 2 * q, 2, kv + kvoff[k]);
+      const int items = ib[kCJ], warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+      auto locate = [&](int it, int& k, int& h, int& i0) {
+        k = 0;
+#pragma unroll
+        for (int c = 1; c < kCJ; ++c) k += ib[c] <= it ? 1 : 0;
+        const int tiles = (H.ring[k].m + 15) >> 4, loc = it - ib[k];
+        h = 2 * q + loc / tiles;
+        i0 = (loc % tiles) * 16;
+      };
+      auto qload = [&](int it, uint32_t* f) {
+        int k, h, i0;
+        locate(it, k, h, i0);
+        const Particles<PM>& P = H.ring[k];
+        q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, n0 + k, h, i); }, f);
+      };
+      uint32_t a[4] = {0u, 0u, 0u, 0u};
+      if (warp < items) qload(warp, a);
+      cp_async_wait_all();
+      __syncthreads();
+      for (int it = warp; it < items; it += nwarp) {
+        uint32_t an[4] = {0u, 0u, 0u, 0u};
+        if (it + nwarp < items) qload(it + nwarp, an);
+        int k, h, i0;
+        locate(it, k, h, i0);
+        const Particles<PM>& P = H.ring[k];
+        const int m = P.m;
+        const uint16_t* kh = kv + kvoff[k] + (h - 2 * q) * (kv16_bytes(m) / 2);
+        const ClusterUBias ub{reinterpret_cast<const __half*>(S.U + H.tri_off[k]), 2 * q};
+        attend_tile16(
+            kh, kh + round16(m) * 16, m, i0, min(16, m - i0), a,
+            [&](int i) { return X.out + qkv_off<PM>(P, J, n0 + k, h, i); }, ub.head(h));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a[e] = an[e];
+      }
+      if (q < K) zero_masked_rows<PM>(H.ring[q], J, X.out, n0 + q);
+    }
+  } else {
+    // one jet per CTA on query blocks, 8-head records in the same space
+    cluster_sync_all();  // the same barriers on both paths
+    if (q < K) {
+      const Particles<PM>& P = H.ring[q];
+      const int m = P.m, cap = kUCap / 4;
+      SmemUSink sink{reinterpret_cast<uint4*>(S.U), cap};
+      const int qb = max(1, cap / max(1, m));
+      for (int i0 = 0; i0 < m && !aborted; i0 += qb) {
+        const int i1 = min(m, i0 + qb);
+        const bool ok = mlp_pass<NG, SL>(H.mlp, JetTiles<PM, RectPairs, true>{&P, (i1 - i0) * m, RectPairs{i0, m}}, sink,
+                                         &phase);
+        aborted = __syncthreads_or(!ok) != 0;
+        if (aborted) break;
+        const RectUBias ub{reinterpret_cast<const __half*>(S.U), i0, m};
+        attention_block<PM>(P, J, X, n0 + q, i0, i1, stage, kStageFloats, ub);
+      }
+      if (!aborted) zero_masked_rows<PM>(P, J, X.out, n0 + q);
+    }
+  }
+  mlp_teardown<NG, SL>(H.mlp, aborted, &phase);
+}
 
 // ================================================= k_wait_selftest (diagnostic)
 //
