@@ -221,7 +221,7 @@ pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb
 bool cluster_applies(const pb::JetArgs& J) {
   int dev = 0, sms = 0;
   if (device_sms(&dev, &sms) != PB_OK) return false;
-  return J.P <= 128 && J.N >= 1 && J.N <= kClusterJetsPerSm * sms;
+  return J.P <= 128 && J.N >= 1 && J.N <= kClusterJetsPerSm * sms && J.N <= pb::kClusterMaxJets;
 }
 
 constexpr long long kGridMaxMaskBytes = 1ll << 21;  // padded N*P scanned by every CTA in phase 0

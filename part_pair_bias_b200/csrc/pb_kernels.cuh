@@ -2280,7 +2280,9 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
 // Cluster barriers are hardware barriers that every CTA reaches on every
 // path; the first one makes sure all 4 CTAs run before any remote store.
 
-constexpr int kCJ = 4;  // jets and CTAs per cluster
+constexpr int kCJ = 4;                // jets and CTAs per cluster
+constexpr int kClusterMaxJets = 256;  // batch size the jet table holds
+constexpr int kMaxJetTiles = (128 * 129 / 2 + kTileM - 1) / kTileM;  // MLP tiles of a full P = 128 jet
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -2312,6 +2314,10 @@ struct ClusterHead {
   int fits;
   int kvoff[kCJ + 1];    // staged K/V of each jet (halves) in the attention
   int ib[kCJ + 1];       // prefix of each jet's (head, query tile) items
+  int jets[kCJ];         // this cluster's jets
+  int cnt[kClusterMaxJets + 1];  // multiplicity of every jet of the batch (cnt[n + 1])
+  int order[kClusterMaxJets];    // jets by decreasing MLP tiles
+  int bin[kMaxJetTiles + 2];     // jets per tile count, then the next free rank of each
 };
 
 template <int PM>
@@ -2368,11 +2374,63 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   constexpr int NG = 4, SL = 2;
   constexpr int kUCap = ClusterSmem<PM>::kUCap;
   const int q = (int)cluster_ctarank();
-  const int n0 = (blockIdx.x / kCJ) * kCJ;
-  const int K = min(kCJ, J.N - n0);  // >= 1: the grid covers the jets
+  const int c = blockIdx.x / kCJ, ncl = gridDim.x / kCJ;
   WeightRegs wr;
-  wr.load(W);
-  stage_jets<PM, true>(H.ring, J, K, [n0](int k) { return n0 + k; });
+  wr.load(W);  // in flight while the jets are counted and staged
+  // Every CTA counts every jet and sorts them by MLP tiles, largest first,
+  // ties in jet order (a stable counting sort: every CTA must come to the
+  // same order); cluster c takes the jets at ranks c, 2 ncl - 1 - c,
+  // 2 ncl + c, ... (a snake over the clusters), so the clusters' tile sums
+  // come out close.
+  for (int t = threadIdx.x; t < kMaxJetTiles + 2; t += blockDim.x) H.bin[t] = 0;
+  jet_counts(J, H.cnt);
+  __syncthreads();
+  auto jet_tiles = [&H](int n) {
+    const int m = H.cnt[n + 1];
+    return min(kMaxJetTiles, (m * (m + 1) / 2 + kTileM - 1) / kTileM);
+  };
+  for (int n = threadIdx.x; n < J.N; n += blockDim.x) atomicAdd(&H.bin[jet_tiles(n)], 1);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    if (lane == 0) {  // first rank of each tile count, largest counts first
+      int run = 0;
+      for (int t = kMaxJetTiles; t >= 0; --t) {
+        const int b = H.bin[t];
+        H.bin[t] = run;
+        run += b;
+      }
+    }
+    __syncwarp();
+    // 32 jets at a time in jet order: equal counts within a chunk take
+    // consecutive ranks by lane, and the last of them advances the count's
+    // next free rank for the following chunks
+    for (int n0 = 0; n0 < J.N; n0 += 32) {
+      const int n = n0 + lane;
+      const int t = n < J.N ? jet_tiles(n) : kMaxJetTiles + 1;
+      const unsigned same = __match_any_sync(0xffffffffu, t);
+      const int before = __popc(same & ((1u << lane) - 1u));
+      const int pos = H.bin[t] + before;
+      __syncwarp();
+      if (n < J.N) {
+        H.order[pos] = n;
+        if ((same >> lane) == 1u) H.bin[t] = pos + 1;  // highest lane of the group
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  int K = 0;
+#pragma unroll
+  for (int r = 0; r < kCJ; ++r) {
+    const int p = r * ncl + ((r & 1) ? ncl - 1 - c : c);
+    if (p < J.N) {
+      if (threadIdx.x == 0) H.jets[K] = H.order[p];
+      ++K;
+    }
+  }
+  __syncthreads();
+  stage_jets<PM, true>(H.ring, J, K, [&H](int k) { return H.jets[k]; });
   mlp_setup<NG, SL>(H.mlp, wr);
   if (threadIdx.x == 0) {
     int pairs = 0, tiles = 0;
@@ -2419,7 +2477,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
       const int* kvoff = H.kvoff;
       const int* ib = H.ib;
       for (int k = 0; k < K; ++k)
-        if (H.ring[k].m > 0) stage_kv16<PM>(H.ring[k], J, X, n0 + k, 2 * q, 2, kv + kvoff[k]);
+        if (H.ring[k].m > 0) stage_kv16<PM>(H.ring[k], J, X, H.jets[k], 2 * q, 2, kv + kvoff[k]);
       const int items = ib[kCJ], warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
       auto locate = [&](int it, int& k, int& h, int& i0) {
         k = 0;
@@ -2433,7 +2491,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
         int k, h, i0;
         locate(it, k, h, i0);
         const Particles<PM>& P = H.ring[k];
-        q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, n0 + k, h, i); }, f);
+        q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, H.jets[k], h, i); }, f);
       };
       uint32_t a[4] = {0u, 0u, 0u, 0u};
       if (warp < items) qload(warp, a);
@@ -2450,11 +2508,11 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
         const ClusterUBias ub{reinterpret_cast<const __half*>(S.U + H.tri_off[k]), 2 * q};
         attend_tile16(
             kh, kh + round16(m) * 16, m, i0, min(16, m - i0), a,
-            [&](int i) { return X.out + qkv_off<PM>(P, J, n0 + k, h, i); }, ub.head(h));
+            [&](int i) { return X.out + qkv_off<PM>(P, J, H.jets[k], h, i); }, ub.head(h));
 #pragma unroll
         for (int e = 0; e < 4; ++e) a[e] = an[e];
       }
-      if (q < K) zero_masked_rows<PM>(H.ring[q], J, X.out, n0 + q);
+      if (q < K) zero_masked_rows<PM>(H.ring[q], J, X.out, H.jets[q]);
     }
   } else {
     // one jet per CTA on query blocks, 8-head records in the same space
@@ -2471,9 +2529,9 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
         aborted = __syncthreads_or(!ok) != 0;
         if (aborted) break;
         const RectUBias ub{reinterpret_cast<const __half*>(S.U), i0, m};
-        attention_block<PM>(P, J, X, n0 + q, i0, i1, stage, kStageFloats, ub);
+        attention_block<PM>(P, J, X, H.jets[q], i0, i1, stage, kStageFloats, ub);
       }
-      if (!aborted) zero_masked_rows<PM>(P, J, X.out, n0 + q);
+      if (!aborted) zero_masked_rows<PM>(P, J, X.out, H.jets[q]);
     }
   }
   mlp_teardown<NG, SL>(H.mlp, aborted, &phase);
