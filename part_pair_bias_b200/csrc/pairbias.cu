@@ -191,7 +191,10 @@ pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArg
 
 // The 4-CTA cluster kernel takes batches of at most this many jets per SM
 // (one jet per CTA); larger batches already balance over the persistent CTAs.
+// Below kClusterMinJets its fixed costs (counting, two cluster barriers)
+// outweigh the imbalance it removes.
 constexpr int kClusterJetsPerSm = 1;
+constexpr int kClusterMinJets = 16;
 
 template <int PM>
 pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s) {
@@ -221,7 +224,7 @@ pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb
 bool cluster_applies(const pb::JetArgs& J) {
   int dev = 0, sms = 0;
   if (device_sms(&dev, &sms) != PB_OK) return false;
-  return J.P <= 128 && J.N >= 1 && J.N <= kClusterJetsPerSm * sms && J.N <= pb::kClusterMaxJets;
+  return J.P <= 128 && J.N >= kClusterMinJets && J.N <= kClusterJetsPerSm * sms && J.N <= pb::kClusterMaxJets;
 }
 
 constexpr long long kGridMaxMaskBytes = 1ll << 21;  // padded N*P scanned by every CTA in phase 0

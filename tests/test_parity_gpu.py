@@ -157,6 +157,33 @@ def test_staging_path_boundaries(oracle_lib, P, mults):
     assert ops.get_device_status() == 0
 
 
+CLUSTER_MULTS = [120, 89, 88, 86, 85, 65, 64, 63, 40, 33, 17, 7, 3, 2, 1, 0, 0]  # 17 jets: 5 clusters
+
+
+@pytest.mark.parametrize("layout", ["padded", "packed"])
+def test_cluster_kernel_mixed_jets(oracle_lib, layout):
+    """Batches of 16 to one-per-SM jets take the 4-CTA cluster kernel: jets
+    dealt to clusters by size (empty, one-particle and 120-particle jets, a
+    last cluster with fewer than 4 jets), biases exchanged between the CTAs."""
+    kw = dict(mask_mode="scrambled") if layout == "padded" else {}
+    b = synth.make_jets(N=len(CLUSTER_MULTS), P=128, layout=layout, mults=CLUSTER_MULTS, seed=33, **kw)
+    d = pt.Device(b)
+    ref = oracle_lib.forward(b)
+    got = pt.to_np(d.fused())
+    pt.check_attention(got, ref, b)
+    assert ops.get_device_status() == 0
+    assert torch.equal(d.fused(), d.fused())
+
+
+def test_cluster_kernel_query_block_fallback(oracle_lib):
+    """16 jets of 90 particles: no cluster's four bias triangles fit, so
+    every CTA runs one jet on query blocks."""
+    b = synth.make_jets(N=16, P=128, mults=[90] * 16, mask_mode="scrambled", seed=34)
+    d = pt.Device(b)
+    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    assert ops.get_device_status() == 0
+
+
 def test_packed_wide_jets(oracle_lib):
     """Packed jets of up to 200 particles (the P = 256 kernels): triangle,
     query-block and balanced paths against the oracle."""
