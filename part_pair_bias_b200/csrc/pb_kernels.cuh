@@ -2275,10 +2275,11 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
 //     pair, written through distributed shared memory (st.shared::cluster);
 //   - a cluster barrier publishes them; CTA q then attends heads 2q, 2q + 1
 //     of each jet from its own shared memory.
-// When the 4 jets' pairs do not fit (kClusterUCap pairs), each CTA runs one
-// of the jets alone on query blocks (8-head records in the same space).
-// Cluster barriers are hardware barriers that every CTA reaches on every
-// path; the first one makes sure all 4 CTAs run before any remote store.
+// When the 4 jets' pairs do not fit the triangles together, consecutive
+// groups of them that fit run one after another (one P <= 128 jet always
+// fits). Cluster barriers are hardware barriers that every CTA reaches the
+// same number of times on every path (a CTA whose wait ran out still takes
+// them); the first one makes sure all 4 CTAs run before any remote store.
 
 constexpr int kCJ = 4;                // jets and CTAs per cluster
 constexpr int kClusterMaxJets = 256;  // batch size the jet table holds
@@ -2310,10 +2311,10 @@ struct ClusterHead {
   Particles<PM> ring[kCJ];
   int tbeg[kCJ + 1];     // prefix of the jets' MLP tiles
   int tri_off[kCJ + 1];  // prefix of the jets' pairs
-  int lo, hi;            // this CTA's tiles of the cluster's list
-  int fits;
-  int kvoff[kCJ + 1];    // staged K/V of each jet (halves) in the attention
-  int ib[kCJ + 1];       // prefix of each jet's (head, query tile) items
+  int lo, hi;            // this CTA's tiles of the current group's list
+  int G;                 // jets in the current group
+  int kvoff[kCJ + 1];    // staged K/V of each jet of the group (halves) in the attention
+  int ib[kCJ + 1];       // prefix of each group jet's (head, query tile) items
   int jets[kCJ];         // this cluster's jets
   int cnt[kClusterMaxJets + 1];  // multiplicity of every jet of the batch (cnt[n + 1])
   int order[kClusterMaxJets];    // jets by decreasing MLP tiles
@@ -2333,6 +2334,7 @@ struct ClusterSmem {
 template <int PM>
 struct ClusterTiles {
   const ClusterHead<PM>* H;
+  int g0;  // the group's first jet
   __device__ __forceinline__ int ntiles() const { return H->hi - H->lo; }
   __device__ __forceinline__ bool row(int t, int r, int& p, int& a, int& b, float f[4]) const {
     const int gt = H->lo + t;
@@ -2340,11 +2342,12 @@ struct ClusterTiles {
 #pragma unroll
     for (int q = 1; q < kCJ; ++q) k += H->tbeg[q] <= gt ? 1 : 0;
     const int pl = (gt - H->tbeg[k]) * kTileM + r;
-    const int m = H->ring[k].m;
+    const Particles<PM>& P = H->ring[g0 + k];
+    const int m = P.m;
     if (pl >= m * (m + 1) / 2) return false;
     TriPairs{}.map(pl, a, b);
     if (!in_bounds(a >= 0 && a <= b && b < m)) return false;
-    pair_feat<PM, true>(H->ring[k], a, b, f);
+    pair_feat<PM, true>(P, a, b, f);
     p = H->tri_off[k] + pl;
     return true;
   }
@@ -2432,66 +2435,82 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   __syncthreads();
   stage_jets<PM, true>(H.ring, J, K, [&H](int k) { return H.jets[k]; });
   mlp_setup<NG, SL>(H.mlp, wr);
-  if (threadIdx.x == 0) {
-    int pairs = 0, tiles = 0;
-    for (int k = 0; k < kCJ; ++k) {
-      const int m = k < K ? H.ring[k].m : 0;
-      H.tri_off[k] = pairs;
-      H.tbeg[k] = tiles;
-      pairs += m * (m + 1) / 2;
-      tiles += (m * (m + 1) / 2 + kTileM - 1) / kTileM;
+  // groups of consecutive jets whose triangles fit together (identical in
+  // every CTA of the cluster: the same jets, the same order); thread 0 lays
+  // out the group starting at jet g0
+  auto plan = [&](int g0) {
+    if (threadIdx.x == 0) {
+      int G = 0, pairs = 0, tiles = 0;
+      while (g0 + G < K) {
+        const int m = H.ring[g0 + G].m, np = m * (m + 1) / 2;
+        if (G > 0 && pairs + np > kUCap) break;
+        H.tri_off[G] = pairs;
+        H.tbeg[G] = tiles;
+        pairs += np;
+        tiles += (np + kTileM - 1) / kTileM;
+        ++G;
+      }
+      for (int k = G; k <= kCJ; ++k) {
+        H.tri_off[k] = pairs;
+        H.tbeg[k] = tiles;
+      }
+      H.kvoff[0] = 0;
+      H.ib[0] = 0;
+      for (int k = 0; k < kCJ; ++k) {
+        const int m = k < G ? H.ring[g0 + k].m : 0;
+        H.kvoff[k + 1] = H.kvoff[k] + (m > 0 ? kv16_bytes(m) : 0);  // two heads of kv16_bytes / 2 halves
+        H.ib[k + 1] = H.ib[k] + (m > 0 ? 2 * ((m + 15) >> 4) : 0);
+      }
+      H.lo = tiles * q / kCJ;
+      H.hi = tiles * (q + 1) / kCJ;
+      H.G = G;
     }
-    H.tri_off[kCJ] = pairs;
-    H.tbeg[kCJ] = tiles;
-    H.kvoff[0] = 0;
-    H.ib[0] = 0;
-    for (int k = 0; k < kCJ; ++k) {
-      const int m = k < K ? H.ring[k].m : 0;
-      H.kvoff[k + 1] = H.kvoff[k] + (m > 0 ? kv16_bytes(m) : 0);  // two heads of kv16_bytes / 2 halves
-      H.ib[k + 1] = H.ib[k] + (m > 0 ? 2 * ((m + 15) >> 4) : 0);
-    }
-    H.lo = tiles * q / kCJ;
-    H.hi = tiles * (q + 1) / kCJ;
-    H.fits = pairs <= kUCap ? 1 : 0;
-  }
+  };
+  plan(0);
   __syncthreads();
   cluster_sync_all();  // all 4 CTAs run: their shared memory may be written
   float* stage = reinterpret_cast<float*>(&H.mlp.A[0][0]);
-  constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
   uint32_t phase = 0u;
   bool aborted = false;
-  if (H.fits) {
-    ClusterUSink sink;
+  ClusterUSink sink;
+  {
     const uint32_t local = smem_u32(S.U);
 #pragma unroll
-    for (int c = 0; c < kCJ; ++c) sink.base[c] = map_shared_rank(local, (uint32_t)c);
+    for (int cc = 0; cc < kCJ; ++cc) sink.base[cc] = map_shared_rank(local, (uint32_t)cc);
     sink.cap = kUCap;
-    const bool ok = mlp_pass<NG, SL>(H.mlp, ClusterTiles<PM>{&H}, sink, &phase);
-    aborted = __syncthreads_or(!ok) != 0;
+  }
+  for (int g0 = 0; g0 < K;) {
+    __syncthreads();
+    const int G = H.G;
+    if (!aborted) {
+      const bool ok = mlp_pass<NG, SL>(H.mlp, ClusterTiles<PM>{&H, g0}, sink, &phase);
+      aborted = !ok;
+    }
+    aborted = __syncthreads_or(aborted) != 0;
     cluster_sync_all();  // every CTA's stores into this one are visible
     if (!aborted) {
-      // heads 2q, 2q + 1 of all the cluster's jets at once: K and V of every
-      // (jet, head) staged together, then the warps take (jet, head, 16-query
-      // tile) items, the next item's Q fragment loaded ahead
+      // heads 2q, 2q + 1 of the group's jets at once: K and V of every (jet,
+      // head) staged together, then the warps take (jet, head, 16-query tile)
+      // items, the next item's Q fragment loaded ahead
       uint16_t* kv = reinterpret_cast<uint16_t*>(stage);
       const int* kvoff = H.kvoff;
       const int* ib = H.ib;
-      for (int k = 0; k < K; ++k)
-        if (H.ring[k].m > 0) stage_kv16<PM>(H.ring[k], J, X, H.jets[k], 2 * q, 2, kv + kvoff[k]);
+      for (int k = 0; k < G; ++k)
+        if (H.ring[g0 + k].m > 0) stage_kv16<PM>(H.ring[g0 + k], J, X, H.jets[g0 + k], 2 * q, 2, kv + kvoff[k]);
       const int items = ib[kCJ], warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
       auto locate = [&](int it, int& k, int& h, int& i0) {
         k = 0;
 #pragma unroll
-        for (int c = 1; c < kCJ; ++c) k += ib[c] <= it ? 1 : 0;
-        const int tiles = (H.ring[k].m + 15) >> 4, loc = it - ib[k];
+        for (int cc = 1; cc < kCJ; ++cc) k += ib[cc] <= it ? 1 : 0;
+        const int tiles = (H.ring[g0 + k].m + 15) >> 4, loc = it - ib[k];
         h = 2 * q + loc / tiles;
         i0 = (loc % tiles) * 16;
       };
       auto qload = [&](int it, uint32_t* f) {
         int k, h, i0;
         locate(it, k, h, i0);
-        const Particles<PM>& P = H.ring[k];
-        q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, H.jets[k], h, i); }, f);
+        const Particles<PM>& P = H.ring[g0 + k];
+        q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, H.jets[g0 + k], h, i); }, f);
       };
       uint32_t a[4] = {0u, 0u, 0u, 0u};
       if (warp < items) qload(warp, a);
@@ -2502,38 +2521,26 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
         if (it + nwarp < items) qload(it + nwarp, an);
         int k, h, i0;
         locate(it, k, h, i0);
-        const Particles<PM>& P = H.ring[k];
+        const Particles<PM>& P = H.ring[g0 + k];
         const int m = P.m;
         const uint16_t* kh = kv + kvoff[k] + (h - 2 * q) * (kv16_bytes(m) / 2);
         const ClusterUBias ub{reinterpret_cast<const __half*>(S.U + H.tri_off[k]), 2 * q};
         attend_tile16(
             kh, kh + round16(m) * 16, m, i0, min(16, m - i0), a,
-            [&](int i) { return X.out + qkv_off<PM>(P, J, H.jets[k], h, i); }, ub.head(h));
+            [&](int i) { return X.out + qkv_off<PM>(P, J, H.jets[g0 + k], h, i); }, ub.head(h));
 #pragma unroll
         for (int e = 0; e < 4; ++e) a[e] = an[e];
       }
-      if (q < K) zero_masked_rows<PM>(H.ring[q], J, X.out, H.jets[q]);
     }
-  } else {
-    // one jet per CTA on query blocks, 8-head records in the same space
-    cluster_sync_all();  // the same barriers on both paths
-    if (q < K) {
-      const Particles<PM>& P = H.ring[q];
-      const int m = P.m, cap = kUCap / 4;
-      SmemUSink sink{reinterpret_cast<uint4*>(S.U), cap};
-      const int qb = max(1, cap / max(1, m));
-      for (int i0 = 0; i0 < m && !aborted; i0 += qb) {
-        const int i1 = min(m, i0 + qb);
-        const bool ok = mlp_pass<NG, SL>(H.mlp, JetTiles<PM, RectPairs, true>{&P, (i1 - i0) * m, RectPairs{i0, m}}, sink,
-                                         &phase);
-        aborted = __syncthreads_or(!ok) != 0;
-        if (aborted) break;
-        const RectUBias ub{reinterpret_cast<const __half*>(S.U), i0, m};
-        attention_block<PM>(P, J, X, H.jets[q], i0, i1, stage, kStageFloats, ub);
-      }
-      if (!aborted) zero_masked_rows<PM>(P, J, X.out, H.jets[q]);
+    g0 += G;
+    if (g0 < K) {
+      __syncthreads();  // the stage and this group's tables are free again
+      plan(g0);
+      __syncthreads();
+      cluster_sync_all();  // no CTA still reads the triangles the next group overwrites
     }
   }
+  if (!aborted && q < K) zero_masked_rows<PM>(H.ring[q], J, X.out, H.jets[q]);
   mlp_teardown<NG, SL>(H.mlp, aborted, &phase);
 }
 

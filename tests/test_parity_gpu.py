@@ -175,13 +175,25 @@ def test_cluster_kernel_mixed_jets(oracle_lib, layout):
     assert torch.equal(d.fused(), d.fused())
 
 
-def test_cluster_kernel_query_block_fallback(oracle_lib):
-    """16 jets of 90 particles: no cluster's four bias triangles fit, so
-    every CTA runs one jet on query blocks."""
-    b = synth.make_jets(N=16, P=128, mults=[90] * 16, mask_mode="scrambled", seed=34)
+GROUP_MULTS = {
+    "groups_of_1": [128] * 16,                 # one triangle at a time, 4 groups per cluster
+    "groups_of_2": [90] * 16,                  # 2 + 2
+    "groups_of_3_1": [75] * 16,                # 3 + 1
+    "mixed": [128, 127, 100, 99, 90, 80, 75, 70, 68, 50, 40, 30, 20, 10, 5, 1],
+}
+
+
+@pytest.mark.parametrize("name", list(GROUP_MULTS))
+def test_cluster_kernel_jet_groups(oracle_lib, name):
+    """Clusters whose four bias triangles do not fit together run their jets
+    in consecutive groups that do (all four CTAs on each group, the same
+    cluster barriers in every CTA)."""
+    b = synth.make_jets(N=16, P=128, mults=GROUP_MULTS[name], mask_mode="scrambled", seed=34)
     d = pt.Device(b)
-    pt.check_attention(pt.to_np(d.fused()), oracle_lib.forward(b), b)
+    got = d.fused()
+    pt.check_attention(pt.to_np(got), oracle_lib.forward(b), b)
     assert ops.get_device_status() == 0
+    assert torch.equal(got, d.fused())
 
 
 def test_packed_wide_jets(oracle_lib):
