@@ -2396,12 +2396,28 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    if (lane == 0) {  // first rank of each tile count, largest counts first
-      int run = 0;
-      for (int t = kMaxJetTiles; t >= 0; --t) {
-        const int b = H.bin[t];
-        H.bin[t] = run;
-        run += b;
+    {  // first rank of each tile count, largest counts first: an exclusive
+       // scan over the bins from kMaxJetTiles down, kPer bins per lane
+      constexpr int kPer = (kMaxJetTiles + 1 + 31) / 32;
+      int v[kPer], sum = 0;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const int t = kMaxJetTiles - (lane * kPer + e);
+        v[e] = t >= 0 ? H.bin[t] : 0;
+        sum += v[e];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      int run = incl - sum;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const int t = kMaxJetTiles - (lane * kPer + e);
+        if (t >= 0) H.bin[t] = run;
+        run += v[e];
       }
     }
     __syncwarp();
@@ -2487,33 +2503,37 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
       aborted = !ok;
     }
     aborted = __syncthreads_or(aborted) != 0;
-    cluster_sync_all();  // every CTA's stores into this one are visible
+    // heads 2q, 2q + 1 of the group's jets at once: K and V of every (jet,
+    // head) staged together, then the warps take (jet, head, 16-query tile)
+    // items, the next item's Q fragment loaded ahead. This CTA's MLP is done,
+    // so the staging (into the MLP's operand buffers) and the first Q
+    // fragment are issued before the barrier that waits for the others.
+    uint16_t* kv = reinterpret_cast<uint16_t*>(stage);
+    const int* kvoff = H.kvoff;
+    const int* ib = H.ib;
+    const int items = ib[kCJ], warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    auto locate = [&](int it, int& k, int& h, int& i0) {
+      k = 0;
+#pragma unroll
+      for (int cc = 1; cc < kCJ; ++cc) k += ib[cc] <= it ? 1 : 0;
+      const int tiles = (H.ring[g0 + k].m + 15) >> 4, loc = it - ib[k];
+      h = 2 * q + loc / tiles;
+      i0 = (loc % tiles) * 16;
+    };
+    auto qload = [&](int it, uint32_t* f) {
+      int k, h, i0;
+      locate(it, k, h, i0);
+      const Particles<PM>& P = H.ring[g0 + k];
+      q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, H.jets[g0 + k], h, i); }, f);
+    };
+    uint32_t a[4] = {0u, 0u, 0u, 0u};
     if (!aborted) {
-      // heads 2q, 2q + 1 of the group's jets at once: K and V of every (jet,
-      // head) staged together, then the warps take (jet, head, 16-query tile)
-      // items, the next item's Q fragment loaded ahead
-      uint16_t* kv = reinterpret_cast<uint16_t*>(stage);
-      const int* kvoff = H.kvoff;
-      const int* ib = H.ib;
       for (int k = 0; k < G; ++k)
         if (H.ring[g0 + k].m > 0) stage_kv16<PM>(H.ring[g0 + k], J, X, H.jets[g0 + k], 2 * q, 2, kv + kvoff[k]);
-      const int items = ib[kCJ], warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-      auto locate = [&](int it, int& k, int& h, int& i0) {
-        k = 0;
-#pragma unroll
-        for (int cc = 1; cc < kCJ; ++cc) k += ib[cc] <= it ? 1 : 0;
-        const int tiles = (H.ring[g0 + k].m + 15) >> 4, loc = it - ib[k];
-        h = 2 * q + loc / tiles;
-        i0 = (loc % tiles) * 16;
-      };
-      auto qload = [&](int it, uint32_t* f) {
-        int k, h, i0;
-        locate(it, k, h, i0);
-        const Particles<PM>& P = H.ring[g0 + k];
-        q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, H.jets[g0 + k], h, i); }, f);
-      };
-      uint32_t a[4] = {0u, 0u, 0u, 0u};
       if (warp < items) qload(warp, a);
+    }
+    cluster_sync_all();  // every CTA's stores into this one are visible
+    if (!aborted) {
       cp_async_wait_all();
       __syncthreads();
       for (int it = warp; it < items; it += nwarp) {
