@@ -11,6 +11,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "pairbias.h"
@@ -35,6 +36,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 constexpr int kMaxDev = 64;
 struct DevInfo {
   int sms = 0;
+  int clusters = -1;  // co-resident 4-CTA clusters of the cluster kernel (-1: not asked yet)
 };
 DevInfo g_dev[kMaxDev];
 std::mutex g_mu;
@@ -196,6 +198,10 @@ pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArg
 constexpr int kClusterJetsPerSm = 1;
 constexpr int kClusterMinJets = 16;
 
+// The jets are dealt over as many clusters as run at once (cluster sizes
+// need not divide a GPC's SMs, so that number comes from the occupancy query,
+// once per device), at most one cluster per jet and never fewer than
+// ceil(N / 4): N = 128 runs on 37 clusters of 3 or 4 jets rather than 32 of 4.
 template <int PM>
 pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s) {
   auto k = pb::k_fused_cluster<PM>;
@@ -205,7 +211,6 @@ pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb
   if (st != PB_OK) return st;
   if ((st = resident_per_sm((const void*)k, dev, smem, 512, &per_sm)) != PB_OK) return st;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((J.N + pb::kCJ - 1) / pb::kCJ * pb::kCJ));
   cfg.blockDim = dim3(512);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -216,6 +221,21 @@ pb_status run_fused_cluster(const pb::JetArgs& J, const pb::MlpArgs& W, const pb
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  int cap = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_dev[dev].clusters < 0) {
+      cfg.gridDim = dim3((unsigned)(sms / pb::kCJ * pb::kCJ));
+      int n = 0;
+      const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      if (e != cudaSuccess) return fail(PB_ECUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
+      g_dev[dev].clusters = n;
+    }
+    cap = g_dev[dev].clusters;
+  }
+  const int need = (J.N + pb::kCJ - 1) / pb::kCJ;
+  const int ncl = std::max(need, std::min(J.N, cap));
+  cfg.gridDim = dim3((unsigned)(ncl * pb::kCJ));
   cudaError_t e = cudaLaunchKernelEx(&cfg, k, J, W, X);
   if (e != cudaSuccess) return fail(PB_ECUDA, "k_fused_cluster launch: %s", cudaGetErrorString(e));
   return PB_OK;

@@ -32,11 +32,12 @@ CASES = {
     "packed_empty": dict(N=6, P=64, layout="packed", mults=[3, 0, 64, 1, 0, 20], seed=6),
     "many_jets": dict(N=700, P=24, dist="uniform", mult_lo=1, mult_hi=24, mask_mode="scrambled", seed=8),
     "tiny_p3": dict(N=8, P=3, mults=[0, 1, 3, 2, 2, 3, 0, 1], mask_mode="scrambled", seed=9),
-    # 16 to one-per-SM jets take the 4-CTA cluster kernel: mixed sizes dealt to
-    # 5 clusters, and clusters whose jets run in groups of 1 to 4
-    "cluster_mixed": dict(N=17, P=128, mults=[120, 89, 88, 86, 85, 65, 64, 63, 40, 33, 17, 7, 3, 2, 1, 0, 0],
+    # 16 to one-per-SM jets take the 4-CTA cluster kernel: mixed sizes dealt
+    # two or three to a cluster, and 37 clusters of 4 jets run in groups of 1 to 4
+    "cluster_mixed": dict(N=85, P=128, mults=[120, 89, 88, 86, 85, 65, 64, 63, 40, 33, 17, 7, 3, 2, 1, 0, 0] * 5,
                           mask_mode="scrambled", seed=33),
-    "cluster_groups": dict(N=16, P=128, mults=[128, 127, 100, 99, 90, 80, 75, 70, 68, 50, 40, 30, 20, 10, 5, 1],
+    "cluster_groups": dict(N=148, P=128,
+                           mults=([128, 127, 100, 99, 90, 80, 75, 70, 68, 50, 40, 30, 20, 10, 5, 1] * 10)[:148],
                            mask_mode="scrambled", seed=34),
 }
 

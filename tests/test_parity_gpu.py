@@ -157,16 +157,19 @@ def test_staging_path_boundaries(oracle_lib, P, mults):
     assert ops.get_device_status() == 0
 
 
-CLUSTER_MULTS = [120, 89, 88, 86, 85, 65, 64, 63, 40, 33, 17, 7, 3, 2, 1, 0, 0]  # 17 jets: 5 clusters
+CLUSTER_MULTS = [120, 89, 88, 86, 85, 65, 64, 63, 40, 33, 17, 7, 3, 2, 1, 0, 0]
 
 
 @pytest.mark.parametrize("layout", ["padded", "packed"])
-def test_cluster_kernel_mixed_jets(oracle_lib, layout):
-    """Batches of 16 to one-per-SM jets take the 4-CTA cluster kernel: jets
-    dealt to clusters by size (empty, one-particle and 120-particle jets, a
-    last cluster with fewer than 4 jets), biases exchanged between the CTAs."""
+@pytest.mark.parametrize("reps", [1, 5])
+def test_cluster_kernel_mixed_jets(oracle_lib, layout, reps):
+    """Batches of 16 to one-per-SM jets take the 4-CTA cluster kernel, the
+    jets dealt over the clusters that run at once by size: 17 jets (one per
+    cluster) and 85 (two or three per cluster), with empty, one-particle and
+    120-particle jets, biases exchanged between the CTAs."""
     kw = dict(mask_mode="scrambled") if layout == "padded" else {}
-    b = synth.make_jets(N=len(CLUSTER_MULTS), P=128, layout=layout, mults=CLUSTER_MULTS, seed=33, **kw)
+    mults = CLUSTER_MULTS * reps
+    b = synth.make_jets(N=len(mults), P=128, layout=layout, mults=mults, seed=33, **kw)
     d = pt.Device(b)
     ref = oracle_lib.forward(b)
     got = pt.to_np(d.fused())
@@ -175,11 +178,12 @@ def test_cluster_kernel_mixed_jets(oracle_lib, layout):
     assert torch.equal(d.fused(), d.fused())
 
 
-GROUP_MULTS = {
-    "groups_of_1": [128] * 16,                 # one triangle at a time, 4 groups per cluster
-    "groups_of_2": [90] * 16,                  # 2 + 2
-    "groups_of_3_1": [75] * 16,                # 3 + 1
-    "mixed": [128, 127, 100, 99, 90, 80, 75, 70, 68, 50, 40, 30, 20, 10, 5, 1],
+_GROUP_MIX = [128, 127, 100, 99, 90, 80, 75, 70, 68, 50, 40, 30, 20, 10, 5, 1]
+GROUP_MULTS = {  # 148 jets: 37 clusters of 4 (one per SM) whatever the device's cluster capacity
+    "groups_of_1": [128] * 148,                  # one triangle at a time, 4 groups per cluster
+    "groups_of_2": [90] * 148,                   # 2 + 2
+    "groups_of_3_1": [75] * 148,                 # 3 + 1
+    "mixed": (_GROUP_MIX * 10)[:148],
 }
 
 
@@ -188,7 +192,7 @@ def test_cluster_kernel_jet_groups(oracle_lib, name):
     """Clusters whose four bias triangles do not fit together run their jets
     in consecutive groups that do (all four CTAs on each group, the same
     cluster barriers in every CTA)."""
-    b = synth.make_jets(N=16, P=128, mults=GROUP_MULTS[name], mask_mode="scrambled", seed=34)
+    b = synth.make_jets(N=148, P=128, mults=GROUP_MULTS[name], mask_mode="scrambled", seed=34)
     d = pt.Device(b)
     got = d.fused()
     pt.check_attention(pt.to_np(got), oracle_lib.forward(b), b)
