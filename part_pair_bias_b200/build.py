@@ -7,7 +7,9 @@ import subprocess
 _HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(_HERE)
 SRC = os.path.join(_HERE, "csrc", "pairbias.cu")
-DEPS = [os.path.join(_HERE, "csrc", f) for f in ("pairbias.cu", "pb_device.cuh", "pb_kernels.cuh")] + [
+CSRC = os.path.join(_HERE, "csrc")
+# every source the library is compiled from (pairbias.cu includes the rest)
+DEPS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))) + [
     os.path.join(ROOT, "include", "pairbias.h")]
 OUT = os.path.join(_HERE, "libpairbias.so")
 # the same library with every computed-index check of PB_DEBUG_BOUNDS compiled in

@@ -39,6 +39,14 @@ def test_every_declared_symbol_is_exported(L):
     assert ops.version().startswith("pairbias-b200")
 
 
+def test_build_watches_every_source():
+    """A change to any file under csrc/ (or the header) makes the library stale."""
+    from part_pair_bias_b200 import build
+    csrc = os.path.join(ROOT, "part_pair_bias_b200", "csrc")
+    sources = {os.path.join(csrc, f) for f in os.listdir(csrc)} | {HEADER}
+    assert sources <= set(build.DEPS)
+
+
 def _jets(N=2, P=8, ptr=False, aligned=True):
     buf = np.zeros(64, np.float32)
     base = buf.ctypes.data + (0 if aligned else 1)
