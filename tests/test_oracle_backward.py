@@ -1,8 +1,8 @@
 """Pins of the fp64 backward oracle (oracle/backward.py), checked against
 things other than itself: central finite differences of the scalar
 sum(O * dO), the C oracle's forward, closed forms of the softmax gradient,
-the U = 0 special case against torch's own attention backward in fp64, and
-the m = 1 jet. A dropped term, a wrong sign or a transposed operand in any of
+the U = 0 special case against torch's own attention backward in fp64, the
+m = 1 jet, and permutation equivariance. A dropped term, a wrong sign or a transposed operand in any of
 the gradient formulas fails at least one of these."""
 import numpy as np
 import pytest
@@ -164,3 +164,25 @@ def test_single_particle_jet(bw):
     assert np.all(r["dq"] == 0) and np.all(r["dk"] == 0)
     for name in bw.FOLDED_NAMES:
         assert np.all(r["folded"][name] == 0.0)
+
+
+def test_permutation_equivariance(bw):
+    """Reordering a jet's slots (momenta, mask, q, k, v and the upstream
+    gradient alike) moves dq, dk, dv with them and leaves the parameter
+    gradients, sums over all pairs, unchanged up to fp64 rounding."""
+    b = tiny(9, mults=(5, 7, 3), P=8)
+    dO = upstream(b, 9)
+    rng = np.random.default_rng(9)
+    perms = np.stack([rng.permutation(b.P) for _ in range(b.N)])
+    c = lambda a: a.reshape(b.N, b.P)[np.arange(b.N)[:, None], perms].reshape(-1).copy()
+    h = lambda a: a.reshape(b.N, 8, b.P, 16)[np.arange(b.N)[:, None, None], np.arange(8)[None, :, None],
+                                             perms[:, None, :]].copy()
+    bp = synth.JetBatch("padded", b.N, b.P, b.mult.copy(), c(b.E), c(b.px), c(b.py), c(b.pz), c(b.mask), None,
+                        h(b.q), h(b.k), h(b.v), b.params)
+    r0, r1 = bw.backward(b, dO), bw.backward(bp, h(dO))
+    for name in ("out", "dq", "dk", "dv"):
+        np.testing.assert_allclose(r1[name].reshape(b.N, 8, b.P, 16), h(r0[name]), rtol=0,
+                                   atol=1e-12 * max(1.0, np.abs(r0[name]).max()))
+    for name in bw.FOLDED_NAMES:
+        np.testing.assert_allclose(r1["folded"][name], r0["folded"][name], rtol=1e-10,
+                                   atol=1e-12 * max(1.0, np.abs(r0["folded"][name]).max()))

@@ -11,7 +11,7 @@ to the composed affine maps (this catches a transposed weight, a misplaced
 affine or a dropped bias).
 Attention: the bias-free and the biased cases against torch's
 scaled_dot_product_attention in fp64, one-particle jets, constant keys, mask
-exclusion, and padded == packed.
+exclusion, padded == packed, and permutation equivariance.
 Block (attention with its in and out projections): against torch's
 multi_head_attention_forward in fp64 jet by jet, reduction to the pinned
 attention under identity projections, masked rows 0, and the output-bias
@@ -247,6 +247,37 @@ def test_mask_exclusion_bitwise(oracle_lib):
         setattr(b, name, np.where(hole4, noise, arr))
     out1 = oracle_lib.forward(b)
     assert np.array_equal(out0, out1)
+
+
+def _permute_slots(b, perms):
+    """The same jets with jet n's slots reordered: new slot s holds old slot perms[n][s]."""
+    c = lambda a: a.reshape(b.N, b.P)[np.arange(b.N)[:, None], perms].reshape(-1).copy()
+    h = lambda a: a[np.arange(b.N)[:, None, None], np.arange(a.shape[1])[None, :, None], perms[:, None, :]].copy()
+    return synth.JetBatch("padded", b.N, b.P, b.mult.copy(), c(b.E), c(b.px), c(b.py), c(b.pz), c(b.mask),
+                          None, h(b.q), h(b.k), h(b.v), b.params)
+
+
+def test_permutation_equivariance(oracle_lib):
+    """Reordering a jet's slots reorders its features, bias and output rows
+    the same way and changes nothing else (the block acts on a set of
+    particles). Features and bias are per-pair values, so they move bit for
+    bit; the output's sums run in another order, so it moves to within fp64
+    rounding. A slot used where a compact index belongs, or the reverse,
+    breaks this."""
+    b = synth.make_jets(N=3, P=24, dist="uniform", mult_lo=3, mult_hi=24, seed=21, mask_mode="scrambled")
+    rng = np.random.default_rng(21)
+    perms = np.stack([rng.permutation(b.P) for _ in range(b.N)])
+    bp = _permute_slots(b, perms)
+    n3 = np.arange(b.N)[:, None, None]
+    f0, f1 = oracle_lib.features(b), oracle_lib.features(bp)
+    assert np.array_equal(f1, f0[n3, perms[:, :, None], perms[:, None, :]])
+    u0, u1 = oracle_lib.pair_bias(b), oracle_lib.pair_bias(bp)
+    assert np.array_equal(u1, u0[n3[..., None], np.arange(8)[None, :, None, None], perms[:, None, :, None],
+                                 perms[:, None, None, :]])
+    o0, o1 = oracle_lib.forward(b), oracle_lib.forward(bp)
+    moved = o0[np.arange(b.N)[:, None, None], np.arange(8)[None, :, None], perms[:, None, :]]
+    np.testing.assert_allclose(o1, moved, rtol=0, atol=1e-12 * max(1.0, np.abs(o0).max()))
+    assert not np.allclose(o1, o0)  # the permutation did move rows
 
 
 def _to_packed(b):
