@@ -21,12 +21,16 @@
  *     pb_fold_affine and pb_unfold_grad (host). Nothing is allocated inside
  *     the library.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
- *     NULL = the legacy default stream), launches exactly one kernel (the
- *     balanced fused path as a cooperative launch; pair_block_forward three
- *     and pair_attention_backward four, in order) and does not synchronise.
- *     Host-side argument errors return before any launch; device-side problems (an invalid ptr array, a bounded wait that
- *     ran out) set bits of a per-device status word, read with
- *     pb_get_device_status.
+ *     NULL = the legacy default stream) and does not synchronise. It launches
+ *     exactly one kernel (the balanced fused path as a cooperative launch),
+ *     except: pair_block_forward launches one (projections fused in) for at
+ *     most one jet per SM and three otherwise; pair_attention_forward_noalloc
+ *     clears its scratch header with one cudaMemsetAsync first;
+ *     pair_attention_backward launches three per chunk of up to 8192 jets
+ *     and one more, in order.
+ *     Host-side argument errors return before any launch; device-side
+ *     problems (an invalid ptr array, a bounded wait that ran out) set bits
+ *     of a per-device status word, read with pb_get_device_status.
  *   - H must be 8 and D must be 16 (the MLP output width fixes H);
  *     1 <= P <= 256. Other values return PB_EUNSUPPORTED.
  *   - Q, K, V, out and U pointers must be 16-byte aligned; momentum, mask and
@@ -200,10 +204,12 @@ size_t pb_workspace_bytes(const pb_jets *jets);
  *   workspace: device memory of at least pb_block_workspace_bytes(jets)
  *         bytes, 256-byte aligned, for Q, K, V and O (bf16, the layout of
  *         pair_attention_forward's q); its contents need no initialisation.
- * Launches, in order on `stream`: the in-projection GEMM (tensor cores),
- * the fused pair-bias attention (pair_attention_forward with mlp), and the
- * output-projection GEMM. Calls that share a workspace must not overlap on
- * the device. Errors as for pair_attention_forward. */
+ * Launches on `stream`: for at most one jet per SM, one kernel that runs
+ * both projections inside the fused pair-bias attention, jet by jet (Q, K,
+ * V and O go through the workspace); otherwise, in order, the in-projection
+ * GEMM (tensor cores), the fused pair-bias attention (pair_attention_forward
+ * with mlp) and the output-projection GEMM. Calls that share a workspace
+ * must not overlap on the device. Errors as for pair_attention_forward. */
 pb_status pair_block_forward(const pb_jets *jets, const pb_mlp *mlp, const pb_proj *proj, int H, int D, int E,
                              const uint16_t *x, uint16_t *y, void *workspace, size_t workspace_bytes,
                              void *stream);
