@@ -27,3 +27,17 @@ def test_reference_arm_json_line(oracle_lib):
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_under_two_ranks(oracle_lib):
+    """Launched as two ranks, only rank 0 runs the oracle and prints its line
+    (n_gpus = 2); rank 1 exits 0 without output."""
+    base = dict(os.environ, WORLD_SIZE="2", LOCAL_RANK="0", MASTER_ADDR="127.0.0.1", MASTER_PORT="29531")
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"]
+    r1 = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=dict(base, RANK="1"))
+    assert r1.returncode == 0, r1.stderr[-2000:]
+    assert not [ln for ln in r1.stdout.splitlines() if ln.startswith("{")]
+    r0 = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=dict(base, RANK="0"))
+    assert r0.returncode == 0, r0.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r0.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
