@@ -220,7 +220,10 @@ pb_status pair_block_forward(const pb_jets *jets, const pb_mlp *mlp, const pb_pr
 size_t pb_block_workspace_bytes(const pb_jets *jets);
 
 /* PB_STATIC_SCRATCH_BYTES -- size of the library's static per-device scratch
- * array used by pair_attention_forward_noalloc (32 MiB). */
+ * array used by pair_attention_forward_noalloc (32 MiB). The array belongs
+ * to the library's one device module, so every process that loads the
+ * library onto a device holds these 32 MiB there until it exits, whichever
+ * entry points it calls. */
 #define PB_STATIC_SCRATCH_BYTES (32u << 20)
 
 /* pair_attention_forward_noalloc -- the fused path of pair_attention_forward
@@ -235,7 +238,9 @@ size_t pb_block_workspace_bytes(const pb_jets *jets);
  *   decided on the host from N, P and tokens before any device call.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture. Every call then clears the array's 256-byte
+ *   before any stream capture. The address is kept for the life of the
+ *   process: after a cudaDeviceReset (or any reset of the device's primary
+ *   context) restart the process before calling this entry point again. Every call then clears the array's 256-byte
  *   header (barrier counters) on `stream` with cudaMemsetAsync and launches
  *   one cooperative kernel. It calls no cudaMalloc, cudaFree or other
  *   allocating routine.
@@ -261,13 +266,21 @@ pb_status pair_attention_forward_noalloc(const pb_jets *jets, const pb_mlp *mlp,
  *   workspace: device memory of at least pb_backward_workspace_bytes(jets)
  *     bytes, 256-byte aligned, no initialisation needed; calls sharing one
  *     workspace must not overlap on the device.
- * Arithmetic: the bias is recomputed by the forward MLP kernel and kept in
- * the workspace as bf16; attention gradients use bf16 tensor-core operands
- * with fp32 accumulation and fp32 softmax statistics, dL/dU is kept as bf16;
- * the MLP is recomputed with bf16 operands (hi + lo terms for the first
- * layer), fp32 accumulation and the erf form of GELU; the weight gradients
- * accumulate in fp32 per CTA and are summed over CTAs in a fixed order, so
- * the result does not depend on timing.
+ * Arithmetic: the bias of every unordered valid pair is recomputed by the
+ * fused path's balanced MLP kernel (the forward's own values: f16 operands,
+ * hidden layers accumulated in f16, the same GELU approximations) and kept
+ * in the workspace as one 16-byte record of 8 f16 values per pair. The
+ * attention gradients use bf16 m16n8k16 tensor-core operands with fp32
+ * accumulation and fp32 softmax statistics; dL/dU[h,i,j] + dL/dU[h,j,i] is
+ * kept as one 32-byte record of 8 fp32 values per unordered pair. The MLP
+ * backward recomputes layers 1-3 on tcgen05 with fp32 accumulation in TMEM
+ * (features and layer-1 weights as bf16 hi + lo terms, h1 and h2 as f16,
+ * W2 and W3 as f16 hi + lo terms) and the tanh approximation of GELU,
+ * GELU(z) = z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))), with its exact
+ * derivative; the products of the backward pass use bf16 operands (weights
+ * as hi + lo terms) with fp32 accumulation. The weight gradients accumulate
+ * in fp32 per CTA and are summed over CTAs in a fixed order, so the result
+ * does not depend on timing.
  * Launches, in order on `stream`: the bias kernel of pairbias_mlp_forward,
  * the attention backward, the MLP backward and a gradient-sum kernel (with
  * N = 0 only the last, writing zeros). Errors as for
@@ -279,10 +292,15 @@ pb_status pair_attention_backward(const pb_jets *jets, const pb_mlp *mlp, int H,
                                   const pb_mlp_grad *dmlp, void *workspace, size_t workspace_bytes,
                                   void *stream);
 
-/* pb_backward_workspace_bytes -- workspace size of pair_attention_backward:
- * N*8*P*P bf16 values (the bias, then dL/dU) plus min(N, 256) partial
- * gradients of PB_FOLDED_FLOATS floats, each part rounded up to 256 bytes.
- * 0 if `jets` is invalid. */
+/* pb_backward_workspace_bytes -- workspace size of pair_attention_backward.
+ * With c = the jets of one chunk (min(N, 8192), and padded also at most
+ * 2^21 / P) and R = the bias-record rows of such a chunk (padded:
+ * c * ceil(P (P + 1) / 2 / 128) * 128; packed: the smaller of that and
+ * tokens * (P + 1) / 2 + 127 c + 128), it is the sum of, each part rounded
+ * up to 256 bytes: a 256-byte header, R * 16 bytes of bias records (8 f16
+ * per pair), R * 32 bytes of gradient records (8 fp32 per pair), (c + 1)
+ * int32 tile offsets and 256 partial gradients of PB_FOLDED_FLOATS fp32
+ * values. 0 if `jets` is invalid. */
 size_t pb_backward_workspace_bytes(const pb_jets *jets);
 
 /* pb_unfold_grad -- host helper, not on the GPU path: gradients of the

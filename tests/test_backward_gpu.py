@@ -3,7 +3,15 @@ backward oracle.
 
 Tolerances (no bar is stated for gradients; these follow from the
 arithmetic of the forward bars and the backward's own roundings):
-  dq, dk, dv      relative L2 over valid rows <= 2e-2, masked rows exactly 0.
+  dq, dk, dv      relative L2 over valid rows <= 2e-2, over the whole batch
+                  and for every (jet, head) on its own (against at least a
+                  tenth of the batch's rms), every element within 0.25 of
+                  that scale; masked rows exactly 0. A gradient element is a
+                  sum of dS-weighted rows in which dS = P (dP - D) cancels,
+                  so single elements carry several times the block's
+                  relative error (largest seen: 0.13 of the scale, on small
+                  jets), while a misrouted row or head is off by about
+                  1.4 times the scale.
                   The bias enters through the forward MLP kernel (bias bar:
                   rel L2 1e-2), the softmax gradient dS = P (dP - D) loses
                   relative accuracy where dP ~ D, and dq, dk, dv are bf16.
@@ -68,11 +76,20 @@ def rel_l2(got, ref):
     return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
 
 
+QKV_OUTLIER = 0.25
+
+
 def check_qkv(got, ref, b):
+    """dq, dk or dv: relative L2 over all valid rows, then per (jet, head)
+    relative L2 and an element bound of QKV_OUTLIER * the block's rms. A
+    block whose gradient nearly cancels (a one-hot softmax, a one-particle
+    jet) is measured against a tenth of the batch's rms instead of its own."""
     vr = pt.valid_rows(b, got.shape)
     rel = rel_l2(got[vr], ref[vr])
     assert rel <= QKV_RELL2, f"rel L2 {rel:.3e}"
     assert np.all(got[~vr] == 0.0), "masked rows must be 0"
+    rms = np.linalg.norm(ref[vr]) / np.sqrt(max(ref[vr].size, 1))
+    pt.check_jet_heads(got, ref, b, QKV_RELL2, QKV_OUTLIER, floor=max(0.1 * rms, 1e-30))
     return rel
 
 

@@ -75,9 +75,12 @@ def test_bias(oracle_lib, name, dtype):
     d = pt.Device(b)
     got = pt.to_np(d.bias(dtype))
     assert ops.get_device_status() == 0
+    worst = (0.0, 0.0)
     for lo, hi in sample_ranges(b):
         s = synth.slice_jets(b, lo, hi)
-        pt.check_bias(got[lo:hi], oracle_lib.pair_bias(s), s, bf16=dtype == torch.bfloat16)
+        e = pt.check_bias(got[lo:hi], oracle_lib.pair_bias(s), s, bf16=dtype == torch.bfloat16)
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+    print(f"\nU error {name} {dtype}: max-abs {worst[0]:.3e}, rel L2 {worst[1]:.3e}")
 
 
 @pytest.mark.parametrize("name", ALL)

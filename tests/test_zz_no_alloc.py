@@ -1,5 +1,7 @@
 """The allocation-free fused entry point (static per-device scratch) against
-the allocating one, through the C ABI, on two calls in a row.
+the allocating one, through the C ABI, on two calls in a row: bit for bit
+against pair_attention_forward given a caller workspace (the same balanced
+kernel, deterministic), and against the fp64 oracle at the attention bar.
 
 Collected last on purpose: it must hold both in a fresh process, where the
 first call performs the per-device set-up, and after every other test has
@@ -25,16 +27,18 @@ def _cuda():
 
 
 @pytest.mark.parametrize("name", ["pr1_n8_p32", "n128_p128"])
-def test_noalloc_matches_fused_entry_point(name):
+def test_noalloc_matches_fused_entry_point(oracle_lib, name):
     b = synth.make_jets(**configs.workload(name, seed=0))
     d = pt.Device(b)
-    ref = pt.to_np(d.fused())                     # the existing entry point, no workspace
+    ref = d.fused(balanced=True)                  # the same kernel with a caller workspace
     assert ops.get_device_status() == 0
+    oref = oracle_lib.forward(b)
     for _call in range(2):
         out = torch.full_like(d.q, float("nan"))
         ops.pair_attention_forward_noalloc(d.jets, d.mlp, d.q, d.k, d.v, out)
         assert ops.get_device_status() == 0
-        pt.check_attention(pt.to_np(out), ref, b)  # rel L2 <= 1e-2, masked rows exactly 0
+        assert torch.equal(out, ref), "noalloc output differs from the workspace call"
+        pt.check_attention(pt.to_np(out), oref, b)
 
 
 def test_noalloc_rejects_batches_beyond_the_static_scratch():
