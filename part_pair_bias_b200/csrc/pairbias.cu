@@ -193,10 +193,10 @@ pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArg
 
 // The 4-CTA cluster kernel takes batches of at most this many jets per SM
 // (one jet per CTA); larger batches already balance over the persistent CTAs.
-// Below kClusterMinJets its fixed costs (counting, two cluster barriers)
-// outweigh the imbalance it removes.
+// Small batches take it too: dealt one jet per cluster, each jet's MLP is
+// split over 4 CTAs.
 constexpr int kClusterJetsPerSm = 1;
-constexpr int kClusterMinJets = 16;
+constexpr int kClusterMinJets = 1;
 
 // The jets are dealt over as many clusters as run at once (cluster sizes
 // need not divide a GPC's SMs, so that number comes from the occupancy query,

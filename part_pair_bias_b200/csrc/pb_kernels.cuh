@@ -287,8 +287,16 @@ __global__ void __launch_bounds__(256) k_pairfeat(JetArgs J, float* __restrict__
 //            max deviation 4.8e-3), on the FMA pipe only. The next layer's
 //            weights carry 1/2 on the tanh columns;
 //   layers 2..4: f16 operands; layer 4 accumulates in fp32; each bias enters
-//            through an extra K step: a constant tile of ones times the
-//            weights' (hi(b), lo(b)) columns.
+//            through an extra K step: a constant column block of ones times
+//            the weights' (hi(b), lo(b)) columns.
+// Data flow: every operand A of the four layers lives in tensor memory. A
+// tile group's 128-column TMEM slot holds its accumulator D (64 columns) and
+// its A operand (40 columns: 64 f16 activations two per column, then the
+// ones block); the epilogue reads D with tcgen05.ld and writes the activated
+// row back with tcgen05.st, and the MMAs read A from TMEM and only the
+// weights (B) from shared memory. An N = 64 MMA whose A and B both came from
+// shared memory would move 6 KB through it, 48 clk at 128 B/clk, against
+// 32 clk of tensor math; with A in TMEM it moves 2 KB.
 
 constexpr int kAK = 64;              // activation tile width
 constexpr int kWK = 80;              // weight K width: 64 activations + 16 bias columns
@@ -318,7 +326,13 @@ struct MlpSmem {
   uint32_t tmem_base;
 };
 
-__host__ __device__ constexpr int kTmemCols(int ng, int sl) { return ng * sl * 64; }
+// TMEM of the MLP: one 128-column slot per tile group (D at +0, A at +64,
+// the ones block of the bias K step at +96); the SL activation tiles of
+// MlpSmem are not used by the MLP and serve the kernels as staging space.
+constexpr int kSlotCols = 128;
+constexpr int kSlotA = 64;
+constexpr int kSlotOnes = kSlotA + 32;
+__host__ __device__ constexpr int kTmemCols(int ng, int) { return ng * kSlotCols; }
 
 // f16 hi/lo split: x = hi + lo to about 22 bits.
 __device__ __forceinline__ void split_half(float x, __half& hi, __half& lo) {
@@ -440,11 +454,10 @@ __device__ void mlp_teardown(MlpSmem<NG, SL>& S, bool aborted, const uint32_t* p
   __syncthreads();
   tc_fence_after();
   if (aborted && (threadIdx.x & 127) == 0) {
-    // A wait that ran out may leave a slot's last commit in flight: give each
-    // slot one more bounded wait before the TMEM they write is released.
+    // A wait that ran out may leave the group's last commit in flight: give
+    // it one more bounded wait before the TMEM it writes is released.
     const int g = threadIdx.x >> 7;
-    if (g < NG)
-      for (int s = 0; s < SL; ++s) mbar_wait(&S.mbar[SL * g + s], ((*phase >> s) & 1u) ^ 1u);
+    if (g < NG) mbar_wait(&S.mbar[g], (*phase & 1u) ^ 1u);
   }
   __syncthreads();
   if ((threadIdx.x >> 5) == 0) tmem_dealloc(S.tmem_base, kTmemCols(NG, SL));
@@ -492,13 +505,13 @@ struct RectPairs {  // ordered pairs (i0 + p / m, p % m): a query block against 
   }
 };
 
-// Runs the 4-layer MLP over `npairs` rows in 128-row tiles. Group g (threads
-// 128g .. 128g+127) takes tiles g, g+NG, ... and keeps up to SL of them in
-// flight (each slot: activation tile, 64 TMEM columns, an mbarrier): while
-// the tensor cores run one slot's layer, the group computes another slot's
-// epilogue. Thread row r of a group owns TMEM lane r. For each valid row the
-// sink gets (p, a, b, u[8]). Bit s of *phase tracks slot s's mbarrier parity.
-// Returns false if the group aborted on a timed-out wait.
+// Runs the 4-layer MLP over the source's rows in 128-row tiles. Group g
+// (threads 128g .. 128g+127) takes tiles g, g+NG, ... one at a time through
+// its TMEM slot; thread row r of a group owns TMEM lane r. The groups run
+// independently, so one group's epilogue overlaps the others' MMAs. For each
+// valid row the sink gets (p, a, b, u[8]). Bit 0 of *phase tracks the
+// group's mbarrier parity. Returns false if the group aborted on a timed-out
+// wait.
 // A source of MLP rows for one pass: ntiles() tiles; row(t, r, ...) gives
 // the features of row r of tile t and the (p, a, b) its sink receives, or
 // false for a padding row.
@@ -520,79 +533,76 @@ struct JetTiles {  // the pairs of one staged jet
 
 template <int NG, int SL, class Source, class Sink>
 __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Source& src, Sink& sink, uint32_t* phase) {
-  static_assert(SL >= 1 && SL <= 4, "one to four tiles in flight per group");
   const int g = threadIdx.x >> 7;
   if (g >= NG) return true;  // threads past the MLP's groups take no tiles
   const int row = threadIdx.x & 127;
   const uint32_t bar_id = 1 + g;
   const bool leader = row == 0;
   const uint32_t w_addr[4] = {smem_u32(S.W1), smem_u32(S.W2), smem_u32(S.W3), smem_u32(S.W4)};
-  const uint32_t ones_addr = smem_u32(S.Ones);
   // layers 1..3 accumulate in f16 (read back packed, no conversion), layer 4 in fp32
   constexpr uint32_t kId64 = idesc_f16_m128(64, false), kId16 = idesc_f16_m128(16, true);
   const int ntiles = src.ntiles();
+  uint64_t* const mbar = &S.mbar[g];
+  const uint32_t lane_off = (uint32_t)(row & 96) << 16;
+  const uint32_t t_d = S.tmem_base + (uint32_t)(g * kSlotCols);  // accumulator, 64 columns
+  const uint32_t t_a = t_d + kSlotA;                             // A operand, 40 columns
   bool ok = true;
 
-  // slot s: activation tile A0 + s*kTileElems, TMEM columns t_d0 + 64 s,
-  // mbarrier S.mbar[SL g + s]; selected arithmetically (no local-memory arrays)
-  constexpr int kTileElems = kTileM * kAK;
-  __half* const A0 = S.A[SL * g];
-  const uint32_t a_addr0 = smem_u32(A0);
-  const uint32_t t_d0 = S.tmem_base + (uint32_t)(SL * g * 64);
-  const uint32_t lane_off = (uint32_t)(row & 96) << 16;
-
-  // Publish this thread's operand writes and TMEM reads, meet the group and
-  // have the leader issue layer L of slot s; completion arrives on its mbarrier.
-  auto issue = [&](int s, int L) -> bool {
-    fence_proxy_async_smem();
+  // Publish this thread's TMEM stores and reads, meet the group and have the
+  // leader issue layer L; its completion arrives on the group's mbarrier.
+  auto issue = [&](int L) -> bool {
     tc_fence_before();
     if (named_bar_or(bar_id, 128, !ok)) return false;
     if (leader) {
       tc_fence_after();
-      const uint32_t a_addr = a_addr0 + (uint32_t)(s * kTileElems * 2);
-      const uint32_t d = t_d0 + 64u * s;
       if (L == 0) {
-        mma_f16(d, smem_desc(a_addr, 128, kASBO), smem_desc(w_addr[0], 128, 256), kId64, 0);
+        mma_f16_ta(t_d, t_a, smem_desc(w_addr[0], 128, 256), kId64, 0u);
       } else {
         const uint32_t w = L == 1 ? w_addr[1] : (L == 2 ? w_addr[2] : w_addr[3]);
         const uint32_t id = L == 3 ? kId16 : kId64;
         // bias step first (initialises the accumulator), then the 64 activations
-        mma_f16(d, smem_desc(ones_addr, 128, 256), smem_desc(w + 1024u, 128, kWSBO), id, 0u);
+        mma_f16_ta(t_d, t_d + kSlotOnes, smem_desc(w + 1024u, 128, kWSBO), id, 0u);
 #pragma unroll
         for (int k = 0; k < kAK / 16; ++k)
-          mma_f16(d, smem_desc(a_addr + 256u * k, 128, kASBO), smem_desc(w + 256u * k, 128, kWSBO), id, 1u);
+          mma_f16_ta(t_d, t_a + 8u * k, smem_desc(w + 256u * k, 128, kWSBO), id, 1u);
       }
-      mma_commit(&S.mbar[SL * g + s]);
+      mma_commit(mbar);
     }
     return true;
   };
-  auto wait = [&](int s) {
-    const bool done = mbar_wait(&S.mbar[SL * g + s], (*phase >> s) & 1u);
+  auto wait = [&]() {
+    const bool done = mbar_wait(mbar, *phase & 1u);
     ok = ok && done;
-    *phase ^= 1u << s;
+    *phase ^= 1u;
     tc_fence_after();
   };
 
-  // TMEM accumulator row (bias included, f16) -> activation in f16x2 -> the slot's A tile.
-  auto hidden = [&](int s) {
-    __half* As = A0 + s * kTileElems;
+  // The ones block of the bias K step, [1 1 0 ... 0] per row (K columns
+  // 64..79 of A); written on every pass, since other users of the TMEM
+  // (the projections) may have overwritten it.
+  {
+    const uint32_t ones[8] = {0x3C003C00u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    tmem_st8_wait(t_d + kSlotOnes + lane_off, ones);
+  }
+
+  // TMEM accumulator row (bias included, f16) -> activation in f16x2 -> the
+  // group's A operand.
+  auto hidden = [&]() {
     uint32_t y[32];
-    tmem_ld64_f16_wait(t_d0 + 64u * s + lane_off, y);
+    tmem_ld64_f16_wait(t_d + lane_off, y);
 #pragma unroll
-    for (int chunk = 0; chunk < 8; ++chunk) {
-      uint32_t w[4];
+    for (int chunk = 0; chunk < 8; ++chunk)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        w[j] = chunk < kTanhChunks ? gelu2_f16x2(y[4 * chunk + j]) : gelu_poly_f16x2(y[4 * chunk + j]);
-      *reinterpret_cast<uint4*>(As + cofs(row, 8 * chunk, kAK)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+        y[4 * chunk + j] = chunk < kTanhChunks ? gelu2_f16x2(y[4 * chunk + j]) : gelu_poly_f16x2(y[4 * chunk + j]);
+    tmem_st32_wait(t_a + lane_off, y);
   };
 
-  // Features of tile t into slot s's layer-1 operand row: [hi(f) | hi(f) |
-  // lo(f) | 1 1 0 0] against [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0]
-  // gives W1 f + b1 to ~22 bits. Returns the row's sink key (-1 for a padding
-  // row) and its particles.
-  auto start = [&](int s, int t, int& p_out, int& a_out, int& b_out) -> bool {
+  // Features of tile t as the layer-1 operand row: [hi(f) | hi(f) | lo(f) |
+  // 1 1 0 0] against [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0] gives
+  // W1 f + b1 to ~22 bits. Returns the row's sink key (-1 for a padding row)
+  // and its particles.
+  auto features = [&](int t, uint32_t* a1, int& p_out, int& a_out, int& b_out) {
     int p = -1, a = 0, b = 0;
     float f[4] = {0.f, 0.f, 0.f, 0.f};
     const bool valid = src.row(t, row, p, a, b, f);
@@ -607,61 +617,47 @@ __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Source& src, Sink& sink, uint
 #pragma unroll
     for (int i = 0; i < 4; ++i) split_half(f[i], hi[i], lo[i]);
     const __half one = __float2half_rn(valid ? 1.f : 0.f), zero = __float2half_rn(0.f);
-    __half* As = A0 + s * kTileElems;
-    *reinterpret_cast<uint4*>(As + cofs(row, 0, kAK)) =
-        make_uint4(h2bits(hi[0], hi[1]), h2bits(hi[2], hi[3]), h2bits(hi[0], hi[1]), h2bits(hi[2], hi[3]));
-    *reinterpret_cast<uint4*>(As + cofs(row, 8, kAK)) =
-        make_uint4(h2bits(lo[0], lo[1]), h2bits(lo[2], lo[3]), h2bits(one, one), h2bits(zero, zero));
-    return issue(s, 0);
+    a1[0] = h2bits(hi[0], hi[1]);
+    a1[1] = h2bits(hi[2], hi[3]);
+    a1[2] = a1[0];
+    a1[3] = a1[1];
+    a1[4] = h2bits(lo[0], lo[1]);
+    a1[5] = h2bits(lo[2], lo[3]);
+    a1[6] = h2bits(one, one);
+    a1[7] = h2bits(zero, zero);
   };
 
-  // per-slot state: tile index (-1 = idle), next layer, row's pair and
-  // particles; slots are visited round-robin with compile-time indices
-  int tile[SL], lay[SL], pk[SL], pa[SL], pb[SL];
-  int next = g;
-#pragma unroll
-  for (int s = 0; s < SL; ++s) {
-    tile[s] = -1;
-    lay[s] = 0;
-    pk[s] = -1;
-    pa[s] = pb[s] = 0;
-    if (next < ntiles) {
-      tile[s] = next;
-      next += NG;
-      lay[s] = 1;
-      if (!start(s, tile[s], pk[s], pa[s], pb[s])) return false;
-    }
-  }
-  bool active = tile[0] >= 0;
+  // Per tile: layer 1 is issued from features computed during the previous
+  // tile's last MMA, and the previous tile's row goes to the sink while this
+  // tile's first MMA runs, so neither sits between two MMAs of the group.
+  uint32_t a1[8];
+  int pk = -1, pa = 0, pb = 0;       // the current tile's row
+  int qk = -1, qa = 0, qb = 0;       // the previous tile's row, waiting for the sink
+  float u[8];
+  int t = g;
+  if (t < ntiles) features(t, a1, pk, pa, pb);
 #pragma unroll 1
-  while (active) {
-    active = false;
-#pragma unroll
-    for (int s = 0; s < SL; ++s) {
-      if (tile[s] >= 0) {
-        wait(s);
-        if (lay[s] <= 3) {
-          hidden(s);
-          if (!issue(s, lay[s])) return false;
-          ++lay[s];
-        } else {
-          float u[8];
-          tmem_ld8_wait(t_d0 + 64u * s + lane_off, u);
-          if (pk[s] >= 0) sink(pk[s], pa[s], pb[s], u);
-          if (next < ntiles) {
-            tile[s] = next;
-            next += NG;
-            lay[s] = 1;
-            if (!start(s, tile[s], pk[s], pa[s], pb[s])) return false;
-          } else {
-            tile[s] = -1;
-          }
-        }
-      }
-      active = active || tile[s] >= 0;
+  while (t < ntiles) {
+    tmem_st8_wait(t_a + lane_off, a1);
+    if (!issue(0)) return false;
+    if (qk >= 0) sink(qk, qa, qb, u);
+#pragma unroll 1
+    for (int L = 1; L <= 3; ++L) {
+      wait();
+      hidden();
+      if (!issue(L)) return false;
     }
+    const int ck = pk, ca = pa, cb = pb;
+    t += NG;
+    if (t < ntiles) features(t, a1, pk, pa, pb);
+    wait();
+    tmem_ld8_wait(t_d + lane_off, u);
+    qk = ck;
+    qa = ca;
+    qb = cb;
   }
-  // the TMEM reads of the last tiles must finish before anyone reuses them
+  if (qk >= 0) sink(qk, qa, qb, u);
+  // the TMEM reads of the last tile must finish before anyone reuses them
   tc_fence_before();
   return ok;
 }
@@ -1772,10 +1768,14 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
     SmemUSink sink{S.U8, kUCap};
     const int np = m * (m + 1) / 2;
     if (np <= kUCap) {
-      // when the bias triangle leaves room, the K and V of all heads are
-      // copied in behind it while the MLP runs
+      // the K and V of all heads are copied in while the MLP runs: into the
+      // stage (the MLP keeps its operands in TMEM), or behind the bias
+      // triangle when the stage is too small (P = 256 jets above 128)
       uint16_t* early = nullptr;
-      if (m > 0 && np + kH * kv16_bytes(m) / 16 <= kUCap) {
+      if (m > 0 && kH * kv16_bytes(m) <= kStageFloats * 4) {
+        early = reinterpret_cast<uint16_t*>(stage);
+        stage_kv16<PM>(S.part, J, X, n, 0, kH, early);
+      } else if (m > 0 && np + kH * kv16_bytes(m) / 16 <= kUCap) {
         early = reinterpret_cast<uint16_t*>(S.U8 + np);
         stage_kv16<PM>(S.part, J, X, n, 0, kH, early);
       }
@@ -2267,9 +2267,10 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
 // ============================================== k_fused_cluster (4-CTA jets)
 //
 // The fused path for batches of few jets, where one CTA per jet would wait
-// for the widest one: a thread-block cluster of 4 CTAs takes 4 jets.
-//   - every CTA stages all 4 jets; the MLP tiles of the 4 jets are split
-//     evenly over the 4 CTAs (contiguous ranges of the cluster's tile list);
+// for the widest one: a thread-block cluster of 4 CTAs takes up to 4 jets
+// (the host deals the jets over as many clusters as run at once).
+//   - every CTA stages the cluster's jets; their MLP tiles are split evenly
+//     over the 4 CTAs (contiguous ranges of the cluster's tile list);
 //   - a tile row's 8 biases go straight to the CTA that owns their heads:
 //     CTA q keeps heads 2q, 2q + 1 of every pair of the 4 jets, 4 bytes per
 //     pair, written through distributed shared memory (st.shared::cluster);
@@ -2498,17 +2499,20 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   for (int g0 = 0; g0 < K;) {
     __syncthreads();
     const int G = H.G;
+    // heads 2q, 2q + 1 of the group's jets at once: K and V of every (jet,
+    // head) are copied into the stage while the MLP runs (its operands live
+    // in TMEM), then the warps take (jet, head, 16-query tile) items, the
+    // next item's Q fragment loaded ahead; the first Q fragment is loaded
+    // before the barrier that waits for the other CTAs' MLP.
+    uint16_t* kv = reinterpret_cast<uint16_t*>(stage);
+    if (!aborted)
+      for (int k = 0; k < G; ++k)
+        if (H.ring[g0 + k].m > 0) stage_kv16<PM>(H.ring[g0 + k], J, X, H.jets[g0 + k], 2 * q, 2, kv + H.kvoff[k]);
     if (!aborted) {
       const bool ok = mlp_pass<NG, SL>(H.mlp, ClusterTiles<PM>{&H, g0}, sink, &phase);
       aborted = !ok;
     }
     aborted = __syncthreads_or(aborted) != 0;
-    // heads 2q, 2q + 1 of the group's jets at once: K and V of every (jet,
-    // head) staged together, then the warps take (jet, head, 16-query tile)
-    // items, the next item's Q fragment loaded ahead. This CTA's MLP is done,
-    // so the staging (into the MLP's operand buffers) and the first Q
-    // fragment are issued before the barrier that waits for the others.
-    uint16_t* kv = reinterpret_cast<uint16_t*>(stage);
     const int* kvoff = H.kvoff;
     const int* ib = H.ib;
     const int items = ib[kCJ], warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
@@ -2527,12 +2531,9 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
       q_frag(i0, min(16, P.m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, H.jets[g0 + k], h, i); }, f);
     };
     uint32_t a[4] = {0u, 0u, 0u, 0u};
-    if (!aborted) {
-      for (int k = 0; k < G; ++k)
-        if (H.ring[g0 + k].m > 0) stage_kv16<PM>(H.ring[g0 + k], J, X, H.jets[g0 + k], 2 * q, 2, kv + kvoff[k]);
-      if (warp < items) qload(warp, a);
-    }
+    if (!aborted && warp < items) qload(warp, a);
     cluster_sync_all();  // every CTA's stores into this one are visible
+    if (aborted) cp_async_wait_all();  // no copy may still land after the kernel
     if (!aborted) {
       cp_async_wait_all();
       __syncthreads();
