@@ -65,6 +65,13 @@ def lib():
             L.orc_pair_bias.argtypes = [C.POINTER(_Jets), C.POINTER(_Params), dp]
             L.orc_attention.argtypes = [C.POINTER(_Jets), dp, u16, u16, u16, C.c_int, dp]
             L.orc_forward.argtypes = [C.POINTER(_Jets), C.POINTER(_Params), u16, u16, u16, C.c_int, dp]
+            i8 = C.POINTER(C.c_int8)
+            L.orc_quantize_act.argtypes = [dp, C.c_int, i8, dp, C.POINTER(C.c_int)]
+            L.orc_quantize_weights.argtypes = [dp, C.c_int, C.c_int, i8, dp]
+            L.orc_int8_linear.argtypes = [dp, C.c_int, dp, dp, C.c_int, dp]
+            L.orc_mlp_row_i8.argtypes = [dp, C.POINTER(_Params), dp]
+            L.orc_pair_bias_i8.argtypes = [C.POINTER(_Jets), C.POINTER(_Params), dp]
+            L.orc_forward_i8.argtypes = [C.POINTER(_Jets), C.POINTER(_Params), u16, u16, u16, C.c_int, dp]
             L.orc_set_threads.argtypes = [C.c_int]
             L.orc_get_threads.restype = C.c_int
             _lib = L
@@ -118,6 +125,69 @@ def mlp_row(f, params) -> np.ndarray:
     st, _keep = _params(params)
     out = np.zeros(8)
     lib().orc_mlp_row(_ptr(f, C.c_double), C.byref(st), _ptr(out, C.c_double))
+    return out
+
+
+def quantize_act(x):
+    """Zero-point int8 quantisation of one input row: (codes int8, s, z)."""
+    x = np.ascontiguousarray(x, np.float64)
+    q = np.zeros(x.shape[0], np.int8)
+    s = C.c_double()
+    z = C.c_int()
+    lib().orc_quantize_act(_ptr(x, C.c_double), int(x.shape[0]), _ptr(q, C.c_int8), C.byref(s), C.byref(z))
+    return q, s.value, z.value
+
+
+def quantize_weights(W):
+    """Per-row symmetric int8 weight codes of W [rows, cols]: (codes, alpha)."""
+    W = np.ascontiguousarray(W, np.float64)
+    T = np.zeros(W.shape, np.int8)
+    alpha = np.zeros(W.shape[0])
+    lib().orc_quantize_weights(_ptr(W, C.c_double), int(W.shape[0]), int(W.shape[1]), _ptr(T, C.c_int8),
+                               _ptr(alpha, C.c_double))
+    return T, alpha
+
+
+def int8_linear(x, W, b) -> np.ndarray:
+    """y = W x + b with x and W quantised to int8 (the int8 variant's layer)."""
+    x = np.ascontiguousarray(x, np.float64)
+    W = np.ascontiguousarray(W, np.float64)
+    b = np.ascontiguousarray(b, np.float64)
+    y = np.zeros(W.shape[0])
+    lib().orc_int8_linear(_ptr(x, C.c_double), int(x.shape[0]), _ptr(W, C.c_double), _ptr(b, C.c_double),
+                          int(W.shape[0]), _ptr(y, C.c_double))
+    return y
+
+
+def mlp_row_i8(f, params) -> np.ndarray:
+    f = np.ascontiguousarray(f, np.float64)
+    st, _keep = _params(params)
+    out = np.zeros(8)
+    lib().orc_mlp_row_i8(_ptr(f, C.c_double), C.byref(st), _ptr(out, C.c_double))
+    return out
+
+
+def pair_bias_i8(b, params=None) -> np.ndarray:
+    """U [N, 8, P, P] float64 of the MLP with int8 hidden-layer inputs."""
+    js, _k = _jets(b)
+    ps, _kp = _params(params if params is not None else b.params)
+    out = np.zeros((b.N, H, b.P, b.P))
+    if lib().orc_pair_bias_i8(C.byref(js), C.byref(ps), _ptr(out, C.c_double)) != 0:
+        raise ValueError("oracle: invalid jet description")
+    return out
+
+
+def forward_i8(b, params=None) -> np.ndarray:
+    """The block with the int8 MLP variant; output in the layout of q."""
+    js, _k = _jets(b)
+    ps, _kp = _params(params if params is not None else b.params)
+    q = np.ascontiguousarray(b.q, np.uint16)
+    k = np.ascontiguousarray(b.k, np.uint16)
+    v = np.ascontiguousarray(b.v, np.uint16)
+    out = np.zeros(q.shape)
+    if lib().orc_forward_i8(C.byref(js), C.byref(ps), _ptr(q, C.c_uint16), _ptr(k, C.c_uint16),
+                            _ptr(v, C.c_uint16), D, _ptr(out, C.c_double)) != 0:
+        raise ValueError("oracle: invalid jet description")
     return out
 
 

@@ -29,6 +29,20 @@
  *      o_i = sum_j softmax_j(q_i.k_j / sqrt(D) + U[h,i,j]) v_j over valid
  *      keys j; masked keys are excluded (score -inf); masked query rows are 0.
  *
+ *   5. (variant) int8 inputs of the hidden layers, the data-type quantisation
+ *      of "Economical Jet Taggers -- Equivariant, Slim and Quantised",
+ *      section "Kwantiseringsstrategieen": the inputs of linear layers are
+ *      int8 with zero-point quantisation, the weights binary or ternary.
+ *      Reading (orc_*_i8): layer 1 keeps its float input (the features);
+ *      for layers 2, 3 and 4 the input row x (64 activations of one pair)
+ *      is quantised on its own: lo = min(0, min x), hi = max(0, max x),
+ *      s = (hi - lo) / 255 (s = 1 when hi == lo), z = -128 - round(lo / s),
+ *      q = clamp(round(x / s) + z, -128, 127), rounding half to even; the
+ *      layer's folded weights W' (rows a_k * W_k, bias a_k b_k + c_k; W4 and
+ *      b4 as they are) are quantised per output row, alpha = max|W'_row| /
+ *      127, T = round(W' / alpha); then y_o = alpha_o s sum_i T_oi (q_i - z)
+ *      + b'_o, evaluated exactly (the integer sum in int64).
+ *
  * Readings where the pages are silent: diagonal pairs (a == b) are included
  * and use the same formulas; pairs with a masked end are never evaluated and
  * their feature / bias entries are 0; Q/K/V are bf16 bit patterns widened
@@ -175,6 +189,113 @@ void orc_mlp_row(const double f[4], const orc_params *w, double u[8]) {
   }
 }
 
+/* ------------------------------------------------ int8 hidden-layer inputs */
+
+/* Round half to even (the rounding of the quantiser). */
+static double round_even(double x) { return nearbyint(x); }
+
+/* Zero-point quantisation of one input row x[n] (see 5. above). */
+void orc_quantize_act(const double *x, int n, int8_t *q, double *s_out, int *z_out) {
+  double lo = 0.0, hi = 0.0;
+  for (int i = 0; i < n; ++i) {
+    if (x[i] < lo) lo = x[i];
+    if (x[i] > hi) hi = x[i];
+  }
+  double s = hi > lo ? (hi - lo) / 255.0 : 1.0;
+  int z = -128 - (int)round_even(lo / s);
+  for (int i = 0; i < n; ++i) {
+    double c = round_even(x[i] / s) + z;
+    q[i] = (int8_t)(c < -128.0 ? -128 : (c > 127.0 ? 127 : c));
+  }
+  *s_out = s;
+  *z_out = z;
+}
+
+/* Symmetric per-row weight codes: alpha = max|W_row| / 127 (1 for a zero
+ * row), T = round(W / alpha). W is [rows][cols] row-major. */
+void orc_quantize_weights(const double *W, int rows, int cols, int8_t *T, double *alpha) {
+  for (int r = 0; r < rows; ++r) {
+    double mx = 0.0;
+    for (int c = 0; c < cols; ++c) mx = fmax(mx, fabs(W[r * cols + c]));
+    double a = mx > 0.0 ? mx / 127.0 : 1.0;
+    for (int c = 0; c < cols; ++c) T[r * cols + c] = (int8_t)round_even(W[r * cols + c] / a);
+    alpha[r] = a;
+  }
+}
+
+/* One linear layer with int8 input and weight codes:
+ * y_o = alpha_o s sum_i T_oi (q_i - z) + b_o. */
+static void int8_layer(const int8_t *q, double s, int z, const int8_t *T, const double *alpha,
+                       const double *b, int nin, int nout, double *y) {
+  for (int o = 0; o < nout; ++o) {
+    int64_t acc = 0;
+    for (int i = 0; i < nin; ++i) acc += (int64_t)T[o * nin + i] * ((int64_t)q[i] - z);
+    y[o] = alpha[o] * s * (double)acc + b[o];
+  }
+}
+
+/* The whole quantised linear map of one row, from float input and float
+ * weights: both are quantised as above, then int8_layer. */
+void orc_int8_linear(const double *x, int nin, const double *W, const double *b, int nout, double *y) {
+  int8_t *q = malloc((size_t)nin), *T = malloc((size_t)nin * nout);
+  double *alpha = malloc(sizeof(double) * nout), s;
+  int z;
+  orc_quantize_act(x, nin, q, &s, &z);
+  orc_quantize_weights(W, nout, nin, T, alpha);
+  int8_layer(q, s, z, T, alpha, b, nin, nout, y);
+  free(q); free(T); free(alpha);
+}
+
+/* Folded and quantised layers 2..4 of one parameter set. */
+typedef struct {
+  int8_t T2[ORC_HID * ORC_HID], T3[ORC_HID * ORC_HID], T4[ORC_NH * ORC_HID];
+  double al2[ORC_HID], al3[ORC_HID], al4[ORC_NH];
+  double b2[ORC_HID], b3[ORC_HID], b4[ORC_NH];
+} orc_i8;
+
+static void fold_quantize_layer(const float *W, const float *b, const float *a, const float *c, int nout,
+                                int8_t *T, double *alpha, double *bf) {
+  double *Wf = malloc(sizeof(double) * nout * ORC_HID);
+  for (int o = 0; o < nout; ++o) {
+    double ao = a ? (double)a[o] : 1.0;
+    for (int i = 0; i < ORC_HID; ++i) Wf[o * ORC_HID + i] = ao * (double)W[o * ORC_HID + i];
+    bf[o] = ao * (double)b[o] + (c ? (double)c[o] : 0.0);
+  }
+  orc_quantize_weights(Wf, nout, ORC_HID, T, alpha);
+  free(Wf);
+}
+
+static void prepare_i8(const orc_params *w, orc_i8 *qw) {
+  fold_quantize_layer(w->W2, w->b2, w->a2, w->c2, ORC_HID, qw->T2, qw->al2, qw->b2);
+  fold_quantize_layer(w->W3, w->b3, w->a3, w->c3, ORC_HID, qw->T3, qw->al3, qw->b3);
+  fold_quantize_layer(w->W4, w->b4, NULL, NULL, ORC_NH, qw->T4, qw->al4, qw->b4);
+}
+
+/* MLP row with int8 inputs to layers 2..4: f[4] -> u[8]. */
+static void mlp_row_i8(const double f[4], const orc_params *w, const orc_i8 *qw, double u[8]) {
+  double x[ORC_NF], h[ORC_HID], y[ORC_HID], s;
+  int8_t q[ORC_HID];
+  int z;
+  for (int i = 0; i < ORC_NF; ++i) x[i] = (double)w->a0[i] * f[i] + (double)w->c0[i];
+  hidden_layer(x, ORC_NF, w->W1, w->b1, w->a1, w->c1, h);
+  orc_quantize_act(h, ORC_HID, q, &s, &z);
+  int8_layer(q, s, z, qw->T2, qw->al2, qw->b2, ORC_HID, ORC_HID, y);
+  for (int i = 0; i < ORC_HID; ++i) h[i] = orc_gelu(y[i]);
+  orc_quantize_act(h, ORC_HID, q, &s, &z);
+  int8_layer(q, s, z, qw->T3, qw->al3, qw->b3, ORC_HID, ORC_HID, y);
+  for (int i = 0; i < ORC_HID; ++i) h[i] = orc_gelu(y[i]);
+  orc_quantize_act(h, ORC_HID, q, &s, &z);
+  int8_layer(q, s, z, qw->T4, qw->al4, qw->b4, ORC_HID, ORC_NH, u);
+}
+
+/* One pair row of the int8 variant (for tests). */
+void orc_mlp_row_i8(const double f[4], const orc_params *w, double u[8]) {
+  orc_i8 *qw = malloc(sizeof(orc_i8));
+  prepare_i8(w, qw);
+  mlp_row_i8(f, w, qw, u);
+  free(qw);
+}
+
 /* ------------------------------------------------------------ jet access */
 
 /* Valid local slots of jet n and their element indices into the momentum
@@ -234,21 +355,25 @@ int orc_features(const orc_jets *j, double *feat) {
   return bad ? -1 : 0;
 }
 
-/* Bias of one jet over its valid ordered pairs: u[(h*m + ia)*m + ib]. */
-static void jet_bias(const orc_jets *j, const orc_params *w, int m, const int64_t *elem, double *u) {
+/* Bias of one jet over its valid ordered pairs: u[(h*m + ia)*m + ib]; with
+ * qw, the int8 variant of the MLP. */
+static void jet_bias(const orc_jets *j, const orc_params *w, const orc_i8 *qw, int m, const int64_t *elem,
+                     double *u) {
   for (int ia = 0; ia < m; ++ia)
     for (int ib = 0; ib < m; ++ib) {
       double pa[4], pb[4], f[4], row[8];
       momentum(j, elem[ia], pa);
       momentum(j, elem[ib], pb);
       orc_pair_features(pa, pb, f);
-      orc_mlp_row(f, w, row);
+      if (qw) mlp_row_i8(f, w, qw, row);
+      else orc_mlp_row(f, w, row);
       for (int h = 0; h < ORC_NH; ++h) u[((int64_t)h * m + ia) * m + ib] = row[h];
     }
 }
 
-/* U [N,8,P,P]: bias of every valid ordered pair, 0 elsewhere. */
-int orc_pair_bias(const orc_jets *j, const orc_params *w, double *U) {
+/* U [N,8,P,P]: bias of every valid ordered pair, 0 elsewhere; with qw the
+ * int8 variant. */
+static int pair_bias(const orc_jets *j, const orc_params *w, const orc_i8 *qw, double *U) {
   int bad = 0;
   memset(U, 0, sizeof(double) * (size_t)j->N * ORC_NH * j->P * j->P);
 #pragma omp parallel for schedule(dynamic) num_threads(orc_get_threads()) reduction(| : bad)
@@ -258,7 +383,7 @@ int orc_pair_bias(const orc_jets *j, const orc_params *w, double *U) {
     int m = jet_slots(j, n, slot, elem);
     if (m < 0) { bad = 1; free(slot); free(elem); continue; }
     double *u = malloc(sizeof(double) * (size_t)ORC_NH * (m ? m : 1) * (m ? m : 1));
-    jet_bias(j, w, m, elem, u);
+    jet_bias(j, w, qw, m, elem, u);
     for (int h = 0; h < ORC_NH; ++h)
       for (int ia = 0; ia < m; ++ia)
         for (int ib = 0; ib < m; ++ib)
@@ -267,6 +392,16 @@ int orc_pair_bias(const orc_jets *j, const orc_params *w, double *U) {
     free(u); free(slot); free(elem);
   }
   return bad ? -1 : 0;
+}
+
+int orc_pair_bias(const orc_jets *j, const orc_params *w, double *U) { return pair_bias(j, w, NULL, U); }
+
+int orc_pair_bias_i8(const orc_jets *j, const orc_params *w, double *U) {
+  orc_i8 *qw = malloc(sizeof(orc_i8));
+  prepare_i8(w, qw);
+  int r = pair_bias(j, w, qw, U);
+  free(qw);
+  return r;
 }
 
 /* Attention of one jet. bias(h, ia, ib) is read from u_local (m x m per head)
@@ -324,9 +459,9 @@ int orc_attention(const orc_jets *j, const double *U, const uint16_t *q, const u
 }
 
 /* out (layout of q): the whole block -- features, MLP bias and attention --
- * with each jet's bias kept local to the jet. */
-int orc_forward(const orc_jets *j, const orc_params *w, const uint16_t *q, const uint16_t *k,
-                const uint16_t *v, int D, double *out) {
+ * with each jet's bias kept local to the jet; with qw the int8 MLP. */
+static int forward(const orc_jets *j, const orc_params *w, const orc_i8 *qw, const uint16_t *q,
+                   const uint16_t *k, const uint16_t *v, int D, double *out) {
   int bad = 0;
   memset(out, 0, sizeof(double) * (size_t)qkv_elems(j, D));
 #pragma omp parallel for schedule(dynamic) num_threads(orc_get_threads()) reduction(| : bad)
@@ -336,9 +471,23 @@ int orc_forward(const orc_jets *j, const orc_params *w, const uint16_t *q, const
     int m = jet_slots(j, n, slot, elem);
     if (m < 0) { bad = 1; free(slot); free(elem); continue; }
     double *u = malloc(sizeof(double) * (size_t)ORC_NH * (m ? m : 1) * (m ? m : 1));
-    jet_bias(j, w, m, elem, u);
+    jet_bias(j, w, qw, m, elem, u);
     jet_attention(j, n, m, slot, u, NULL, q, k, v, D, out);
     free(u); free(slot); free(elem);
   }
   return bad ? -1 : 0;
+}
+
+int orc_forward(const orc_jets *j, const orc_params *w, const uint16_t *q, const uint16_t *k,
+                const uint16_t *v, int D, double *out) {
+  return forward(j, w, NULL, q, k, v, D, out);
+}
+
+int orc_forward_i8(const orc_jets *j, const orc_params *w, const uint16_t *q, const uint16_t *k,
+                   const uint16_t *v, int D, double *out) {
+  orc_i8 *qw = malloc(sizeof(orc_i8));
+  prepare_i8(w, qw);
+  int r = forward(j, w, qw, q, k, v, D, out);
+  free(qw);
+  return r;
 }

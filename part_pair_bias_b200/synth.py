@@ -120,19 +120,39 @@ def _constituents(rng, m, pt_lo, pt_hi, prongs):
     return pt * np.cosh(eta), pt * np.cos(phi), pt * np.sin(phi), pt * np.sinh(eta)
 
 
-def make_params(rng) -> Dict[str, np.ndarray]:
-    """Unfolded pair-embedding MLP parameters (4 -> 64 -> 64 -> 64 -> 8), float32."""
+def _ternary(rng, rows, fan):
+    """Rows tau * t with t in {-1, 0, +1} (P(0) = 1/3) and one tau per row,
+    tau = sqrt(1.5 / fan): the variance 1/fan of the Gaussian weights."""
+    t = rng.integers(-1, 2, size=(rows, fan)).astype(np.float64)
+    return np.sqrt(1.5 / fan) * rng.uniform(0.8, 1.2, size=(rows, 1)) * t
+
+
+def make_params(rng, weights: str = "gaussian") -> Dict[str, np.ndarray]:
+    """Unfolded pair-embedding MLP parameters (4 -> 64 -> 64 -> 64 -> 8), float32.
+
+    ``weights="ternary"`` draws the Linear weights of layers 2..4 (the layers
+    whose inputs are hidden activations) as one scale per output row times
+    {-1, 0, +1}, the weights of a ternary-quantised network; layer 1 and every
+    other parameter keep their Gaussian / uniform draws."""
+    if weights not in ("gaussian", "ternary"):
+        raise ValueError(f"unknown weight kind {weights!r}")
     p = {}
     p["a0"] = rng.uniform(0.5, 1.5, N_FEAT)
     p["c0"] = rng.normal(0.0, 0.1, N_FEAT)
     fan = N_FEAT
     for k in (1, 2, 3):
-        p[f"W{k}"] = rng.normal(0.0, 1.0 / np.sqrt(fan), (HIDDEN, fan))
+        if weights == "ternary" and k > 1:
+            p[f"W{k}"] = _ternary(rng, HIDDEN, fan)
+        else:
+            p[f"W{k}"] = rng.normal(0.0, 1.0 / np.sqrt(fan), (HIDDEN, fan))
         p[f"b{k}"] = rng.normal(0.0, 0.1, HIDDEN)
         p[f"a{k}"] = rng.uniform(0.5, 1.5, HIDDEN)
         p[f"c{k}"] = rng.normal(0.0, 0.1, HIDDEN)
         fan = HIDDEN
-    p["W4"] = rng.normal(0.0, 1.0 / np.sqrt(HIDDEN), (H_HEADS, HIDDEN))
+    if weights == "ternary":
+        p["W4"] = _ternary(rng, H_HEADS, HIDDEN)
+    else:
+        p["W4"] = rng.normal(0.0, 1.0 / np.sqrt(HIDDEN), (H_HEADS, HIDDEN))
     p["b4"] = rng.normal(0.0, 0.1, H_HEADS)
     return {k: np.ascontiguousarray(v, dtype=np.float32) for k, v in p.items()}
 
@@ -140,19 +160,20 @@ def make_params(rng) -> Dict[str, np.ndarray]:
 def make_jets(*, N: int, P: int, layout: str = "padded", dist: str = "poisson",
               mult_lo: int = 2, mult_hi: Optional[int] = None, lam: float = 40.0,
               pt_lo: float = 500.0, pt_hi: float = 550.0, prongs: int = 1,
-              mask_mode: str = "prefix", seed: int = 0, mults=None) -> JetBatch:
+              mask_mode: str = "prefix", seed: int = 0, mults=None, weights: str = "gaussian") -> JetBatch:
     """Draw one batch of jets, MLP parameters and Q/K/V from PCG64(seed).
 
     ``mask_mode="prefix"`` puts the m valid particles in slots 0..m-1;
     ``"scrambled"`` places them in m random slots of the P (padded only).
-    ``mults`` fixes the multiplicity of every jet instead of drawing it.
+    ``mults`` fixes the multiplicity of every jet instead of drawing it;
+    ``weights`` selects Gaussian or ternary hidden-layer weights (make_params).
     Draw order: parameters, multiplicities, per-jet kinematics, slot
     permutations, Q, K, V.
     """
     if mult_hi is None:
         mult_hi = P
     rng = np.random.Generator(np.random.PCG64(seed))
-    params = make_params(rng)
+    params = make_params(rng, weights)
     mult = _multiplicities(rng, N, dist, mult_lo, mult_hi, lam, mults)
     kin = [_constituents(rng, int(m), pt_lo, pt_hi, prongs) for m in mult]
 
