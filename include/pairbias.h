@@ -145,6 +145,29 @@ typedef struct {
   float *W4, *b4;  /* [8][64], [8]    */
 } pb_mlp_grad;
 
+/* The MLP with int8 inputs to its hidden layers ("Economical Jet Taggers",
+ * section "Kwantiseringsstrategieen": the inputs of linear layers are int8
+ * with zero-point quantisation, the weights binary or ternary). Device
+ * pointers. Layer 1 keeps its fp32 weights (W1, b1 as in pb_mlp, folded);
+ * layers 2, 3 and 4 hold int8 weight codes T (row-major [out][in], 16-byte
+ * aligned: 64x64, 64x64, 8x64) and one fp32 scale per output row, so that
+ * the folded weight is alpha_o * T_oi; b2, b3, b4 are the folded fp32
+ * biases. pb_quantize_mlp_i8 makes T and alpha from pb_fold_affine's output
+ * (exactly, for weights that are a per-row scale times {-1, 0, +1}). */
+typedef struct pb_mlp_i8 {
+  const float *W1, *b1;             /* [64][4], [64]                   */
+  const int8_t *T2, *T3, *T4;       /* [64][64], [64][64], [8][64]      */
+  const float *a2, *a3, *a4;        /* [64], [64], [8] row scales       */
+  const float *b2, *b3, *b4;        /* [64], [64], [8] folded biases    */
+} pb_mlp_i8;
+
+/* Offsets inside the buffers that pb_quantize_mlp_i8 writes: codes
+ * (PB_I8_CODES int8 values) and alpha (PB_I8_ALPHAS floats). */
+enum {
+  PB_I8_T2 = 0, PB_I8_T3 = 4096, PB_I8_T4 = 8192, PB_I8_CODES = 8704,
+  PB_I8_A2 = 0, PB_I8_A3 = 64, PB_I8_A4 = 128, PB_I8_ALPHAS = 136
+};
+
 /* pairfeat_compute -- the four pair features of every slot pair.
  * feat: fp32 [N, P, P, 4], channel order (ln kT, ln z, ln dR, ln m^2);
  * feat[n, i, j] == feat[n, j, i] bit for bit; pairs with a masked (or, packed,
@@ -177,6 +200,36 @@ pb_status pair_attention_forward(const pb_jets *jets, const pb_mlp *mlp, const u
                                  int H, int D, const uint16_t *q, const uint16_t *k,
                                  const uint16_t *v, uint16_t *out, void *workspace,
                                  size_t workspace_bytes, void *stream);
+
+/* pairbias_mlp_forward_i8 -- pairbias_mlp_forward with the int8 MLP
+ * (pb_mlp_i8). Per pair row: y1 = W1 f + b1 (f16 hi + lo operands, fp32
+ * accumulation); for each of layers 2, 3 and 4 the 64 inputs h of the row
+ * (h = GELU(y) of the layer before, erf form, fp32) are quantised on their
+ * own: lo = min(0, min h), hi = max(0, max h), s = (hi - lo) / 255 (1 if
+ * hi == lo), z = -128 - rint(lo / s), q = clamp(rint(h / s) + z, -128, 127)
+ * (rint rounds half to even); the layer runs on int8 tensor cores (s32
+ * accumulation) and y_o = alpha_o s (sum_i T_oi q_i - z sum_i T_oi) + b_o in
+ * fp32. U as in pairbias_mlp_forward. Codes near a rounding boundary may
+ * land on the other side than in exact arithmetic (one quantisation step).
+ * Source: "Fusion 2" with the quantisation of "Economical Jet Taggers". */
+pb_status pairbias_mlp_forward_i8(const pb_jets *jets, const pb_mlp_i8 *mlp, void *U, pb_dtype dtype,
+                                  void *stream);
+
+/* pair_attention_forward_i8 -- the fused path of pair_attention_forward
+ * with the int8 MLP (arithmetic of pairbias_mlp_forward_i8), one CTA per jet
+ * at a time, the bias kept in shared memory. Arguments and errors as
+ * pair_attention_forward with mlp given and no workspace. */
+pb_status pair_attention_forward_i8(const pb_jets *jets, const pb_mlp_i8 *mlp, int H, int D,
+                                    const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                    uint16_t *out, void *stream);
+
+/* pb_quantize_mlp_i8 -- host helper, not on the GPU path: per output row of
+ * the folded W2, W3 and W4 (pb_fold_affine's buffer, PB_OFF_* layout),
+ * alpha = max |w| / 127 (1 for a zero row) and codes round(w / alpha), in
+ * double. codes: host buffer of PB_I8_CODES int8 (PB_I8_T* offsets);
+ * alpha: host buffer of PB_I8_ALPHAS floats (PB_I8_A* offsets). Returns
+ * PB_EINVAL for a NULL pointer. */
+pb_status pb_quantize_mlp_i8(const float *folded, int8_t *codes, float *alpha);
 
 /* pb_workspace_bytes -- size of the optional workspace of the fused path.
  * With a workspace of at least this size (device memory, 256-byte aligned,

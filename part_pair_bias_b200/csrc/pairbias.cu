@@ -61,7 +61,7 @@ pb_status device_sms(int* dev_out, int* sms_out) {
 // Resident CTAs per SM of a kernel instance on a device, found once (the
 // shared-memory attribute is raised at the same time) and cached, so that a
 // launch costs no runtime queries after the first.
-constexpr int kMaxKernels = 32;
+constexpr int kMaxKernels = 64;
 struct KernelFacts {
   const void* fn = nullptr;
   int per_sm[kMaxDev] = {};
@@ -144,6 +144,16 @@ pb_status check_mlp(const pb_mlp* w, pb::MlpArgs* out) {
   return PB_OK;
 }
 
+pb_status check_mlp_i8(const pb_mlp_i8* w, pb::MlpI8Args* out) {
+  if (!w) return fail(PB_EINVAL, "mlp is NULL");
+  if (!w->W1 || !w->b1 || !w->T2 || !w->T3 || !w->T4 || !w->a2 || !w->a3 || !w->a4 || !w->b2 || !w->b3 || !w->b4)
+    return fail(PB_EINVAL, "an int8 MLP parameter pointer is NULL");
+  if (!aligned(w->T2, 16) || !aligned(w->T3, 16) || !aligned(w->T4, 16))
+    return fail(PB_EINVAL, "the weight code arrays must be 16-byte aligned");
+  *out = pb::MlpI8Args{w->W1, w->b1, w->T2, w->T3, w->T4, w->a2, w->a3, w->a4, w->b2, w->b3, w->b4};
+  return PB_OK;
+}
+
 constexpr int kGroups = 4;  // tensor-core tile groups per CTA (128 threads each)
 
 template <int PM>
@@ -157,9 +167,9 @@ pb_status run_pairfeat(const pb::JetArgs& J, float* feat, cudaStream_t s) {
   return launched("k_pairfeat");
 }
 
-template <int PM, bool F32>
-pb_status run_mlp_bias(const pb::JetArgs& J, const pb::MlpArgs& W, void* U, cudaStream_t s) {
-  auto k = pb::k_mlp_bias<PM, kGroups, F32>;
+template <int PM, bool F32, class WA = pb::MlpArgs>
+pb_status run_mlp_bias(const pb::JetArgs& J, const WA& W, void* U, cudaStream_t s) {
+  auto k = pb::k_mlp_bias<PM, kGroups, F32, WA>;
   const size_t smem = sizeof(pb::MlpBiasSmem<PM, kGroups>);
   int grid = 0;
   pb_status st = prepare(k, smem, kGroups * 128, J.N, &grid);
@@ -179,10 +189,10 @@ pb_status run_attn_bias(const pb::JetArgs& J, const pb::QkvArgs& X, const uint16
   return launched("k_attn_bias");
 }
 
-template <int PM, bool kProj = false>
-pb_status run_fused(const pb::JetArgs& J, const pb::MlpArgs& W, const pb::QkvArgs& X, cudaStream_t s,
+template <int PM, bool kProj = false, class WA = pb::MlpArgs>
+pb_status run_fused(const pb::JetArgs& J, const WA& W, const pb::QkvArgs& X, cudaStream_t s,
                     const pb::ProjArgs& Pin = pb::ProjArgs{}, const pb::ProjArgs& Pout = pb::ProjArgs{}) {
-  auto k = pb::k_fused<PM, kGroups, kProj>;
+  auto k = pb::k_fused<PM, kGroups, kProj, WA>;
   const size_t smem = sizeof(pb::FusedSmem<PM, kGroups>);
   int grid = 0;
   pb_status st = prepare(k, smem, kGroups * 128, J.N, &grid);
@@ -438,6 +448,56 @@ pb_status pairbias_mlp_forward(const pb_jets* jets, const pb_mlp* mlp, void* U, 
   if (dtype == PB_F32)
     return J.P <= 128 ? run_mlp_bias<128, true>(J, W, U, s) : run_mlp_bias<256, true>(J, W, U, s);
   return J.P <= 128 ? run_mlp_bias<128, false>(J, W, U, s) : run_mlp_bias<256, false>(J, W, U, s);
+}
+
+pb_status pairbias_mlp_forward_i8(const pb_jets* jets, const pb_mlp_i8* mlp, void* U, pb_dtype dtype,
+                                  void* stream) {
+  pb::JetArgs J;
+  pb::MlpI8Args W;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK || J.N == 0) return st;
+  if ((st = check_mlp_i8(mlp, &W)) != PB_OK) return st;
+  if (!U || !aligned(U, 16)) return fail(PB_EINVAL, "U must be a non-NULL 16-byte aligned pointer");
+  if (dtype != PB_BF16 && dtype != PB_F32) return fail(PB_EINVAL, "dtype %d is not PB_BF16 or PB_F32", (int)dtype);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == PB_F32)
+    return J.P <= 128 ? run_mlp_bias<128, true>(J, W, U, s) : run_mlp_bias<256, true>(J, W, U, s);
+  return J.P <= 128 ? run_mlp_bias<128, false>(J, W, U, s) : run_mlp_bias<256, false>(J, W, U, s);
+}
+
+pb_status pair_attention_forward_i8(const pb_jets* jets, const pb_mlp_i8* mlp, int H, int D, const uint16_t* q,
+                                    const uint16_t* k, const uint16_t* v, uint16_t* out, void* stream) {
+  pb::JetArgs J;
+  pb::MlpI8Args W;
+  pb_status st = check_jets(jets, &J);
+  if (st != PB_OK) return st;
+  if (H != pb::kH || D != pb::kD) return fail(PB_EUNSUPPORTED, "H = %d, D = %d; only H = 8, D = 16", H, D);
+  if ((st = check_mlp_i8(mlp, &W)) != PB_OK) return st;
+  if (J.N == 0) return PB_OK;
+  if (!q || !k || !v || !out) return fail(PB_EINVAL, "q, k, v and out must be non-NULL");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return fail(PB_EINVAL, "q, k, v and out must be 16-byte aligned");
+  const pb::QkvArgs X{q, k, v, out};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return J.P <= 128 ? run_fused<128, false>(J, W, X, s) : run_fused<256, false>(J, W, X, s);
+}
+
+pb_status pb_quantize_mlp_i8(const float* folded, int8_t* codes, float* alpha) {
+  if (!folded || !codes || !alpha) return fail(PB_EINVAL, "NULL argument");
+  struct Layer {
+    int off, rows, code_off, alpha_off;
+  } const L[3] = {{PB_OFF_W2, 64, PB_I8_T2, PB_I8_A2}, {PB_OFF_W3, 64, PB_I8_T3, PB_I8_A3},
+                  {PB_OFF_W4, 8, PB_I8_T4, PB_I8_A4}};
+  for (const Layer& l : L)
+    for (int r = 0; r < l.rows; ++r) {
+      const float* w = folded + l.off + r * 64;
+      double mx = 0.0;
+      for (int c = 0; c < 64; ++c) mx = fmax(mx, fabs((double)w[c]));
+      const double a = mx > 0.0 ? mx / 127.0 : 1.0;
+      for (int c = 0; c < 64; ++c) codes[l.code_off + r * 64 + c] = (int8_t)nearbyint((double)w[c] / a);
+      alpha[l.alpha_off + r] = (float)a;
+    }
+  return PB_OK;
 }
 
 size_t pb_workspace_bytes(const pb_jets* jets) {

@@ -14,6 +14,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "pb_device.cuh"
 
 namespace pb {
@@ -32,6 +34,16 @@ struct JetArgs {
 
 struct MlpArgs {
   const float *W1, *b1, *W2, *b2, *W3, *b3, *W4, *b4;
+};
+
+// The MLP with int8 inputs to layers 2..4: layer 1 as MlpArgs (fp32,
+// folded); layers 2..4 as int8 weight codes T (row-major [out][in]), one
+// fp32 scale alpha per output row (W' = alpha T) and the folded fp32 bias.
+struct MlpI8Args {
+  const float *W1, *b1;
+  const int8_t *T2, *T3, *T4;
+  const float *a2, *a3, *a4;
+  const float *b2, *b3, *b4;
 };
 
 struct QkvArgs {
@@ -662,6 +674,284 @@ __device__ bool mlp_pass(MlpSmem<NG, SL>& S, const Source& src, Sink& sink, uint
   return ok;
 }
 
+// ============================================== int8 engine (kind::i8)
+//
+// The variant of the MLP whose hidden layers take int8 inputs with zero
+// points and int8 weights ("Economical Jet Taggers", section
+// "Kwantiseringsstrategieen": inputs of linear layers int8 with zero-point
+// quantisation, weights binary or ternary). Per pair row:
+//   layer 1  y1 = W1 f + b1 as in the f16 engine (f16 hi + lo operands), but
+//            accumulated in fp32;
+//   hidden   h = GELU(y) in fp32 with erff (an approximation of GELU would
+//            move codes across rounding boundaries); the row's 64 values are
+//            quantised on their own: lo = min(0, min h), hi = max(0, max h),
+//            s = (hi - lo) / 255 (1 if hi == lo), z = -128 - rint(lo / s),
+//            q = clamp(rint(h / s) + z, -128, 127) (round half to even);
+//            the 64 codes go to TMEM as the next layer's A operand;
+//   layers 2..4  tcgen05.mma kind::i8 (s8 x s8 -> s32, K = 32 per MMA, A
+//            from TMEM, four codes per column; B, the weight codes, from
+//            shared memory); then y_o = alpha_o s (acc_o - z sum_i T_oi) +
+//            b_o in fp32, the zero-point term being an exact integer.
+// Shared memory: the f16 engine's W2 / W3 / W4 tiles hold instead the code
+// tiles (K-major, 16-byte core-matrix rows of 16 codes) and each layer's
+// alpha, bias and code row sums.
+
+constexpr int kI8TileBytes = 64 * 64;     // one 64 x 64 code tile
+constexpr int kI8Alpha = kI8TileBytes;    // byte offsets inside a layer's region
+constexpr int kI8Bias = kI8Alpha + 256;
+constexpr int kI8Tsum = kI8Bias + 256;
+constexpr int kI8W4Alpha = 16 * 64;       // layer 4: 16 code rows (8 used), then 8 + 8 + 8 values
+constexpr int kI8W4Bias = kI8W4Alpha + 32;
+constexpr int kI8W4Tsum = kI8W4Bias + 32;
+
+// Byte offset of code (row r, column k) of a K-major code tile with 64
+// columns: 8 x 16-byte core matrices, 4 along K per 8-row group.
+__device__ __forceinline__ int i8ofs(int r, int k) { return (((r >> 3) * 4 + (k >> 4)) << 7) + ((r & 7) << 4) + (k & 15); }
+
+// kind::i8 instruction descriptor: s8 A and B, both K-major, s32 D, M = 128.
+__host__ __device__ constexpr uint32_t idesc_i8_m128(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_i8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16_wait_u(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Once per CTA: layer 1 as in the f16 engine, the code tiles and per-row
+// constants of layers 2..4, mbarriers, TMEM.
+template <int NG, int SL>
+__device__ void mlp_setup_i8(MlpSmem<NG, SL>& S, const MlpI8Args& W) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  unsigned char* R2 = reinterpret_cast<unsigned char*>(S.W2);
+  unsigned char* R3 = reinterpret_cast<unsigned char*>(S.W3);
+  unsigned char* R4 = reinterpret_cast<unsigned char*>(S.W4);
+  for (int e = tid; e < 64 * 64 / 4; e += nthr) {  // 4 codes of one row at a time
+    const int r = e >> 4, k = (e & 15) * 4;
+    *reinterpret_cast<uint32_t*>(R2 + i8ofs(r, k)) = reinterpret_cast<const uint32_t*>(W.T2)[e];
+    *reinterpret_cast<uint32_t*>(R3 + i8ofs(r, k)) = reinterpret_cast<const uint32_t*>(W.T3)[e];
+    if (r < 16) *reinterpret_cast<uint32_t*>(R4 + i8ofs(r, k)) = r < 8 ? reinterpret_cast<const uint32_t*>(W.T4)[e] : 0u;
+  }
+  if (tid < 64) {
+    const int r = tid;
+    int s2 = 0, s3 = 0, s4 = 0;
+    for (int k = 0; k < 64; ++k) {
+      s2 += W.T2[r * 64 + k];
+      s3 += W.T3[r * 64 + k];
+      if (r < 8) s4 += W.T4[r * 64 + k];
+    }
+    reinterpret_cast<float*>(R2 + kI8Alpha)[r] = W.a2[r];
+    reinterpret_cast<float*>(R2 + kI8Bias)[r] = W.b2[r];
+    reinterpret_cast<int*>(R2 + kI8Tsum)[r] = s2;
+    reinterpret_cast<float*>(R3 + kI8Alpha)[r] = W.a3[r];
+    reinterpret_cast<float*>(R3 + kI8Bias)[r] = W.b3[r];
+    reinterpret_cast<int*>(R3 + kI8Tsum)[r] = s3;
+    if (r < 8) {
+      reinterpret_cast<float*>(R4 + kI8W4Alpha)[r] = W.a4[r];
+      reinterpret_cast<float*>(R4 + kI8W4Bias)[r] = W.b4[r];
+      reinterpret_cast<int*>(R4 + kI8W4Tsum)[r] = s4;
+    }
+    // layer-1 row r: [hi(W1) | lo(W1) | hi(W1) | hi(b1) lo(b1) 0 0] (K = 16)
+    __half h[4], l[4], bh, bl;
+    const float w1[4] = {W.W1[4 * r], W.W1[4 * r + 1], W.W1[4 * r + 2], W.W1[4 * r + 3]};
+    for (int i = 0; i < 4; ++i) split_half(w1[i], h[i], l[i]);
+    split_half(W.b1[r], bh, bl);
+    const __half z = __float2half_rn(0.f);
+    *reinterpret_cast<uint4*>(S.W1 + cofs(r, 0, 16)) =
+        make_uint4(h2bits(h[0], h[1]), h2bits(h[2], h[3]), h2bits(l[0], l[1]), h2bits(l[2], l[3]));
+    *reinterpret_cast<uint4*>(S.W1 + cofs(r, 8, 16)) =
+        make_uint4(h2bits(h[0], h[1]), h2bits(h[2], h[3]), h2bits(bh, bl), h2bits(z, z));
+  }
+  if (tid == 0) {
+    for (int i = 0; i < NG * SL; ++i) mbar_init(&S.mbar[i], 1);
+    fence_mbar_init();
+  }
+  if ((tid >> 5) == 0) tmem_alloc(&S.tmem_base, kTmemCols(NG, SL));
+  fence_proxy_async_smem();  // code and weight tiles are read by the tensor cores
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+__device__ __forceinline__ float gelu_erf(float y) { return 0.5f * y * (1.f + erff(y * 0.70710678118654752f)); }
+
+// The int8 variant of mlp_pass (same scheduling, sources and sinks).
+template <int NG, int SL, class Source, class Sink>
+__device__ bool mlp_pass_i8(MlpSmem<NG, SL>& S, const Source& src, Sink& sink, uint32_t* phase) {
+  const int g = threadIdx.x >> 7;
+  if (g >= NG) return true;
+  const int row = threadIdx.x & 127;
+  const uint32_t bar_id = 1 + g;
+  const bool leader = row == 0;
+  const unsigned char* const R2 = reinterpret_cast<const unsigned char*>(S.W2);
+  const unsigned char* const R3 = reinterpret_cast<const unsigned char*>(S.W3);
+  const unsigned char* const R4 = reinterpret_cast<const unsigned char*>(S.W4);
+  auto region = [&](int L) { return L == 1 ? R2 : (L == 2 ? R3 : R4); };  // layer L + 1's constants
+  const uint32_t w1_addr = smem_u32(S.W1);
+  constexpr uint32_t kIdL1 = idesc_f16_m128(64, true), kId64 = idesc_i8_m128(64), kId16 = idesc_i8_m128(16);
+  const int ntiles = src.ntiles();
+  uint64_t* const mbar = &S.mbar[g];
+  const uint32_t lane_off = (uint32_t)(row & 96) << 16;
+  const uint32_t t_d = S.tmem_base + (uint32_t)(g * kSlotCols);
+  const uint32_t t_a = t_d + kSlotA;
+  bool ok = true;
+
+  auto issue = [&](int L) -> bool {
+    tc_fence_before();
+    if (named_bar_or(bar_id, 128, !ok)) return false;
+    if (leader) {
+      tc_fence_after();
+      if (L == 0) {
+        mma_f16_ta(t_d, t_a, smem_desc(w1_addr, 128, 256), kIdL1, 0u);
+      } else {
+        const uint32_t w = smem_u32(region(L));
+        const uint32_t id = L == 3 ? kId16 : kId64;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) mma_i8_ta(t_d, t_a + 8u * k, smem_desc(w + 256u * k, 128, 512), id, k);
+      }
+      mma_commit(mbar);
+    }
+    return true;
+  };
+  auto wait = [&]() {
+    const bool done = mbar_wait(mbar, *phase & 1u);
+    ok = ok && done;
+    *phase ^= 1u;
+    tc_fence_after();
+  };
+  // y of one output column o of layer L (1..3: hidden; the accumulator word
+  // is fp32 for layer 1, s32 for the others) from the row's scale and zero point
+  auto dequant = [&](int L, int o, uint32_t accw, float s, int z) -> float {
+    if (L == 0) return __uint_as_float(accw);
+    const unsigned char* Rl = region(L);
+    const bool last = L == 3;
+    const float al = reinterpret_cast<const float*>(Rl + (last ? kI8W4Alpha : kI8Alpha))[o];
+    const float bi = reinterpret_cast<const float*>(Rl + (last ? kI8W4Bias : kI8Bias))[o];
+    const int ts = reinterpret_cast<const int*>(Rl + (last ? kI8W4Tsum : kI8Tsum))[o];
+    const int d = (int)accw - z * ts;
+    return fmaf((float)d, al * s, bi);
+  };
+  // Layer L's accumulators -> GELU -> int8 codes of the next layer's input;
+  // the row's new scale and zero point replace (s, z).
+  auto hidden = [&](int L, float& s, int& z) {
+    float h[64];
+    {
+      uint32_t w[64];
+      tmem_ld64_wait(t_d + lane_off, reinterpret_cast<float*>(w));
+#pragma unroll
+      for (int o = 0; o < 64; ++o) h[o] = gelu_erf(dequant(L, o, w[o], s, z));
+    }
+    float lo = 0.f, hi = 0.f;
+#pragma unroll
+    for (int o = 0; o < 64; ++o) {
+      lo = fminf(lo, h[o]);
+      hi = fmaxf(hi, h[o]);
+    }
+    const float sn = hi > lo ? (hi - lo) / 255.f : 1.f;
+    const float inv = 1.f / sn;
+    const int zn = -128 - __float2int_rn(lo / sn);
+    uint32_t codes[16];
+#pragma unroll
+    for (int w4 = 0; w4 < 16; ++w4) {
+      int c[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) c[j] = max(-128, min(127, __float2int_rn(h[4 * w4 + j] * inv) + zn));
+      codes[w4] = (uint32_t)(c[0] & 255) | ((uint32_t)(c[1] & 255) << 8) | ((uint32_t)(c[2] & 255) << 16) |
+                  ((uint32_t)(c[3] & 255) << 24);
+    }
+    tmem_st16_wait_u(t_a + lane_off, codes);
+    s = sn;
+    z = zn;
+  };
+  auto features = [&](int t, uint32_t* a1, int& p_out, int& a_out, int& b_out) {
+    int p = -1, a = 0, b = 0;
+    float f[4] = {0.f, 0.f, 0.f, 0.f};
+    const bool valid = src.row(t, row, p, a, b, f);
+    if (!valid) {
+      f[0] = f[1] = f[2] = f[3] = 0.f;
+      a = b = 0;
+    }
+    p_out = valid ? p : -1;
+    a_out = a;
+    b_out = b;
+    __half hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split_half(f[i], hi[i], lo[i]);
+    const __half one = __float2half_rn(valid ? 1.f : 0.f), zero = __float2half_rn(0.f);
+    a1[0] = h2bits(hi[0], hi[1]);
+    a1[1] = h2bits(hi[2], hi[3]);
+    a1[2] = a1[0];
+    a1[3] = a1[1];
+    a1[4] = h2bits(lo[0], lo[1]);
+    a1[5] = h2bits(lo[2], lo[3]);
+    a1[6] = h2bits(one, one);
+    a1[7] = h2bits(zero, zero);
+  };
+
+  uint32_t a1[8];
+  int pk = -1, pa = 0, pb = 0, qk = -1, qa = 0, qb = 0;
+  float u[8];
+  int t = g;
+  if (t < ntiles) features(t, a1, pk, pa, pb);
+#pragma unroll 1
+  while (t < ntiles) {
+    tmem_st8_wait(t_a + lane_off, a1);
+    if (!issue(0)) return false;
+    if (qk >= 0) sink(qk, qa, qb, u);
+    float s = 1.f;
+    int z = 0;
+#pragma unroll 1
+    for (int L = 0; L < 3; ++L) {
+      wait();
+      hidden(L, s, z);
+      if (!issue(L + 1)) return false;
+    }
+    const int ck = pk, ca = pa, cb = pb;
+    t += NG;
+    if (t < ntiles) features(t, a1, pk, pa, pb);
+    wait();
+    {
+      float w[8];
+      tmem_ld8_wait(t_d + lane_off, w);
+#pragma unroll
+      for (int o = 0; o < 8; ++o) u[o] = dequant(3, o, __float_as_uint(w[o]), s, z);
+    }
+    qk = ck;
+    qa = ca;
+    qb = cb;
+  }
+  if (qk >= 0) sink(qk, qa, qb, u);
+  tc_fence_before();
+  return ok;
+}
+
+// The engine of a weight-argument type: f16 (MlpArgs) or int8 (MlpI8Args).
+template <int NG, int SL>
+__device__ void mlp_setup_any(MlpSmem<NG, SL>& S, const MlpArgs& W) { mlp_setup<NG, SL>(S, W); }
+template <int NG, int SL>
+__device__ void mlp_setup_any(MlpSmem<NG, SL>& S, const MlpI8Args& W) { mlp_setup_i8<NG, SL>(S, W); }
+
+template <class WA, int NG, int SL, class Source, class Sink>
+__device__ bool mlp_run(MlpSmem<NG, SL>& S, const Source& src, Sink& sink, uint32_t* phase) {
+  if constexpr (std::is_same<WA, MlpI8Args>::value) return mlp_pass_i8<NG, SL>(S, src, sink, phase);
+  else return mlp_pass<NG, SL>(S, src, sink, phase);
+}
+
 // ----------------------------------------------- k_mlp_bias (materialised U)
 
 template <int PM, bool F32OUT>
@@ -710,11 +1000,11 @@ struct MlpBiasSmem {
   Particles<PM> part;
 };
 
-template <int PM, int NG, bool F32OUT>
-__global__ void __launch_bounds__(NG * 128, 1) k_mlp_bias(JetArgs J, MlpArgs W, void* __restrict__ U) {
+template <int PM, int NG, bool F32OUT, class WA = MlpArgs>
+__global__ void __launch_bounds__(NG * 128, 1) k_mlp_bias(JetArgs J, WA W, void* __restrict__ U) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   MlpBiasSmem<PM, NG>& S = *reinterpret_cast<MlpBiasSmem<PM, NG>*>(smem_raw);
-  mlp_setup<NG, 2>(S.mlp, W);
+  mlp_setup_any<NG, 2>(S.mlp, W);
   uint32_t phase = 0u;
   bool aborted = false;
   for (int n = blockIdx.x; n < J.N; n += gridDim.x) {
@@ -722,7 +1012,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_mlp_bias(JetArgs J, MlpArgs W, 
     zero_masked_pairs<PM, F32OUT>(S.part, U, n, J.P);
     const int m = S.part.m;
     GlobalUSink<PM, F32OUT> sink{&S.part, U, n, J.P};
-    const bool ok = mlp_pass<NG, 2>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, m * (m + 1) / 2, TriPairs{}}, sink, &phase);
+    const bool ok = mlp_run<WA, NG, 2>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, m * (m + 1) / 2, TriPairs{}}, sink, &phase);
     aborted = __syncthreads_or(!ok) != 0;
     if (aborted) break;
   }
@@ -1696,8 +1986,8 @@ struct FusedSmem {
 // kProj: the jet's Q, K, V (X.q/k/v) are first computed from its embeddings
 // (Pin: x, Wqkv, bqkv) and its output O (X.out) is finally projected to y
 // (Pout: O, Wo, bo); see "per-jet projections inside k_fused" above.
-template <int PM, int NG, bool kProj>
-__global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, QkvArgs X, ProjArgs Pin,
+template <int PM, int NG, bool kProj, class WA = MlpArgs>
+__global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, WA W, QkvArgs X, ProjArgs Pin,
                                                        ProjArgs Pout) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FusedSmem<PM, NG>& S = *reinterpret_cast<FusedSmem<PM, NG>*>(smem_raw);
@@ -1709,11 +1999,16 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
       fence_mbar_init();  // made visible by the barrier at the end of mlp_setup
     }
   }
-  // the weights' loads are in flight while the first jet is staged
-  WeightRegs wr;
-  wr.load(W);
-  if (blockIdx.x < J.N) stage_jet<PM>(S.part, J, blockIdx.x);
-  mlp_setup<MG, SL>(S.mlp, wr);
+  if constexpr (std::is_same<WA, MlpArgs>::value) {
+    // the weights' loads are in flight while the first jet is staged
+    WeightRegs wr;
+    wr.load(W);
+    if (blockIdx.x < J.N) stage_jet<PM>(S.part, J, blockIdx.x);
+    mlp_setup<MG, SL>(S.mlp, wr);
+  } else {
+    if (blockIdx.x < J.N) stage_jet<PM>(S.part, J, blockIdx.x);
+    mlp_setup_i8<MG, SL>(S.mlp, W);
+  }
   // during attention the activation tiles hold K and V
   float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
   constexpr int kStageFloats = MG * SL * kTileM * kAK / 2;
@@ -1779,7 +2074,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
         early = reinterpret_cast<uint16_t*>(S.U8 + np);
         stage_kv16<PM>(S.part, J, X, n, 0, kH, early);
       }
-      const bool ok = mlp_pass<MG, SL>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, np, TriPairs{}}, sink, &phase);
+      const bool ok = mlp_run<WA, MG, SL>(S.mlp, JetTiles<PM, TriPairs, true>{&S.part, np, TriPairs{}}, sink, &phase);
       aborted = __syncthreads_or(!ok) != 0;
       if (aborted) {
         if (early) cp_async_wait_all();
@@ -1791,7 +2086,7 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, MlpArgs W, Qkv
       const int qb = kUCap / m;
       for (int i0 = 0; i0 < m; i0 += qb) {
         const int i1 = min(m, i0 + qb);
-        const bool ok = mlp_pass<MG, SL>(S.mlp, JetTiles<PM, RectPairs, true>{&S.part, (i1 - i0) * m, RectPairs{i0, m}}, sink, &phase);
+        const bool ok = mlp_run<WA, MG, SL>(S.mlp, JetTiles<PM, RectPairs, true>{&S.part, (i1 - i0) * m, RectPairs{i0, m}}, sink, &phase);
         aborted = __syncthreads_or(!ok) != 0;
         if (aborted) break;
         RectUBias ub{reinterpret_cast<const __half*>(S.U8), i0, m};

@@ -7,8 +7,9 @@ on first use and its absence is an error -- there is no fallback.
 Entry points mirror ``include/pairbias.h``: ``pairfeat_compute``,
 ``pairbias_mlp_forward``, ``pair_attention_forward``,
 ``pair_attention_forward_noalloc``, ``pair_block_forward``,
-``pair_attention_backward``, ``get_device_status`` and the host helpers
-``fold_affine`` and ``unfold_grad``.
+``pair_attention_backward``, the int8 variants ``pairbias_mlp_forward_i8``
+and ``pair_attention_forward_i8``, ``get_device_status`` and the host
+helpers ``fold_affine``, ``unfold_grad`` and ``quantize_mlp_i8``.
 """
 from __future__ import annotations
 
@@ -40,6 +41,10 @@ UNFOLDED_OFFSETS = dict(a0=(0, (4,)), c0=(4, (4,)), W1=(8, (64, 4)), b1=(264, (6
                         c2=(4680, (64,)), W3=(4744, (64, 64)), b3=(8840, (64,)), a3=(8904, (64,)),
                         c3=(8968, (64,)), W4=(9032, (8, 64)), b4=(9544, (8,)))
 UNFOLDED_FLOATS = 9552
+# offsets of pb_quantize_mlp_i8's outputs (PB_I8_* in the header)
+I8_CODES, I8_ALPHAS = 8704, 136
+I8_CODE_OFFSETS = dict(T2=(0, (64, 64)), T3=(4096, (64, 64)), T4=(8192, (8, 64)))
+I8_ALPHA_OFFSETS = dict(a2=(0, 64), a3=(64, 64), a4=(128, 8))
 
 
 class PairBiasError(RuntimeError):
@@ -60,6 +65,10 @@ class _Mlp(C.Structure):
 
 class _Proj(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("Wqkv", "bqkv", "Wo", "bo")]
+
+
+class _MlpI8(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("W1", "b1", "T2", "T3", "T4", "a2", "a3", "a4", "b2", "b3", "b4")]
 
 
 class _MlpUnfolded(C.Structure):
@@ -127,9 +136,14 @@ def load(path: str):
     L.pb_backward_workspace_bytes.argtypes = [C.POINTER(_Jets)]
     L.pb_backward_workspace_bytes.restype = C.c_size_t
     L.pb_unfold_grad.argtypes = [C.POINTER(_MlpUnfolded), C.POINTER(C.c_float), C.POINTER(C.c_float)]
+    L.pb_quantize_mlp_i8.argtypes = [C.POINTER(C.c_float), C.POINTER(C.c_int8), C.POINTER(C.c_float)]
+    L.pairbias_mlp_forward_i8.argtypes = [C.POINTER(_Jets), C.POINTER(_MlpI8), vp, C.c_int, vp]
+    L.pair_attention_forward_i8.argtypes = [C.POINTER(_Jets), C.POINTER(_MlpI8), C.c_int, C.c_int, vp, vp, vp, vp,
+                                            vp]
     for f in (L.pairfeat_compute, L.pairbias_mlp_forward, L.pair_attention_forward, L.pb_selftest_wait_timeouts,
               L.pair_attention_forward_noalloc, L.pair_block_forward, L.pb_get_device_status,
-              L.pb_fold_affine, L.pair_attention_backward, L.pb_unfold_grad):
+              L.pb_fold_affine, L.pair_attention_backward, L.pb_unfold_grad, L.pb_quantize_mlp_i8,
+              L.pairbias_mlp_forward_i8, L.pair_attention_forward_i8):
         f.restype = C.c_int
     return L
 
@@ -212,6 +226,63 @@ def fold_affine(params: Dict[str, np.ndarray]) -> np.ndarray:
 
 def folded_mlp(params: Dict[str, np.ndarray], device="cuda") -> FoldedMLP:
     return FoldedMLP(torch.from_numpy(fold_affine(params)).to(device))
+
+
+@dataclass
+class MlpI8:
+    """The int8 MLP (see pb_mlp_i8 in the header): the folded fp32 buffer
+    (for W1, b1 and the biases) plus the int8 weight codes and row scales of
+    layers 2..4, all on the device."""
+
+    flat: torch.Tensor
+    codes: torch.Tensor
+    alpha: torch.Tensor
+
+    def struct(self) -> _MlpI8:
+        f, c, a = self.flat.data_ptr(), self.codes.data_ptr(), self.alpha.data_ptr()
+        return _MlpI8(W1=f + 4 * FOLDED_OFFSETS["W1"][0], b1=f + 4 * FOLDED_OFFSETS["b1"][0],
+                      T2=c + I8_CODE_OFFSETS["T2"][0], T3=c + I8_CODE_OFFSETS["T3"][0],
+                      T4=c + I8_CODE_OFFSETS["T4"][0], a2=a + 4 * I8_ALPHA_OFFSETS["a2"][0],
+                      a3=a + 4 * I8_ALPHA_OFFSETS["a3"][0], a4=a + 4 * I8_ALPHA_OFFSETS["a4"][0],
+                      b2=f + 4 * FOLDED_OFFSETS["b2"][0], b3=f + 4 * FOLDED_OFFSETS["b3"][0],
+                      b4=f + 4 * FOLDED_OFFSETS["b4"][0])
+
+
+def quantize_mlp_i8(folded: np.ndarray):
+    """int8 codes (PB_I8_CODES) and row scales (PB_I8_ALPHAS) of the folded
+    layers 2..4 (host, C library)."""
+    f = np.ascontiguousarray(folded, np.float32)
+    assert f.size == FOLDED_FLOATS
+    codes = np.zeros(I8_CODES, np.int8)
+    alpha = np.zeros(I8_ALPHAS, np.float32)
+    _check(lib().pb_quantize_mlp_i8(f.ctypes.data_as(C.POINTER(C.c_float)), codes.ctypes.data_as(C.POINTER(C.c_int8)),
+                                    alpha.ctypes.data_as(C.POINTER(C.c_float))))
+    return codes, alpha
+
+
+def mlp_i8(params: Dict[str, np.ndarray], device="cuda") -> MlpI8:
+    folded = fold_affine(params)
+    codes, alpha = quantize_mlp_i8(folded)
+    to = lambda a: torch.from_numpy(a).to(device)  # noqa: E731
+    return MlpI8(to(folded), to(codes), to(alpha))
+
+
+def pairbias_mlp_forward_i8(jets: Jets, mlp: MlpI8, U: torch.Tensor, stream=None) -> None:
+    """U (bfloat16 or float32 [N, 8, P, P]) with the int8 MLP."""
+    assert U.is_contiguous() and U.dtype in (torch.bfloat16, torch.float32)
+    js, ms = jets.struct(), mlp.struct()
+    dtype = PB_F32 if U.dtype == torch.float32 else PB_BF16
+    _check(lib().pairbias_mlp_forward_i8(C.byref(js), C.byref(ms), U.data_ptr(), dtype, _stream(stream)))
+
+
+def pair_attention_forward_i8(jets: Jets, mlp: MlpI8, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              out: torch.Tensor, stream=None) -> None:
+    """The fused path with the int8 MLP; bf16 q/k/v/out."""
+    for t in (q, k, v, out):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    js, ms = jets.struct(), mlp.struct()
+    _check(lib().pair_attention_forward_i8(C.byref(js), C.byref(ms), H, D, q.data_ptr(), k.data_ptr(),
+                                           v.data_ptr(), out.data_ptr(), _stream(stream)))
 
 
 def jets_to_device(b, device="cuda") -> Jets:

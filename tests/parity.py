@@ -114,6 +114,37 @@ def check_jet_heads(got, ref, b, rel_tol, outlier, floor=None):
     return worst
 
 
+I8_RELL2 = 1e-2      # the benchmark's U bar
+I8_AGREE = 1e-3      # a row with no code on the other side of a rounding boundary
+I8_AGREE_FRAC = 0.99
+I8_FLIP = 0.25       # a row with a few codes one step away
+
+
+def check_bias_i8(got, ref, b):
+    """U of the int8 variant against the int8 oracle. The quantiser is
+    discontinuous: where a pre-quantisation value lies within rounding of a
+    code boundary, the kernel and the oracle may pick neighbouring codes (one
+    step s = row range / 255 apart), which moves that row's outputs by about
+    alpha * s per code. So: relative L2 over valid pairs <= 1e-2; at least
+    99 % of valid pair rows within 1e-3 on all 8 heads (no such code); every
+    row within 0.25 (a few such codes); masked pairs 0; U[i,j] == U[j,i].
+    Returns (fraction of agreeing rows, largest row error, relative L2)."""
+    vp = valid_pairs(b)
+    g = np.moveaxis(got, 1, -1)[vp]      # [rows, 8]
+    o = np.moveaxis(ref, 1, -1)[vp]
+    rel = np.linalg.norm(g - o) / np.linalg.norm(o)
+    assert rel <= I8_RELL2, f"int8 U rel L2 {rel:.3e}"
+    row = np.abs(g - o).max(axis=1) if g.size else np.zeros(0)
+    frac = float(np.mean(row <= I8_AGREE)) if row.size else 1.0
+    assert frac >= I8_AGREE_FRAC, f"only {frac * 100:.2f} % of pair rows within {I8_AGREE}"
+    worst = float(row.max()) if row.size else 0.0
+    assert worst <= I8_FLIP, f"int8 U row error {worst:.3e} > {I8_FLIP}"
+    mask = np.broadcast_to(vp[:, None], got.shape)
+    assert np.all(got[~mask] == 0.0), "masked pairs of U must be 0"
+    assert np.array_equal(got, got.transpose(0, 1, 3, 2)), "U[i,j] != U[j,i]"
+    return frac, worst, float(rel)
+
+
 def check_attention(got, ref, b):
     """Attention output against the oracle: per (jet, head) relative L2 and
     element bounds, masked rows exactly 0. Returns the batch-wide relative
@@ -142,6 +173,7 @@ class Device:
         self.b = b
         self.jets = ops.jets_to_device(b, dev)
         self.mlp = ops.folded_mlp(b.params, dev)
+        self.mlp_i8 = ops.mlp_i8(b.params, dev)
         self.q, self.k, self.v = (ops.bf16_to_device(x, dev) for x in (b.q, b.k, b.v))
 
     def features(self):
@@ -165,6 +197,16 @@ class Device:
         if balanced:
             torch.cuda.synchronize()
             assert torch.all(ws[:256] == 0), "the workspace header must be left zero"
+        return out
+
+    def bias_i8(self, dtype=torch.float32):
+        U = torch.full((self.b.N, 8, self.b.P, self.b.P), float("nan"), device=self.q.device, dtype=dtype)
+        ops.pairbias_mlp_forward_i8(self.jets, self.mlp_i8, U)
+        return U
+
+    def fused_i8(self):
+        out = torch.full_like(self.q, float("nan"))
+        ops.pair_attention_forward_i8(self.jets, self.mlp_i8, self.q, self.k, self.v, out)
         return out
 
     def with_bias(self, U_bf16):

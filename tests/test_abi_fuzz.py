@@ -45,6 +45,8 @@ ENTRY_VIOLATIONS = {
               "xy_misaligned", "ws_null", "ws_misaligned", "ws_small"],
     "backward": ["hd_bad", "mlp_null", "dmlp_null", "dmlp_field_null", "dmlp_misaligned", "qkv_grad_null",
                  "qkv_grad_misaligned", "ws_null", "ws_misaligned", "ws_small"],
+    "mlp_forward_i8": ["mlp_null", "i8_field_null", "i8_codes_misaligned", "u_null", "u_misaligned", "dtype_bad"],
+    "attention_i8": ["hd_bad", "mlp_null", "i8_field_null", "i8_codes_misaligned", "qkvo_null", "qkvo_misaligned"],
 }
 
 
@@ -82,6 +84,18 @@ def _call(L, entry, jets, v):
     mlp_ref = None if mlp is None else C.byref(mlp)
     q, k, vv, out = (None if "qkvo_null" in v and i == 3 else mis(_ptr(12 + i), "qkvo_misaligned" in v and i == 1)
                      for i in range(4))
+    m8 = ops._MlpI8(*([_ptr(90 + i) for i in range(11)]))
+    if "i8_field_null" in v:
+        m8.a3 = None
+    if "i8_codes_misaligned" in v:
+        m8.T4 = _ptr(94) + 4
+    m8_ref = None if "mlp_null" in v else C.byref(m8)
+    if entry == "mlp_forward_i8":
+        U = None if "u_null" in v else mis(_ptr(20), "u_misaligned" in v)
+        return L.pairbias_mlp_forward_i8(jets, m8_ref, U, 5 if "dtype_bad" in v else 0, None)
+    if entry == "attention_i8":
+        H, D = (8, 8) if "hd_bad" in v else (8, 16)
+        return L.pair_attention_forward_i8(jets, m8_ref, H, D, q, k, vv, out, None)
     if entry == "pairfeat":
         return L.pairfeat_compute(jets, None if "feat_null" in v else mis(d, "feat_misaligned" in v), None)
     if entry == "mlp_forward":
