@@ -530,6 +530,11 @@ def run_sweep(args):
                           inp + qkv + 256 * slots, True))
         paths.append(("block", lambda: ops.pair_block_forward(jets, mlp, proj, x, y, bws),
                       inp + 256 * slots + 256 * slots, True))
+        mlp8 = ops.mlp_i8(b.params, dev)
+        paths.append(("bias_bf16_int8", lambda: ops.pairbias_mlp_forward_i8(jets, mlp8, U),
+                      inp + 2 * 8 * b.N * b.P * b.P, True))
+        paths.append(("fused_int8", lambda: ops.pair_attention_forward_i8(jets, mlp8, q, k, v, out),
+                      inp + qkv + 256 * slots, True))
         dout = ops.bf16_to_device(synth.make_upstream(b, args.seed), dev)
         dq, dk, dv = (torch.empty_like(q) for _ in range(3))
         grad = ops.MlpGrad(dev)

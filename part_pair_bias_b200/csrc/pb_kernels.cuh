@@ -137,7 +137,7 @@ __device__ void stage_jets(Particles<PM>* ring, const JetArgs& J, int K, const J
           S.px[c] = px;
           S.py[c] = py;
           S.pt[c] = (float)pt;
-          S.lnpt[c] = (float)log(pt);
+          S.lnpt[c] = logf((float)pt);
         }
       }
       if (t == 0) {
@@ -223,7 +223,7 @@ __device__ void stage_jet(Particles<PM>& S, const JetArgs& J, int n) {
       S.px[c] = px;
       S.py[c] = py;
       S.pt[c] = (float)pt;
-      S.lnpt[c] = (float)log(pt);
+      S.lnpt[c] = logf((float)pt);
     }
   }
   if (tid == 0) {
@@ -2249,7 +2249,10 @@ __device__ __forceinline__ int nonzero_bytes(uint32_t w) { return __popc(__vcmpn
 // Phase 0: the valid particles of every jet into T[1..N], all threads in
 // parallel (bounds of a packed jet as stage_jets checks them; a padded mask
 // read 16 bytes at a time when its rows allow it).
-__device__ void jet_counts(const JetArgs& J, int* T) {
+// With `ends` (padded layout), ends[n] receives one past the last slot that
+// may be valid: the end of jet n's last 16-slot chunk holding a valid slot
+// (exact on the byte-wise path), 0 for an empty jet.
+__device__ void jet_counts(const JetArgs& J, int* T, int* ends = nullptr) {
   const int tid = threadIdx.x, nthr = blockDim.x, N = J.N;
   if (J.ptr) {
 #pragma unroll 4
@@ -2259,7 +2262,10 @@ __device__ void jet_counts(const JetArgs& J, int* T) {
     }
     return;
   }
-  for (int n = tid; n < N; n += nthr) T[n + 1] = 0;
+  for (int n = tid; n < N; n += nthr) {
+    T[n + 1] = 0;
+    if (ends) ends[n] = 0;
+  }
   __syncthreads();
   if ((J.P & 15) == 0 && (reinterpret_cast<uintptr_t>(J.mask) & 15) == 0) {
     const int cpj = J.P >> 4;  // 16-byte chunks per jet
@@ -2269,14 +2275,31 @@ __device__ void jet_counts(const JetArgs& J, int* T) {
     for (int c = tid; c < nc; c += nthr) {
       const uint4 w = mk[c];
       const int k = nonzero_bytes(w.x) + nonzero_bytes(w.y) + nonzero_bytes(w.z) + nonzero_bytes(w.w);
-      if (k) atomicAdd(&T[c / cpj + 1], k);
+      if (k) {
+        atomicAdd(&T[c / cpj + 1], k);
+        if (ends) atomicMax(&ends[c / cpj], (c % cpj + 1) * 16);
+      }
     }
   } else {
     const int ne = N * J.P;
 #pragma unroll 4
     for (int e = tid; e < ne; e += nthr)
-      if (J.mask[e]) atomicAdd(&T[e / J.P + 1], 1);
+      if (J.mask[e]) {
+        atomicAdd(&T[e / J.P + 1], 1);
+        if (ends) atomicMax(&ends[e / J.P], e % J.P + 1);
+      }
   }
+}
+
+// This CTA's share (part of parts) of [base, base + bytes) into L2, in whole
+// 16-byte units; nothing for an array that is not 16-byte aligned. One thread.
+__device__ __forceinline__ void prefetch_slice(const void* base, size_t bytes, int part, int parts) {
+  if (reinterpret_cast<uintptr_t>(base) & 15) return;
+  const size_t chunk = ((bytes + parts - 1) / parts + 15) & ~(size_t)15;
+  const size_t lo = chunk * (size_t)part;
+  if (lo >= bytes) return;
+  const size_t n = (bytes - lo < chunk ? bytes - lo : chunk) & ~(size_t)15;
+  if (n) prefetch_l2(static_cast<const char*>(base) + lo, (uint32_t)n);
 }
 
 // kBiasOnly: phase 0 and phase A only (no barrier, no attention, counters
@@ -2613,8 +2636,9 @@ struct ClusterHead {
   int ib[kCJ + 1];       // prefix of each group jet's (head, query tile) items
   int jets[kCJ];         // this cluster's jets
   int cnt[kClusterMaxJets + 1];  // multiplicity of every jet of the batch (cnt[n + 1])
-  int order[kClusterMaxJets];    // jets by decreasing MLP tiles
+  int ends[kClusterMaxJets];     // padded: one past the last slot that may be valid
   int bin[kMaxJetTiles + 2];     // jets per tile count, then the next free rank of each
+  int order[kClusterMaxJets];    // jets by decreasing MLP tiles
 };
 
 template <int PM>
@@ -2674,6 +2698,13 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   constexpr int kUCap = ClusterSmem<PM>::kUCap;
   const int q = (int)cluster_ctarank();
   const int c = blockIdx.x / kCJ, ncl = gridDim.x / kCJ;
+  if (threadIdx.x == 0) {  // this CTA's slice of the momenta into L2, for the staging below
+    const size_t bytes = (J.ptr ? (size_t)J.tokens : (size_t)J.N * J.P) * 4;
+    prefetch_slice(J.E, bytes, blockIdx.x, gridDim.x);
+    prefetch_slice(J.px, bytes, blockIdx.x, gridDim.x);
+    prefetch_slice(J.py, bytes, blockIdx.x, gridDim.x);
+    prefetch_slice(J.pz, bytes, blockIdx.x, gridDim.x);
+  }
   WeightRegs wr;
   wr.load(W);  // in flight while the jets are counted and staged
   // Every CTA counts every jet and sorts them by MLP tiles, largest first,
@@ -2682,7 +2713,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   // 2 ncl + c, ... (a snake over the clusters), so the clusters' tile sums
   // come out close.
   for (int t = threadIdx.x; t < kMaxJetTiles + 2; t += blockDim.x) H.bin[t] = 0;
-  jet_counts(J, H.cnt);
+  jet_counts(J, H.cnt, J.ptr ? nullptr : H.ends);
   __syncthreads();
   auto jet_tiles = [&H](int n) {
     const int m = H.cnt[n + 1];
@@ -2745,6 +2776,23 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
     }
   }
   __syncthreads();
+  // the rows of Q, K and V this CTA attends (heads 2q, 2q + 1 of the
+  // cluster's jets) into L2: one thread per (jet, head, tensor); packed jets
+  // hold all heads of a row together, so CTA q takes tensor q there
+  if (threadIdx.x < kCJ * 2 * 3) {
+    const int k = threadIdx.x / 6, hh = (threadIdx.x / 3) & 1, tsel = threadIdx.x % 3;
+    const uint16_t* T = tsel == 0 ? X.q : (tsel == 1 ? X.k : X.v);
+    if (k < K) {
+      const int n = H.jets[k];
+      if (J.ptr) {
+        const long long lo = J.ptr[n], hi = J.ptr[n + 1];
+        if (hh == 0 && tsel == q && lo >= 0 && hi > lo && hi <= J.tokens)
+          prefetch_l2(T + (size_t)lo * kH * kD, (uint32_t)(hi - lo) * kH * kD * 2);
+      } else if (H.ends[n] > 0) {
+        prefetch_l2(T + ((size_t)n * kH + 2 * q + hh) * J.P * kD, (uint32_t)min(H.ends[n], J.P) * kD * 2);
+      }
+    }
+  }
   stage_jets<PM, true>(H.ring, J, K, [&H](int k) { return H.jets[k]; });
   mlp_setup<NG, SL>(H.mlp, wr);
   // groups of consecutive jets whose triangles fit together (identical in

@@ -278,3 +278,22 @@ def test_tiny_jets_elementwise(oracle_lib, P):
     pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
     pt.check_attention(pt.to_np(d.with_bias(d.bias(torch.bfloat16))), ref, b)
     assert ops.get_device_status() == 0
+
+
+def test_hybrid_lorentzpart_interaction_embed(oracle_lib):
+    """The hybrid Lorentz-equivariant ParT's pair-bias path (InteractionEmbed
+    [64, 64, 64], one output per head of 8): the same MLP shape on the same
+    four pair features with the hybrid model's own parameters, through the
+    bias, fused, balanced and int8 entry points."""
+    from part_pair_bias_b200 import configs as cf
+    e = cf.HYBRID_INTERACTION_EMBED
+    assert e["hidden"] == (64, 64, 64) and e["heads"] == ops.H and e["features"] == 4
+    b = synth.make_jets(**cf.workload("hybrid_n128_p128", seed=0))
+    assert b.params["W1"].shape == (64, 4) and b.params["W4"].shape == (8, 64)
+    d = pt.Device(b)
+    pt.check_bias(pt.to_np(d.bias()), oracle_lib.pair_bias(b), b)
+    ref = oracle_lib.forward(b)
+    pt.check_attention(pt.to_np(d.fused()), ref, b)
+    pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
+    pt.check_attention(pt.to_np(d.fused_i8()), oracle_lib.forward_i8(b), b)
+    assert ops.get_device_status() == 0
