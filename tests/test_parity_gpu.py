@@ -297,3 +297,18 @@ def test_hybrid_lorentzpart_interaction_embed(oracle_lib):
     pt.check_attention(pt.to_np(d.fused(balanced=True)), ref, b)
     pt.check_attention(pt.to_np(d.fused_i8()), oracle_lib.forward_i8(b), b)
     assert ops.get_device_status() == 0
+
+
+@pytest.mark.parametrize("N", [20, 300])
+def test_balanced_full_jets(oracle_lib, N):
+    """Full P = 128 jets on the balanced path: a jet's records and K/V do not
+    fit the stage together, so its attention reads the bias from the
+    records, the heads of one jet split over CTAs (N = 20) or whole jets per
+    CTA (N = 300)."""
+    b = synth.make_jets(N=N, P=128, dist="full", seed=41)
+    d = pt.Device(b)
+    got = pt.to_np(d.fused(balanced=True))
+    assert ops.get_device_status() == 0
+    lo, hi = (0, N) if N <= 20 else (N - 12, N)
+    s = synth.slice_jets(b, lo, hi)
+    pt.check_attention(got[lo:hi], oracle_lib.forward(s), s)
