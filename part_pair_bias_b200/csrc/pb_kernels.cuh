@@ -2249,10 +2249,7 @@ __device__ __forceinline__ int nonzero_bytes(uint32_t w) { return __popc(__vcmpn
 // Phase 0: the valid particles of every jet into T[1..N], all threads in
 // parallel (bounds of a packed jet as stage_jets checks them; a padded mask
 // read 16 bytes at a time when its rows allow it).
-// With `ends` (padded layout), ends[n] receives one past the last slot that
-// may be valid: the end of jet n's last 16-slot chunk holding a valid slot
-// (exact on the byte-wise path), 0 for an empty jet.
-__device__ void jet_counts(const JetArgs& J, int* T, int* ends = nullptr) {
+__device__ void jet_counts(const JetArgs& J, int* T) {
   const int tid = threadIdx.x, nthr = blockDim.x, N = J.N;
   if (J.ptr) {
 #pragma unroll 4
@@ -2262,10 +2259,7 @@ __device__ void jet_counts(const JetArgs& J, int* T, int* ends = nullptr) {
     }
     return;
   }
-  for (int n = tid; n < N; n += nthr) {
-    T[n + 1] = 0;
-    if (ends) ends[n] = 0;
-  }
+  for (int n = tid; n < N; n += nthr) T[n + 1] = 0;
   __syncthreads();
   if ((J.P & 15) == 0 && (reinterpret_cast<uintptr_t>(J.mask) & 15) == 0) {
     const int cpj = J.P >> 4;  // 16-byte chunks per jet
@@ -2275,19 +2269,13 @@ __device__ void jet_counts(const JetArgs& J, int* T, int* ends = nullptr) {
     for (int c = tid; c < nc; c += nthr) {
       const uint4 w = mk[c];
       const int k = nonzero_bytes(w.x) + nonzero_bytes(w.y) + nonzero_bytes(w.z) + nonzero_bytes(w.w);
-      if (k) {
-        atomicAdd(&T[c / cpj + 1], k);
-        if (ends) atomicMax(&ends[c / cpj], (c % cpj + 1) * 16);
-      }
+      if (k) atomicAdd(&T[c / cpj + 1], k);
     }
   } else {
     const int ne = N * J.P;
 #pragma unroll 4
     for (int e = tid; e < ne; e += nthr)
-      if (J.mask[e]) {
-        atomicAdd(&T[e / J.P + 1], 1);
-        if (ends) atomicMax(&ends[e / J.P], e % J.P + 1);
-      }
+      if (J.mask[e]) atomicAdd(&T[e / J.P + 1], 1);
   }
 }
 
@@ -2587,8 +2575,9 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
 // The fused path for batches of few jets, where one CTA per jet would wait
 // for the widest one: a thread-block cluster of 4 CTAs takes up to 4 jets
 // (the host deals the jets over as many clusters as run at once).
-//   - every CTA stages the cluster's jets; their MLP tiles are split evenly
-//     over the 4 CTAs (contiguous ranges of the cluster's tile list);
+//   - every CTA stages the cluster's jets; their unordered pairs, one jet
+//     after another, are packed into 128-row MLP tiles (no padding between
+//     jets), split evenly over the 4 CTAs (contiguous tile ranges);
 //   - a tile row's 8 biases go straight to the CTA that owns their heads:
 //     CTA q keeps heads 2q, 2q + 1 of every pair of the 4 jets, 4 bytes per
 //     pair, written through distributed shared memory (st.shared::cluster);
@@ -2598,7 +2587,8 @@ __host__ __device__ inline size_t grid_workspace_bytes(int N, int P, long long t
 // groups of them that fit run one after another (one P <= 128 jet always
 // fits). Cluster barriers are hardware barriers that every CTA reaches the
 // same number of times on every path (a CTA whose wait ran out still takes
-// them); the first one makes sure all 4 CTAs run before any remote store.
+// them); the first one makes sure all 4 CTAs run before any remote store:
+// each CTA arrives on it at its start and waits on it right before its MLP.
 
 constexpr int kCJ = 4;                // jets and CTAs per cluster
 constexpr int kClusterMaxJets = 256;  // batch size the jet table holds
@@ -2623,12 +2613,17 @@ __device__ __forceinline__ void cluster_sync_all() {
       "barrier.cluster.wait.acquire.aligned;" ::
           : "memory");
 }
+// The two halves of a cluster barrier that publishes nothing (it only tells
+// that every CTA of the cluster runs): arrive early, wait where it matters.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 template <int PM>
 struct ClusterHead {
   MlpSmem<4, 2> mlp;  // activation tiles double as the attention stage
   Particles<PM> ring[kCJ];
-  int tbeg[kCJ + 1];     // prefix of the jets' MLP tiles
   int tri_off[kCJ + 1];  // prefix of the jets' pairs
   int lo, hi;            // this CTA's tiles of the current group's list
   int G;                 // jets in the current group
@@ -2636,7 +2631,6 @@ struct ClusterHead {
   int ib[kCJ + 1];       // prefix of each group jet's (head, query tile) items
   int jets[kCJ];         // this cluster's jets
   int cnt[kClusterMaxJets + 1];  // multiplicity of every jet of the batch (cnt[n + 1])
-  int ends[kClusterMaxJets];     // padded: one past the last slot that may be valid
   int bin[kMaxJetTiles + 2];     // jets per tile count, then the next free rank of each
   int order[kClusterMaxJets];    // jets by decreasing MLP tiles
 };
@@ -2649,26 +2643,29 @@ struct ClusterSmem {
   alignas(16) uint32_t U[kUCap];  // heads 2q, 2q + 1 of every pair (f16x2), jet after jet; or 16-byte 8-head records
 };
 
-// The rows of this CTA's tiles of the cluster's 4 jets; the sink key is the
-// pair's index in the cluster's triangles.
+// The rows of this CTA's tiles of the group's jets: the jets' unordered
+// pairs one jet after another, packed into 128-row tiles without padding
+// between jets; the row's index there is also the sink key (the pair's index
+// in the group's triangles).
 template <int PM>
 struct ClusterTiles {
   const ClusterHead<PM>* H;
   int g0;  // the group's first jet
   __device__ __forceinline__ int ntiles() const { return H->hi - H->lo; }
   __device__ __forceinline__ bool row(int t, int r, int& p, int& a, int& b, float f[4]) const {
-    const int gt = H->lo + t;
+    const int pg = (H->lo + t) * kTileM + r;
+    if (pg >= H->tri_off[kCJ]) return false;
     int k = 0;
 #pragma unroll
-    for (int q = 1; q < kCJ; ++q) k += H->tbeg[q] <= gt ? 1 : 0;
-    const int pl = (gt - H->tbeg[k]) * kTileM + r;
+    for (int q = 1; q < kCJ; ++q) k += H->tri_off[q] <= pg ? 1 : 0;
+    const int pl = pg - H->tri_off[k];
     const Particles<PM>& P = H->ring[g0 + k];
     const int m = P.m;
-    if (pl >= m * (m + 1) / 2) return false;
+    if (!in_bounds(pl < m * (m + 1) / 2)) return false;
     TriPairs{}.map(pl, a, b);
     if (!in_bounds(a >= 0 && a <= b && b < m)) return false;
     pair_feat<PM, true>(P, a, b, f);
-    p = H->tri_off[k] + pl;
+    p = pg;
     return true;
   }
 };
@@ -2698,6 +2695,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   constexpr int kUCap = ClusterSmem<PM>::kUCap;
   const int q = (int)cluster_ctarank();
   const int c = blockIdx.x / kCJ, ncl = gridDim.x / kCJ;
+  cluster_arrive_relaxed();  // this CTA runs; waited for before the first remote store
   if (threadIdx.x == 0) {  // this CTA's slice of the momenta into L2, for the staging below
     const size_t bytes = (J.ptr ? (size_t)J.tokens : (size_t)J.N * J.P) * 4;
     prefetch_slice(J.E, bytes, blockIdx.x, gridDim.x);
@@ -2713,7 +2711,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   // 2 ncl + c, ... (a snake over the clusters), so the clusters' tile sums
   // come out close.
   for (int t = threadIdx.x; t < kMaxJetTiles + 2; t += blockDim.x) H.bin[t] = 0;
-  jet_counts(J, H.cnt, J.ptr ? nullptr : H.ends);
+  jet_counts(J, H.cnt);
   __syncthreads();
   auto jet_tiles = [&H](int n) {
     const int m = H.cnt[n + 1];
@@ -2776,23 +2774,6 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
     }
   }
   __syncthreads();
-  // the rows of Q, K and V this CTA attends (heads 2q, 2q + 1 of the
-  // cluster's jets) into L2: one thread per (jet, head, tensor); packed jets
-  // hold all heads of a row together, so CTA q takes tensor q there
-  if (threadIdx.x < kCJ * 2 * 3) {
-    const int k = threadIdx.x / 6, hh = (threadIdx.x / 3) & 1, tsel = threadIdx.x % 3;
-    const uint16_t* T = tsel == 0 ? X.q : (tsel == 1 ? X.k : X.v);
-    if (k < K) {
-      const int n = H.jets[k];
-      if (J.ptr) {
-        const long long lo = J.ptr[n], hi = J.ptr[n + 1];
-        if (hh == 0 && tsel == q && lo >= 0 && hi > lo && hi <= J.tokens)
-          prefetch_l2(T + (size_t)lo * kH * kD, (uint32_t)(hi - lo) * kH * kD * 2);
-      } else if (H.ends[n] > 0) {
-        prefetch_l2(T + ((size_t)n * kH + 2 * q + hh) * J.P * kD, (uint32_t)min(H.ends[n], J.P) * kD * 2);
-      }
-    }
-  }
   stage_jets<PM, true>(H.ring, J, K, [&H](int k) { return H.jets[k]; });
   mlp_setup<NG, SL>(H.mlp, wr);
   // groups of consecutive jets whose triangles fit together (identical in
@@ -2800,20 +2781,16 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   // out the group starting at jet g0
   auto plan = [&](int g0) {
     if (threadIdx.x == 0) {
-      int G = 0, pairs = 0, tiles = 0;
+      int G = 0, pairs = 0;
       while (g0 + G < K) {
         const int m = H.ring[g0 + G].m, np = m * (m + 1) / 2;
         if (G > 0 && pairs + np > kUCap) break;
         H.tri_off[G] = pairs;
-        H.tbeg[G] = tiles;
         pairs += np;
-        tiles += (np + kTileM - 1) / kTileM;
         ++G;
       }
-      for (int k = G; k <= kCJ; ++k) {
-        H.tri_off[k] = pairs;
-        H.tbeg[k] = tiles;
-      }
+      for (int k = G; k <= kCJ; ++k) H.tri_off[k] = pairs;
+      const int tiles = (pairs + kTileM - 1) / kTileM;  // the group's pairs, packed
       H.kvoff[0] = 0;
       H.ib[0] = 0;
       for (int k = 0; k < kCJ; ++k) {
@@ -2828,7 +2805,7 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   };
   plan(0);
   __syncthreads();
-  cluster_sync_all();  // all 4 CTAs run: their shared memory may be written
+  cluster_wait();  // all 4 CTAs run: their shared memory may be written
   float* stage = reinterpret_cast<float*>(&H.mlp.A[0][0]);
   uint32_t phase = 0u;
   bool aborted = false;
