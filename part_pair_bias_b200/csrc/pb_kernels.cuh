@@ -366,8 +366,9 @@ struct WeightRegs {
   static constexpr int kPer = (2 * 1024 + 255) / 256;  // float4 loads of W2 and W3 per thread (>= 256 threads)
   float4 w[kPer], w4, w1;
   float bias1, bias2, bias3, bias4;
-  __device__ void load(const MlpArgs& W) {
-    const int tid = threadIdx.x, nthr = blockDim.x;
+  // Threads tid = 0 .. nthr - 1 of the loading set (by default the block).
+  __device__ void load(const MlpArgs& W) { load(W, threadIdx.x, blockDim.x); }
+  __device__ void load(const MlpArgs& W, int tid, int nthr) {
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int q = tid + j * nthr;
@@ -382,10 +383,10 @@ struct WeightRegs {
   }
 };
 
-// Weight tiles in the canonical layout, from the registers of WeightRegs.
+// Weight tiles in the canonical layout, from the registers of WeightRegs
+// (loaded by the same set of threads tid = 0 .. nthr - 1).
 template <int NG, int SL>
-__device__ void store_weights(MlpSmem<NG, SL>& S, const WeightRegs& R) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
+__device__ void store_weights(MlpSmem<NG, SL>& S, const WeightRegs& R, int tid, int nthr) {
 #pragma unroll
   for (int j = 0; j < WeightRegs::kPer; ++j) {
     const int q = tid + j * nthr;
@@ -441,7 +442,7 @@ __device__ void store_weights(MlpSmem<NG, SL>& S, const WeightRegs& R) {
 // allocates NG*SL*64 columns).
 template <int NG, int SL>
 __device__ void mlp_setup(MlpSmem<NG, SL>& S, const WeightRegs& R) {
-  store_weights<NG, SL>(S, R);
+  store_weights<NG, SL>(S, R, threadIdx.x, blockDim.x);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NG * SL; ++i) mbar_init(&S.mbar[i], 1);
     fence_mbar_init();
@@ -451,6 +452,21 @@ __device__ void mlp_setup(MlpSmem<NG, SL>& S, const WeightRegs& R) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+}
+
+// The part of mlp_setup that threads tid = 0 .. nthr - 1 of warps 1 and up
+// do while warp 0 is busy elsewhere (the set's first thread initialises the
+// mbarriers). Warp 0 then allocates the TMEM (it also frees it in
+// mlp_teardown) and the caller completes the set-up with tc_fence_before, a
+// block barrier and tc_fence_after.
+template <int NG, int SL>
+__device__ void mlp_setup_part(MlpSmem<NG, SL>& S, const WeightRegs& R, int tid, int nthr) {
+  store_weights<NG, SL>(S, R, tid, nthr);
+  if (tid == 0) {
+    for (int i = 0; i < NG * SL; ++i) mbar_init(&S.mbar[i], 1);
+    fence_mbar_init();
+  }
+  fence_proxy_async_smem();  // weight tiles are read by the tensor cores
 }
 
 template <int NG, int SL>
@@ -2703,8 +2719,11 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
     prefetch_slice(J.py, bytes, blockIdx.x, gridDim.x);
     prefetch_slice(J.pz, bytes, blockIdx.x, gridDim.x);
   }
+  // warps 1.. load the weights (in flight while the jets are counted) and
+  // set up the MLP while warp 0 sorts the jets
+  const int wt = (int)threadIdx.x - 32, wn = (int)blockDim.x - 32;
   WeightRegs wr;
-  wr.load(W);  // in flight while the jets are counted and staged
+  if (wt >= 0) wr.load(W, wt, wn);
   // Every CTA counts every jet and sorts them by MLP tiles, largest first,
   // ties in jet order (a stable counting sort: every CTA must come to the
   // same order); cluster c takes the jets at ranks c, 2 ncl - 1 - c,
@@ -2762,8 +2781,13 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
       }
       __syncwarp();
     }
+    tmem_alloc(&H.mlp.tmem_base, kTmemCols(NG, SL));
+  } else {
+    mlp_setup_part<NG, SL>(H.mlp, wr, wt, wn);
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   int K = 0;
 #pragma unroll
   for (int r = 0; r < kCJ; ++r) {
@@ -2775,7 +2799,6 @@ __global__ void __launch_bounds__(512, 1) k_fused_cluster(JetArgs J, MlpArgs W, 
   }
   __syncthreads();
   stage_jets<PM, true>(H.ring, J, K, [&H](int k) { return H.jets[k]; });
-  mlp_setup<NG, SL>(H.mlp, wr);
   // groups of consecutive jets whose triangles fit together (identical in
   // every CTA of the cluster: the same jets, the same order); thread 0 lays
   // out the group starting at jet g0
