@@ -2147,9 +2147,13 @@ __global__ void __launch_bounds__(NG * 128, 1) k_fused(JetArgs J, WA W, QkvArgs 
 //   phase B  the 8 N (jet, head) attention items, weighted by the jet's tiles,
 //            are split evenly over the CTAs and run with the bias read back
 //            from the records.
+// Phases A and B run in rounds of consecutive jets whose records fit
+// kRoundTiles tiles (24 MB), a grid barrier between rounds, so that the
+// records of a round stay in L2 however large the batch.
 // Jets of any multiplicity up to P use the unordered triangle.
 
 constexpr int kGridMaxJets = 8192;    // jet-table capacity (shared memory)
+constexpr long long kRoundTiles = 12288;  // MLP tiles per round: 24 MB of bias records, kept in L2
 constexpr size_t kWsHeader = 256;     // barrier counters, then the records
 
 template <int PM>
@@ -2360,71 +2364,222 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
     }
   }
   __syncthreads();
-  const long long Ttot = S.T[N];
-
-  // phase B's share of this CTA: item (n, h) costs tiles_n + 1 and starts at
-  // 8 (T[n] + n) + h (tiles_n + 1)
-  const long long CB = 8ll * (Ttot + N);
-  const long long loB = CB * b / G, hiB = CB * (b + 1) / G;
-  int nB = 0;
-  {
-    int l = 0, r = N;  // smallest n whose items end past loB
-    while (l < r) {
-      const int mid = (l + r) >> 1;
-      if (8ll * ((long long)S.T[mid + 1] + mid + 1) > loB) r = mid; else l = mid + 1;
-    }
-    nB = l;
-  }
 
   mlp_setup<NG, SL>(S.mlp, wr);
   uint32_t phase = 0u;
   bool aborted = false;
 
-  // ---------------------------------------------------------------- phase A
-  {
-    const long long lo = Ttot * b / G, hi = Ttot * (b + 1) / G;
-    // first jet whose tiles reach past lo
-    int n = 0;
+  // Rounds: consecutive jets whose records fit kRoundTiles tiles (at least
+  // one jet), so that a round's records stay in L2 between its MLP and its
+  // attention; a round's records are indexed from its first tile. The
+  // bias-only launch keeps every record: one round. Every CTA takes the same
+  // barriers in every round, a CTA that aborted included.
+  for (int r0 = 0; r0 < N;) {
+    const long long T0 = S.T[r0];
+    int r1 = N;
+    if (!kBiasOnly) {  // the largest r1 > r0 with T[r1] - T0 <= kRoundTiles
+      int l = r0 + 1, r = N;
+      while (l < r) {
+        const int mid = (l + r + 1) >> 1;
+        if (S.T[mid] - T0 <= kRoundTiles) l = mid; else r = mid - 1;
+      }
+      r1 = l;
+    }
+    const long long Tr = S.T[r1] - T0;
+    const int Nr = r1 - r0;
+    // ---------------------------------------------------------------- phase A
     {
-      int l = 0, r = N;  // smallest n with T[n + 1] > lo
+      const long long lo = T0 + Tr * b / G, hi = T0 + Tr * (b + 1) / G;
+      // first jet whose tiles reach past lo
+      int n = r0;
+      {
+        int l = r0, r = r1;  // smallest n with T[n + 1] > lo
+        while (l < r) {
+          const int mid = (l + r) >> 1;
+          if (S.T[mid + 1] > lo) r = mid; else l = mid + 1;
+        }
+        n = l;
+      }
+      while (!aborted && n < r1 && S.T[n] < hi) {
+        // gather up to JB jets with tiles in [lo, hi)
+        if (tid == 0) {
+          int K = 0, acc = 0;
+          int nn = n;
+          while (K < JB && nn < r1 && S.T[nn] < hi) {
+            const long long a0 = max((long long)S.T[nn], lo), a1 = min((long long)S.T[nn + 1], hi);
+            if (a1 > a0) {
+              S.batch.tbeg[K] = acc;
+              S.batch.t_lo[K] = (int)(a0 - S.T[nn]);
+              S.batch.rowbase[K] = (long long)(S.T[nn] - T0) * kTileM;
+              S.batch.jet[K] = nn;
+              acc += (int)(a1 - a0);
+              ++K;
+            }
+            ++nn;
+          }
+          S.batch.tbeg[K] = acc;
+          S.batch.K = K;
+          S.flag = nn;  // next jet to look at
+        }
+        __syncthreads();
+        const int K = S.batch.K;
+        const int n_next = S.flag;
+        stage_jets<PM, true>(S.ring, J, K, [&S](int k) { return S.batch.jet[k]; });
+        if (tid == 0)
+          for (int k = 0; k < K; ++k) S.batch.npairs[k] = S.ring[k].m * (S.ring[k].m + 1) / 2;
+        __syncthreads();
+        RecordSink sink{rec, Tr * kTileM};
+        const bool ok = mlp_pass<NG, SL>(S.mlp, BatchTiles<PM>{S.ring, &S.batch}, sink, &phase);
+        aborted = __syncthreads_or(!ok) != 0;
+        n = n_next;
+      }
+    }
+
+    if (kBiasOnly) break;
+
+    // --------------------------------------------------------------- barrier
+    const bool passed = grid_barrier(bar_ctr, (unsigned)G, &S.flag);
+    aborted = aborted || !passed;
+
+    // phase B's share of this CTA: item (n, h) of the round costs tiles_n + 1
+    // and starts at 8 (T[n] - T0 + n - r0) + h (tiles_n + 1)
+    const long long CB = 8ll * (Tr + Nr);
+    const long long loB = CB * b / G, hiB = CB * (b + 1) / G;
+    int nB = r0;
+    {
+      int l = r0, r = r1;  // smallest n whose items end past loB
       while (l < r) {
         const int mid = (l + r) >> 1;
-        if (S.T[mid + 1] > lo) r = mid; else l = mid + 1;
+        if (8ll * ((long long)(S.T[mid + 1] - T0) + mid + 1 - r0) > loB) r = mid; else l = mid + 1;
       }
-      n = l;
+      nB = l;
     }
-    while (!aborted && n < N && S.T[n] < hi) {
-      // gather up to JB jets with tiles in [lo, hi)
-      if (tid == 0) {
-        int K = 0, acc = 0;
-        int nn = n;
-        while (K < JB && nn < N && S.T[nn] < hi) {
-          const long long a0 = max((long long)S.T[nn], lo), a1 = min((long long)S.T[nn + 1], hi);
-          if (a1 > a0) {
-            S.batch.tbeg[K] = acc;
-            S.batch.t_lo[K] = (int)(a0 - S.T[nn]);
-            S.batch.rowbase[K] = (long long)S.T[nn] * kTileM;
-            S.batch.jet[K] = nn;
-            acc += (int)(a1 - a0);
-            ++K;
+
+    // ---------------------------------------------------------------- phase B
+    if (!aborted) {
+      const long long lo = loB, hi = hiB;
+      int n = nB;
+      float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
+      constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
+      AttnBatch<PM>& A = S.ab;
+      while (n < r1 && 8ll * ((long long)(S.T[n] - T0) + n - r0) < hi) {
+        // up to JB jets with heads in [lo, hi), staged (slots only) together
+        if (tid == 0) {
+          int K = 0, nn = n;
+          while (K < JB && nn < r1 && 8ll * ((long long)(S.T[nn] - T0) + nn - r0) < hi) {
+            const long long base = 8ll * ((long long)(S.T[nn] - T0) + nn - r0);
+            const long long c = (long long)(S.T[nn + 1] - S.T[nn]) + 1;
+            int h_lo = 0, h_hi = 0;
+            for (int h = 0; h < kH; ++h) {
+              const long long st = base + h * c;
+              if (st < lo) h_lo = h + 1;
+              if (st < hi) h_hi = h + 1;
+            }
+            if (h_lo < h_hi) {
+              A.jet[K] = nn;
+              A.hl[K] = h_lo;
+              A.hh[K] = h_hi;
+              ++K;
+            }
+            ++nn;
           }
-          ++nn;
+          A.K = K;
+          A.next = nn;
         }
-        S.batch.tbeg[K] = acc;
-        S.batch.K = K;
-        S.flag = nn;  // next jet to look at
+        __syncthreads();
+        const int K = A.K;
+        stage_jets<PM, false>(S.ring, J, K, [&A](int k) { return A.jet[k]; });
+        // the leading jets whose records and K/V fit in the stage together
+        if (tid == 0) {
+          int used = 0, items = 0, Kf = 0;
+          for (; Kf < K; ++Kf) {
+            const int m = S.ring[Kf].m, hr = A.hh[Kf] - A.hl[Kf];
+            const int need = m * (m + 1) / 2 * 4 + hr * (kv16_bytes(m) / 4);
+            if (used + need > kStageFloats) break;
+            A.uoff[Kf] = used;
+            A.kvoff[Kf] = used + m * (m + 1) / 2 * 4;
+            A.ib[Kf] = items;
+            used += need;
+            items += hr * ((m + 15) >> 4);
+          }
+          A.ib[Kf] = items;
+          A.Kf = Kf;
+          // jets that did not fit are staged again in the next round
+          if (Kf > 0 && Kf < K) A.next = A.jet[Kf];
+          else if (Kf == 0 && K > 1) A.next = A.jet[1];
+        }
+        __syncthreads();
+        const int Kf = A.Kf, n_next = A.next;
+        if (K == 0) {
+          // [lo, hi) lies inside one jet's head: nothing to do in this round
+        } else if (Kf == 0) {
+          // one jet too wide for the stage: its bias is read from the records
+          const int nj = A.jet[0];
+          RecordUBias ub{reinterpret_cast<const __half*>(rec + (size_t)(S.T[nj] - T0) * kTileM)};
+          attention_block<PM>(S.ring[0], J, X, nj, 0, S.ring[0].m, stage, kStageFloats, ub, A.hl[0], A.hh[0]);
+          if (A.hl[0] == 0) zero_masked_rows<PM>(S.ring[0], J, X.out, nj);
+        } else {
+          // warp items: (jet, head, 16-query tile); Q fragments are loaded ahead
+          const int items = A.ib[Kf], nwarp = (int)(blockDim.x >> 5);
+          auto qload = [&](int it, uint32_t* f) {
+            int k = 0;
+  #pragma unroll
+            for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= it) ? 1 : 0;
+            const Particles<PM>& P = S.ring[k];
+            const int m = P.m, tiles = (m + 15) >> 4, loc = it - A.ib[k];
+            const int h = A.hl[k] + loc / tiles, i0 = (loc % tiles) * 16, nj = A.jet[k];
+            q_frag(i0, min(16, m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, nj, h, i); }, f);
+          };
+          uint32_t a[4] = {0u, 0u, 0u, 0u};
+          if (warp < items) qload(warp, a);
+          for (int k = 0; k < Kf; ++k) {
+            const int nj = A.jet[k], m = S.ring[k].m, np = m * (m + 1) / 2;
+            const uint4* jrec = rec + (size_t)(S.T[nj] - T0) * kTileM;
+            uint4* U8 = reinterpret_cast<uint4*>(stage + A.uoff[k]);
+            for (int r0 = tid; r0 < np; r0 += 4 * (int)blockDim.x) {
+              uint4 v[4];
+  #pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int r = r0 + u * (int)blockDim.x;
+                v[u] = r < np ? __ldcg(jrec + r) : make_uint4(0, 0, 0, 0);
+              }
+  #pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (r0 + u * (int)blockDim.x < np) U8[r0 + u * (int)blockDim.x] = v[u];
+            }
+            stage_kv16<PM>(S.ring[k], J, X, nj, A.hl[k], A.hh[k] - A.hl[k], reinterpret_cast<uint16_t*>(stage + A.kvoff[k]));
+          }
+          cp_async_wait_all();
+          __syncthreads();
+          for (int it = warp; it < items; it += nwarp) {
+            uint32_t an[4] = {0u, 0u, 0u, 0u};
+            if (it + nwarp < items) qload(it + nwarp, an);
+            int k = 0;
+  #pragma unroll
+            for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= it) ? 1 : 0;
+            const Particles<PM>& P = S.ring[k];
+            const int m = P.m, tiles = (m + 15) >> 4, loc = it - A.ib[k];
+            const int hh = loc / tiles, i0 = (loc % tiles) * 16, h = A.hl[k] + hh, nj = A.jet[k];
+            const uint16_t* kh = reinterpret_cast<const uint16_t*>(stage + A.kvoff[k]) + hh * (kv16_bytes(m) / 2);
+            const TriBlock ub{reinterpret_cast<const __half*>(stage + A.uoff[k]) + h};
+            attend_tile16(
+                kh, kh + round16(m) * 16, m, i0, min(16, m - i0), a,
+                [&](int i) { return X.out + qkv_off<PM>(P, J, nj, h, i); }, ub);
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) a[e] = an[e];
+          }
+          for (int k = 0; k < Kf; ++k)
+            if (A.hl[k] == 0) zero_masked_rows<PM>(S.ring[k], J, X.out, A.jet[k]);
+        }
+        __syncthreads();
+        n = n_next;
       }
-      __syncthreads();
-      const int K = S.batch.K;
-      const int n_next = S.flag;
-      stage_jets<PM, true>(S.ring, J, K, [&S](int k) { return S.batch.jet[k]; });
-      if (tid == 0)
-        for (int k = 0; k < K; ++k) S.batch.npairs[k] = S.ring[k].m * (S.ring[k].m + 1) / 2;
-      __syncthreads();
-      RecordSink sink{rec, Ttot * kTileM};
-      const bool ok = mlp_pass<NG, SL>(S.mlp, BatchTiles<PM>{S.ring, &S.batch}, sink, &phase);
-      aborted = __syncthreads_or(!ok) != 0;
-      n = n_next;
+    }
+
+    r0 = r1;
+    if (r0 < N) {  // the next round overwrites the records this one read
+      const bool again = grid_barrier(bar_ctr, (unsigned)G, &S.flag);
+      aborted = aborted || !again;
     }
   }
 
@@ -2433,131 +2588,6 @@ __global__ void __launch_bounds__(512, 1) k_fused_grid(JetArgs J, MlpArgs W, Qkv
       for (int n = tid; n <= N; n += blockDim.x) Tout[n] = S.T[n];
     mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
     return;
-  }
-
-  // --------------------------------------------------------------- barrier
-  const bool passed = grid_barrier(bar_ctr, (unsigned)G, &S.flag);
-  aborted = aborted || !passed;
-
-  // ---------------------------------------------------------------- phase B
-  if (!aborted) {
-    const long long lo = loB, hi = hiB;
-    int n = nB;
-    float* stage = reinterpret_cast<float*>(&S.mlp.A[0][0]);
-    constexpr int kStageFloats = NG * SL * kTileM * kAK / 2;
-    AttnBatch<PM>& A = S.ab;
-    while (n < N && 8ll * ((long long)S.T[n] + n) < hi) {
-      // up to JB jets with heads in [lo, hi), staged (slots only) together
-      if (tid == 0) {
-        int K = 0, nn = n;
-        while (K < JB && nn < N && 8ll * ((long long)S.T[nn] + nn) < hi) {
-          const long long base = 8ll * ((long long)S.T[nn] + nn);
-          const long long c = (long long)(S.T[nn + 1] - S.T[nn]) + 1;
-          int h_lo = 0, h_hi = 0;
-          for (int h = 0; h < kH; ++h) {
-            const long long st = base + h * c;
-            if (st < lo) h_lo = h + 1;
-            if (st < hi) h_hi = h + 1;
-          }
-          if (h_lo < h_hi) {
-            A.jet[K] = nn;
-            A.hl[K] = h_lo;
-            A.hh[K] = h_hi;
-            ++K;
-          }
-          ++nn;
-        }
-        A.K = K;
-        A.next = nn;
-      }
-      __syncthreads();
-      const int K = A.K;
-      stage_jets<PM, false>(S.ring, J, K, [&A](int k) { return A.jet[k]; });
-      // the leading jets whose records and K/V fit in the stage together
-      if (tid == 0) {
-        int used = 0, items = 0, Kf = 0;
-        for (; Kf < K; ++Kf) {
-          const int m = S.ring[Kf].m, hr = A.hh[Kf] - A.hl[Kf];
-          const int need = m * (m + 1) / 2 * 4 + hr * (kv16_bytes(m) / 4);
-          if (used + need > kStageFloats) break;
-          A.uoff[Kf] = used;
-          A.kvoff[Kf] = used + m * (m + 1) / 2 * 4;
-          A.ib[Kf] = items;
-          used += need;
-          items += hr * ((m + 15) >> 4);
-        }
-        A.ib[Kf] = items;
-        A.Kf = Kf;
-        // jets that did not fit are staged again in the next round
-        if (Kf > 0 && Kf < K) A.next = A.jet[Kf];
-        else if (Kf == 0 && K > 1) A.next = A.jet[1];
-      }
-      __syncthreads();
-      const int Kf = A.Kf, n_next = A.next;
-      if (K == 0) {
-        // [lo, hi) lies inside one jet's head: nothing to do in this round
-      } else if (Kf == 0) {
-        // one jet too wide for the stage: its bias is read from the records
-        const int nj = A.jet[0];
-        RecordUBias ub{reinterpret_cast<const __half*>(rec + (size_t)S.T[nj] * kTileM)};
-        attention_block<PM>(S.ring[0], J, X, nj, 0, S.ring[0].m, stage, kStageFloats, ub, A.hl[0], A.hh[0]);
-        if (A.hl[0] == 0) zero_masked_rows<PM>(S.ring[0], J, X.out, nj);
-      } else {
-        // warp items: (jet, head, 16-query tile); Q fragments are loaded ahead
-        const int items = A.ib[Kf], nwarp = (int)(blockDim.x >> 5);
-        auto qload = [&](int it, uint32_t* f) {
-          int k = 0;
-#pragma unroll
-          for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= it) ? 1 : 0;
-          const Particles<PM>& P = S.ring[k];
-          const int m = P.m, tiles = (m + 15) >> 4, loc = it - A.ib[k];
-          const int h = A.hl[k] + loc / tiles, i0 = (loc % tiles) * 16, nj = A.jet[k];
-          q_frag(i0, min(16, m - i0), [&](int i) { return X.q + qkv_off<PM>(P, J, nj, h, i); }, f);
-        };
-        uint32_t a[4] = {0u, 0u, 0u, 0u};
-        if (warp < items) qload(warp, a);
-        for (int k = 0; k < Kf; ++k) {
-          const int nj = A.jet[k], m = S.ring[k].m, np = m * (m + 1) / 2;
-          const uint4* jrec = rec + (size_t)S.T[nj] * kTileM;
-          uint4* U8 = reinterpret_cast<uint4*>(stage + A.uoff[k]);
-          for (int r0 = tid; r0 < np; r0 += 4 * (int)blockDim.x) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int r = r0 + u * (int)blockDim.x;
-              v[u] = r < np ? __ldcg(jrec + r) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              if (r0 + u * (int)blockDim.x < np) U8[r0 + u * (int)blockDim.x] = v[u];
-          }
-          stage_kv16<PM>(S.ring[k], J, X, nj, A.hl[k], A.hh[k] - A.hl[k], reinterpret_cast<uint16_t*>(stage + A.kvoff[k]));
-        }
-        cp_async_wait_all();
-        __syncthreads();
-        for (int it = warp; it < items; it += nwarp) {
-          uint32_t an[4] = {0u, 0u, 0u, 0u};
-          if (it + nwarp < items) qload(it + nwarp, an);
-          int k = 0;
-#pragma unroll
-          for (int q = 1; q < JB; ++q) k += (q < Kf && A.ib[q] <= it) ? 1 : 0;
-          const Particles<PM>& P = S.ring[k];
-          const int m = P.m, tiles = (m + 15) >> 4, loc = it - A.ib[k];
-          const int hh = loc / tiles, i0 = (loc % tiles) * 16, h = A.hl[k] + hh, nj = A.jet[k];
-          const uint16_t* kh = reinterpret_cast<const uint16_t*>(stage + A.kvoff[k]) + hh * (kv16_bytes(m) / 2);
-          const TriBlock ub{reinterpret_cast<const __half*>(stage + A.uoff[k]) + h};
-          attend_tile16(
-              kh, kh + round16(m) * 16, m, i0, min(16, m - i0), a,
-              [&](int i) { return X.out + qkv_off<PM>(P, J, nj, h, i); }, ub);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) a[e] = an[e];
-        }
-        for (int k = 0; k < Kf; ++k)
-          if (A.hl[k] == 0) zero_masked_rows<PM>(S.ring[k], J, X.out, A.jet[k]);
-      }
-      __syncthreads();
-      n = n_next;
-    }
   }
 
   mlp_teardown<NG, SL>(S.mlp, aborted, &phase);
