@@ -87,7 +87,10 @@ typedef struct pb_jets {
   int64_t tokens;        /* packed only: length of the momentum arrays */
 } pb_jets;
 
-/* Folded pair-embedding MLP, fp32, device pointers, row-major [out][in]. */
+/* Folded pair-embedding MLP, fp32, device pointers, row-major [out][in]; the
+ * matrices W1..W4 16-byte aligned (the kernels read them as float4; a
+ * misaligned one returns PB_EINVAL). The flat buffer of pb_fold_affine,
+ * 16-byte aligned, meets this at every offset below. */
 typedef struct pb_mlp {
   const float *W1, *b1;  /* [64][4], [64]  (input affine and layer-1 affine folded in) */
   const float *W2, *b2;  /* [64][64], [64] (layer-2 affine folded in)                  */

@@ -140,6 +140,8 @@ pb_status check_mlp(const pb_mlp* w, pb::MlpArgs* out) {
   if (!w) return fail(PB_EINVAL, "mlp is NULL");
   if (!w->W1 || !w->b1 || !w->W2 || !w->b2 || !w->W3 || !w->b3 || !w->W4 || !w->b4)
     return fail(PB_EINVAL, "an MLP parameter pointer is NULL");
+  if (!aligned(w->W1, 16) || !aligned(w->W2, 16) || !aligned(w->W3, 16) || !aligned(w->W4, 16))
+    return fail(PB_EINVAL, "the MLP weight matrices W1..W4 must be 16-byte aligned");
   *out = pb::MlpArgs{w->W1, w->b1, w->W2, w->b2, w->W3, w->b3, w->W4, w->b4};
   return PB_OK;
 }
@@ -378,7 +380,7 @@ pb_status run_backward_chunk(const pb::JetArgs& J, const pb::MlpArgs& W, const p
     if ((st = launched("k_attn_bwd")) != PB_OK) return st;
   }
   auto k = pb::k_mlp_bwd<PM>;
-  k<<<mlp_grid, 512, sizeof(pb::MlpBwdSmem<PM>), s>>>(J, W, X, partials, accumulate ? 1 : 0);
+  k<<<mlp_grid, pb::kBwdThreads, sizeof(pb::MlpBwdSmem<PM>), s>>>(J, W, X, partials, accumulate ? 1 : 0);
   return launched("k_mlp_bwd");
 }
 
@@ -396,7 +398,7 @@ pb_status run_backward(const pb::JetArgs& J, const pb::MlpArgs& W, pb::BwdArgs X
   pb_status st = device_sms(&dev, &sms);
   if (st != PB_OK) return st;
   auto kb = pb::k_mlp_bwd<PM>;
-  if ((st = resident_per_sm((const void*)kb, dev, sizeof(pb::MlpBwdSmem<PM>), 512, &per_sm)) != PB_OK) return st;
+  if ((st = resident_per_sm((const void*)kb, dev, sizeof(pb::MlpBwdSmem<PM>), pb::kBwdThreads, &per_sm)) != PB_OK) return st;
   const int mlp_grid = sms * per_sm < pb::kBwdMaxCtas ? sms * per_sm : pb::kBwdMaxCtas;
   const int nc = bwd_chunk_jets(J);
   for (int c0 = 0; c0 < J.N; c0 += nc) {
@@ -413,7 +415,7 @@ pb_status run_backward(const pb::JetArgs& J, const pb::MlpArgs& W, pb::BwdArgs X
     }
     if ((st = run_backward_chunk<PM>(Jc, W, Xc, ws, table, partials, mlp_grid, c0 > 0, s)) != PB_OK) return st;
   }
-  pb::k_grad_reduce<<<pb::kReduceCtas, 256, 0, s>>>(partials, mlp_grid, G);
+  pb::k_grad_reduce<<<pb::kReduceCtas, 32 * pb::kReduceWarps, 0, s>>>(partials, mlp_grid, G);
   return launched("k_grad_reduce");
 }
 
@@ -641,7 +643,7 @@ pb_status pair_attention_backward(const pb_jets* jets, const pb_mlp* mlp, int H,
   const pb::GradArgs G{gp[0], gp[1], gp[2], gp[3], gp[4], gp[5], gp[6], gp[7]};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (J.N == 0) {  // no pairs: the weight gradients are zero
-    pb::k_grad_reduce<<<pb::kReduceCtas, 256, 0, s>>>(nullptr, 0, G);
+    pb::k_grad_reduce<<<pb::kReduceCtas, 32 * pb::kReduceWarps, 0, s>>>(nullptr, 0, G);
     return launched("k_grad_reduce");
   }
   if (!q || !k || !v || !dout || !dq || !dk || !dv) return fail(PB_EINVAL, "q, k, v, dout, dq, dk and dv must be non-NULL");

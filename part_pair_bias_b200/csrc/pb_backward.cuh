@@ -10,9 +10,9 @@
 //                  fp32 record per unordered pair
 //   k_mlp_bwd      the pairs' 128-row tiles split evenly over the CTAs: the
 //                  MLP recomputed on tcgen05 (GELU' kept in TMEM), the
-//                  backward through it on tcgen05, the weight gradients on
-//                  m16n8k16 tensor cores in registers that persist over all
-//                  the CTA's tiles (and chunks)
+//                  backward through it and the weight gradients on tcgen05,
+//                  the latter accumulated in TMEM over all the CTA's tiles
+//                  (and summed into the CTA's partial slot over chunks)
 // then, once, k_grad_reduce: the per-CTA partials summed in CTA order.
 //
 // Source: "Event Classification with Masked Transformer Autoencoders",
@@ -354,18 +354,21 @@ __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
 // g_h = dS_h[a, b] + dS_h[b, a] (a != b) or dS_h[a, a], the record that the
 // attention backward accumulated. Per tile of 128 such rows (one CTA, 512
 // threads; thread (row r, quarter c) owns TMEM lane r and columns 16c ..
-// 16c + 15 of each 64-wide accumulator):
-//   z1 = W1' f + b1', h1 = GELU(z1), z2 = W2' h1 + b2', ... h3   (tcgen05)
+// 16c + 15 of each 64-wide accumulator), all products on tcgen05:
+//   z1 = W1' f + b1', h1 = GELU(z1), z2 = W2' h1 + b2', ... h3
 //   e3 = g W4 (issued with z1), d3 = e3 * GELU'(z3), e2 = d3 W3', d2, e1 = d2 W2', d1
-//   dW4 += g^T h3, dWk' += dk^T h(k-1) (h0 = f), dbk' += column sums of dk
-// with bf16 operands and fp32 accumulation; f, g and the folded layer-1
-// weights enter as bf16 hi + lo terms. GELU is the tanh form the forward
-// kernels use (tanh.approx); GELU'(z) is computed with h and parked in TMEM
-// over z until the backward step needs it. The weight gradients are 31
-// (layer, 16-row block, up to three 8-column blocks) parts spread over the
-// 16 warps as m16n8k16 MMAs whose A operand (d^T) and B operand (h) come
-// from the row-major tiles through ldmatrix.trans; a column block of ones
-// gives the bias gradients.
+//   [dW2' | db2'; dW1' | db1'] += [d2 | d1]^T [f | h1 | 1]
+//   [dW3' | db3'; dW4 | db4]   += [d3 | g]^T  [h2 | h3 | 1]
+// The recompute multiplies f16 h (two per TMEM column, the A operand read
+// from TMEM) by f16 hi + lo weights; the backward products take bf16 d and
+// bf16 hi + lo weights; f, g and the folded layer-1 weights enter as bf16
+// hi + lo terms. The weight gradients are two MMAs per tile over the tile's
+// rows (K = 128) with both operands read transposed (MN-major) from the same
+// row-major tiles, accumulated in fp32 TMEM over all the CTA's tiles; the
+// second overlaps the next tile's feature and gradient-record loads. GELU is
+// the tanh form the forward kernels use; GELU'(z) is computed with h and
+// parked in TMEM (f16, in the first half of the quarter's z columns, h in
+// the second half) until the backward step needs it.
 
 constexpr int kBwdMaxCtas = 256;     // partial-gradient slots in the workspace
 constexpr int kFoldedFloats = 9160;  // W1 b1 W2 b2 W3 b3 W4 b4, as pb_fold_affine lays them out
@@ -376,13 +379,21 @@ struct GradArgs {
   float *W1, *b1, *W2, *b2, *W3, *b3, *W4, *b4;
 };
 
+// Operand tiles of one 128-row tile (bf16, columns as listed; each in the
+// canonical no-swizzle layout of cofs with its own width):
+//   F1  [hi f | lo f | hi f | 0 | h1 | 1 | 0]  96 wide: A of z1 (columns 0..15), B of the first gradient MMA
+//   H23 [h2 | h3 | 1 | 0]                     144 wide: B of the second gradient MMA
+//   D12 [d1 | d2]                             128 wide: A of e1 (columns 64..127), A^T of the first
+//   D3G [d3 | hi g | lo g | 0]                128 wide: A of e2 (0..63) and e3 (64..79), A^T of the second
+constexpr int kF1W = 96, kH23W = 144, kDW = 128;
+constexpr int kF1Ones = 80, kH23Ones = 128, kD3G = 64;
+
 template <int PM>
 struct MlpBwdSmem {
-  __nv_bfloat16 A0[kTileM * 16];     // [hi(f) | lo(f) | hi(f) | 0]
-  __nv_bfloat16 G4[kTileM * 16];     // [hi(g) | lo(g)] (8 heads each)
-  __half Hf[2][kTileM * 64];         // h1, h2 in f16: operands of z2, z3
-  __nv_bfloat16 Hs[3][kTileM * 64];  // h1, h2, h3 in bf16: operands of the weight gradients
-  __nv_bfloat16 Ds[3][kTileM * 64];  // d1, d2, d3 = dL/dz
+  __nv_bfloat16 F1[kTileM * kF1W];
+  __nv_bfloat16 H23[kTileM * kH23W];
+  __nv_bfloat16 D12[kTileM * kDW];
+  __nv_bfloat16 D3G[kTileM * kDW];
   __nv_bfloat16 W1f[64 * 16];        // [hi(W1') | hi(W1') | lo(W1') | 0] per output row
   __half Wf[2][2][64 * 64];          // W2', W3' as [out][in], f16: hi, lo
   __nv_bfloat16 Wt[2][2][64 * 64];   // W2'^T, W3'^T as [in][out]: hi, lo
@@ -390,229 +401,354 @@ struct MlpBwdSmem {
   float bias[3][64];                 // b1', b2', b3'
   uint64_t mbar;
   uint32_t tmem_base;
+  int stop;  // set by the epilogue warps at a hand-off: the issuer stops
+  int n0;    // the CTA's first jet
   Particles<PM> part;
 };
+// The kernel takes all 512 TMEM columns: one CTA per SM.
+static_assert(sizeof(MlpBwdSmem<128>) > 116 * 1024, "k_mlp_bwd must not fit twice on an SM");
 
-// Weights in the canonical K-major layouts of their MMA roles.
-template <int PM>
-__device__ void bwd_load_weights(MlpBwdSmem<PM>& S, const MlpArgs& W) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  for (int e = tid; e < 64 * 64; e += nthr) {
-    const int o = e >> 6, i = e & 63;
-    const float w[2] = {W.W2[e], W.W3[e]};
+// TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192), e3 / e2 / e1
+// [192, 256), the gradient accumulators [256, 352) and [352, 496).
+constexpr uint32_t kTmG12 = 256, kTmG3G = 352, kBwdTmemCols = 512;
+
+// Weights in the canonical K-major layouts of their MMA roles, and the
+// constant columns of the operand tiles (ones, zeros). load() issues every
+// global load of the thread at once (one round trip); store() converts and
+// writes whole 8- or 16-byte pieces of core-matrix rows: Wf rows from float4
+// of 4 consecutive inputs, Wt rows (8 consecutive outputs of one input) from
+// 8 loads coalesced across the warp's consecutive inputs, W1f and W4t rows
+// (16 columns) from one row of W1 or one column of W4. Needs >= 512 threads.
+struct BwdWeightLoad {
+  static constexpr int kWfJobs = 2 * 1024, kWtJobs = 2 * 512;  // (layer, float4), (layer, input, 8-output block)
+  static constexpr int kPer = (kWfJobs + kWtJobs + 511) / 512;
+  float v[kPer][8];
+  float4 w1;   // threads 0..63: row tid of W1
+  float w4[8];  // threads 64..127: column tid - 64 of W4
+  float b;      // threads 128..319: b1, b2, b3
+  __device__ void load(const MlpArgs& W, int tid, int nthr) {
 #pragma unroll
-    for (int L = 0; L < 2; ++L) {
-      const __half fh = __float2half_rn(w[L]), fl = __float2half_rn(w[L] - __half2float(fh));
-      S.Wf[L][0][cofs(o, i, 64)] = fh;
-      S.Wf[L][1][cofs(o, i, 64)] = fl;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(w[L]), lo = __float2bfloat16_rn(w[L] - __bfloat162float(hi));
-      S.Wt[L][0][cofs(i, o, 64)] = hi;
-      S.Wt[L][1][cofs(i, o, 64)] = lo;
+    for (int j = 0; j < kPer; ++j) {
+      const int q = tid + j * nthr;
+      if (q < kWfJobs) {
+        const float4 x = reinterpret_cast<const float4*>(q < 1024 ? W.W2 : W.W3)[q & 1023];
+        v[j][0] = x.x; v[j][1] = x.y; v[j][2] = x.z; v[j][3] = x.w;
+      } else if (q < kWfJobs + kWtJobs) {
+        const int t = q - kWfJobs, i = t & 63, ob = (t >> 6) & 7;
+        const float* Wl = t < 512 ? W.W2 : W.W3;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[j][u] = Wl[(ob * 8 + u) * 64 + i];
+      }
+    }
+    if (tid < 64) w1 = reinterpret_cast<const float4*>(W.W1)[tid];
+    if (tid >= 64 && tid < 128) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) w4[u] = W.W4[u * 64 + tid - 64];
+    }
+    if (tid >= 128 && tid < 320) {
+      const int e = tid - 128;
+      b = (e < 64 ? W.b1 : (e < 128 ? W.b2 : W.b3))[e & 63];
     }
   }
-  for (int e = tid; e < 64 * 16; e += nthr) {
-    const int r = e >> 4, k = e & 15;  // W1f row = output r, W4t row = input r
-    const float w1 = k < 12 ? W.W1[r * 4 + (k & 3)] : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w1);
-    S.W1f[cofs(r, k, 16)] = (k >= 8 && k < 12) ? __float2bfloat16_rn(w1 - __bfloat162float(hi)) : hi;
-    const float w4 = W.W4[(k & 7) * 64 + r];
-    const __nv_bfloat16 h4 = __float2bfloat16_rn(w4);
-    S.W4t[0][cofs(r, k, 16)] = h4;
-    S.W4t[1][cofs(r, k, 16)] = __float2bfloat16_rn(w4 - __bfloat162float(h4));
+  template <class Smem>
+  __device__ void store(Smem& S, int tid, int nthr) const {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int q = tid + j * nthr;
+      if (q < kWfJobs) {
+        const int L = q >> 10, e = (q & 1023) * 4, o = e >> 6, i = e & 63;
+        uint32_t hw[2], lw[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          hw[u] = cvt_f16x2(v[j][2 * u], v[j][2 * u + 1]);
+          const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hw[u]));
+          lw[u] = cvt_f16x2(v[j][2 * u] - hf.x, v[j][2 * u + 1] - hf.y);
+        }
+        *reinterpret_cast<uint2*>(&S.Wf[L][0][cofs(o, i, 64)]) = make_uint2(hw[0], hw[1]);
+        *reinterpret_cast<uint2*>(&S.Wf[L][1][cofs(o, i, 64)]) = make_uint2(lw[0], lw[1]);
+      } else if (q < kWfJobs + kWtJobs) {
+        const int t = q - kWfJobs, L = t >> 9, i = t & 63, ob = (t >> 6) & 7;
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          hw[u] = cvt_bf16x2(v[j][2 * u], v[j][2 * u + 1]);
+          lw[u] = cvt_bf16x2(v[j][2 * u] - bf16lo(hw[u]), v[j][2 * u + 1] - bf16hi(hw[u]));
+        }
+        *reinterpret_cast<uint4*>(&S.Wt[L][0][cofs(i, ob * 8, 64)]) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(&S.Wt[L][1][cofs(i, ob * 8, 64)]) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    }
+    if (tid < 64) {  // W1f row tid: [hi W1 | hi W1 | lo W1 | 0]
+      const uint32_t h01 = cvt_bf16x2(w1.x, w1.y), h23 = cvt_bf16x2(w1.z, w1.w);
+      const uint32_t l01 = cvt_bf16x2(w1.x - bf16lo(h01), w1.y - bf16hi(h01));
+      const uint32_t l23 = cvt_bf16x2(w1.z - bf16lo(h23), w1.w - bf16hi(h23));
+      *reinterpret_cast<uint4*>(&S.W1f[cofs(tid, 0, 16)]) = make_uint4(h01, h23, h01, h23);
+      *reinterpret_cast<uint4*>(&S.W1f[cofs(tid, 8, 16)]) = make_uint4(l01, l23, 0u, 0u);
+    }
+    if (tid >= 64 && tid < 128) {  // W4t rows (input tid - 64): [W4^T | W4^T], hi and lo
+      const int i = tid - 64;
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        hw[u] = cvt_bf16x2(w4[2 * u], w4[2 * u + 1]);
+        lw[u] = cvt_bf16x2(w4[2 * u] - bf16lo(hw[u]), w4[2 * u + 1] - bf16hi(hw[u]));
+      }
+      const uint4 h = make_uint4(hw[0], hw[1], hw[2], hw[3]), l = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      *reinterpret_cast<uint4*>(&S.W4t[0][cofs(i, 0, 16)]) = h;
+      *reinterpret_cast<uint4*>(&S.W4t[0][cofs(i, 8, 16)]) = h;
+      *reinterpret_cast<uint4*>(&S.W4t[1][cofs(i, 0, 16)]) = l;
+      *reinterpret_cast<uint4*>(&S.W4t[1][cofs(i, 8, 16)]) = l;
+    }
+    if (tid >= 128 && tid < 320) S.bias[(tid - 128) >> 6][(tid - 128) & 63] = b;
+    // constant columns, 8 at a time: F1 [80, 96) = 1 1 1 1 1 1 1 1 | 0 ..., H23 [128, 144) alike, D3G [80, 128) = 0
+    const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u), zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int e = tid; e < kTileM * 10; e += nthr) {
+      const int r = e & 127, g = e >> 7;  // g: 0, 1 of F1; 2, 3 of H23; 4..9 of D3G
+      if (g < 2) *reinterpret_cast<uint4*>(&S.F1[cofs(r, kF1Ones + 8 * g, kF1W)]) = g == 0 ? ones : zero;
+      else if (g < 4) *reinterpret_cast<uint4*>(&S.H23[cofs(r, kH23Ones + 8 * (g - 2), kH23W)]) = g == 2 ? ones : zero;
+      else *reinterpret_cast<uint4*>(&S.D3G[cofs(r, kD3G + 16 + 8 * (g - 4), kDW)]) = zero;
+    }
   }
-  for (int e = tid; e < 3 * 64; e += nthr) S.bias[e >> 6][e & 63] = (e < 64 ? W.b1 : (e < 128 ? W.b2 : W.b3))[e & 63];
-}
+};
 
-// GELU(z) = z/2 (1 + tanh(u)), u = sqrt(2/pi) (z + 0.044715 z^3), and its
-// derivative Phi + z/2 sech^2(u) sqrt(2/pi) (1 + 3 0.044715 z^2), where
-// Phi = (1 + tanh u) / 2. Both come from w = exp(-2|u|): Phi = 1 / (1 + w)
-// (u >= 0) or w / (1 + w), sech^2 u = 4 w / (1 + w)^2, which stay accurate
-// where tanh saturates (1 - tanh^2 from an approximate tanh would not, and
-// its error there is the same for every pair with large |u|).
+// GELU(z) = z s and GELU'(z) = s + 2 s (1 - s) z u'(z), with s = sigma(2u) =
+// (1 + tanh u) / 2, u = sqrt(2/pi) (z + 0.044715 z^3). s comes from
+// exp(-2u) and one reciprocal, so 1 - s and the sech^2 u = 4 s (1 - s) term
+// keep their accuracy where tanh saturates (1 - tanh^2 of an approximate
+// tanh would not, and its error there is the same for every pair with large
+// |u|). For very negative z, exp(-2u) overflows to +inf and s, h and GELU'
+// all come out 0, their limits.
 __device__ __forceinline__ void gelu_tanh_and_grad(float z, float& h, float& dh) {
   constexpr float kC0 = 0.7978845608028654f, kC1 = 0.044715f;
-  const float z2 = z * z, c0z = kC0 * z;
-  const float u = c0z * fmaf(kC1, z2, 1.f);
-  const float w = ex2(-2.f * kLog2e * fabsf(u));
-  const float r = __fdividef(1.f, 1.f + w);
-  const float phi = u >= 0.f ? r : w * r;
-  h = z * phi;
-  const float sech2 = 4.f * w * r * r;
-  dh = fmaf(0.5f * sech2, c0z * fmaf(3.f * kC1, z2, 1.f), phi);
+  constexpr float kA0 = -2.f * kLog2e * kC0, kA1 = kA0 * kC1;  // -2 log2(e) u = z (kA0 + kA1 z^2)
+  constexpr float kQ0 = 2.f * kC0, kQ1 = 6.f * kC0 * kC1;      // 2 u'(z) = kQ0 + kQ1 z^2
+  const float z2 = z * z;
+  const float w = ex2(z * fmaf(kA1, z2, kA0));
+  float s;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(s) : "f"(1.f + w));
+  h = z * s;
+  const float ss = fmaf(-s, s, s);
+  dh = fmaf(z * fmaf(kQ1, z2, kQ0), ss, s);
 }
 
-// TMEM <- registers, 32 lanes x 16 columns (thread t of the warp writes lane
-// quadrant base + t), then wait for the stores.
-__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const float* v) {
+// The k-th 16-column quarter of a row's packed f16 pair words, as floats.
+__device__ __forceinline__ void unpack_f16x8(const uint32_t* w, float* v) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ void tmem_ld8u_wait(uint32_t taddr, uint32_t* r) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
       : "memory");
 }
 
-// One weight-gradient part: layer L (1..4), 16-row block mb of dW, column
-// blocks nb0 .. nb0 + nc - 1 (the last block index of a layer is the ones
-// column: 8 for L = 2..4, 1 for L = 1).
-struct GradPart {
-  int L, mb, nb0, nc;
+// Instruction descriptor of the weight-gradient MMAs: bf16, M = 128, both
+// operands MN-major (the tiles' row index is the contraction index).
+__host__ __device__ constexpr uint32_t idesc_bf16_m128_mn(int n) {
+  return idesc_bf16_m128(n) | (1u << 15) | (1u << 16);
+}
+
+// One 16-column chunk of a gradient accumulator row into the CTA's partial
+// (folded layout), staged in shared memory. `lane` is the accumulator row
+// (= A^T row), `col` the chunk's first column; the caller's warp holds all 32
+// lanes of its quadrant. Every folded element is written exactly once.
+struct GradOut {
+  float* stage;
+  __device__ __forceinline__ void put(int idx, float v) const { stage[idx] = v; }
+  // first accumulator: rows 0..63 d1 (W1, b1), rows 64..127 d2 (W2, b2)
+  __device__ void g12(int lane, int col, const float* v) const {
+    if (lane < 64) {
+      if (col == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) put(kOffW1 + lane * 4 + i, v[i] + v[4 + i]);  // hi f + lo f
+      } else if (col == kF1Ones) {
+        put(kOffB1 + lane, v[0]);
+      }
+    } else if (col >= 16 && col < 80) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) put(kOffW2 + (lane - 64) * 64 + col - 16 + i, v[i]);
+    } else if (col == kF1Ones) {
+      put(kOffB2 + lane - 64, v[0]);
+    }
+  }
+  // second accumulator: rows 0..63 d3 (W3, b3), rows 64..71 hi g and
+  // 72..79 lo g (W4, b4: their sum), rows 80..127 zero
+  __device__ void g3g(int lane, int col, float* v) const {
+    if (lane >= 64 && lane < 96) {  // one warp: add the lo-g rows to the hi-g rows
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] += __shfl_down_sync(0xffffffffu, v[i], 8);
+    }
+    if (lane < 64) {
+      if (col < 64) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) put(kOffW3 + lane * 64 + col + i, v[i]);
+      } else if (col == kH23Ones) {
+        put(kOffB3 + lane, v[0]);
+      }
+    } else if (lane < 72) {
+      if (col >= 64 && col < 128) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) put(kOffW4 + (lane - 64) * 64 + col - 64 + i, v[i]);
+      } else if (col == kH23Ones) {
+        put(kOffB4 + lane - 64, v[0]);
+      }
+    }
+  }
 };
-
-__device__ __forceinline__ GradPart grad_part(int q) {
-  if (q < 3) return GradPart{4, 0, 3 * q, 3};
-  if (q < 15) return GradPart{3, (q - 3) / 3, 3 * ((q - 3) % 3), 3};
-  if (q < 27) return GradPart{2, (q - 15) / 3, 3 * ((q - 15) % 3), 3};
-  return GradPart{1, q - 27, 0, 2};
-}
-constexpr int kGradParts = 31;
-
-template <int PM>
-__device__ __forceinline__ void grad_tiles(const MlpBwdSmem<PM>& S, const GradPart& gp, const __nv_bfloat16*& Dt,
-                                           int& Kd, const __nv_bfloat16*& Bt, int& Kb, int& ones) {
-  Dt = gp.L == 4 ? S.G4 : S.Ds[gp.L - 1];
-  Kd = gp.L == 4 ? 16 : 64;
-  Bt = gp.L == 1 ? S.A0 : S.Hs[gp.L - 2];
-  Kb = gp.L == 1 ? 16 : 64;
-  ones = gp.L == 1 ? 1 : 8;
-}
-
-// acc[j] += d^T h over the tile's 128 rows for the part's column blocks.
-// Lane addresses are formed once; each 16-row step moves both operands by
-// two 8-row core groups.
-template <int PM>
-__device__ __forceinline__ void grad_mma(const MlpBwdSmem<PM>& S, const GradPart& gp, float (*acc)[4]) {
-  const int lane = threadIdx.x & 31;
-  const __nv_bfloat16 *Dt, *Bt;
-  int Kd, Kb, ones;
-  grad_tiles(S, gp, Dt, Kd, Bt, Kb, ones);
-  const int mi = lane >> 3;
-  const uint32_t a_addr = smem_u32(Dt) + 2u * cofs((lane & 7) + (mi >> 1) * 8, gp.mb * 16 + (mi & 1) * 8, Kd);
-  const uint32_t b_row = smem_u32(Bt) + 2u * cofs((lane & 7) + ((lane >> 3) & 1) * 8, 0, Kb);
-  const uint32_t a_step = (uint32_t)Kd * 32u, b_step = (uint32_t)Kb * 32u;  // 16 rows
-  uint32_t b_addr[3];
-  bool is_one[3];
-#pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    const int nb = gp.nb0 + j;
-    is_one[j] = nb == ones;
-    b_addr[j] = b_row + 128u * (uint32_t)(is_one[j] ? 0 : nb);
-  }
-#pragma unroll 2
-  for (int k = 0; k < kTileM / 16; ++k) {
-    uint32_t a[4];
-    ldsm_x4_t(a_addr + a_step * k, a);
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      if (j >= gp.nc) break;
-      uint32_t b[2];
-      if (is_one[j]) {
-        b[0] = b[1] = 0x3F803F80u;  // bf16 1.0 in both halves
-      } else {
-        ldsm_x2_t(b_addr[j] + b_step * k, b);
-      }
-      mma_16816(acc[j], a, b[0], b[1]);
-    }
-  }
-}
-
-// The part's accumulators into the CTA's partial (folded layout), added to
-// what the slot holds when `accumulate`.
-__device__ void grad_store(const GradPart& gp, float (*acc)[4], float* part, bool accumulate) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int oa = gp.mb * 16 + g, ob = oa + 8;
-  auto put = [&](int idx, float v) { part[idx] = accumulate ? part[idx] + v : v; };
-  for (int j = 0; j < gp.nc; ++j) {
-    const int nb = gp.nb0 + j;
-    const float* c = acc[j];
-    if (gp.L == 1) {
-      // columns 0..3 hold sum d hi(f), 4..7 sum d lo(f)
-      const float p0 = __shfl_down_sync(0xffffffffu, c[0], 2), p1 = __shfl_down_sync(0xffffffffu, c[1], 2);
-      const float p2 = __shfl_down_sync(0xffffffffu, c[2], 2), p3 = __shfl_down_sync(0xffffffffu, c[3], 2);
-      if (nb == 0) {
-        if (t < 2) {
-          put(kOffW1 + oa * 4 + 2 * t, c[0] + p0);
-          put(kOffW1 + oa * 4 + 2 * t + 1, c[1] + p1);
-          put(kOffW1 + ob * 4 + 2 * t, c[2] + p2);
-          put(kOffW1 + ob * 4 + 2 * t + 1, c[3] + p3);
-        }
-      } else if (t == 0) {
-        put(kOffB1 + oa, c[0]);
-        put(kOffB1 + ob, c[2]);
-      }
-    } else if (gp.L == 4) {  // rows g: sum hi(g) h3, rows g + 8: sum lo(g) h3
-      if (nb < 8) {
-        put(kOffW4 + g * 64 + nb * 8 + 2 * t, c[0] + c[2]);
-        put(kOffW4 + g * 64 + nb * 8 + 2 * t + 1, c[1] + c[3]);
-      } else if (t == 0) {
-        put(kOffB4 + g, c[0] + c[2]);
-      }
-    } else {
-      const int offW = gp.L == 2 ? kOffW2 : kOffW3, offB = gp.L == 2 ? kOffB2 : kOffB3;
-      if (nb < 8) {
-        put(offW + oa * 64 + nb * 8 + 2 * t, c[0]);
-        put(offW + oa * 64 + nb * 8 + 2 * t + 1, c[1]);
-        put(offW + ob * 64 + nb * 8 + 2 * t, c[2]);
-        put(offW + ob * 64 + nb * 8 + 2 * t + 1, c[3]);
-      } else if (t == 0) {
-        put(offB + oa, c[0]);
-        put(offB + ob, c[2]);
-      }
-    }
-  }
-}
 
 // The T[N] tiles are split evenly over the CTAs (a CTA's range may start and
 // end inside a jet); the CTA's weight-gradient partial goes to slot
 // blockIdx.x, added to it when `accumulate` (later chunks of a batch).
+// Warps 0..15 stage the operands and run the epilogues; warp 16 issues the
+// MMAs. Each hand-off is an OR-barrier of the 16 warps (any failed wait
+// stops the tile) followed by warp 0's arrive on a barrier the issuer waits
+// on; the epilogue warps then wait for the step's commit, so the issuer has
+// always taken one hand-off before the next one is offered.
+constexpr int kBwdThreads = 544, kBwdIssuer = 16;
+constexpr uint32_t kBarHandoff = 1, kBarEpi = 2;
+enum BwdStep : int { kStepZ1, kStepZ2, kStepZ3, kStepE2, kStepE1, kStepG12, kBwdSteps };
+
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <int PM>
-__global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArgs X, float* __restrict__ partials,
-                                                    int accumulate) {
+__global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArgs X,
+                                                            float* __restrict__ partials, int accumulate) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   MlpBwdSmem<PM>& S = *reinterpret_cast<MlpBwdSmem<PM>*>(smem_raw);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int r = tid & 127, c = tid >> 7;  // tile row (TMEM lane) and column quarter
-  bwd_load_weights<PM>(S, W);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool issuer = warp == kBwdIssuer;
+  const int r = tid & 127, c = (tid >> 7) & 3;  // tile row (TMEM lane) and column quarter (epilogue warps)
+  // this CTA's tiles [lo, hi) of the T[N] and the first jet n0 whose tiles
+  // reach past lo: T is nondecreasing, so n0 is the least n with
+  // T[n + 1] > lo, found by all threads at once (one round trip of loads)
+  BwdWeightLoad wl;
+  wl.load(W, tid, blockDim.x);  // in flight during the search
+  const long long Ttot = X.T[J.N];
+  const long long lo = Ttot * blockIdx.x / gridDim.x, hi = Ttot * (blockIdx.x + 1) / gridDim.x;
+  if (tid == 0) S.n0 = J.N;
+  __syncthreads();
+  {
+    int first = J.N;
+#pragma unroll 4
+    for (int i = tid; i < J.N; i += blockDim.x) {  // independent loads, no early exit
+      const bool past = X.T[i + 1] > lo;
+      first = (past && i < first) ? i : first;
+    }
+    if (first < J.N) atomicMin(&S.n0, first);
+  }
+  __syncthreads();
+  const int n0 = S.n0;
+  if (tid == 32 && lo < hi) prefetch_jet(J, n0);  // into L2 while the weights are converted
+  wl.store(S, tid, blockDim.x);
   if (tid == 0) {
     mbar_init(&S.mbar, 1);
     fence_mbar_init();
+    S.stop = 0;
   }
-  if (warp == 0) tmem_alloc(&S.tmem_base, 256);
+  if (warp == 0) tmem_alloc(&S.tmem_base, kBwdTmemCols);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192) (then GELU'), e3 / e2 / e1 [192, 256)
   const uint32_t tm = S.tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  constexpr uint32_t kId = idesc_bf16_m128(64);
-  const uint32_t a0 = smem_u32(S.A0), g4 = smem_u32(S.G4), w1f = smem_u32(S.W1f);
-  const uint32_t w4t_hi = smem_u32(S.W4t[0]), w4t_lo = smem_u32(S.W4t[1]);
   uint32_t phase = 0u;
-  bool ok = true, aborted = false;
+  bool ok = true, aborted = false, pending = false, any_tile = false;
 
-  const GradPart gp0 = grad_part(warp), gp1 = grad_part(min(warp + 16, kGradParts - 1));
-  const bool has1 = warp + 16 < kGradParts;
-  float acc0[3][4], acc1[3][4];
+  // ---- issuer (warp 16, lane 0 issues): one hand-off per step
+  constexpr uint32_t kId = idesc_bf16_m128(64), kIdF16 = idesc_f16_m128(64);
+  constexpr uint32_t kIdG12 = idesc_bf16_m128_mn(kF1W), kIdG3G = idesc_bf16_m128_mn(kH23W);
+  constexpr uint32_t kF1Sbo = kF1W / 8 * 128, kH23Sbo = kH23W / 8 * 128, kDSbo = kDW / 8 * 128;
+  // D = A (W_hi + W_lo), K = 64, A from TMEM (K step j at column 16j + 8 of
+  // the layer's 64-column block): the weights' rounding error is the same for
+  // every pair row and would not average out of the gradient sums, so they
+  // enter as two terms
+  auto gemm64_ta = [&](uint32_t d, uint32_t a_tm, uint32_t b_hi, uint32_t b_lo, uint32_t id) {
 #pragma unroll
-  for (int j = 0; j < 3; ++j)
+    for (int part = 0; part < 2; ++part)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc0[j][e] = acc1[j][e] = 0.f;
+      for (int k = 0; k < 4; ++k)
+        mma_f16_ta(d, a_tm + 16u * k + 8u, smem_desc((part ? b_lo : b_hi) + 256u * k, 128, 1024), id,
+                   (part | k) != 0 ? 1u : 0u);
+  };
+  // D += A^T B over the tile's 128 rows (K steps of 16 rows = two 8-row
+  // groups); MN-major descriptors: lbo = 8-row group stride, sbo = 8-column
+  // group stride. The first tile's first step overwrites.
+  auto gemm_grad = [&](uint32_t d, uint32_t a, uint32_t a_rows, uint32_t b, uint32_t b_rows, uint32_t id) {
+#pragma unroll
+    for (int k = 0; k < kTileM / 16; ++k)
+      mma_f16(d, smem_desc(a + 2u * a_rows * k, a_rows, 128), smem_desc(b + 2u * b_rows * k, b_rows, 128), id,
+              (any_tile || k != 0) ? 1u : 0u);
+  };
+  auto issue_step = [&](int step) {
+    const uint32_t f1 = smem_u32(S.F1), h23 = smem_u32(S.H23), d12 = smem_u32(S.D12), d3g = smem_u32(S.D3G);
+    switch (step) {
+      case kStepZ1: {  // z1 = [hi f | lo f | hi f] [hi W1 | hi W1 | lo W1]; behind it e3 = [hi g | lo g] [W4 | W4]
+        mma_f16(tm, smem_desc(f1, 128, kF1Sbo), smem_desc(smem_u32(S.W1f), 128, 256), kId, 0u);
+        mma_commit(&S.mbar);
+        const uint64_t ga = smem_desc(d3g + kD3G / 8 * 128, 128, kDSbo);
+        mma_f16(tm + 192u, ga, smem_desc(smem_u32(S.W4t[0]), 128, 256), kId, 0u);
+        mma_f16(tm + 192u, ga, smem_desc(smem_u32(S.W4t[1]), 128, 256), kId, 1u);
+        break;
+      }
+      case kStepZ2:  // its commit also covers e3
+        gemm64_ta(tm + 64u, tm, smem_u32(S.Wf[0][0]), smem_u32(S.Wf[0][1]), kIdF16);
+        mma_commit(&S.mbar);
+        break;
+      case kStepZ3:
+        gemm64_ta(tm + 128u, tm + 64u, smem_u32(S.Wf[1][0]), smem_u32(S.Wf[1][1]), kIdF16);
+        mma_commit(&S.mbar);
+        break;
+      case kStepE2:  // e2 = d3 W3' (d3 bf16 in TMEM over z3)
+        gemm64_ta(tm + 192u, tm + 128u, smem_u32(S.Wt[1][0]), smem_u32(S.Wt[1][1]), kId);
+        mma_commit(&S.mbar);
+        break;
+      case kStepE1:  // e1 = d2 W2', then (not delaying e1) [d3 | g]^T [h2 | h3 | 1]
+        gemm64_ta(tm + 192u, tm + 64u, smem_u32(S.Wt[0][0]), smem_u32(S.Wt[0][1]), kId);
+        mma_commit(&S.mbar);
+        gemm_grad(tm + kTmG3G, d3g, kDSbo, h23, kH23Sbo, kIdG3G);
+        break;
+      default:  // [d1 | d2]^T [f | h1 | 1]; its commit also covers the one above
+        gemm_grad(tm + kTmG12, d12, kDSbo, f1, kF1Sbo, kIdG12);
+        mma_commit(&S.mbar);
+        break;
+    }
+  };
+  // one tile's steps; false when the epilogue warps stopped
+  auto issue_tile = [&]() -> bool {
+    for (int step = 0; step < kBwdSteps; ++step) {
+      named_bar(kBarHandoff, 64);
+      tc_fence_after();
+      if (*reinterpret_cast<volatile int*>(&S.stop)) return false;
+      if (lane == 0) issue_step(step);
+      __syncwarp();
+    }
+    any_tile = true;
+    return true;
+  };
 
-  // operand writes published, then thread 0 issues `body` and commits
-  auto issue = [&](auto&& body) -> bool {
+  // ---- epilogue warps
+  // operand writes published and offered to the issuer; false (for all 16
+  // warps) once any of their waits has failed
+  auto handoff = [&]() -> bool {
     fence_proxy_async_smem();
     tc_fence_before();
-    if (__syncthreads_or(!ok)) return false;
-    if (tid == 0) {
-      tc_fence_after();
-      body();
-      mma_commit(&S.mbar);
+    const bool stop = named_bar_or(kBarEpi, 512, !ok);
+    if (warp == 0) {
+      if (lane == 0) S.stop = stop ? 1 : 0;
+      __syncwarp();
+      named_bar_arrive(kBarHandoff, 64);
     }
-    return true;
+    return !stop;
   };
   auto wait = [&]() {
     const bool done = mbar_wait(&S.mbar, phase);
@@ -620,31 +756,25 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
     ok = ok && done;
     tc_fence_after();
   };
-  // D = A (W_hi + W_lo): the weights' rounding error is the same for every
-  // pair row and would not average out of the gradient sums, so they enter as
-  // two terms. The recompute's products (A = h, f16) use kind::f16 with f16
-  // operands, the backward's (A = d, bf16) bf16 operands.
-  auto gemm64 = [&](uint32_t d, uint32_t aa, uint32_t b_hi, uint32_t b_lo, uint32_t id) {
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      const uint32_t bb = part ? b_lo : b_hi;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_f16(d, smem_desc(aa + 256u * k, 128, 1024), smem_desc(bb + 256u * k, 128, 1024), id,
-                (part | k) != 0 ? 1u : 0u);
-    }
-  };
-  constexpr uint32_t kIdF16 = idesc_f16_m128(64);
-  auto store16 = [&](void* T, const float* v, bool f16) {
+  auto store16 = [&](__nv_bfloat16* T, int width, int col, const float* v) {
     uint32_t w[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = f16 ? cvt_f16x2(v[2 * i], v[2 * i + 1]) : cvt_bf16x2(v[2 * i], v[2 * i + 1]);
-    uint16_t* T16 = static_cast<uint16_t*>(T);
-    *reinterpret_cast<uint4*>(T16 + cofs(r, 16 * c, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(T16 + cofs(r, 16 * c + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
+    for (int i = 0; i < 8; ++i) w[i] = cvt_bf16x2(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4*>(T + cofs(r, col, width)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(T + cofs(r, col + 8, width)) = make_uint4(w[4], w[5], w[6], w[7]);
   };
-  // h_k = GELU(z_k + b_k) to the operand tile, GELU'(z_k + b_k) back over z_k in TMEM
-  auto hidden = [&](int k) {
+  // d (bf16) into the second half of the quarter's TMEM columns of block k:
+  // the A operand of the next backward product
+  auto d_to_tmem = [&](int k, const float* v) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = cvt_bf16x2(v[2 * i], v[2 * i + 1]);
+    tmem_st8_wait(tm + lane_off + 64u * k + 16u * c + 8u, w);
+  };
+  // z_k + b_k -> h (bf16 to `T` at column `col`; for k < 2 f16 into TMEM as
+  // the next layer's A operand) and GELU' (f16 into TMEM, k < 2) or, for
+  // k = 2, d3 = e3 GELU'(z3) to D3G and TMEM
+  auto hidden = [&](int k, __nv_bfloat16* T, int width, int col) {
     float z[16], h[16];
     const uint32_t ta = tm + lane_off + 64u * k + 16u * c;
     tmem_ld16_wait(ta, z);
@@ -659,157 +789,230 @@ __global__ void __launch_bounds__(512, 1) k_mlp_bwd(JetArgs J, MlpArgs W, BwdArg
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) gelu_tanh_and_grad(z[i], h[i], z[i]);
-    if (k < 2) store16(S.Hf[k], h, true);  // the next layer's operand
-    store16(S.Hs[k], h, false);
-    tmem_st16_wait(ta, z);
+    store16(T, width, col, h);
+    if (k < 2) {
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        w[i] = cvt_f16x2(z[2 * i], z[2 * i + 1]);
+        w[8 + i] = cvt_f16x2(h[2 * i], h[2 * i + 1]);
+      }
+      tmem_st16_wait_u(ta, w);
+    } else {
+      float e[16];
+      tmem_ld16_wait(tm + lane_off + 192u + 16u * c, e);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) e[i] *= z[i];
+      store16(S.D3G, kDW, 16 * c, e);
+      d_to_tmem(2, e);
+    }
   };
-  // d_k = e * GELU'(z_k + b_k)
+  // d_k = e_k GELU'(z_k) (k = 1, 0) into D12 (and d2 into TMEM)
   auto delta = [&](int k) {
+    uint32_t gw[8];
     float gp[16], e[16];
-    tmem_ld16_wait(tm + lane_off + 64u * k + 16u * c, gp);
+    tmem_ld8u_wait(tm + lane_off + 64u * k + 16u * c, gw);
     tmem_ld16_wait(tm + lane_off + 192u + 16u * c, e);
+    unpack_f16x8(gw, gp);
 #pragma unroll
     for (int i = 0; i < 16; ++i) e[i] *= gp[i];
-    store16(S.Ds[k], e, false);
+    store16(S.D12, kDW, 64 * k + 16 * c, e);
+    if (k == 1) d_to_tmem(1, e);
+  };
+  // tile t's row r as operand words: features (c = 0: [hi f | lo f], [hi f | 0])
+  // or the gradient record (c = 1: hi g, lo g); zero past the jet's pairs
+  auto prep = [&](int t, int m, const float* gjet, uint4& w0, uint4& w1) {
+    const int p = t * kTileM + r;
+    bool valid = p < m * (m + 1) / 2;
+    w0 = make_uint4(0u, 0u, 0u, 0u);
+    w1 = w0;
+    if (c == 0) {
+      int a = 0, b = 0;
+      if (valid) {
+        TriPairs{}.map(p, a, b);
+        valid = in_bounds(a >= 0 && a <= b && b < m);
+      }
+      float f[4] = {0.f, 0.f, 0.f, 0.f};
+      if (valid) pair_feat<PM, true>(S.part, a, b, f);  // the forward MLP's features
+      const uint32_t h01 = cvt_bf16x2(f[0], f[1]), h23w = cvt_bf16x2(f[2], f[3]);
+      const uint32_t l01 = cvt_bf16x2(f[0] - bf16lo(h01), f[1] - bf16hi(h01));
+      const uint32_t l23 = cvt_bf16x2(f[2] - bf16lo(h23w), f[3] - bf16hi(h23w));
+      w0 = make_uint4(h01, h23w, l01, l23);
+      w1 = make_uint4(h01, h23w, 0u, 0u);
+    } else if (c == 1) {
+      float gv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (valid) {
+        const float4 u0 = *reinterpret_cast<const float4*>(gjet + (size_t)p * 8);
+        const float4 u1 = *reinterpret_cast<const float4*>(gjet + (size_t)p * 8 + 4);
+        gv[0] = u0.x; gv[1] = u0.y; gv[2] = u0.z; gv[3] = u0.w;
+        gv[4] = u1.x; gv[5] = u1.y; gv[6] = u1.z; gv[7] = u1.w;
+      }
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        hw[i] = cvt_bf16x2(gv[2 * i], gv[2 * i + 1]);
+        lw[i] = cvt_bf16x2(gv[2 * i] - bf16lo(hw[i]), gv[2 * i + 1] - bf16hi(hw[i]));
+      }
+      w0 = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      w1 = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+  };
+  // one tile; false when stopped
+  auto epilogue_tile = [&](int t, int t_last, int m, const float* gjet, uint4& w0, uint4& w1, bool& have) -> bool {
+    if (!have) prep(t, m, gjet, w0, w1);
+    have = false;
+    if (pending) {  // the previous tile's gradient MMAs read F1, H23, D12 and D3G
+      wait();
+      pending = false;
+    }
+    if (c == 0) {
+      *reinterpret_cast<uint4*>(S.F1 + cofs(r, 0, kF1W)) = w0;
+      *reinterpret_cast<uint4*>(S.F1 + cofs(r, 8, kF1W)) = w1;
+    } else if (c == 1) {
+      *reinterpret_cast<uint4*>(S.D3G + cofs(r, kD3G, kDW)) = w0;
+      *reinterpret_cast<uint4*>(S.D3G + cofs(r, kD3G + 8, kDW)) = w1;
+    }
+    if (!handoff()) return false;  // z1, e3
+    wait();
+    hidden(0, S.F1, kF1W, 16 + 16 * c);
+    if (!handoff()) return false;  // z2
+    wait();
+    hidden(1, S.H23, kH23W, 16 * c);
+    if (!handoff()) return false;  // z3
+    wait();
+    hidden(2, S.H23, kH23W, 64 + 16 * c);
+    if (!handoff()) return false;  // e2
+    if (t + 1 < t_last) {          // the next tile's operand words while e2 runs
+      prep(t + 1, m, gjet, w0, w1);
+      have = true;
+    }
+    wait();
+    delta(1);
+    if (!handoff()) return false;  // e1, then the [d3 | g] gradient
+    wait();
+    delta(0);
+    if (!handoff()) return false;  // the [d1 | d2] gradient
+    pending = true;
+    any_tile = true;
+    return true;
   };
 
-  const long long Ttot = X.T[J.N];
-  const long long lo = Ttot * blockIdx.x / gridDim.x, hi = Ttot * (blockIdx.x + 1) / gridDim.x;
-  int n = 0;
-  {
-    int l = 0, rr = J.N;  // first jet whose tiles reach past lo
-    while (l < rr) {
-      const int mid = (l + rr) >> 1;
-      if (X.T[mid + 1] > lo) rr = mid; else l = mid + 1;
-    }
-    n = l;
-  }
+  int n = n0;
+  uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
   for (; n < J.N && X.T[n] < hi && !aborted; ++n) {
     const long long tj0 = X.T[n], tj1 = X.T[n + 1];
     if (tj1 <= tj0) continue;  // no pairs
     stage_jet<PM>(S.part, J, n);
+    if (tid == 32 && X.T[n + 1] < hi) prefetch_jet(J, n + 1);  // this CTA's next jet, if it has one
     const int m = S.part.m;
-    const int npairs = m * (m + 1) / 2;
     const float* gjet = X.grec + (size_t)tj0 * kTileM * 8;
     const int t_first = (int)(max(lo, tj0) - tj0), t_last = (int)(min(hi, tj1) - tj0);
-    for (int t = t_first; t < t_last; ++t) {
-      // row r: the unordered pair p = b(b+1)/2 + a; features (c = 0) and g (c = 1)
-      const int p = t * kTileM + r;
-      int a = 0, b = 0;
-      bool valid = p < npairs;
-      if (valid && c == 0) {
-        TriPairs{}.map(p, a, b);
-        valid = in_bounds(a >= 0 && a <= b && b < m);
-      }
-      if (c == 0) {
-        float f[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) pair_feat<PM, true>(S.part, a, b, f);  // the forward MLP's features
-        const uint32_t h01 = cvt_bf16x2(f[0], f[1]), h23 = cvt_bf16x2(f[2], f[3]);
-        const uint32_t l01 = cvt_bf16x2(f[0] - bf16lo(h01), f[1] - bf16hi(h01));
-        const uint32_t l23 = cvt_bf16x2(f[2] - bf16lo(h23), f[3] - bf16hi(h23));
-        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 0, 16)) = make_uint4(h01, h23, l01, l23);
-        *reinterpret_cast<uint4*>(S.A0 + cofs(r, 8, 16)) = make_uint4(h01, h23, 0u, 0u);
-      } else if (c == 1) {
-        float gv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (valid) {
-          const float4 u0 = *reinterpret_cast<const float4*>(gjet + (size_t)p * 8);
-          const float4 u1 = *reinterpret_cast<const float4*>(gjet + (size_t)p * 8 + 4);
-          gv[0] = u0.x; gv[1] = u0.y; gv[2] = u0.z; gv[3] = u0.w;
-          gv[4] = u1.x; gv[5] = u1.y; gv[6] = u1.z; gv[7] = u1.w;
-        }
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          hw[i] = cvt_bf16x2(gv[2 * i], gv[2 * i + 1]);
-          lw[i] = cvt_bf16x2(gv[2 * i] - bf16lo(hw[i]), gv[2 * i + 1] - bf16hi(hw[i]));
-        }
-        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 0, 16)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(S.G4 + cofs(r, 8, 16)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      }
-      // forward: z1 (and e3 = g W4, which needs nothing else), z2, z3
-      if (!issue([&] {
-            mma_f16(tm, smem_desc(a0, 128, 256), smem_desc(w1f, 128, 256), kId, 0u);
-            mma_f16(tm + 192u, smem_desc(g4, 128, 256), smem_desc(w4t_hi, 128, 256), kId, 0u);
-            mma_f16(tm + 192u, smem_desc(g4, 128, 256), smem_desc(w4t_lo, 128, 256), kId, 1u);
-          })) {
-        aborted = true;
-        break;
-      }
-      wait();
-      hidden(0);
-      if (!issue([&] { gemm64(tm + 64u, smem_u32(S.Hf[0]), smem_u32(S.Wf[0][0]), smem_u32(S.Wf[0][1]), kIdF16); })) {
-        aborted = true;
-        break;
-      }
-      wait();
-      hidden(1);
-      if (!issue([&] { gemm64(tm + 128u, smem_u32(S.Hf[1]), smem_u32(S.Wf[1][0]), smem_u32(S.Wf[1][1]), kIdF16); })) {
-        aborted = true;
-        break;
-      }
-      wait();
-      hidden(2);
-      delta(2);
-      // backward: e2 = d3 W3', e1 = d2 W2'
-      if (!issue([&] { gemm64(tm + 192u, smem_u32(S.Ds[2]), smem_u32(S.Wt[1][0]), smem_u32(S.Wt[1][1]), kId); })) {
-        aborted = true;
-        break;
-      }
-      wait();
-      delta(1);
-      if (!issue([&] { gemm64(tm + 192u, smem_u32(S.Ds[1]), smem_u32(S.Wt[0][0]), smem_u32(S.Wt[0][1]), kId); })) {
-        aborted = true;
-        break;
-      }
-      wait();
-      delta(0);
-      __syncthreads();  // every tile row written before the weight-gradient MMAs read them
-      grad_mma(S, gp0, acc0);
-      if (has1) grad_mma(S, gp1, acc1);
-      tc_fence_before();
-      __syncthreads();  // operands and TMEM free for the next tile
-      tc_fence_after();
-    }
+    bool have = false;
+    for (int t = t_first; t < t_last && !aborted; ++t)
+      aborted = issuer ? !issue_tile() : !epilogue_tile(t, t_last, m, gjet, w0, w1, have);
     aborted = __syncthreads_or(aborted || !ok) != 0;
   }
-  float* part = partials + (size_t)blockIdx.x * kFoldedFloats;
-  grad_store(gp0, acc0, part, accumulate != 0);
-  if (has1) grad_store(gp1, acc1, part, accumulate != 0);
+  if (pending && !aborted) wait();
+  aborted = __syncthreads_or(aborted || !ok) != 0;
+  tc_fence_after();
+  any_tile = __syncthreads_or(any_tile) != 0;
+  // the accumulators (all-zero when the CTA had no tile) into the partial,
+  // through shared memory (the gradient operand tiles, free now) so that the
+  // global writes are whole float4 rows
+  float* stage = reinterpret_cast<float*>(S.D12);
+  static_assert(sizeof(S.D12) + sizeof(S.D3G) >= kFoldedFloats * sizeof(float) &&
+                    offsetof(MlpBwdSmem<PM>, D3G) == offsetof(MlpBwdSmem<PM>, D12) + sizeof(S.D12),
+                "the staged partial spans D12 and D3G");
+  if (!aborted && !issuer) {
+    const GradOut go{stage};
+    // quarter c reads the 16-column chunks c, c + 4, ... of the 15 (6 + 9)
+    for (int q = c; q < (kF1W + kH23W) / 16; q += 4) {
+      float v[16];
+      const bool g12 = q < kF1W / 16;
+      const int col = g12 ? 16 * q : 16 * q - kF1W;
+      if (any_tile) {
+        tmem_ld16_wait(tm + lane_off + (g12 ? kTmG12 : kTmG3G) + (uint32_t)col, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      }
+      if (g12) go.g12(r, col, v); else go.g3g(r, col, v);
+    }
+  }
   tc_fence_before();
   __syncthreads();
+  if (!aborted) {
+    float4* part = reinterpret_cast<float4*>(partials + (size_t)blockIdx.x * kFoldedFloats);
+    const float4* st4 = reinterpret_cast<const float4*>(stage);
+    for (int q = tid; q < kFoldedFloats / 4; q += blockDim.x) {
+      float4 v = st4[q];
+      if (accumulate) {
+        const float4 o = part[q];
+        v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+      }
+      part[q] = v;
+    }
+  }
   if (aborted && tid == 0) (void)mbar_wait(&S.mbar, phase ^ 1u);  // bounded: the last commit before TMEM is freed
   __syncthreads();
-  if (warp == 0) tmem_dealloc(S.tmem_base, 256);
+  if (warp == 0) tmem_dealloc(S.tmem_base, kBwdTmemCols);
 }
 
 // Weight gradients: the sum over the CTAs' partials in a fixed order. CTA
-// x owns 32 consecutive elements; warp w sums the slots w, w + 8, ... in
-// order, then the eight warp sums are added in warp order.
-constexpr int kReduceCtas = (kFoldedFloats + 31) / 32;
+// x owns 32 consecutive float4 columns (128 elements); warp w of 16 sums the
+// slots w, w + 16, ... in order (all its loads in flight at once), then the
+// sixteen warp sums are added in warp order. The folded arrays start at
+// multiples of 4 elements, so a column never straddles two of them.
+constexpr int kReduceCols = kFoldedFloats / 4;
+constexpr int kReduceCtas = (kReduceCols + 31) / 32;
+constexpr int kReduceWarps = 16;
+static_assert(kBwdMaxCtas <= 16 * kReduceWarps, "one fully unrolled pass over the slots");
+static_assert(kFoldedFloats % 4 == 0 && kOffB1 % 4 == 0 && kOffW2 % 4 == 0 && kOffB2 % 4 == 0 &&
+                  kOffW3 % 4 == 0 && kOffB3 % 4 == 0 && kOffW4 % 4 == 0 && kOffB4 % 4 == 0,
+              "float4 columns of the folded layout");
 
-__global__ void __launch_bounds__(256) k_grad_reduce(const float* __restrict__ partials, int nparts, GradArgs G) {
-  __shared__ float wsum[8][32];
+__global__ void __launch_bounds__(32 * kReduceWarps) k_grad_reduce(const float* __restrict__ partials, int nparts,
+                                                                   GradArgs G) {
+  __shared__ float4 wsum[kReduceWarps][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int e = blockIdx.x * 32 + lane;
-  float s = 0.f;
-  if (e < kFoldedFloats) {
-#pragma unroll 4
-    for (int c = w; c < nparts; c += 8) s += partials[(size_t)c * kFoldedFloats + e];
+  const int j = blockIdx.x * 32 + lane;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (j < kReduceCols) {
+    const float4* P = reinterpret_cast<const float4*>(partials) + j;
+    float4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = w + i * kReduceWarps;
+      v[i] = c < nparts ? P[(size_t)c * kReduceCols] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      s.x += v[i].x; s.y += v[i].y; s.z += v[i].z; s.w += v[i].w;
+    }
   }
   wsum[w][lane] = s;
   __syncthreads();
-  if (w != 0 || e >= kFoldedFloats) return;
-  float t = 0.f;
+  if (w != 0 || j >= kReduceCols) return;
+  float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) t += wsum[q][lane];
-  if (e < kOffB1) G.W1[e - kOffW1] = t;
-  else if (e < kOffW2) G.b1[e - kOffB1] = t;
-  else if (e < kOffB2) G.W2[e - kOffW2] = t;
-  else if (e < kOffW3) G.b2[e - kOffB2] = t;
-  else if (e < kOffB3) G.W3[e - kOffW3] = t;
-  else if (e < kOffW4) G.b3[e - kOffB3] = t;
-  else if (e < kOffB4) G.W4[e - kOffW4] = t;
-  else G.b4[e - kOffB4] = t;
+  for (int q = 0; q < kReduceWarps; ++q) {
+    const float4 v = wsum[q][lane];
+    t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+  }
+  const int e = 4 * j;
+  float* dst;
+  if (e < kOffB1) dst = G.W1 + (e - kOffW1);
+  else if (e < kOffW2) dst = G.b1 + (e - kOffB1);
+  else if (e < kOffB2) dst = G.W2 + (e - kOffW2);
+  else if (e < kOffW3) dst = G.b2 + (e - kOffB2);
+  else if (e < kOffB3) dst = G.W3 + (e - kOffW3);
+  else if (e < kOffW4) dst = G.b3 + (e - kOffB3);
+  else if (e < kOffB4) dst = G.W4 + (e - kOffW4);
+  else dst = G.b4 + (e - kOffB4);
+  dst[0] = t.x;
+  dst[1] = t.y;
+  dst[2] = t.z;
+  dst[3] = t.w;
 }
 
 }  // namespace pb

@@ -37,13 +37,13 @@ JET_VIOLATIONS = ["jets_null", "n_negative", "p_zero", "p_too_big", "momentum_nu
                   "layout_missing", "ptr_misaligned", "tokens_negative"]
 ENTRY_VIOLATIONS = {
     "pairfeat": ["feat_null", "feat_misaligned"],
-    "mlp_forward": ["mlp_null", "mlp_field_null", "u_null", "u_misaligned", "dtype_bad"],
+    "mlp_forward": ["mlp_null", "mlp_field_null", "mlp_misaligned", "u_null", "u_misaligned", "dtype_bad"],
     "attention": ["hd_bad", "mlp_and_u", "neither", "qkvo_null", "qkvo_misaligned", "u_misaligned",
-                  "mlp_field_null", "ws_misaligned"],
-    "noalloc": ["hd_bad", "mlp_null", "mlp_field_null", "qkvo_null", "qkvo_misaligned"],
-    "block": ["hde_bad", "mlp_null", "proj_null", "proj_field_null", "proj_misaligned", "xy_null",
+                  "mlp_field_null", "mlp_misaligned", "ws_misaligned"],
+    "noalloc": ["hd_bad", "mlp_null", "mlp_field_null", "mlp_misaligned", "qkvo_null", "qkvo_misaligned"],
+    "block": ["hde_bad", "mlp_null", "mlp_misaligned", "proj_null", "proj_field_null", "proj_misaligned", "xy_null",
               "xy_misaligned", "ws_null", "ws_misaligned", "ws_small"],
-    "backward": ["hd_bad", "mlp_null", "dmlp_null", "dmlp_field_null", "dmlp_misaligned", "qkv_grad_null",
+    "backward": ["hd_bad", "mlp_null", "mlp_misaligned", "dmlp_null", "dmlp_field_null", "dmlp_misaligned", "qkv_grad_null",
                  "qkv_grad_misaligned", "ws_null", "ws_misaligned", "ws_small"],
     "mlp_forward_i8": ["mlp_null", "i8_field_null", "i8_codes_misaligned", "u_null", "u_misaligned", "dtype_bad"],
     "attention_i8": ["hd_bad", "mlp_null", "i8_field_null", "i8_codes_misaligned", "qkvo_null", "qkvo_misaligned"],
@@ -81,6 +81,8 @@ def _call(L, entry, jets, v):
     d = _ptr(8)
     mis = lambda p, bad: p + 2 if bad else p  # noqa: E731
     mlp = None if "mlp_null" in v else ops._Mlp(*([_ptr(10)] * 7 + [0 if "mlp_field_null" in v else _ptr(11)]))
+    if mlp is not None and "mlp_misaligned" in v:
+        mlp.W3 = _ptr(10) + 4  # 4-byte aligned floats, but the matrices need 16
     mlp_ref = None if mlp is None else C.byref(mlp)
     q, k, vv, out = (None if "qkvo_null" in v and i == 3 else mis(_ptr(12 + i), "qkvo_misaligned" in v and i == 1)
                      for i in range(4))
