@@ -64,31 +64,21 @@ struct BwdArgs {
 __host__ __device__ constexpr int bwd_tensor_bytes(int m) { return round16(m) * kKStride * 2; }
 __host__ __device__ constexpr int bwd_head_bytes(int m) { return 4 * bwd_tensor_bytes(m) + 8 * round16(m); }
 
+// Asynchronous 16-byte copies, committed as one group with whatever the
+// caller issued before; the caller waits (cp_async_wait_all and a barrier).
 template <int PM>
 __device__ void stage_bwd(const Particles<PM>& S, const JetArgs& J, const BwdArgs& X, int n, int h0, int hr,
                           unsigned char* buf) {
   const int m = S.m, m16 = round16(m), hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m);
   const int total = hr * m16 * 8, nthr = blockDim.x;
-  for (int base = threadIdx.x; base < total; base += 4 * nthr) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int idx = base + u * nthr;
-      const int part = idx & 7, j = (idx >> 3) % m16, hh = (idx >> 3) / m16;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (idx < total && j < m) {
-        const uint16_t* src = part < 2 ? X.q : (part < 4 ? X.k : (part < 6 ? X.v : X.dout));
-        v[u] = *reinterpret_cast<const uint4*>(src + qkv_off<PM>(S, J, n, h0 + hh, j) + (part & 1) * 8);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int idx = base + u * nthr;
-      if (idx >= total) break;
-      const int part = idx & 7, j = (idx >> 3) % m16, hh = (idx >> 3) / m16;
-      *reinterpret_cast<uint4*>(buf + hh * hb + (part >> 1) * tb + j * kKStride * 2 + (part & 1) * 16) = v[u];
-    }
+  for (int idx = threadIdx.x; idx < total; idx += nthr) {
+    const int part = idx & 7, j = (idx >> 3) % m16, hh = (idx >> 3) / m16;
+    const bool valid = j < m;
+    const uint16_t* src = part < 2 ? X.q : (part < 4 ? X.k : (part < 6 ? X.v : X.dout));
+    cp_async16(buf + hh * hb + (part >> 1) * tb + j * kKStride * 2 + (part & 1) * 16,
+               src + (valid ? qkv_off<PM>(S, J, n, h0 + hh, j) : 0) + (part & 1) * 8, valid ? 16u : 0u);
   }
+  cp_async_commit();
   // lse and D of rows m .. m16-1 (read, masked, by the key pass) are 0
   for (int idx = threadIdx.x; idx < hr * 2 * m16; idx += nthr) {
     const int hh = idx / (2 * m16), r = idx % (2 * m16);
@@ -297,6 +287,36 @@ struct AttnBwdSmem {
   Particles<PM> part;
 };
 
+// The CTA's kHG heads of a jet's bias triangle, copied from the records into
+// shared memory (kHG halves per pair): one asynchronous 8-byte copy per pair
+// (the record's heads h0 .. h0 + 3), left uncommitted for the next commit.
+template <int kHG>
+__device__ void stage_bias_heads(const uint4* __restrict__ rec, int npairs, int h0, __half* U) {
+  static_assert(kHG == 4, "8-byte pieces of 4 heads");
+  const uint32_t u0 = smem_u32(U);
+  const char* src0 = reinterpret_cast<const char*>(rec) + h0 * 2;
+  for (int p = threadIdx.x; p < npairs; p += blockDim.x)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(u0 + 8u * (uint32_t)p), "l"(src0 + 16 * (size_t)p)
+                 : "memory");
+}
+
+struct SmemUBias4 {  // the CTA's 4 heads from h0, staged by stage_bias_heads
+  const __half* U;
+  int h0;
+  __device__ __forceinline__ TriBlockS<4> head(int h) const { return TriBlockS<4>{U + (h - h0)}; }
+};
+
+// Masked rows (slot s with comp[s] < 0) of `out`, every head: 16 threads per
+// slot, thread (head, half) of it, no division.
+template <int PM>
+__device__ void zero_masked_rows_bwd(const Particles<PM>& S, const JetArgs& J, uint16_t* out, int n) {
+  if (J.ptr) return;
+  const int P = J.P, hh = (threadIdx.x >> 1) & 7, half = threadIdx.x & 1;
+  for (int s = threadIdx.x >> 4; s < P; s += blockDim.x >> 4)
+    if (S.comp[s] < 0)
+      *reinterpret_cast<uint4*>(out + (((size_t)n * kH + hh) * P + s) * kD + half * 8) = make_uint4(0, 0, 0, 0);
+}
+
 template <int PM>
 __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -311,12 +331,17 @@ __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
     if (m > 0) {
       const int hb = bwd_head_bytes(m), tb = bwd_tensor_bytes(m), m16 = round16(m);
       const int HR = max(1, min(kHG, kBwdStageBytes / hb));
-      const int tiles = (m + 15) >> 4;
-      const RecordUBias ub{reinterpret_cast<const __half*>(X.urec + rowbase)};
-      if (in_bounds(hb <= kBwdStageBytes)) {
+      const int tiles = (m + 15) >> 4, npairs = m * (m + 1) / 2;
+      // the bias from shared memory when all the CTA's heads and their
+      // triangle fit the stage at once, else from the records in L2
+      const bool u_smem = HR == kHG && kHG * hb + npairs * kHG * 2 <= kBwdStageBytes;
+      __half* Us = reinterpret_cast<__half*>(S.stage + kHG * hb);
+      auto pass = [&](const auto& ub) {
         for (int h0 = hg * kHG; h0 < (hg + 1) * kHG; h0 += HR) {
           const int hr = min(HR, (hg + 1) * kHG - h0);
+          if (u_smem) stage_bias_heads<kHG>(X.urec + rowbase, npairs, hg * kHG, Us);
           stage_bwd<PM>(S.part, J, X, n, h0, hr, S.stage);
+          cp_async_wait_all();
           __syncthreads();
           for (int it = warp; it < hr * tiles; it += nwarp) {
             const int hh = it / tiles, h = h0 + hh;
@@ -336,13 +361,18 @@ __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
           }
           __syncthreads();
         }
+      };
+      if (in_bounds(hb <= kBwdStageBytes)) {
+        if (u_smem) pass(SmemUBias4{Us, hg * kHG});
+        else pass(RecordUBias{reinterpret_cast<const __half*>(X.urec + rowbase)});
       }
     }
-    if (hg == 0) {  // masked rows of every head
-      zero_masked_rows<PM>(S.part, J, X.dq, n);
-      zero_masked_rows<PM>(S.part, J, X.dk, n);
-      zero_masked_rows<PM>(S.part, J, X.dv, n);
+    // masked rows of every head: dq and dk by the jet's first CTA, dv by its second
+    if (hg == 0) {
+      zero_masked_rows_bwd<PM>(S.part, J, X.dq, n);
+      zero_masked_rows_bwd<PM>(S.part, J, X.dk, n);
     }
+    if (hg == kBwdHeadGroups - 1) zero_masked_rows_bwd<PM>(S.part, J, X.dv, n);
     __syncthreads();
   }
 }
