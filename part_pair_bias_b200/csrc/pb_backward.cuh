@@ -390,9 +390,10 @@ __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
 //   [dW2' | db2'; dW1' | db1'] += [d2 | d1]^T [f | h1 | 1]
 //   [dW3' | db3'; dW4 | db4]   += [d3 | g]^T  [h2 | h3 | 1]
 // The recompute multiplies f16 h (two per TMEM column, the A operand read
-// from TMEM) by f16 hi + lo weights; the backward products take bf16 d and
-// bf16 hi + lo weights; f, g and the folded layer-1 weights enter as bf16
-// hi + lo terms. The weight gradients are two MMAs per tile over the tile's
+// from TMEM) by the f16 weights, as the forward kernels do, and adds the
+// layer's bias through one more MMA (a TMEM block of ones times [hi b | lo b]);
+// the backward products take bf16 d and bf16 hi + lo weights; f, g and the
+// folded layer-1 weights and bias enter as bf16 hi + lo terms. The weight gradients are two MMAs per tile over the tile's
 // rows (K = 128) with both operands read transposed (MN-major) from the same
 // row-major tiles, accumulated in fp32 TMEM over all the CTA's tiles; the
 // second overlaps the next tile's feature and gradient-record loads. GELU is
@@ -411,12 +412,18 @@ struct GradArgs {
 
 // Operand tiles of one 128-row tile (bf16, columns as listed; each in the
 // canonical no-swizzle layout of cofs with its own width):
-//   F1  [hi f | lo f | hi f | 0 | h1 | 1 | 0]  96 wide: A of z1 (columns 0..15), B of the first gradient MMA
-//   H23 [h2 | h3 | 1 | 0]                     144 wide: B of the second gradient MMA
-//   D12 [d1 | d2]                             128 wide: A of e1 (columns 64..127), A^T of the first
-//   D3G [d3 | hi g | lo g | 0]                128 wide: A of e2 (0..63) and e3 (64..79), A^T of the second
+//   Z1A [hi f | lo f | hi f | 1 1 0 0]           16 wide: A of z1 (the ones carry b1)
+//   G4  [hi g | lo g]                            16 wide: A of e3
+//   F1  [hi f | lo f | hi f | 0 | h1 | 1 | 0]    96 wide: B of the first gradient MMA
+//   H23 [h2 | h3 | 1 | 0]                       144 wide: B of the second gradient MMA
+//   D12 [d1 | d2]                               128 wide: A^T of the first gradient MMA
+//   D3G [d3 | hi g | lo g | 0]                  128 wide: A^T of the second gradient MMA
+// Z1A and G4 are written at a tile's start; the f and g columns of F1 and D3G
+// only once the tile's z1 is done, which in MMA order is after the previous
+// tile's gradient MMAs: the next tile never waits for those.
 constexpr int kF1W = 96, kH23W = 144, kDW = 128;
 constexpr int kF1Ones = 80, kH23Ones = 128, kD3G = 64;
+constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;  // bf16 1.0 in both halves
 
 template <int PM>
 struct MlpBwdSmem {
@@ -424,12 +431,15 @@ struct MlpBwdSmem {
   __nv_bfloat16 H23[kTileM * kH23W];
   __nv_bfloat16 D12[kTileM * kDW];
   __nv_bfloat16 D3G[kTileM * kDW];
-  __nv_bfloat16 W1f[64 * 16];        // [hi(W1') | hi(W1') | lo(W1') | 0] per output row
-  __half Wf[2][2][64 * 64];          // W2', W3' as [out][in], f16: hi, lo
+  __nv_bfloat16 Z1A[kTileM * 16];
+  __nv_bfloat16 G4[kTileM * 16];
+  __nv_bfloat16 W1f[64 * 16];        // [hi(W1') | hi(W1') | lo(W1') | hi b1' lo b1' 0 0] per output row
+  __half Wf[2][64 * 64];             // W2', W3' as [out][in], f16
+  __half Bz[2][64 * 16];             // [hi b | lo b | 0] per output row, f16: b2', b3'
   __nv_bfloat16 Wt[2][2][64 * 64];   // W2'^T, W3'^T as [in][out]: hi, lo
   __nv_bfloat16 W4t[2][64 * 16];     // [W4^T | W4^T] as [in][out]: hi, lo
-  float bias[3][64];                 // b1', b2', b3'
-  uint64_t mbar;
+  uint64_t mbar;                     // the tile's chain of MMAs
+  uint64_t mbar_g;                   // the tile's gradient MMAs
   uint32_t tmem_base;
   int stop;  // set by the epilogue warps at a hand-off: the issuer stops
   int n0;    // the CTA's first jet
@@ -439,8 +449,9 @@ struct MlpBwdSmem {
 static_assert(sizeof(MlpBwdSmem<128>) > 116 * 1024, "k_mlp_bwd must not fit twice on an SM");
 
 // TMEM columns: z1 [0, 64), z2 [64, 128), z3 [128, 192), e3 / e2 / e1
-// [192, 256), the gradient accumulators [256, 352) and [352, 496).
-constexpr uint32_t kTmG12 = 256, kTmG3G = 352, kBwdTmemCols = 512;
+// [192, 256), the gradient accumulators [256, 352) and [352, 496), a block
+// of ones [496, 504) (f16: K elements 0 and 1 of every row are 1).
+constexpr uint32_t kTmG12 = 256, kTmG3G = 352, kTmOnes = 496, kBwdTmemCols = 512;
 
 // Weights in the canonical K-major layouts of their MMA roles, and the
 // constant columns of the operand tiles (ones, zeros). load() issues every
@@ -454,8 +465,8 @@ struct BwdWeightLoad {
   static constexpr int kPer = (kWfJobs + kWtJobs + 511) / 512;
   float v[kPer][8];
   float4 w1;   // threads 0..63: row tid of W1
+  float b;      // threads 0..63: b1[tid]; 128..255: b2, b3
   float w4[8];  // threads 64..127: column tid - 64 of W4
-  float b;      // threads 128..319: b1, b2, b3
   __device__ void load(const MlpArgs& W, int tid, int nthr) {
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
@@ -470,15 +481,15 @@ struct BwdWeightLoad {
         for (int u = 0; u < 8; ++u) v[j][u] = Wl[(ob * 8 + u) * 64 + i];
       }
     }
-    if (tid < 64) w1 = reinterpret_cast<const float4*>(W.W1)[tid];
+    if (tid < 64) {
+      w1 = reinterpret_cast<const float4*>(W.W1)[tid];
+      b = W.b1[tid];
+    }
     if (tid >= 64 && tid < 128) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) w4[u] = W.W4[u * 64 + tid - 64];
     }
-    if (tid >= 128 && tid < 320) {
-      const int e = tid - 128;
-      b = (e < 64 ? W.b1 : (e < 128 ? W.b2 : W.b3))[e & 63];
-    }
+    if (tid >= 128 && tid < 256) b = (tid < 192 ? W.b2 : W.b3)[tid & 63];
   }
   template <class Smem>
   __device__ void store(Smem& S, int tid, int nthr) const {
@@ -487,15 +498,8 @@ struct BwdWeightLoad {
       const int q = tid + j * nthr;
       if (q < kWfJobs) {
         const int L = q >> 10, e = (q & 1023) * 4, o = e >> 6, i = e & 63;
-        uint32_t hw[2], lw[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          hw[u] = cvt_f16x2(v[j][2 * u], v[j][2 * u + 1]);
-          const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hw[u]));
-          lw[u] = cvt_f16x2(v[j][2 * u] - hf.x, v[j][2 * u + 1] - hf.y);
-        }
-        *reinterpret_cast<uint2*>(&S.Wf[L][0][cofs(o, i, 64)]) = make_uint2(hw[0], hw[1]);
-        *reinterpret_cast<uint2*>(&S.Wf[L][1][cofs(o, i, 64)]) = make_uint2(lw[0], lw[1]);
+        *reinterpret_cast<uint2*>(&S.Wf[L][cofs(o, i, 64)]) =
+            make_uint2(cvt_f16x2(v[j][0], v[j][1]), cvt_f16x2(v[j][2], v[j][3]));
       } else if (q < kWfJobs + kWtJobs) {
         const int t = q - kWfJobs, L = t >> 9, i = t & 63, ob = (t >> 6) & 7;
         uint32_t hw[4], lw[4];
@@ -508,12 +512,13 @@ struct BwdWeightLoad {
         *reinterpret_cast<uint4*>(&S.Wt[L][1][cofs(i, ob * 8, 64)]) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
     }
-    if (tid < 64) {  // W1f row tid: [hi W1 | hi W1 | lo W1 | 0]
+    if (tid < 64) {  // W1f row tid: [hi W1 | hi W1 | lo W1 | hi b1 lo b1 0 0]
       const uint32_t h01 = cvt_bf16x2(w1.x, w1.y), h23 = cvt_bf16x2(w1.z, w1.w);
       const uint32_t l01 = cvt_bf16x2(w1.x - bf16lo(h01), w1.y - bf16hi(h01));
       const uint32_t l23 = cvt_bf16x2(w1.z - bf16lo(h23), w1.w - bf16hi(h23));
+      const float bh = bf16lo(cvt_bf16x2(b, 0.f));
       *reinterpret_cast<uint4*>(&S.W1f[cofs(tid, 0, 16)]) = make_uint4(h01, h23, h01, h23);
-      *reinterpret_cast<uint4*>(&S.W1f[cofs(tid, 8, 16)]) = make_uint4(l01, l23, 0u, 0u);
+      *reinterpret_cast<uint4*>(&S.W1f[cofs(tid, 8, 16)]) = make_uint4(l01, l23, cvt_bf16x2(bh, b - bh), 0u);
     }
     if (tid >= 64 && tid < 128) {  // W4t rows (input tid - 64): [W4^T | W4^T], hi and lo
       const int i = tid - 64;
@@ -529,7 +534,12 @@ struct BwdWeightLoad {
       *reinterpret_cast<uint4*>(&S.W4t[1][cofs(i, 0, 16)]) = l;
       *reinterpret_cast<uint4*>(&S.W4t[1][cofs(i, 8, 16)]) = l;
     }
-    if (tid >= 128 && tid < 320) S.bias[(tid - 128) >> 6][(tid - 128) & 63] = b;
+    if (tid >= 128 && tid < 256) {  // Bz row: [hi b | lo b | 0], f16
+      const float bh = __half2float(__float2half_rn(b));
+      __half* row = &S.Bz[(tid - 128) >> 6][cofs(tid & 63, 0, 16)];
+      *reinterpret_cast<uint4*>(row) = make_uint4(cvt_f16x2(bh, b - bh), 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(&S.Bz[(tid - 128) >> 6][cofs(tid & 63, 8, 16)]) = make_uint4(0u, 0u, 0u, 0u);
+    }
     // constant columns, 8 at a time: F1 [80, 96) = 1 1 1 1 1 1 1 1 | 0 ..., H23 [128, 144) alike, D3G [80, 128) = 0
     const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u), zero = make_uint4(0u, 0u, 0u, 0u);
     for (int e = tid; e < kTileM * 10; e += nthr) {
@@ -682,6 +692,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
   wl.store(S, tid, blockDim.x);
   if (tid == 0) {
     mbar_init(&S.mbar, 1);
+    mbar_init(&S.mbar_g, 1);
     fence_mbar_init();
     S.stop = 0;
   }
@@ -691,17 +702,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = S.tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  uint32_t phase = 0u;
+  if (warp < 4) {  // the ones block, every lane: f16 1.0 as K elements 0 and 1
+    const uint32_t ones[8] = {0x3C003C00u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    tmem_st8_wait(tm + lane_off + kTmOnes, ones);
+  }
+  uint32_t phase = 0u, phase_g = 0u;
   bool ok = true, aborted = false, pending = false, any_tile = false;
+  bool g_open = false;  // a gradient commit not yet seen complete (its parity: phase_g)
 
   // ---- issuer (warp 16, lane 0 issues): one hand-off per step
   constexpr uint32_t kId = idesc_bf16_m128(64), kIdF16 = idesc_f16_m128(64);
   constexpr uint32_t kIdG12 = idesc_bf16_m128_mn(kF1W), kIdG3G = idesc_bf16_m128_mn(kH23W);
   constexpr uint32_t kF1Sbo = kF1W / 8 * 128, kH23Sbo = kH23W / 8 * 128, kDSbo = kDW / 8 * 128;
-  // D = A (W_hi + W_lo), K = 64, A from TMEM (K step j at column 16j + 8 of
-  // the layer's 64-column block): the weights' rounding error is the same for
-  // every pair row and would not average out of the gradient sums, so they
-  // enter as two terms
+  // z = b + A W, K = 64, A (f16 h) from TMEM (K step j at column 16j + 8 of
+  // the layer's 64-column block), the bias through the ones block
+  auto gemm_z = [&](uint32_t d, uint32_t a_tm, uint32_t w, uint32_t bz) {
+    mma_f16_ta(d, tm + kTmOnes, smem_desc(bz, 128, 256), kIdF16, 0u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mma_f16_ta(d, a_tm + 16u * k + 8u, smem_desc(w + 256u * k, 128, 1024), kIdF16, 1u);
+  };
+  // D = A (W_hi + W_lo), K = 64, A (bf16 d) from TMEM: the weights' rounding
+  // error is the same for every pair row and would not average out of the
+  // gradient sums, so they enter as two terms
   auto gemm64_ta = [&](uint32_t d, uint32_t a_tm, uint32_t b_hi, uint32_t b_lo, uint32_t id) {
 #pragma unroll
     for (int part = 0; part < 2; ++part)
@@ -722,20 +744,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
   auto issue_step = [&](int step) {
     const uint32_t f1 = smem_u32(S.F1), h23 = smem_u32(S.H23), d12 = smem_u32(S.D12), d3g = smem_u32(S.D3G);
     switch (step) {
-      case kStepZ1: {  // z1 = [hi f | lo f | hi f] [hi W1 | hi W1 | lo W1]; behind it e3 = [hi g | lo g] [W4 | W4]
-        mma_f16(tm, smem_desc(f1, 128, kF1Sbo), smem_desc(smem_u32(S.W1f), 128, 256), kId, 0u);
+      case kStepZ1: {  // z1 = [hi f | lo f | hi f | 1 1] [hi W1 | hi W1 | lo W1 | hi b1 lo b1]; behind it e3 = [hi g | lo g] [W4 | W4]
+        mma_f16(tm, smem_desc(smem_u32(S.Z1A), 128, 256), smem_desc(smem_u32(S.W1f), 128, 256), kId, 0u);
         mma_commit(&S.mbar);
-        const uint64_t ga = smem_desc(d3g + kD3G / 8 * 128, 128, kDSbo);
+        const uint64_t ga = smem_desc(smem_u32(S.G4), 128, 256);
         mma_f16(tm + 192u, ga, smem_desc(smem_u32(S.W4t[0]), 128, 256), kId, 0u);
         mma_f16(tm + 192u, ga, smem_desc(smem_u32(S.W4t[1]), 128, 256), kId, 1u);
         break;
       }
       case kStepZ2:  // its commit also covers e3
-        gemm64_ta(tm + 64u, tm, smem_u32(S.Wf[0][0]), smem_u32(S.Wf[0][1]), kIdF16);
+        gemm_z(tm + 64u, tm, smem_u32(S.Wf[0]), smem_u32(S.Bz[0]));
         mma_commit(&S.mbar);
         break;
       case kStepZ3:
-        gemm64_ta(tm + 128u, tm + 64u, smem_u32(S.Wf[1][0]), smem_u32(S.Wf[1][1]), kIdF16);
+        gemm_z(tm + 128u, tm + 64u, smem_u32(S.Wf[1]), smem_u32(S.Bz[1]));
         mma_commit(&S.mbar);
         break;
       case kStepE2:  // e2 = d3 W3' (d3 bf16 in TMEM over z3)
@@ -747,9 +769,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
         mma_commit(&S.mbar);
         gemm_grad(tm + kTmG3G, d3g, kDSbo, h23, kH23Sbo, kIdG3G);
         break;
-      default:  // [d1 | d2]^T [f | h1 | 1]; its commit also covers the one above
+      default:  // [d1 | d2]^T [f | h1 | 1]; its commit (on the gradient barrier) also covers the one above
         gemm_grad(tm + kTmG12, d12, kDSbo, f1, kF1Sbo, kIdG12);
-        mma_commit(&S.mbar);
+        mma_commit(&S.mbar_g);
         break;
     }
   };
@@ -786,6 +808,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
     ok = ok && done;
     tc_fence_after();
   };
+  auto wait_g = [&]() {  // one commit per tile, waited before the next tile's is issued
+    const bool done = mbar_wait(&S.mbar_g, phase_g);
+    if (done) {
+      phase_g ^= 1u;
+      g_open = false;
+    }
+    ok = ok && done;
+    tc_fence_after();
+  };
   auto store16 = [&](__nv_bfloat16* T, int width, int col, const float* v) {
     uint32_t w[8];
 #pragma unroll
@@ -801,22 +832,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
     for (int i = 0; i < 8; ++i) w[i] = cvt_bf16x2(v[2 * i], v[2 * i + 1]);
     tmem_st8_wait(tm + lane_off + 64u * k + 16u * c + 8u, w);
   };
-  // z_k + b_k -> h (bf16 to `T` at column `col`; for k < 2 f16 into TMEM as
-  // the next layer's A operand) and GELU' (f16 into TMEM, k < 2) or, for
-  // k = 2, d3 = e3 GELU'(z3) to D3G and TMEM
+  // z_k (bias included) -> h (bf16 to `T` at column `col`; for k < 2 f16
+  // into TMEM as the next layer's A operand) and GELU' (f16 into TMEM, k < 2)
+  // or, for k = 2, d3 = e3 GELU'(z3) to D3G and TMEM
   auto hidden = [&](int k, __nv_bfloat16* T, int width, int col) {
     float z[16], h[16];
     const uint32_t ta = tm + lane_off + 64u * k + 16u * c;
     tmem_ld16_wait(ta, z);
-    const float4* bq = reinterpret_cast<const float4*>(&S.bias[k][16 * c]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 bb = bq[i];
-      z[4 * i] += bb.x;
-      z[4 * i + 1] += bb.y;
-      z[4 * i + 2] += bb.z;
-      z[4 * i + 3] += bb.w;
-    }
 #pragma unroll
     for (int i = 0; i < 16; ++i) gelu_tanh_and_grad(z[i], h[i], z[i]);
     store16(T, width, col, h);
@@ -849,7 +871,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
     store16(S.D12, kDW, 64 * k + 16 * c, e);
     if (k == 1) d_to_tmem(1, e);
   };
-  // tile t's row r as operand words: features (c = 0: [hi f | lo f], [hi f | 0])
+  // tile t's row r as operand words: features (c = 0: [hi f | lo f], [hi f | 0 0])
   // or the gradient record (c = 1: hi g, lo g); zero past the jet's pairs
   auto prep = [&](int t, int m, const float* gjet, uint4& w0, uint4& w1) {
     const int p = t * kTileM + r;
@@ -891,19 +913,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
   auto epilogue_tile = [&](int t, int t_last, int m, const float* gjet, uint4& w0, uint4& w1, bool& have) -> bool {
     if (!have) prep(t, m, gjet, w0, w1);
     have = false;
-    if (pending) {  // the previous tile's gradient MMAs read F1, H23, D12 and D3G
-      wait();
+    // z1's and e3's operands (the previous tile's z1 and e3 are long done)
+    if (c == 0) {
+      *reinterpret_cast<uint4*>(S.Z1A + cofs(r, 0, 16)) = w0;
+      *reinterpret_cast<uint4*>(S.Z1A + cofs(r, 8, 16)) = make_uint4(w1.x, w1.y, kOnesBf16x2, 0u);
+    } else if (c == 1) {
+      *reinterpret_cast<uint4*>(S.G4 + cofs(r, 0, 16)) = w0;
+      *reinterpret_cast<uint4*>(S.G4 + cofs(r, 8, 16)) = w1;
+    }
+    if (!handoff()) return false;  // z1, e3
+    wait();
+    if (pending) {  // the previous tile's gradient MMAs read F1, H23, D12 and D3G (done before z1 was)
+      wait_g();
       pending = false;
     }
-    if (c == 0) {
+    if (c == 0) {  // f and g for this tile's gradient MMAs
       *reinterpret_cast<uint4*>(S.F1 + cofs(r, 0, kF1W)) = w0;
       *reinterpret_cast<uint4*>(S.F1 + cofs(r, 8, kF1W)) = w1;
     } else if (c == 1) {
       *reinterpret_cast<uint4*>(S.D3G + cofs(r, kD3G, kDW)) = w0;
       *reinterpret_cast<uint4*>(S.D3G + cofs(r, kD3G + 8, kDW)) = w1;
     }
-    if (!handoff()) return false;  // z1, e3
-    wait();
     hidden(0, S.F1, kF1W, 16 + 16 * c);
     if (!handoff()) return false;  // z2
     wait();
@@ -923,6 +953,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
     delta(0);
     if (!handoff()) return false;  // the [d1 | d2] gradient
     pending = true;
+    g_open = true;
     any_tile = true;
     return true;
   };
@@ -942,7 +973,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
       aborted = issuer ? !issue_tile() : !epilogue_tile(t, t_last, m, gjet, w0, w1, have);
     aborted = __syncthreads_or(aborted || !ok) != 0;
   }
-  if (pending && !aborted) wait();
+  if (pending && !aborted) wait_g();
   aborted = __syncthreads_or(aborted || !ok) != 0;
   tc_fence_after();
   any_tile = __syncthreads_or(any_tile) != 0;
@@ -983,7 +1014,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
       part[q] = v;
     }
   }
-  if (aborted && tid == 0) (void)mbar_wait(&S.mbar, phase ^ 1u);  // bounded: the last commit before TMEM is freed
+  if (aborted && tid == 0) {  // bounded: the last commits before TMEM is freed
+    (void)mbar_wait(&S.mbar, phase ^ 1u);
+    if (g_open) (void)mbar_wait(&S.mbar_g, phase_g);
+  }
   __syncthreads();
   if (warp == 0) tmem_dealloc(S.tmem_base, kBwdTmemCols);
 }
