@@ -51,7 +51,7 @@ BWD_FLOP_PER_PAIR = 2 * (4 * 64 + 2 * 64 * 64) + 2 * (8 * 64 + 2 * 64 * 64) + 2 
 BWD_MMA_FLOP_PER_ROW = 2 * (2 * 16 * 64 + 4 * 64 * 64) + 2 * (16 * 72 + 2 * 64 * 72 + 64 * 16)
 PROFILE = os.path.join(ROOT, "profiles", "k_fused_cluster_n128_p128.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "part_pair_bias_b200", "csrc", f)
-                  for f in ("pb_kernels.cuh", "pb_device.cuh", "pairbias.cu")]
+                  for f in ("pb_kernels.cuh", "pb_backward.cuh", "pb_device.cuh", "pairbias.cu")]
 
 
 def parse():
