@@ -306,17 +306,6 @@ struct SmemUBias4 {  // the CTA's 4 heads from h0, staged by stage_bias_heads
   __device__ __forceinline__ TriBlockS<4> head(int h) const { return TriBlockS<4>{U + (h - h0)}; }
 };
 
-// Masked rows (slot s with comp[s] < 0) of `out`, every head: 16 threads per
-// slot, thread (head, half) of it, no division.
-template <int PM>
-__device__ void zero_masked_rows_bwd(const Particles<PM>& S, const JetArgs& J, uint16_t* out, int n) {
-  if (J.ptr) return;
-  const int P = J.P, hh = (threadIdx.x >> 1) & 7, half = threadIdx.x & 1;
-  for (int s = threadIdx.x >> 4; s < P; s += blockDim.x >> 4)
-    if (S.comp[s] < 0)
-      *reinterpret_cast<uint4*>(out + (((size_t)n * kH + hh) * P + s) * kD + half * 8) = make_uint4(0, 0, 0, 0);
-}
-
 template <int PM>
 __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -369,10 +358,10 @@ __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
     }
     // masked rows of every head: dq and dk by the jet's first CTA, dv by its second
     if (hg == 0) {
-      zero_masked_rows_bwd<PM>(S.part, J, X.dq, n);
-      zero_masked_rows_bwd<PM>(S.part, J, X.dk, n);
+      zero_masked_rows<PM>(S.part, J, X.dq, n);
+      zero_masked_rows<PM>(S.part, J, X.dk, n);
     }
-    if (hg == kBwdHeadGroups - 1) zero_masked_rows_bwd<PM>(S.part, J, X.dv, n);
+    if (hg == kBwdHeadGroups - 1) zero_masked_rows<PM>(S.part, J, X.dv, n);
     __syncthreads();
   }
 }

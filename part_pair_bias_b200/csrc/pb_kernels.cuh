@@ -1458,17 +1458,18 @@ __device__ void attention_block(const Particles<PM>& S, const JetArgs& J, const 
   }
 }
 
-// Masked query rows of a padded jet are 0 (all of them when the jet is empty).
+// Masked query rows of a padded jet are 0 (all of them when the jet is
+// empty). Block-wide (blockDim.x a multiple of 16): 16 threads per slot,
+// thread (head, half) of it, no division.
 template <int PM>
 __device__ void zero_masked_rows(const Particles<PM>& S, const JetArgs& J, uint16_t* out, int n) {
   if (J.ptr) return;
-  const int P = J.P;
-  for (int idx = threadIdx.x; idx < kH * P * 2; idx += blockDim.x) {
-    const int half = idx & 1, s = (idx >> 1) % P, h = (idx >> 1) / P;
+  const int P = J.P, h = (threadIdx.x >> 1) & 7, half = threadIdx.x & 1;
+  for (int s = threadIdx.x >> 4; s < P; s += blockDim.x >> 4)
     if (S.comp[s] < 0)
       *reinterpret_cast<uint4*>(out + (((size_t)n * kH + h) * P + s) * kD + half * 8) = make_uint4(0, 0, 0, 0);
-  }
 }
+static_assert(kH == 8, "zero_masked_rows maps 16 threads to (head, half) of a slot");
 
 // ------------------------------------------- k_attn_bias (bias read from HBM)
 
