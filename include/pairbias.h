@@ -330,15 +330,18 @@ pb_status pair_attention_forward_noalloc(const pb_jets *jets, const pb_mlp *mlp,
  * accumulation and fp32 softmax statistics; dL/dU[h,i,j] + dL/dU[h,j,i] is
  * kept as one 32-byte record of 8 fp32 values per unordered pair. The MLP
  * backward recomputes layers 1-3 on tcgen05 with fp32 accumulation in TMEM
- * (features and layer-1 weights as bf16 hi + lo terms, h1 and h2 as f16,
- * W2 and W3 as f16 hi + lo terms) and the tanh approximation of GELU,
+ * (features, layer-1 weights and bias as bf16 hi + lo terms; h1, h2, W2 and
+ * W3 as f16, the forward's own operands; b2, b3 as f16 hi + lo terms) and
+ * the tanh approximation of GELU,
  * GELU(z) = z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))), with its exact
  * derivative; the products of the backward pass use bf16 operands (weights
- * as hi + lo terms) with fp32 accumulation. The weight gradients accumulate
- * in fp32 per CTA and are summed over CTAs in a fixed order, so the result
- * does not depend on timing.
- * Launches, in order on `stream`: the bias kernel of pairbias_mlp_forward,
- * the attention backward, the MLP backward and a gradient-sum kernel (with
+ * as hi + lo terms) with fp32 accumulation. The weight gradients are tcgen05
+ * products (bf16 d and h, fp32 accumulation in TMEM over each CTA's tiles)
+ * and are summed over CTAs in a fixed order, so the result does not depend
+ * on timing.
+ * Launches, in order on `stream`: the balanced kernel's MLP phase (the bias
+ * records), the attention backward, the MLP backward and a gradient-sum
+ * kernel (per chunk of up to 8192 jets the first three; with
  * N = 0 only the last, writing zeros). Errors as for
  * pair_attention_forward; PB_EINVAL also for a missing or small workspace
  * or a NULL gradient buffer. */
