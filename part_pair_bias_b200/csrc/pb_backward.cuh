@@ -382,13 +382,15 @@ __global__ void __launch_bounds__(256, 2) k_attn_bwd(JetArgs J, BwdArgs X) {
 // from TMEM) by the f16 weights, as the forward kernels do, and adds the
 // layer's bias through one more MMA (a TMEM block of ones times [hi b | lo b]);
 // the backward products take bf16 d and bf16 hi + lo weights; f, g and the
-// folded layer-1 weights and bias enter as bf16 hi + lo terms. The weight gradients are two MMAs per tile over the tile's
-// rows (K = 128) with both operands read transposed (MN-major) from the same
-// row-major tiles, accumulated in fp32 TMEM over all the CTA's tiles; the
-// second overlaps the next tile's feature and gradient-record loads. GELU is
-// the tanh form the forward kernels use; GELU'(z) is computed with h and
-// parked in TMEM (f16, in the first half of the quarter's z columns, h in
-// the second half) until the backward step needs it.
+// folded layer-1 weights and bias enter as bf16 hi + lo terms. The weight
+// gradients are two MMAs per tile over the tile's rows (K = 128) with both
+// operands read transposed (MN-major) from the same row-major tiles,
+// accumulated in fp32 TMEM over all the CTA's tiles; issued behind e1 and
+// after the last delta step, they run while the next tile's z1 is staged
+// and computed. GELU is the tanh form the forward kernels use; GELU'(z) is
+// computed with h and parked in TMEM (f16, in the first half of the
+// quarter's z columns, h in the second half) until the backward step needs
+// it.
 
 constexpr int kBwdMaxCtas = 256;     // partial-gradient slots in the workspace
 constexpr int kFoldedFloats = 9160;  // W1 b1 W2 b2 W3 b3 W4 b4, as pb_fold_affine lays them out
@@ -530,7 +532,8 @@ struct BwdWeightLoad {
       *reinterpret_cast<uint4*>(&S.Bz[(tid - 128) >> 6][cofs(tid & 63, 8, 16)]) = make_uint4(0u, 0u, 0u, 0u);
     }
     // constant columns, 8 at a time: F1 [80, 96) = 1 1 1 1 1 1 1 1 | 0 ..., H23 [128, 144) alike, D3G [80, 128) = 0
-    const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u), zero = make_uint4(0u, 0u, 0u, 0u);
+    const uint4 ones = make_uint4(kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2);
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     for (int e = tid; e < kTileM * 10; e += nthr) {
       const int r = e & 127, g = e >> 7;  // g: 0, 1 of F1; 2, 3 of H23; 4..9 of D3G
       if (g < 2) *reinterpret_cast<uint4*>(&S.F1[cofs(r, kF1Ones + 8 * g, kF1W)]) = g == 0 ? ones : zero;
@@ -733,7 +736,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) k_mlp_bwd(JetArgs J, MlpArgs W
   auto issue_step = [&](int step) {
     const uint32_t f1 = smem_u32(S.F1), h23 = smem_u32(S.H23), d12 = smem_u32(S.D12), d3g = smem_u32(S.D3G);
     switch (step) {
-      case kStepZ1: {  // z1 = [hi f | lo f | hi f | 1 1] [hi W1 | hi W1 | lo W1 | hi b1 lo b1]; behind it e3 = [hi g | lo g] [W4 | W4]
+      case kStepZ1: {  // z1 = [hi f | lo f | hi f | 1 1] [hi W1 | hi W1 | lo W1 | hi b1 lo b1];
+                       // behind it e3 = [hi g | lo g] [W4 | W4]
         mma_f16(tm, smem_desc(smem_u32(S.Z1A), 128, 256), smem_desc(smem_u32(S.W1f), 128, 256), kId, 0u);
         mma_commit(&S.mbar);
         const uint64_t ga = smem_desc(smem_u32(S.G4), 128, 256);
